@@ -1,0 +1,555 @@
+// C ABI of the LSA hot path (declarations and contracts in include/lsa.h).
+//
+// Host side only: argument validation, workspace layout, TMA tensor-map
+// encoding and kernel launches. Nothing here allocates device memory or
+// synchronises the stream (except lsa_device_status, which exists to do so).
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "internal.h"
+#include "lsa.h"
+#include "ptx.cuh"
+
+namespace lsa {
+
+// Per-device status word: kernels that give up waiting OR LSA_ERR_TIMEOUT into it.
+__device__ int g_device_status = 0;
+
+namespace {
+
+thread_local char g_err[512] = {0};
+
+lsa_status_t fail(lsa_status_t st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+lsa_status_t cuda_fail(cudaError_t e, const char* what) {
+  return fail(LSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+#define LSA_CHECK_CUDA(expr, what)                  \
+  do {                                              \
+    cudaError_t _e = (expr);                        \
+    if (_e != cudaSuccess) return cuda_fail(_e, what); \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+bool is_pow2_in(int x, int lo, int hi) { return x >= lo && x <= hi && (x & (x - 1)) == 0; }
+
+// ------------------------------------------------------------ tensor maps --
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D row-major tensor [rows, inner] with 128-byte swizzled boxes [box_rows, box_inner].
+lsa_status_t make_tmap(CUtensorMap* m, const void* base, bool fp8, uint64_t inner, uint64_t rows,
+                       uint32_t box_inner, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return fail(LSA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  const uint32_t elt = fp8 ? 1 : 2;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * elt};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(LSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return LSA_OK;
+}
+
+// --------------------------------------------------------------- validation --
+lsa_status_t check_budget(lsa_budget_t bu) {
+  if (bu.k < 1 || bu.k > 8192) return fail(LSA_ERR_UNSUPPORTED, "budget k=%d outside [1, 8192]", bu.k);
+  if (bu.sink < 0 || bu.window < 0) return fail(LSA_ERR_INVALID_ARG, "negative sink/window");
+  if (static_cast<long long>(bu.sink) + bu.window > bu.k)
+    return fail(LSA_ERR_INVALID_ARG, "sink (%d) + window (%d) exceed the budget k=%d", bu.sink, bu.window, bu.k);
+  return LSA_OK;
+}
+
+lsa_status_t check_indexer(const lsa_indexer_in_t* in, bool allow_fp8) {
+  if (!in) return fail(LSA_ERR_INVALID_ARG, "null indexer descriptor");
+  if (in->B < 1 || in->T < 1 || in->L_max < 1) return fail(LSA_ERR_INVALID_ARG, "B, T and L_max must be >= 1");
+  if (in->d != 64 && in->d != 128) return fail(LSA_ERR_UNSUPPORTED, "indexer d=%d not in {64, 128}", in->d);
+  if (!is_pow2_in(in->H, 4, 128)) return fail(LSA_ERR_UNSUPPORTED, "indexer H=%d not in {4,...,128} (power of 2)", in->H);
+  if (in->L_max % 128 != 0) return fail(LSA_ERR_UNSUPPORTED, "L_max=%d must be a multiple of 128", in->L_max);
+  if (static_cast<long long>(in->B) * in->L_max >= (1ll << 31) ||
+      static_cast<long long>(in->B) * in->T * in->H >= (1ll << 31))
+    return fail(LSA_ERR_UNSUPPORTED, "tensor too large for 32-bit row coordinates");
+  if (!in->seq_len || !in->q || !in->w || !in->k) return fail(LSA_ERR_INVALID_ARG, "null indexer tensor");
+  if (!aligned16(in->q) || !aligned16(in->k) || !aligned16(in->w))
+    return fail(LSA_ERR_INVALID_ARG, "indexer tensors must be 16-byte aligned");
+  if (in->dtype == LSA_E4M3) {
+    if (!allow_fp8) return fail(LSA_ERR_UNSUPPORTED, "e4m3 inputs are supported by flat indexing only");
+    if (in->d != 128) return fail(LSA_ERR_UNSUPPORTED, "e4m3 indexer requires d = 128");
+    if (!in->q_scale || !in->k_scale) return fail(LSA_ERR_INVALID_ARG, "e4m3 inputs need q_scale and k_scale");
+  } else if (in->dtype != LSA_BF16) {
+    return fail(LSA_ERR_INVALID_ARG, "unknown dtype %d", static_cast<int>(in->dtype));
+  }
+  return LSA_OK;
+}
+
+lsa_status_t check_attn(const lsa_attn_in_t* at, int k) {
+  if (!at) return fail(LSA_ERR_INVALID_ARG, "null attention descriptor");
+  if (at->B < 1 || at->T < 1 || at->L_max < 1) return fail(LSA_ERR_INVALID_ARG, "B, T and L_max must be >= 1");
+  if (at->Hq < 1 || at->Hq > 128) return fail(LSA_ERR_UNSUPPORTED, "Hq=%d outside [1, 128]", at->Hq);
+  const bool mla = at->d_qk == 576 && at->d_v == 512;
+  const bool small = at->d_qk == 64 && at->d_v == 64;
+  if (!mla && !small) return fail(LSA_ERR_UNSUPPORTED, "(d_qk, d_v) = (%d, %d) unsupported", at->d_qk, at->d_v);
+  if (!at->seq_len || !at->q || !at->k || !at->v) return fail(LSA_ERR_INVALID_ARG, "null attention tensor");
+  if (!aligned16(at->q) || !aligned16(at->k) || !aligned16(at->v))
+    return fail(LSA_ERR_INVALID_ARG, "attention tensors must be 16-byte aligned");
+  if (at->k_row_stride < at->d_qk || at->k_row_stride % 8 || at->v_row_stride < at->d_v || at->v_row_stride % 8)
+    return fail(LSA_ERR_INVALID_ARG, "row strides must cover the row and be multiples of 8 elements");
+  const bool alias = at->v == at->k && at->v_row_stride == at->k_row_stride;
+  if (mla && !alias) return fail(LSA_ERR_UNSUPPORTED, "d_qk=576/d_v=512 requires v == k (MLA latent rows)");
+  if (!(at->scale > 0.f) || !std::isfinite(at->scale)) return fail(LSA_ERR_INVALID_ARG, "scale must be finite and > 0");
+  if (k < 1 || k > 8192) return fail(LSA_ERR_UNSUPPORTED, "index row length %d outside [1, 8192]", k);
+  if (static_cast<long long>(at->B) * at->T * at->Hq >= (1ll << 31))
+    return fail(LSA_ERR_UNSUPPORTED, "too many query rows");
+  return LSA_OK;
+}
+
+// ---------------------------------------------------------- plan helpers --
+struct FlatPlan {
+  int NQ, N, G, n_tiles;
+};
+
+FlatPlan flat_plan(int T, int H, int L_rows) {
+  FlatPlan p;
+  int n = 16;
+  while (n < 256 && n < T * H) n <<= 1;
+  if (n < H) n = H;
+  p.N = n;
+  p.NQ = n / H;
+  p.G = (T + p.NQ - 1) / p.NQ;
+  p.n_tiles = (L_rows + 127) / 128;
+  return p;
+}
+
+struct AttnPlan {
+  int n_split, bps, nvp;
+};
+
+AttnPlan attn_plan(const lsa_attn_in_t* at, int k) {
+  AttnPlan p;
+  const int rows = at->B * at->T;
+  p.nvp = at->d_v >= 512 ? 2 : 1;
+  const int nblk = (k + kAttnBN - 1) / kAttnBN;
+  int ns = device_sm_count() / (rows * p.nvp);
+  if (ns < 1) ns = 1;
+  if (ns > nblk) ns = nblk;
+  p.bps = (nblk + ns - 1) / ns;
+  p.n_split = (nblk + p.bps - 1) / p.bps;
+  return p;
+}
+
+size_t attn_ws_bytes(const lsa_attn_in_t* at, int k) {
+  const AttnPlan p = attn_plan(at, k);
+  if (p.n_split <= 1) return 0;
+  const size_t rows = static_cast<size_t>(at->B) * at->T;
+  const size_t nm = rows * p.n_split * at->Hq;
+  return align_up(nm * at->d_v * 4, 256) + 2 * align_up(nm * 4, 256);
+}
+
+size_t hier_ws_bytes(const lsa_indexer_in_t* in, int P, int M, bool pages_external) {
+  const size_t rows = static_cast<size_t>(in->B) * in->T;
+  size_t s = align_up(rows * (in->L_max / P) * 4, 256);          // page scores
+  if (!pages_external) s += align_up(rows * M * 4, 256);          // recalled pages
+  s += align_up(rows * static_cast<size_t>(M) * P * 4, 256);      // fine candidate scores
+  return s;
+}
+
+size_t flat_ws_bytes(const lsa_indexer_in_t* in, bool scores_external) {
+  if (scores_external) return 0;
+  return align_up(static_cast<size_t>(in->B) * in->T * in->L_max * 4, 256);
+}
+
+// ------------------------------------------------------------ launchers --
+lsa_status_t run_flat_scores(const lsa_indexer_in_t* in, const void* keys, int L_rows, int vis_div,
+                             float* scores, cudaStream_t st) {
+  const bool fp8 = in->dtype == LSA_E4M3;
+  const FlatPlan fp = flat_plan(in->T, in->H, L_rows);
+  CUtensorMap tm_k, tm_q;
+  const uint32_t box_inner = fp8 ? 128 : 64;
+  lsa_status_t s = make_tmap(&tm_k, keys, fp8, in->d, static_cast<uint64_t>(in->B) * L_rows, box_inner, 128);
+  if (s != LSA_OK) return s;
+  s = make_tmap(&tm_q, in->q, fp8, in->d, static_cast<uint64_t>(in->B) * in->T * in->H, box_inner, fp.N);
+  if (s != LSA_OK) return s;
+  IndexerArgs a{};
+  a.B = in->B; a.T = in->T; a.H = in->H; a.d = in->d;
+  a.L_rows = L_rows; a.L_max = in->L_max;
+  a.NQ = fp.NQ; a.N = fp.N; a.G = fp.G; a.n_tiles = fp.n_tiles;
+  a.vis_div = vis_div; a.gather = 0;
+  indexer_pick_pipeline(in->d, fp8, fp.N, &a.stages, &a.nbuf_b);
+  a.n_items = static_cast<long long>(in->B) * fp.G * fp.n_tiles;
+  a.seq_len = in->seq_len; a.w = in->w; a.q_scale = in->q_scale; a.k_scale = in->k_scale;
+  a.out = scores; a.out_row_stride = L_rows;
+  a.inv_sqrt_d = 1.0f / std::sqrt(static_cast<float>(in->d));
+  a.status = device_status_ptr();
+  const int grid = static_cast<int>(std::min<long long>(a.n_items, device_sm_count()));
+  if (grid < 1) return LSA_OK;
+  LSA_CHECK_CUDA(launch_indexer(tm_k, tm_q, a, fp8, grid, st), "indexer launch");
+  return LSA_OK;
+}
+
+lsa_status_t run_select(int mode, int B, int T, int L_max, const int* seq_len, const float* scores,
+                        long long row_stride, int n_slots, lsa_budget_t bu, int P, int M, const int* pages,
+                        int* out, int out_len, cudaStream_t st) {
+  SelectArgs a{};
+  a.mode = mode; a.B = B; a.T = T; a.L_max = L_max; a.seq_len = seq_len;
+  a.scores = scores; a.row_stride = row_stride; a.n_slots = n_slots;
+  a.k = bu.k; a.sink = bu.sink; a.window = bu.window; a.P = P; a.M = M; a.pages = pages;
+  a.out = out; a.out_len = out_len;
+  int cap = 0;
+  const int C = select_cluster_size(B * T, n_slots, device_sm_count(), &cap);
+  a.cap = cap;
+  LSA_CHECK_CUDA(launch_select(a, C, st), "select launch");
+  return LSA_OK;
+}
+
+lsa_status_t run_hier(const lsa_indexer_in_t* in, const void* page_keys, int P, int M, lsa_budget_t bu,
+                      int* idx, int* pages_out, void* ws, cudaStream_t st) {
+  const size_t rows = static_cast<size_t>(in->B) * in->T;
+  const int n_pages = in->L_max / P;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  float* page_scores = reinterpret_cast<float*>(w);
+  w += align_up(rows * n_pages * 4, 256);
+  int* pages = pages_out;
+  if (!pages) {
+    pages = reinterpret_cast<int*>(w);
+    w += align_up(rows * M * 4, 256);
+  }
+  float* cand = reinterpret_cast<float*>(w);
+
+  // 1) coarse scores over full, fully visible pages
+  lsa_status_t s = run_flat_scores(in, page_keys, n_pages, P, page_scores, st);
+  if (s != LSA_OK) return s;
+  // 2) recall: forced sink/window pages + top pages of the dynamic region (ascending)
+  s = run_select(kSelectPages, in->B, in->T, in->L_max, in->seq_len, page_scores, n_pages, n_pages, bu, P, M,
+                 nullptr, pages, M, st);
+  if (s != LSA_OK) return s;
+  // 3) fine scores over the recalled pages' tokens
+  {
+    CUtensorMap tm_k, tm_q;
+    s = make_tmap(&tm_k, in->k, false, in->d, static_cast<uint64_t>(in->B) * in->L_max, 64, P);
+    if (s != LSA_OK) return s;
+    const int N = in->H < 16 ? 16 : in->H;
+    s = make_tmap(&tm_q, in->q, false, in->d, static_cast<uint64_t>(in->B) * in->T * in->H, 64, N);
+    if (s != LSA_OK) return s;
+    IndexerArgs a{};
+    a.B = in->B; a.T = in->T; a.H = in->H; a.d = in->d;
+    a.L_rows = in->L_max; a.L_max = in->L_max;
+    a.NQ = 1; a.N = N; a.G = in->T;
+    a.n_tiles = (M * P + 127) / 128;
+    a.vis_div = 1; a.gather = 1;
+    indexer_pick_pipeline(in->d, false, N, &a.stages, &a.nbuf_b);
+    a.n_items = static_cast<long long>(rows) * a.n_tiles;
+    a.seq_len = in->seq_len; a.w = in->w;
+    a.out = cand; a.out_row_stride = static_cast<long long>(M) * P;
+    a.inv_sqrt_d = 1.0f / std::sqrt(static_cast<float>(in->d));
+    a.pages = pages; a.M = M; a.P = P; a.sink = bu.sink; a.window = bu.window;
+    a.status = device_status_ptr();
+    const int grid = static_cast<int>(std::min<long long>(a.n_items, device_sm_count()));
+    LSA_CHECK_CUDA(launch_indexer(tm_k, tm_q, a, false, grid, st), "fine indexer launch");
+  }
+  // 4) token selection restricted to the recalled pages
+  return run_select(kSelectHierTokens, in->B, in->T, in->L_max, in->seq_len, cand, static_cast<long long>(M) * P,
+                    M * P, bu, P, M, pages, idx, bu.k, st);
+}
+
+lsa_status_t run_attn(const lsa_attn_in_t* at, const int* idx, int k, void* out, float* lse, void* ws,
+                      cudaStream_t st) {
+  const AttnPlan p = attn_plan(at, k);
+  CUtensorMap tm_q;
+  lsa_status_t s = make_tmap(&tm_q, at->q, false, at->d_qk, static_cast<uint64_t>(at->B) * at->T * at->Hq, 64, 128);
+  if (s != LSA_OK) return s;
+  AttnArgs a{};
+  a.B = at->B; a.T = at->T; a.Hq = at->Hq; a.L_max = at->L_max;
+  a.d_qk = at->d_qk; a.d_v = at->d_v; a.k = k;
+  a.scale_log2 = at->scale * 1.4426950408889634f;
+  a.idx = idx;
+  a.kp = static_cast<const uint16_t*>(at->k);
+  a.vp = static_cast<const uint16_t*>(at->v);
+  a.k_stride = at->k_row_stride; a.v_stride = at->v_row_stride;
+  a.sep_v = !(at->v == at->k && at->v_row_stride == at->k_row_stride);
+  a.n_split = p.n_split; a.blocks_per_split = p.bps;
+  a.out = static_cast<uint16_t*>(out);
+  a.lse = lse;
+  a.status = device_status_ptr();
+  if (p.n_split > 1) {
+    const size_t nm = static_cast<size_t>(at->B) * at->T * p.n_split * at->Hq;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    a.part_o = reinterpret_cast<float*>(w);
+    w += align_up(nm * at->d_v * 4, 256);
+    a.part_m = reinterpret_cast<float*>(w);
+    w += align_up(nm * 4, 256);
+    a.part_l = reinterpret_cast<float*>(w);
+  }
+  LSA_CHECK_CUDA(launch_attn(tm_q, a, st), "attention launch");
+  if (p.n_split > 1) LSA_CHECK_CUDA(launch_attn_combine(a, st), "attention combine launch");
+  return LSA_OK;
+}
+
+lsa_status_t check_ws(void* ws, size_t have, size_t need) {
+  if (have < need) return fail(LSA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", have, need);
+  if (need > 0 && (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)))
+    return fail(LSA_ERR_INVALID_ARG, "workspace must be non-null and 256-byte aligned");
+  return LSA_OK;
+}
+
+lsa_status_t check_hier_params(const lsa_indexer_in_t* in, int P, int M, lsa_budget_t bu) {
+  if (in->dtype != LSA_BF16) return fail(LSA_ERR_UNSUPPORTED, "hierarchical indexing takes bf16 inputs");
+  if (!is_pow2_in(P, 16, 128)) return fail(LSA_ERR_UNSUPPORTED, "page size P=%d not in {16,32,64,128}", P);
+  if (in->L_max % P) return fail(LSA_ERR_INVALID_ARG, "L_max must be a multiple of P");
+  const int forced_max = (bu.sink + P - 1) / P + (bu.window + P - 1) / P + 1;
+  if (M < forced_max) return fail(LSA_ERR_INVALID_ARG, "M=%d below the %d pages sink/window can force", M, forced_max);
+  if (static_cast<long long>(M) * P > (1 << 24)) return fail(LSA_ERR_UNSUPPORTED, "M * P too large");
+  return LSA_OK;
+}
+
+}  // namespace
+
+int* device_status_ptr() {
+  static int* cache[64] = {nullptr};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (!cache[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_status) == cudaSuccess) cache[dev] = static_cast<int*>(p);
+  }
+  return cache[dev];
+}
+
+int device_sm_count() {
+  static int cache[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (!cache[dev]) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = n > 0 ? n : 148;
+  }
+  return cache[dev];
+}
+
+cudaError_t set_max_smem(const void* func, size_t bytes) {
+  return cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+}
+
+}  // namespace lsa
+
+using namespace lsa;
+
+extern "C" {
+
+const char* lsa_status_string(lsa_status_t s) {
+  switch (s) {
+    case LSA_OK: return "ok";
+    case LSA_ERR_INVALID_ARG: return "invalid argument";
+    case LSA_ERR_UNSUPPORTED: return "unsupported shape or option";
+    case LSA_ERR_WORKSPACE: return "workspace too small";
+    case LSA_ERR_CUDA: return "CUDA error";
+    case LSA_ERR_TIMEOUT: return "kernel gave up waiting on a barrier";
+  }
+  return "unknown status";
+}
+
+const char* lsa_last_error(void) { return g_err; }
+
+lsa_status_t lsa_workspace_size(lsa_op_t op, const lsa_op_args_t* args, size_t* bytes) {
+  if (!args || !bytes) return fail(LSA_ERR_INVALID_ARG, "null argument");
+  *bytes = 0;
+  lsa_status_t s;
+  switch (op) {
+    case LSA_OP_INDEX_FLAT:
+      if ((s = check_indexer(args->indexer, true)) != LSA_OK) return s;
+      *bytes = flat_ws_bytes(args->indexer, args->scores_external != 0);
+      return LSA_OK;
+    case LSA_OP_INDEX_HIER:
+      if ((s = check_indexer(args->indexer, false)) != LSA_OK) return s;
+      if ((s = check_hier_params(args->indexer, args->P, args->M, args->budget)) != LSA_OK) return s;
+      *bytes = hier_ws_bytes(args->indexer, args->P, args->M, false);
+      return LSA_OK;
+    case LSA_OP_SELECT:
+      *bytes = 0;
+      return LSA_OK;
+    case LSA_OP_SPARSE_ATTN:
+      if ((s = check_attn(args->attn, args->budget.k)) != LSA_OK) return s;
+      *bytes = attn_ws_bytes(args->attn, args->budget.k);
+      return LSA_OK;
+    case LSA_OP_LAYER_GROUP: {
+      if ((s = check_indexer(args->indexer, args->P == 0)) != LSA_OK) return s;
+      if (args->n_layers < 1 || !args->attn) return fail(LSA_ERR_INVALID_ARG, "need n_layers >= 1 attention inputs");
+      const lsa_indexer_in_t* in = args->indexer;
+      size_t idx_bytes = align_up(static_cast<size_t>(in->B) * in->T * args->budget.k * 4, 256);
+      size_t ix = 0;
+      if (args->P) {
+        if ((s = check_hier_params(in, args->P, args->M, args->budget)) != LSA_OK) return s;
+        ix = hier_ws_bytes(in, args->P, args->M, false);
+      } else {
+        ix = flat_ws_bytes(in, false);
+      }
+      size_t at = 0;
+      for (int i = 0; i < args->n_layers; ++i) {
+        if ((s = check_attn(&args->attn[i], args->budget.k)) != LSA_OK) return s;
+        at = std::max(at, attn_ws_bytes(&args->attn[i], args->budget.k));
+      }
+      *bytes = idx_bytes + std::max(ix, at);
+      return LSA_OK;
+    }
+  }
+  return fail(LSA_ERR_INVALID_ARG, "unknown op %d", static_cast<int>(op));
+}
+
+lsa_status_t lsa_index_flat(const lsa_indexer_in_t* in, lsa_budget_t budget, int32_t* idx, float* scores_out,
+                            void* workspace, size_t workspace_bytes, lsa_stream_t stream) {
+  lsa_status_t s;
+  if ((s = check_indexer(in, true)) != LSA_OK) return s;
+  if ((s = check_budget(budget)) != LSA_OK) return s;
+  if (!idx && !scores_out) return fail(LSA_ERR_INVALID_ARG, "need idx or scores_out");
+  if ((idx && !aligned16(idx)) || (scores_out && !aligned16(scores_out)))
+    return fail(LSA_ERR_INVALID_ARG, "outputs must be 16-byte aligned");
+  const size_t need = flat_ws_bytes(in, scores_out != nullptr);
+  if ((s = check_ws(workspace, workspace_bytes, need)) != LSA_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  float* scores = scores_out ? scores_out : static_cast<float*>(workspace);
+  if ((s = run_flat_scores(in, in->k, in->L_max, 1, scores, st)) != LSA_OK) return s;
+  if (idx)
+    return run_select(kSelectTokens, in->B, in->T, in->L_max, in->seq_len, scores, in->L_max, in->L_max, budget, 0,
+                      0, nullptr, idx, budget.k, st);
+  return LSA_OK;
+}
+
+lsa_status_t lsa_select_streaming(const float* scores, const int32_t* seq_len, int32_t B, int32_t T,
+                                  int32_t L_max, lsa_budget_t budget, int32_t* idx, void* workspace,
+                                  size_t workspace_bytes, lsa_stream_t stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  lsa_status_t s;
+  if ((s = check_budget(budget)) != LSA_OK) return s;
+  if (!scores || !seq_len || !idx) return fail(LSA_ERR_INVALID_ARG, "null tensor");
+  if (B < 1 || T < 1 || L_max < 1) return fail(LSA_ERR_INVALID_ARG, "B, T and L_max must be >= 1");
+  if (static_cast<long long>(B) * T > 65535) return fail(LSA_ERR_UNSUPPORTED, "at most 65535 query rows per call");
+  return run_select(kSelectTokens, B, T, L_max, seq_len, scores, L_max, L_max, budget, 0, 0, nullptr, idx,
+                    budget.k, reinterpret_cast<cudaStream_t>(stream));
+}
+
+lsa_status_t lsa_pool_pages(const void* k, const int32_t* seq_len, int32_t B, int32_t L_max, int32_t d, int32_t P,
+                            void* page_keys, lsa_stream_t stream) {
+  if (!k || !seq_len || !page_keys) return fail(LSA_ERR_INVALID_ARG, "null tensor");
+  if (!aligned16(k) || !aligned16(page_keys)) return fail(LSA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  if (B < 1 || L_max < 1) return fail(LSA_ERR_INVALID_ARG, "B and L_max must be >= 1");
+  if (d != 64 && d != 128) return fail(LSA_ERR_UNSUPPORTED, "d=%d not in {64, 128}", d);
+  if (!is_pow2_in(P, 16, 128)) return fail(LSA_ERR_UNSUPPORTED, "page size P=%d not in {16,32,64,128}", P);
+  if (L_max % P) return fail(LSA_ERR_INVALID_ARG, "L_max must be a multiple of P");
+  LSA_CHECK_CUDA(launch_pool(static_cast<const uint16_t*>(k), seq_len, B, L_max, d, P,
+                             static_cast<uint16_t*>(page_keys), reinterpret_cast<cudaStream_t>(stream)),
+                 "pool launch");
+  return LSA_OK;
+}
+
+lsa_status_t lsa_index_hier(const lsa_indexer_in_t* in, const void* page_keys, int32_t P, int32_t M,
+                            lsa_budget_t budget, int32_t* idx, int32_t* pages_out, void* workspace,
+                            size_t workspace_bytes, lsa_stream_t stream) {
+  lsa_status_t s;
+  if ((s = check_indexer(in, false)) != LSA_OK) return s;
+  if ((s = check_budget(budget)) != LSA_OK) return s;
+  if ((s = check_hier_params(in, P, M, budget)) != LSA_OK) return s;
+  if (!page_keys || !idx) return fail(LSA_ERR_INVALID_ARG, "null page_keys or idx");
+  if (!aligned16(page_keys) || !aligned16(idx) || (pages_out && !aligned16(pages_out)))
+    return fail(LSA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  if (static_cast<long long>(in->B) * in->T > 65535) return fail(LSA_ERR_UNSUPPORTED, "at most 65535 query rows per call");
+  const size_t need = hier_ws_bytes(in, P, M, pages_out != nullptr);
+  if ((s = check_ws(workspace, workspace_bytes, need)) != LSA_OK) return s;
+  return run_hier(in, page_keys, P, M, budget, idx, pages_out, workspace, reinterpret_cast<cudaStream_t>(stream));
+}
+
+lsa_status_t lsa_sparse_attn(const lsa_attn_in_t* in, const int32_t* idx, int32_t k, void* out, float* lse,
+                             void* workspace, size_t workspace_bytes, lsa_stream_t stream) {
+  lsa_status_t s;
+  if ((s = check_attn(in, k)) != LSA_OK) return s;
+  if (!idx || !out) return fail(LSA_ERR_INVALID_ARG, "null idx or out");
+  if (!aligned16(out) || (lse && !aligned16(lse))) return fail(LSA_ERR_INVALID_ARG, "outputs must be 16-byte aligned");
+  if (static_cast<long long>(in->B) * in->T > 65535) return fail(LSA_ERR_UNSUPPORTED, "at most 65535 query rows per call");
+  if ((s = check_ws(workspace, workspace_bytes, attn_ws_bytes(in, k))) != LSA_OK) return s;
+  return run_attn(in, idx, k, out, lse, workspace, reinterpret_cast<cudaStream_t>(stream));
+}
+
+lsa_status_t lsa_layer_group(const lsa_indexer_in_t* in, const void* page_keys, int32_t P, int32_t M,
+                             lsa_budget_t budget, int32_t n_layers, const lsa_attn_in_t* layers, void* const* outs,
+                             float* const* lse_outs, int32_t* idx, void* workspace, size_t workspace_bytes,
+                             lsa_stream_t stream) {
+  lsa_status_t s;
+  if ((s = check_indexer(in, P == 0)) != LSA_OK) return s;
+  if ((s = check_budget(budget)) != LSA_OK) return s;
+  if (n_layers < 1 || !layers || !outs) return fail(LSA_ERR_INVALID_ARG, "need n_layers >= 1 layers and outputs");
+  if (P) {
+    if ((s = check_hier_params(in, P, M, budget)) != LSA_OK) return s;
+    if (!page_keys) return fail(LSA_ERR_INVALID_ARG, "hierarchical group needs page_keys");
+  }
+  if (static_cast<long long>(in->B) * in->T > 65535) return fail(LSA_ERR_UNSUPPORTED, "at most 65535 query rows per call");
+  for (int i = 0; i < n_layers; ++i) {
+    if ((s = check_attn(&layers[i], budget.k)) != LSA_OK) return s;
+    if (layers[i].B != in->B || layers[i].T != in->T || layers[i].L_max != in->L_max)
+      return fail(LSA_ERR_INVALID_ARG, "layer %d shapes differ from the indexer's", i);
+    if (!outs[i] || !aligned16(outs[i])) return fail(LSA_ERR_INVALID_ARG, "layer %d output null or unaligned", i);
+  }
+  lsa_op_args_t wa{};
+  wa.indexer = in; wa.attn = layers; wa.budget = budget; wa.P = P; wa.M = M; wa.n_layers = n_layers;
+  size_t need = 0;
+  if ((s = lsa_workspace_size(LSA_OP_LAYER_GROUP, &wa, &need)) != LSA_OK) return s;
+  if ((s = check_ws(workspace, workspace_bytes, need)) != LSA_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  int32_t* idx_buf = idx ? idx : reinterpret_cast<int32_t*>(w);
+  w += align_up(static_cast<size_t>(in->B) * in->T * budget.k * 4, 256);
+  if (P) {
+    if ((s = run_hier(in, page_keys, P, M, budget, idx_buf, nullptr, w, st)) != LSA_OK) return s;
+  } else {
+    float* scores = reinterpret_cast<float*>(w);
+    if ((s = run_flat_scores(in, in->k, in->L_max, 1, scores, st)) != LSA_OK) return s;
+    if ((s = run_select(kSelectTokens, in->B, in->T, in->L_max, in->seq_len, scores, in->L_max, in->L_max, budget,
+                        0, 0, nullptr, idx_buf, budget.k, st)) != LSA_OK)
+      return s;
+  }
+  for (int i = 0; i < n_layers; ++i) {
+    float* lse = lse_outs ? lse_outs[i] : nullptr;
+    if ((s = run_attn(&layers[i], idx_buf, budget.k, outs[i], lse, w, st)) != LSA_OK) return s;
+  }
+  return LSA_OK;
+}
+
+lsa_status_t lsa_device_status(lsa_stream_t stream) {
+  LSA_CHECK_CUDA(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)), "stream synchronize");
+  int v = 0;
+  LSA_CHECK_CUDA(cudaMemcpyFromSymbol(&v, lsa::g_device_status, sizeof(int)), "status read");
+  const int zero = 0;
+  LSA_CHECK_CUDA(cudaMemcpyToSymbol(lsa::g_device_status, &zero, sizeof(int)), "status reset");
+  if (v) return fail(LSA_ERR_TIMEOUT, "a kernel gave up waiting on a barrier");
+  return LSA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,391 @@
+// Gathered-KV sparse MQA / MLA attention (DSA Lightning Indexer article,
+// "Sparse Attention Calculator": attention computed only over the selected
+// top-k entries; LSA paper abstract: the selection reads only those KV rows).
+//
+//   o[r, h, :] = sum_j softmax_j(scale * q[r, h, :] . K[idx_j, :]) V[idx_j, :]
+//
+// over the valid (>= 0) entries idx_j of query row r; lse = log of the softmax
+// denominator plus the max. For MLA one latent row per token serves as K
+// (d_qk = 576) and its first d_v = 512 columns as V.
+//
+// One CTA = (v part, KV split, query row). Heads (<= 128, zero-padded) sit on
+// the MMA M dimension; q is resident in shared memory. KV rows are gathered 32
+// at a time with 16-byte cp.async into 128-byte-swizzled tiles (double
+// buffered), used K-major for S = q K^T and MN-major for O += P V. S (32
+// columns) and O (d_v / n_parts <= 256 columns, the fp32 accumulator) live in
+// TMEM; one thread per head runs the online softmax on its S row (lazy
+// rescaling: the running max moves only when a block raises it by > 2^8) and
+// writes bf16 P to shared memory for the PV MMA. With several KV splits each
+// CTA writes an unnormalised partial (O, m, l) and a combine kernel merges them.
+#include <cuda_bf16.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace lsa {
+namespace {
+
+constexpr int kThreads = 128;
+constexpr int BN = kAttnBN;
+
+template <int DQK, int DV, bool SEP_V>
+struct ACfg {
+  static constexpr int kQChunks = DQK / 64;
+  static constexpr int kVN = DV < 256 ? DV : 256;
+  static constexpr int kNVP = DV / kVN;
+  static constexpr int kQBytes = kQChunks * 128 * 128;
+  static constexpr int kChunkBytes = BN * 128;
+  static constexpr int kKVBytes = kQChunks * kChunkBytes;
+  static constexpr int kVBytes = SEP_V ? (DV / 64) * kChunkBytes : 0;
+  static constexpr int kPBytes = 128 * BN * 2;
+  static constexpr int kSCol = kVN;
+  static constexpr int kTmemCols = (kVN + BN) <= 128 ? 128 : ((kVN + BN) <= 256 ? 256 : 512);
+  static constexpr int kRowUnits = DQK / 8;
+  static constexpr int kVRowUnits = DV / 8;
+  static constexpr size_t kSmem = 1024 + kQBytes + 2 * kKVBytes + 2 * kVBytes + kPBytes + 2 * BN * 4 + 64;
+};
+
+__device__ __forceinline__ void spin_ns(unsigned long long ns) {
+  const unsigned long long t0 = globaltimer_ns();
+  while (globaltimer_ns() - t0 < ns) {
+  }
+}
+
+template <int DQK, int DV, bool SEP_V>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_kernel(const __grid_constant__ CUtensorMap tm_q, const AttnArgs a) {
+  using C = ACfg<DQK, DV, SEP_V>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = base;
+  uint8_t* sKV = sQ + C::kQBytes;
+  uint8_t* sV = sKV + 2 * C::kKVBytes;
+  uint8_t* sP = sV + 2 * C::kVBytes;
+  int* idx_s = reinterpret_cast<int*>(sP + C::kPBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(idx_s + 2 * BN);
+  uint64_t* q_full = bars;
+  uint64_t* s_full = bars + 1;
+  uint64_t* pv_done = bars + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int vp = blockIdx.x, split = blockIdx.y, r = blockIdx.z;
+  const int b = r / a.T;
+  const int h = tid;
+
+  const int nblk_total = (a.k + BN - 1) / BN;
+  const int blk0 = split * a.blocks_per_split;
+  const int nblk = max(0, min(a.blocks_per_split, nblk_total - blk0));
+  const int* idx_row = a.idx + static_cast<long long>(r) * a.k;
+
+  if (tid == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(s_full, 1);
+    mbar_init(pv_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+  const uint32_t tO = tmem;
+  const uint32_t tS = tmem + C::kSCol;
+
+  if (tid == 0 && nblk > 0) {
+    prefetch_tmap(&tm_q);
+    mbar_arrive_expect_tx(q_full, C::kQBytes);
+    for (int c = 0; c < C::kQChunks; ++c) tma_load_2d(sQ + c * 16384, &tm_q, q_full, c * 64, r * a.Hq);
+  }
+
+  auto load_block = [&](int blk, int buf) {
+    if (tid < BN) {
+      const int ip = (blk0 + blk) * BN + tid;
+      int id = ip < a.k ? __ldg(idx_row + ip) : -1;
+      if (id >= a.L_max) id = -1;
+      idx_s[buf * BN + tid] = id;
+    }
+    __syncthreads();
+    uint8_t* kv = sKV + buf * C::kKVBytes;
+    const long long row0 = static_cast<long long>(b) * a.L_max;
+    for (int u = tid; u < BN * C::kRowUnits; u += kThreads) {
+      const int j = u / C::kRowUnits, cu = u % C::kRowUnits;
+      const int id = idx_s[buf * BN + j];
+      uint8_t* dst = kv + (cu >> 3) * C::kChunkBytes + j * 128 + (((cu & 7) ^ (j & 7)) << 4);
+      const uint16_t* src = id >= 0 ? a.kp + (row0 + id) * a.k_stride + cu * 8 : a.kp;
+      cp_async_16(dst, src, id >= 0 ? 16u : 0u);
+    }
+    if (SEP_V) {
+      uint8_t* vv = sV + buf * C::kVBytes;
+      for (int u = tid; u < BN * C::kVRowUnits; u += kThreads) {
+        const int j = u / C::kVRowUnits, cu = u % C::kVRowUnits;
+        const int id = idx_s[buf * BN + j];
+        uint8_t* dst = vv + (cu >> 3) * C::kChunkBytes + j * 128 + (((cu & 7) ^ (j & 7)) << 4);
+        const uint16_t* src = id >= 0 ? a.vp + (row0 + id) * a.v_stride + cu * 8 : a.vp;
+        cp_async_16(dst, src, id >= 0 ? 16u : 0u);
+      }
+    }
+    cp_async_commit();
+  };
+
+  const uint32_t idesc_qk = make_idesc(1, 1, 128, BN, 0, 0);
+  const uint32_t idesc_pv = make_idesc(1, 1, 128, C::kVN, 0, 1);
+  float m_run = -INFINITY, l_run = 0.f;   // log2 domain
+
+  // Failure decisions are block-uniform (__syncthreads_and), so no thread can
+  // be left waiting at a barrier the others skipped.
+  bool fail = false;
+  if (nblk > 0) load_block(0, 0);
+  for (int blk = 0; blk < nblk; ++blk) {
+    const int buf = blk & 1;
+    const bool pv_ok = blk >= 1 ? mbar_wait(pv_done, (blk - 1) & 1, a.status) : true;   // frees buf^1, P and O
+    if (!__syncthreads_and(pv_ok)) { fail = true; break; }
+    if (blk + 1 < nblk) {
+      load_block(blk + 1, buf ^ 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      const bool q_ok = blk > 0 || mbar_wait(q_full, 0, a.status);
+      if (!q_ok) {
+        *abort_flag = 1;
+      } else {
+        tc_fence_after();
+        const uint32_t q0 = smem_u32(sQ), k0 = smem_u32(sKV + buf * C::kKVBytes);
+#pragma unroll 1
+        for (int c = 0; c < C::kQChunks; ++c) {
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) {
+            const uint64_t ad = make_sdesc(q0 + c * 16384 + ks * 32, 16, 1024, kLayoutSW128);
+            const uint64_t bd = make_sdesc(k0 + c * C::kChunkBytes + ks * 32, 16, 1024, kLayoutSW128);
+            umma_f16(tS, ad, bd, idesc_qk, (c | ks) ? 1u : 0u);
+          }
+        }
+        umma_commit(s_full);
+      }
+    }
+    __syncthreads();
+    if (*abort_flag) { fail = true; break; }
+    const bool s_ok = mbar_wait(s_full, blk & 1, a.status);
+    if (!__syncthreads_and(s_ok)) { fail = true; break; }
+    tc_fence_after();
+
+    uint32_t sv[32];
+    tmem_ld32(tS + lane_off, sv);
+    tmem_ld_wait();
+    float x[32];
+    float mb = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const bool valid = idx_s[buf * BN + j] >= 0;
+      x[j] = valid ? __uint_as_float(sv[j]) * a.scale_log2 : -INFINITY;
+      mb = fmaxf(mb, x[j]);
+    }
+    const float m_new = fmaxf(m_run, mb);
+    const bool move = m_new != -INFINITY && (m_run == -INFINITY || m_new > m_run + 8.f);
+    float corr = 1.f;
+    if (move) {
+      corr = m_run == -INFINITY ? 0.f : exp2f(m_run - m_new);
+      l_run *= corr;
+      m_run = m_new;
+    }
+    // O holds data from earlier blocks: rescale it (warp-uniform TMEM access)
+    if (blk > 0 && __any_sync(0xffffffffu, move)) {
+#pragma unroll 1
+      for (int c0 = 0; c0 < C::kVN; c0 += 32) {
+        uint32_t ov[32];
+        tmem_ld32(tO + lane_off + c0, ov);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * corr);
+        tmem_st32(tO + lane_off + c0, ov);
+      }
+      tmem_st_wait();
+    }
+    float psum = 0.f;
+    uint32_t pk[16];
+#pragma unroll
+    for (int j = 0; j < 32; j += 2) {
+      const float p0 = m_run == -INFINITY ? 0.f : exp2f(x[j] - m_run);
+      const float p1 = m_run == -INFINITY ? 0.f : exp2f(x[j + 1] - m_run);
+      psum += p0 + p1;
+      const __nv_bfloat162 v2 = __floats2bfloat162_rn(p0, p1);
+      pk[j >> 1] = *reinterpret_cast<const uint32_t*>(&v2);
+    }
+    l_run += psum;
+    uint8_t* prow = sP + (h >> 3) * 512 + (h & 7) * 16;
+#pragma unroll
+    for (int kc = 0; kc < 4; ++kc)
+      *reinterpret_cast<uint4*>(prow + kc * 128) = make_uint4(pk[4 * kc], pk[4 * kc + 1], pk[4 * kc + 2], pk[4 * kc + 3]);
+    tc_fence_before();
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t p0 = smem_u32(sP);
+      const uint32_t v0 = SEP_V ? smem_u32(sV + buf * C::kVBytes)
+                                : smem_u32(sKV + buf * C::kKVBytes) + vp * (C::kVN / 64) * C::kChunkBytes;
+#pragma unroll
+      for (int ks = 0; ks < BN / 16; ++ks) {
+        const uint64_t ad = make_sdesc(p0 + ks * 256, 128, 512, kLayoutNone);
+        const uint64_t bd = make_sdesc(v0 + ks * 2048, C::kChunkBytes, 1024, kLayoutSW128);
+        umma_f16(tO, ad, bd, idesc_pv, (blk > 0 || ks > 0) ? 1u : 0u);
+      }
+      umma_commit(pv_done);
+    }
+  }
+  {
+    const bool last_ok = (!fail && nblk > 0) ? mbar_wait(pv_done, (nblk - 1) & 1, a.status) : true;
+    if (!__syncthreads_and(last_ok)) fail = true;
+  }
+  if (fail && tid == 0) *abort_flag = 1;
+  __syncthreads();
+  tc_fence_after();
+
+  const bool have = nblk > 0 && !*abort_flag;
+  const bool write_row = h < a.Hq;
+  if (a.n_split == 1) {
+    const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+    uint16_t* orow = a.out + (static_cast<long long>(r) * a.Hq + h) * DV + vp * C::kVN;
+#pragma unroll 1
+    for (int c0 = 0; c0 < C::kVN; c0 += 32) {
+      uint32_t ov[32];
+      if (have) {
+        tmem_ld32(tO + lane_off + c0, ov);
+        tmem_ld_wait();
+      }
+      if (write_row) {
+        uint32_t pkd[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const float o0 = have ? __uint_as_float(ov[i]) * inv_l : 0.f;
+          const float o1 = have ? __uint_as_float(ov[i + 1]) * inv_l : 0.f;
+          const __nv_bfloat162 v2 = __floats2bfloat162_rn(o0, o1);
+          pkd[i >> 1] = *reinterpret_cast<const uint32_t*>(&v2);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) dst[q] = make_uint4(pkd[4 * q], pkd[4 * q + 1], pkd[4 * q + 2], pkd[4 * q + 3]);
+      }
+    }
+    if (vp == 0 && write_row && a.lse)
+      a.lse[static_cast<long long>(r) * a.Hq + h] =
+          l_run > 0.f ? (m_run + log2f(l_run)) * 0.69314718055994530942f : -INFINITY;
+  } else {
+    const long long prow = (static_cast<long long>(r) * a.n_split + split) * a.Hq + h;
+    float* po = a.part_o + prow * DV + vp * C::kVN;
+#pragma unroll 1
+    for (int c0 = 0; c0 < C::kVN; c0 += 32) {
+      uint32_t ov[32];
+      if (have) {
+        tmem_ld32(tO + lane_off + c0, ov);
+        tmem_ld_wait();
+      }
+      if (write_row) {
+        float4* dst = reinterpret_cast<float4*>(po + c0);
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          dst[q] = have ? make_float4(__uint_as_float(ov[4 * q]), __uint_as_float(ov[4 * q + 1]),
+                                      __uint_as_float(ov[4 * q + 2]), __uint_as_float(ov[4 * q + 3]))
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    if (vp == 0 && write_row) {
+      a.part_m[prow] = have ? m_run : -INFINITY;
+      a.part_l[prow] = have ? l_run : 0.f;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag) spin_ns(50000);
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// Merge KV-split partials: m* = max m_s; o = sum O_s 2^(m_s - m*) / sum l_s 2^(m_s - m*).
+__global__ void __launch_bounds__(128) combine_kernel(const AttnArgs a) {
+  const int r = blockIdx.x, h = blockIdx.y;
+  const int c = threadIdx.x * 4;
+  if (c >= a.d_v) return;
+  const long long base = static_cast<long long>(r) * a.n_split * a.Hq + h;
+  float M = -INFINITY;
+  for (int s = 0; s < a.n_split; ++s) {
+    const long long i = base + static_cast<long long>(s) * a.Hq;
+    if (a.part_l[i] > 0.f) M = fmaxf(M, a.part_m[i]);
+  }
+  float den = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int s = 0; s < a.n_split; ++s) {
+    const long long i = base + static_cast<long long>(s) * a.Hq;
+    const float l = a.part_l[i];
+    if (l > 0.f) {
+      const float f = exp2f(a.part_m[i] - M);
+      den += l * f;
+      const float4 o = *reinterpret_cast<const float4*>(a.part_o + i * a.d_v + c);
+      acc[0] += o.x * f;
+      acc[1] += o.y * f;
+      acc[2] += o.z * f;
+      acc[3] += o.w * f;
+    }
+  }
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  const __nv_bfloat162 v01 = __floats2bfloat162_rn(acc[0] * inv, acc[1] * inv);
+  const __nv_bfloat162 v23 = __floats2bfloat162_rn(acc[2] * inv, acc[3] * inv);
+  uint2 pk;
+  pk.x = *reinterpret_cast<const uint32_t*>(&v01);
+  pk.y = *reinterpret_cast<const uint32_t*>(&v23);
+  *reinterpret_cast<uint2*>(a.out + (static_cast<long long>(r) * a.Hq + h) * a.d_v + c) = pk;
+  if (threadIdx.x == 0 && a.lse)
+    a.lse[static_cast<long long>(r) * a.Hq + h] = den > 0.f ? (M + log2f(den)) * 0.69314718055994530942f : -INFINITY;
+}
+
+template <int DQK, int DV, bool SEP_V>
+cudaError_t launch_t(const CUtensorMap& tm_q, const AttnArgs& a, cudaStream_t stream) {
+  using C = ACfg<DQK, DV, SEP_V>;
+  const void* fn = reinterpret_cast<const void*>(&attn_kernel<DQK, DV, SEP_V>);
+  size_t smem = C::kSmem;
+  if (smem < 60 * 1024) smem = 60 * 1024;   // at most 3 CTAs per SM: TMEM demand stays <= 512 columns
+  cudaError_t e = set_max_smem(fn, smem);
+  if (e != cudaSuccess) return e;
+  const dim3 grid(C::kNVP, a.n_split, a.B * a.T);
+  void* args[] = {const_cast<CUtensorMap*>(&tm_q), const_cast<AttnArgs*>(&a)};
+  return cudaLaunchKernel(fn, grid, dim3(kThreads), args, smem, stream);
+}
+
+}  // namespace
+
+size_t attn_smem_bytes(int d_qk, int d_v, bool sep_v) {
+  if (d_qk == 576 && d_v == 512) return sep_v ? ACfg<576, 512, true>::kSmem : ACfg<576, 512, false>::kSmem;
+  return ACfg<64, 64, true>::kSmem;
+}
+
+cudaError_t launch_attn(const CUtensorMap& tm_q, const AttnArgs& a, cudaStream_t stream) {
+  if (a.d_qk == 576 && a.d_v == 512) {
+    if (a.sep_v) return cudaErrorNotSupported;   // MLA keeps V inside the latent row
+    return launch_t<576, 512, false>(tm_q, a, stream);
+  }
+  if (a.d_qk == 64 && a.d_v == 64) {
+    if (a.sep_v) return launch_t<64, 64, true>(tm_q, a, stream);
+    return launch_t<64, 64, false>(tm_q, a, stream);
+  }
+  return cudaErrorNotSupported;
+}
+
+cudaError_t launch_attn_combine(const AttnArgs& a, cudaStream_t stream) {
+  const dim3 grid(a.B * a.T, a.Hq);
+  combine_kernel<<<grid, a.d_v / 4, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace lsa

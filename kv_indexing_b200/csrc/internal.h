@@ -1,0 +1,99 @@
+// Internal launch interfaces between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace lsa {
+
+// ----------------------------------------------------------------- indexer --
+// One work item = one 128-key tile against one query group (NQ queries x H
+// heads = N MMA columns). FLAT: key rows [128 j, 128 j + 128) of sequence b.
+// GATHER: the 128 candidate slots [128 j, 128 j + 128) of query row r, made of
+// 128 / P recalled pages (page ids from `pages`).
+struct IndexerArgs {
+  int B, T, H, d;
+  int L_rows;            // key rows per sequence in the key array
+  int L_max;             // token capacity per sequence (seq_len clamp; gather rows)
+  int NQ, N, G;          // queries per tile, MMA N (= NQ * H), query groups per sequence
+  int n_tiles;           // tiles per group (FLAT) or per query row (GATHER)
+  int vis_div;           // FLAT: key s visible to pos iff s < (pos + 1) / vis_div
+  int gather;            // 0 = FLAT, 1 = GATHER
+  int stages, nbuf_b;    // A-tile ring depth, B-tile buffers (1 or 2)
+  long long n_items;
+  const int* seq_len;
+  const float* w;
+  const float* q_scale;  // e4m3 only
+  const float* k_scale;  // e4m3 only (indexed by b * L_rows + s)
+  float* out;
+  long long out_row_stride;
+  float inv_sqrt_d;
+  // GATHER
+  const int* pages;
+  int M, P, sink, window;
+  int* status;           // per-device status word
+};
+
+size_t indexer_smem_bytes(int d, bool fp8, int N, int stages, int nbuf_b);
+void indexer_pick_pipeline(int d, bool fp8, int N, int* stages, int* nbuf_b);
+cudaError_t launch_indexer(const CUtensorMap& tm_k, const CUtensorMap& tm_q, const IndexerArgs& a,
+                           bool fp8, int grid, cudaStream_t stream);
+
+// --------------------------------------------------------- streaming select --
+enum SelectMode { kSelectTokens = 0, kSelectHierTokens = 1, kSelectPages = 2 };
+
+struct SelectArgs {
+  int mode;
+  int B, T;
+  int L_max;
+  const int* seq_len;
+  const float* scores;
+  long long row_stride;   // floats between consecutive (b, t) rows
+  int n_slots;            // slots per row
+  int k, sink, window;    // token budget
+  int P, M;               // pages / hier
+  const int* pages;       // kSelectHierTokens: [B*T, M]
+  int* out;
+  int out_len;            // k (tokens) or M (pages)
+  int cap;                // keys cached in shared memory per CTA (0 = stream from global)
+};
+
+cudaError_t launch_select(const SelectArgs& a, int cluster, cudaStream_t stream);
+int select_cluster_size(int rows, int max_dyn, int num_sms, int* cap);
+
+// ------------------------------------------------------------------ pooling --
+cudaError_t launch_pool(const uint16_t* k, const int* seq_len, int B, int L_max, int d, int P,
+                        uint16_t* page_keys, cudaStream_t stream);
+
+// ---------------------------------------------------------- sparse attention --
+struct AttnArgs {
+  int B, T, Hq, L_max;
+  int d_qk, d_v;
+  int k;                  // index row length
+  float scale_log2;       // scale * log2(e)
+  const int* idx;
+  const uint16_t* kp;     // K rows
+  const uint16_t* vp;     // V rows (may alias kp)
+  long long k_stride, v_stride;
+  int sep_v;              // V rows loaded separately (not a prefix of the K row)
+  int n_split, blocks_per_split;
+  uint16_t* out;          // [rows, Hq, d_v] bf16
+  float* lse;             // [rows, Hq] or null
+  float* part_o;          // [rows, n_split, Hq, d_v]
+  float* part_m;          // [rows, n_split, Hq]
+  float* part_l;          // [rows, n_split, Hq]
+  int* status;            // per-device status word
+};
+
+constexpr int kAttnBN = 32;  // KV rows per block
+size_t attn_smem_bytes(int d_qk, int d_v, bool sep_v);
+cudaError_t launch_attn(const CUtensorMap& tm_q, const AttnArgs& a, cudaStream_t stream);
+cudaError_t launch_attn_combine(const AttnArgs& a, cudaStream_t stream);
+
+// --------------------------------------------------------------------- misc --
+int device_sm_count();
+int* device_status_ptr();
+cudaError_t set_max_smem(const void* func, size_t bytes);
+
+}  // namespace lsa

@@ -1,0 +1,107 @@
+"""C-ABI boundary checks that need no GPU: the library loads, exports every
+function include/lsa.h declares, and rejects bad arguments on the host before
+touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from kv_indexing_b200 import lsa as L
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "lsa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(lsa_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    fns = header_functions()
+    for name in ["lsa_index_flat", "lsa_index_hier", "lsa_select_streaming", "lsa_sparse_attn",
+                 "lsa_layer_group", "lsa_pool_pages", "lsa_workspace_size", "lsa_status_string"]:
+        assert name in fns
+    assert sorted(L.EXPORTS) == fns
+
+
+def test_library_exports_every_declared_symbol():
+    lib = L.load()
+    for name in header_functions():
+        assert hasattr(lib, name), name
+    raw = ctypes.CDLL(L.LIB_PATH)
+    for name in header_functions():
+        getattr(raw, name)
+
+
+def test_status_strings():
+    lib = L.load()
+    for st in range(6):
+        assert lib.lsa_status_string(st)
+    assert lib.lsa_status_string(99) == b"unknown status"
+
+
+def _indexer(**kw):
+    base = dict(B=1, T=1, H=64, d=128, L_max=1024, dtype=L.LSA_BF16, seq_len=16, q=32, q_scale=None, w=48, k=64,
+                k_scale=None)
+    base.update(kw)
+    return L.IndexerIn(*[base[f] for f, _ in L.IndexerIn._fields_])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(B=0), L.LSA_ERR_INVALID_ARG),
+    (dict(d=96), L.LSA_ERR_UNSUPPORTED),
+    (dict(H=6), L.LSA_ERR_UNSUPPORTED),
+    (dict(L_max=1000), L.LSA_ERR_UNSUPPORTED),
+    (dict(q=None), L.LSA_ERR_INVALID_ARG),
+    (dict(k=72), L.LSA_ERR_INVALID_ARG),              # misaligned pointer
+    (dict(dtype=L.LSA_E4M3), L.LSA_ERR_INVALID_ARG),  # e4m3 without scales
+    (dict(dtype=L.LSA_E4M3, q_scale=16, k_scale=16, d=64), L.LSA_ERR_UNSUPPORTED),
+])
+def test_index_flat_rejects_bad_indexer_on_host(kw, code):
+    lib = L.load()
+    ii = _indexer(**kw)
+    st = lib.lsa_index_flat(ctypes.byref(ii), L.Budget(2048, 64, 960), 16, None, None, 0, None)
+    assert st == code, lib.lsa_last_error()
+    assert lib.lsa_last_error()
+
+
+@pytest.mark.parametrize("budget,code", [
+    ((0, 0, 0), L.LSA_ERR_UNSUPPORTED),
+    ((100, 60, 60), L.LSA_ERR_INVALID_ARG),
+    ((100, -1, 0), L.LSA_ERR_INVALID_ARG),
+    ((9000, 0, 0), L.LSA_ERR_UNSUPPORTED),
+])
+def test_budget_validation(budget, code):
+    lib = L.load()
+    ii = _indexer()
+    assert lib.lsa_index_flat(ctypes.byref(ii), L.Budget(*budget), 16, None, None, 0, None) == code
+
+
+def test_workspace_checks_and_sizes():
+    lib = L.load()
+    ii = _indexer(B=8, T=1, L_max=131072)
+    n = L.workspace_size(L.LSA_OP_INDEX_FLAT, indexer=ii, budget=(2048, 64, 960))
+    assert n == 8 * 131072 * 4
+    assert L.workspace_size(L.LSA_OP_INDEX_FLAT, indexer=ii, budget=(2048, 64, 960), scores_external=True) == 0
+    st = lib.lsa_index_flat(ctypes.byref(ii), L.Budget(2048, 64, 960), 16, None, 256, n - 1, None)
+    assert st == L.LSA_ERR_WORKSPACE
+    hi = L.workspace_size(L.LSA_OP_INDEX_HIER, indexer=_indexer(B=2, L_max=1 << 20), budget=(2048, 64, 960),
+                          P=64, M=256)
+    assert hi == 2 * (1 << 14) * 4 + 2 * 256 * 4 + 2 * 256 * 64 * 4
+
+
+def test_hier_parameter_validation():
+    lib = L.load()
+    ii = _indexer(L_max=4096)
+    bu = L.Budget(2048, 64, 960)
+    assert lib.lsa_index_hier(ctypes.byref(ii), 16, 48, 256, bu, 16, None, None, 0, None) == L.LSA_ERR_UNSUPPORTED
+    assert lib.lsa_index_hier(ctypes.byref(ii), 16, 64, 8, bu, 16, None, None, 0, None) == L.LSA_ERR_INVALID_ARG
+
+
+def test_pool_and_select_validation():
+    lib = L.load()
+    assert lib.lsa_pool_pages(16, 16, 1, 4096, 128, 24, 16, None) == L.LSA_ERR_UNSUPPORTED
+    assert lib.lsa_pool_pages(16, 16, 1, 4000, 128, 64, 16, None) == L.LSA_ERR_INVALID_ARG
+    assert lib.lsa_select_streaming(None, 16, 1, 1, 128, L.Budget(8, 2, 2), 16, None, 0, None) == L.LSA_ERR_INVALID_ARG

@@ -1,0 +1,102 @@
+"""Sparse MQA / MLA attention on the GPU vs the oracle (2e-2 max-abs, 1e-2 relative)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from kv_indexing_b200 import inputs as I
+from kv_indexing_b200 import lsa as L
+from tests.parity import assert_attention_close, dev, host
+
+pytestmark = pytest.mark.gpu
+
+
+def rand_idx(rng, B, T, k, L, seq_len, n_valid=None):
+    idx = np.full((B, T, k), -1, np.int32)
+    for b in range(B):
+        for t in range(T):
+            pos = int(seq_len[b]) - T + t
+            nv = min(k, pos + 1) if n_valid is None else min(n_valid, pos + 1)
+            if nv > 0:
+                idx[b, t, :nv] = np.sort(rng.choice(pos + 1, size=nv, replace=False))
+    return idx
+
+
+def run(w, x, idx, seq_len):
+    sl = dev(seq_len, "i32")
+    q = dev(x["qa"], "bf16")
+    lse = torch.empty(idx.shape[:2] + (w.Hq,), dtype=torch.float32, device="cuda")
+    if w.mla:
+        out, _ = L.lsa_sparse_attn(q, dev(idx, "i32"), sl, w.scale, kv=dev(x["kv"], "bf16"), d_v=w.d_v, lse=lse)
+    else:
+        out, _ = L.lsa_sparse_attn(q, dev(idx, "i32"), sl, w.scale, k=dev(x["k"], "bf16"), v=dev(x["v"], "bf16"),
+                                   lse=lse)
+    torch.cuda.synchronize()
+    L.lsa_device_status()
+    return O.bf16_to_f64(host(out)), host(lse)
+
+
+def oracle_attn(w, x, idx, seq_len):
+    if w.mla:
+        return O.sparse_attention(x["qa"], idx, seq_len, scale=w.scale, d_v=w.d_v, kv=x["kv"])
+    return O.sparse_attention(x["qa"], idx, seq_len, scale=w.scale, d_v=w.d_v, k=x["k"], v=x["v"])
+
+
+@pytest.mark.parametrize("seed", [1, 2])
+def test_attention_tiny_mqa(seed):
+    w = I.WORKLOADS["tiny_l2k"]
+    rng = np.random.default_rng(seed)
+    x = I.make_attn_inputs(w, seed)
+    sl = np.array([w.L], np.int32)
+    idx = rand_idx(rng, w.B, w.T, w.k, w.L, sl)
+    g, gl = run(w, x, idx, sl)
+    o, ol = oracle_attn(w, x, idx, sl)
+    assert_attention_close(g, o)
+    assert np.allclose(gl, ol, atol=1e-3, rtol=1e-3)
+
+
+def test_attention_mla_decode_splits():
+    w = I.scaled(I.WORKLOADS["flat_decode_128k"], B=2, L=8192)
+    rng = np.random.default_rng(3)
+    x = I.make_attn_inputs(w, 3)
+    sl = np.array([8192, 6000], np.int32)
+    idx = rand_idx(rng, w.B, w.T, w.k, w.L, sl)
+    g, gl = run(w, x, idx, sl)
+    o, ol = oracle_attn(w, x, idx, sl)
+    assert_attention_close(g, o)
+    assert np.allclose(gl, ol, atol=1e-3, rtol=1e-3)
+
+
+def test_attention_mla_many_rows_padding_and_empty():
+    w = I.scaled(I.WORKLOADS["flat_decode_128k"], B=1, L=4096, T=40)
+    rng = np.random.default_rng(4)
+    x = I.make_attn_inputs(w, 4)
+    sl = np.array([4096], np.int32)
+    idx = rand_idx(rng, w.B, w.T, w.k, w.L, sl, n_valid=700)    # -1 padded tails
+    idx[0, 5] = -1                                               # a row with nothing selected
+    g, gl = run(w, x, idx, sl)
+    o, ol = oracle_attn(w, x, idx, sl)
+    assert_attention_close(g, o)
+    assert (g[0, 5] == 0).all() and np.isneginf(gl[0, 5]).all()
+    fin = np.isfinite(ol)
+    assert np.allclose(gl[fin], ol[fin], atol=1e-3, rtol=1e-3)
+
+
+def test_attention_select_all_equals_dense():
+    # k >= pos + 1 with every visible token selected == dense causal attention
+    w = I.Workload(name="dense", B=1, L=256, T=8, H=4, d=64, k=256, sink=0, window=0, Hq=16, d_qk=64, d_v=64,
+                   mla=False, scale=0.125)
+    x = I.make_attn_inputs(w, 9)
+    sl = np.array([256], np.int32)
+    idx = np.full((1, 8, 256), -1, np.int32)
+    for t in range(8):
+        idx[0, t, :256 - 8 + t + 1] = np.arange(256 - 8 + t + 1)
+    g, _ = run(w, x, idx, sl)
+    qt = torch.from_numpy(O.bf16_to_f64(x["qa"][0])).permute(1, 0, 2)
+    kt = torch.from_numpy(O.bf16_to_f64(x["k"][0]))[None].expand(16, 256, 64)
+    vt = torch.from_numpy(O.bf16_to_f64(x["v"][0]))[None].expand(16, 256, 64)
+    mask = torch.zeros(8, 256, dtype=torch.bool)
+    for t in range(8):
+        mask[t, :256 - 8 + t + 1] = True
+    ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask, scale=0.125)
+    assert_attention_close(g[0], ref.permute(1, 0, 2).numpy())

@@ -1,0 +1,76 @@
+"""Streaming top-k on the GPU vs the oracle, given the oracle's own scores:
+bit-exact index rows (sink, window, dynamic ascending, -1 padding)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from kv_indexing_b200 import inputs as I
+from kv_indexing_b200 import lsa as L
+from tests.parity import dev, host
+
+pytestmark = pytest.mark.gpu
+
+
+def run_select(scores, seq_len, T, budget):
+    idx = L.lsa_select_streaming(dev(scores, "f32"), dev(seq_len, "i32"), budget)
+    torch.cuda.synchronize()
+    L.lsa_device_status()
+    return host(idx)
+
+
+def oracle_scores(w, seed, rows=None):
+    x = I.make_indexer_inputs(w, seed)
+    return O.indexer_scores(x["q_idx"], x["w"], x["k_idx"], x["seq_len"], rows=rows), x["seq_len"]
+
+
+@pytest.mark.parametrize("seed", [1, 2, 3])
+def test_select_tiny_workload_bit_exact(seed):
+    w = I.WORKLOADS["tiny_l2k"]
+    sc, sl = oracle_scores(w, seed)
+    budget = (w.k, w.sink, w.window)
+    got = run_select(sc, sl, w.T, budget)
+    ref = O.select_streaming(sc, sl, w.T, *budget)
+    assert np.array_equal(got, ref)
+
+
+def test_select_heavy_ties_negative_zero_and_short_rows():
+    rng = np.random.default_rng(5)
+    B, T, L_max = 3, 7, 3000
+    sc = (rng.integers(0, 6, size=(B, T, L_max)) * 0.5).astype(np.float32)
+    sc[rng.random(sc.shape) < 0.05] = -0.0
+    sl = np.array([3000, 700, 40], np.int32)
+    for t in range(T):                       # invisible slots carry -inf, like the indexer writes
+        for b in range(B):
+            sc[b, t, sl[b] - T + t + 1:] = -np.inf
+    for budget in [(256, 64, 64), (64, 0, 0), (100, 20, 0), (50, 0, 50), (8, 3, 5)]:
+        got = run_select(sc, sl, T, budget)
+        ref = O.select_streaming(sc, sl, T, *budget)
+        assert np.array_equal(got, ref), budget
+
+
+def test_select_negative_scores_and_empty_rows():
+    rng = np.random.default_rng(6)
+    B, T, L_max = 2, 4, 512
+    sc = rng.standard_normal((B, T, L_max)).astype(np.float32) * 100
+    sl = np.array([2, 512], np.int32)        # b=0: queries 0,1 have pos < 0
+    for b in range(B):
+        for t in range(T):
+            sc[b, t, max(0, sl[b] - T + t + 1):] = -np.inf
+    got = run_select(sc, sl, T, (64, 4, 8))
+    ref = O.select_streaming(sc, sl, T, 64, 4, 8)
+    assert np.array_equal(got, ref)
+    assert (got[0, 0] == -1).all() and (got[0, 1] == -1).all()
+
+
+@pytest.mark.parametrize("B,L_max", [(8, 131072), (2, 1 << 20)])
+def test_select_long_rows_cluster_paths(B, L_max):
+    # 128K rows use the shared-memory-cached path, 1M rows the streaming path
+    rng = np.random.default_rng(L_max)
+    sc = rng.standard_normal((B, 1, L_max)).astype(np.float32)
+    sc = np.abs(sc) + np.float32(3.0)
+    sc[:, :, rng.integers(0, L_max, size=4000)] = np.float32(9.5)     # a block of exact ties
+    sl = np.full((B,), L_max, np.int32)
+    got = run_select(sc, sl, 1, (2048, 64, 960))
+    ref = O.select_streaming(sc, sl, 1, 2048, 64, 960)
+    assert np.array_equal(got, ref)
