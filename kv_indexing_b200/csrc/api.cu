@@ -78,6 +78,22 @@ lsa_status_t make_tmap(CUtensorMap* m, const void* base, bool fp8, uint64_t inne
   return LSA_OK;
 }
 
+// bf16 rows of `inner` elements spaced `row_stride` elements apart.
+lsa_status_t make_tmap_strided(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t row_stride,
+                               uint32_t box_inner, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return fail(LSA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {row_stride * 2};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(LSA_ERR_CUDA, "cuTensorMapEncodeTiled (rows) failed (%d)", static_cast<int>(r));
+  return LSA_OK;
+}
+
 // --------------------------------------------------------------- validation --
 lsa_status_t check_budget(lsa_budget_t bu) {
   if (bu.k < 1 || bu.k > 8192) return fail(LSA_ERR_UNSUPPORTED, "budget k=%d outside [1, 8192]", bu.k);
@@ -159,6 +175,7 @@ AttnPlan attn_plan(const lsa_attn_in_t* at, int k) {
   int ns = device_sm_count() / (rows * p.nvp);
   if (ns < 1) ns = 1;
   if (ns > nblk) ns = nblk;
+  if (ns > 64) ns = 64;   // the split combine merges at most 64 partials
   p.bps = (nblk + ns - 1) / ns;
   p.n_split = (nblk + p.bps - 1) / p.bps;
   return p;
@@ -172,21 +189,30 @@ size_t attn_ws_bytes(const lsa_attn_in_t* at, int k) {
   return align_up(nm * at->d_v * 4, 256) + 2 * align_up(nm * 4, 256);
 }
 
-size_t hier_ws_bytes(const lsa_indexer_in_t* in, int P, int M, bool pages_external) {
-  const size_t rows = static_cast<size_t>(in->B) * in->T;
-  size_t s = align_up(rows * (in->L_max / P) * 4, 256);          // page scores
-  if (!pages_external) s += align_up(rows * M * 4, 256);          // recalled pages
-  s += align_up(rows * static_cast<size_t>(M) * P * 4, 256);      // fine candidate scores
+SelectPlan token_select_plan(int rows, int n_slots, lsa_budget_t bu) {
+  return select_plan(rows, n_slots, std::max(0, bu.k - bu.sink - bu.window), device_sm_count());
+}
+
+SelectPlan page_select_plan(int rows, int n_pages, int M) { return select_plan(rows, n_pages, M, device_sm_count()); }
+
+size_t hier_ws_bytes(const lsa_indexer_in_t* in, int P, int M, lsa_budget_t bu, bool pages_external) {
+  const int rows = in->B * in->T;
+  size_t s = align_up(static_cast<size_t>(rows) * (in->L_max / P) * 4, 256);   // page scores
+  if (!pages_external) s += align_up(static_cast<size_t>(rows) * M * 4, 256);   // recalled pages
+  s += align_up(static_cast<size_t>(rows) * M * P * 4, 256);                     // fine candidate scores
+  s += std::max(select_ws_bytes(rows, page_select_plan(rows, in->L_max / P, M)),
+                select_ws_bytes(rows, token_select_plan(rows, M * P, bu)));      // selection scratch
   return s;
 }
 
-size_t flat_ws_bytes(const lsa_indexer_in_t* in, bool scores_external) {
-  if (scores_external) return 0;
-  return align_up(static_cast<size_t>(in->B) * in->T * in->L_max * 4, 256);
+size_t flat_ws_bytes(const lsa_indexer_in_t* in, lsa_budget_t bu, bool scores_external) {
+  const int rows = in->B * in->T;
+  size_t s = scores_external ? 0 : align_up(static_cast<size_t>(rows) * in->L_max * 4, 256);
+  return s + select_ws_bytes(rows, token_select_plan(rows, in->L_max, bu));
 }
 
 // ------------------------------------------------------------ launchers --
-lsa_status_t run_flat_scores(const lsa_indexer_in_t* in, const void* keys, int L_rows, int vis_div,
+lsa_status_t run_flat_scores(const lsa_indexer_in_t* in, const void* keys, int L_rows, int vis_shift,
                              float* scores, cudaStream_t st) {
   const bool fp8 = in->dtype == LSA_E4M3;
   const FlatPlan fp = flat_plan(in->T, in->H, L_rows);
@@ -200,8 +226,9 @@ lsa_status_t run_flat_scores(const lsa_indexer_in_t* in, const void* keys, int L
   a.B = in->B; a.T = in->T; a.H = in->H; a.d = in->d;
   a.L_rows = L_rows; a.L_max = in->L_max;
   a.NQ = fp.NQ; a.N = fp.N; a.G = fp.G; a.n_tiles = fp.n_tiles;
-  a.vis_div = vis_div; a.gather = 0;
+  a.vis_shift = vis_shift; a.gather = 0;
   indexer_pick_pipeline(in->d, fp8, fp.N, &a.stages, &a.nbuf_b);
+  a.n_acc = indexer_n_acc(fp.N);
   a.n_items = static_cast<long long>(in->B) * fp.G * fp.n_tiles;
   a.seq_len = in->seq_len; a.w = in->w; a.q_scale = in->q_scale; a.k_scale = in->k_scale;
   a.out = scores; a.out_row_stride = L_rows;
@@ -215,16 +242,16 @@ lsa_status_t run_flat_scores(const lsa_indexer_in_t* in, const void* keys, int L
 
 lsa_status_t run_select(int mode, int B, int T, int L_max, const int* seq_len, const float* scores,
                         long long row_stride, int n_slots, lsa_budget_t bu, int P, int M, const int* pages,
-                        int* out, int out_len, cudaStream_t st) {
+                        int* out, int out_len, void* sws, cudaStream_t st) {
   SelectArgs a{};
   a.mode = mode; a.B = B; a.T = T; a.L_max = L_max; a.seq_len = seq_len;
   a.scores = scores; a.row_stride = row_stride; a.n_slots = n_slots;
   a.k = bu.k; a.sink = bu.sink; a.window = bu.window; a.P = P; a.M = M; a.pages = pages;
   a.out = out; a.out_len = out_len;
-  int cap = 0;
-  const int C = select_cluster_size(B * T, n_slots, device_sm_count(), &cap);
-  a.cap = cap;
-  LSA_CHECK_CUDA(launch_select(a, C, st), "select launch");
+  a.status = device_status_ptr();
+  const SelectPlan p = mode == kSelectPages ? page_select_plan(B * T, n_slots, M)
+                                            : token_select_plan(B * T, n_slots, bu);
+  LSA_CHECK_CUDA(launch_select(a, p, sws, st), "select launch");
   return LSA_OK;
 }
 
@@ -241,13 +268,17 @@ lsa_status_t run_hier(const lsa_indexer_in_t* in, const void* page_keys, int P, 
     w += align_up(rows * M * 4, 256);
   }
   float* cand = reinterpret_cast<float*>(w);
+  w += align_up(rows * static_cast<size_t>(M) * P * 4, 256);
+  void* sws = w;   // selection scratch (reused by both selections)
 
   // 1) coarse scores over full, fully visible pages
-  lsa_status_t s = run_flat_scores(in, page_keys, n_pages, P, page_scores, st);
+  int p_shift = 0;
+  while ((1 << p_shift) < P) ++p_shift;
+  lsa_status_t s = run_flat_scores(in, page_keys, n_pages, p_shift, page_scores, st);
   if (s != LSA_OK) return s;
   // 2) recall: forced sink/window pages + top pages of the dynamic region (ascending)
   s = run_select(kSelectPages, in->B, in->T, in->L_max, in->seq_len, page_scores, n_pages, n_pages, bu, P, M,
-                 nullptr, pages, M, st);
+                 nullptr, pages, M, sws, st);
   if (s != LSA_OK) return s;
   // 3) fine scores over the recalled pages' tokens
   {
@@ -262,8 +293,9 @@ lsa_status_t run_hier(const lsa_indexer_in_t* in, const void* page_keys, int P, 
     a.L_rows = in->L_max; a.L_max = in->L_max;
     a.NQ = 1; a.N = N; a.G = in->T;
     a.n_tiles = (M * P + 127) / 128;
-    a.vis_div = 1; a.gather = 1;
+    a.vis_shift = 0; a.gather = 1;
     indexer_pick_pipeline(in->d, false, N, &a.stages, &a.nbuf_b);
+    a.n_acc = indexer_n_acc(N);
     a.n_items = static_cast<long long>(rows) * a.n_tiles;
     a.seq_len = in->seq_len; a.w = in->w;
     a.out = cand; a.out_row_stride = static_cast<long long>(M) * P;
@@ -275,15 +307,20 @@ lsa_status_t run_hier(const lsa_indexer_in_t* in, const void* page_keys, int P, 
   }
   // 4) token selection restricted to the recalled pages
   return run_select(kSelectHierTokens, in->B, in->T, in->L_max, in->seq_len, cand, static_cast<long long>(M) * P,
-                    M * P, bu, P, M, pages, idx, bu.k, st);
+                    M * P, bu, P, M, pages, idx, bu.k, sws, st);
 }
 
 lsa_status_t run_attn(const lsa_attn_in_t* at, const int* idx, int k, void* out, float* lse, void* ws,
                       cudaStream_t st) {
   const AttnPlan p = attn_plan(at, k);
-  CUtensorMap tm_q;
-  lsa_status_t s = make_tmap(&tm_q, at->q, false, at->d_qk, static_cast<uint64_t>(at->B) * at->T * at->Hq, 64, 128);
+  AttnMaps maps;
+  lsa_status_t s = make_tmap(&maps.q, at->q, false, at->d_qk, static_cast<uint64_t>(at->B) * at->T * at->Hq, 64, 128);
   if (s != LSA_OK) return s;
+  const uint64_t kv_rows = static_cast<uint64_t>(at->B) * at->L_max;
+  if ((s = make_tmap_strided(&maps.k_tile, at->k, at->d_qk, kv_rows, at->k_row_stride, 64, kAttnBN)) != LSA_OK) return s;
+  if ((s = make_tmap_strided(&maps.k_rows, at->k, at->d_qk, kv_rows, at->k_row_stride, 64, 1)) != LSA_OK) return s;
+  if ((s = make_tmap_strided(&maps.v_tile, at->v, at->d_v, kv_rows, at->v_row_stride, 64, kAttnBN)) != LSA_OK) return s;
+  if ((s = make_tmap_strided(&maps.v_rows, at->v, at->d_v, kv_rows, at->v_row_stride, 64, 1)) != LSA_OK) return s;
   AttnArgs a{};
   a.B = at->B; a.T = at->T; a.Hq = at->Hq; a.L_max = at->L_max;
   a.d_qk = at->d_qk; a.d_v = at->d_v; a.k = k;
@@ -306,7 +343,7 @@ lsa_status_t run_attn(const lsa_attn_in_t* at, const int* idx, int k, void* out,
     w += align_up(nm * 4, 256);
     a.part_l = reinterpret_cast<float*>(w);
   }
-  LSA_CHECK_CUDA(launch_attn(tm_q, a, st), "attention launch");
+  LSA_CHECK_CUDA(launch_attn(maps, a, st), "attention launch");
   if (p.n_split > 1) LSA_CHECK_CUDA(launch_attn_combine(a, st), "attention combine launch");
   return LSA_OK;
 }
@@ -324,6 +361,7 @@ lsa_status_t check_hier_params(const lsa_indexer_in_t* in, int P, int M, lsa_bud
   if (in->L_max % P) return fail(LSA_ERR_INVALID_ARG, "L_max must be a multiple of P");
   const int forced_max = (bu.sink + P - 1) / P + (bu.window + P - 1) / P + 1;
   if (M < forced_max) return fail(LSA_ERR_INVALID_ARG, "M=%d below the %d pages sink/window can force", M, forced_max);
+  if (M > 8192) return fail(LSA_ERR_UNSUPPORTED, "recall M=%d above 8192", M);
   if (static_cast<long long>(M) * P > (1 << 24)) return fail(LSA_ERR_UNSUPPORTED, "M * P too large");
   return LSA_OK;
 }
@@ -386,15 +424,19 @@ lsa_status_t lsa_workspace_size(lsa_op_t op, const lsa_op_args_t* args, size_t* 
   switch (op) {
     case LSA_OP_INDEX_FLAT:
       if ((s = check_indexer(args->indexer, true)) != LSA_OK) return s;
-      *bytes = flat_ws_bytes(args->indexer, args->scores_external != 0);
+      if ((s = check_budget(args->budget)) != LSA_OK) return s;
+      *bytes = flat_ws_bytes(args->indexer, args->budget, args->scores_external != 0);
       return LSA_OK;
     case LSA_OP_INDEX_HIER:
       if ((s = check_indexer(args->indexer, false)) != LSA_OK) return s;
       if ((s = check_hier_params(args->indexer, args->P, args->M, args->budget)) != LSA_OK) return s;
-      *bytes = hier_ws_bytes(args->indexer, args->P, args->M, false);
+      if ((s = check_budget(args->budget)) != LSA_OK) return s;
+      *bytes = hier_ws_bytes(args->indexer, args->P, args->M, args->budget, false);
       return LSA_OK;
     case LSA_OP_SELECT:
-      *bytes = 0;
+      if ((s = check_budget(args->budget)) != LSA_OK) return s;
+      if (args->B < 1 || args->T < 1 || args->L_max < 1) return fail(LSA_ERR_INVALID_ARG, "B, T and L_max must be >= 1");
+      *bytes = select_ws_bytes(args->B * args->T, token_select_plan(args->B * args->T, args->L_max, args->budget));
       return LSA_OK;
     case LSA_OP_SPARSE_ATTN:
       if ((s = check_attn(args->attn, args->budget.k)) != LSA_OK) return s;
@@ -408,9 +450,9 @@ lsa_status_t lsa_workspace_size(lsa_op_t op, const lsa_op_args_t* args, size_t* 
       size_t ix = 0;
       if (args->P) {
         if ((s = check_hier_params(in, args->P, args->M, args->budget)) != LSA_OK) return s;
-        ix = hier_ws_bytes(in, args->P, args->M, false);
+        ix = hier_ws_bytes(in, args->P, args->M, args->budget, false);
       } else {
-        ix = flat_ws_bytes(in, false);
+        ix = flat_ws_bytes(in, args->budget, false);
       }
       size_t at = 0;
       for (int i = 0; i < args->n_layers; ++i) {
@@ -432,29 +474,34 @@ lsa_status_t lsa_index_flat(const lsa_indexer_in_t* in, lsa_budget_t budget, int
   if (!idx && !scores_out) return fail(LSA_ERR_INVALID_ARG, "need idx or scores_out");
   if ((idx && !aligned16(idx)) || (scores_out && !aligned16(scores_out)))
     return fail(LSA_ERR_INVALID_ARG, "outputs must be 16-byte aligned");
-  const size_t need = flat_ws_bytes(in, scores_out != nullptr);
+  const size_t need = flat_ws_bytes(in, budget, scores_out != nullptr);
   if ((s = check_ws(workspace, workspace_bytes, need)) != LSA_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  float* scores = scores_out ? scores_out : static_cast<float*>(workspace);
-  if ((s = run_flat_scores(in, in->k, in->L_max, 1, scores, st)) != LSA_OK) return s;
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  float* scores = scores_out;
+  if (!scores) {
+    scores = reinterpret_cast<float*>(w);
+    w += align_up(static_cast<size_t>(in->B) * in->T * in->L_max * 4, 256);
+  }
+  if ((s = run_flat_scores(in, in->k, in->L_max, 0, scores, st)) != LSA_OK) return s;
   if (idx)
     return run_select(kSelectTokens, in->B, in->T, in->L_max, in->seq_len, scores, in->L_max, in->L_max, budget, 0,
-                      0, nullptr, idx, budget.k, st);
+                      0, nullptr, idx, budget.k, w, st);
   return LSA_OK;
 }
 
 lsa_status_t lsa_select_streaming(const float* scores, const int32_t* seq_len, int32_t B, int32_t T,
                                   int32_t L_max, lsa_budget_t budget, int32_t* idx, void* workspace,
                                   size_t workspace_bytes, lsa_stream_t stream) {
-  (void)workspace;
-  (void)workspace_bytes;
   lsa_status_t s;
   if ((s = check_budget(budget)) != LSA_OK) return s;
   if (!scores || !seq_len || !idx) return fail(LSA_ERR_INVALID_ARG, "null tensor");
   if (B < 1 || T < 1 || L_max < 1) return fail(LSA_ERR_INVALID_ARG, "B, T and L_max must be >= 1");
   if (static_cast<long long>(B) * T > 65535) return fail(LSA_ERR_UNSUPPORTED, "at most 65535 query rows per call");
+  const size_t need = select_ws_bytes(B * T, token_select_plan(B * T, L_max, budget));
+  if ((s = check_ws(workspace, workspace_bytes, need)) != LSA_OK) return s;
   return run_select(kSelectTokens, B, T, L_max, seq_len, scores, L_max, L_max, budget, 0, 0, nullptr, idx,
-                    budget.k, reinterpret_cast<cudaStream_t>(stream));
+                    budget.k, workspace, reinterpret_cast<cudaStream_t>(stream));
 }
 
 lsa_status_t lsa_pool_pages(const void* k, const int32_t* seq_len, int32_t B, int32_t L_max, int32_t d, int32_t P,
@@ -482,7 +529,7 @@ lsa_status_t lsa_index_hier(const lsa_indexer_in_t* in, const void* page_keys, i
   if (!aligned16(page_keys) || !aligned16(idx) || (pages_out && !aligned16(pages_out)))
     return fail(LSA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
   if (static_cast<long long>(in->B) * in->T > 65535) return fail(LSA_ERR_UNSUPPORTED, "at most 65535 query rows per call");
-  const size_t need = hier_ws_bytes(in, P, M, pages_out != nullptr);
+  const size_t need = hier_ws_bytes(in, P, M, budget, pages_out != nullptr);
   if ((s = check_ws(workspace, workspace_bytes, need)) != LSA_OK) return s;
   return run_hier(in, page_keys, P, M, budget, idx, pages_out, workspace, reinterpret_cast<cudaStream_t>(stream));
 }
@@ -530,9 +577,10 @@ lsa_status_t lsa_layer_group(const lsa_indexer_in_t* in, const void* page_keys, 
     if ((s = run_hier(in, page_keys, P, M, budget, idx_buf, nullptr, w, st)) != LSA_OK) return s;
   } else {
     float* scores = reinterpret_cast<float*>(w);
-    if ((s = run_flat_scores(in, in->k, in->L_max, 1, scores, st)) != LSA_OK) return s;
+    uint8_t* sws = w + align_up(static_cast<size_t>(in->B) * in->T * in->L_max * 4, 256);
+    if ((s = run_flat_scores(in, in->k, in->L_max, 0, scores, st)) != LSA_OK) return s;
     if ((s = run_select(kSelectTokens, in->B, in->T, in->L_max, in->seq_len, scores, in->L_max, in->L_max, budget,
-                        0, 0, nullptr, idx_buf, budget.k, st)) != LSA_OK)
+                        0, 0, nullptr, idx_buf, budget.k, sws, st)) != LSA_OK)
       return s;
   }
   for (int i = 0; i < n_layers; ++i) {

@@ -9,9 +9,9 @@
 // (d_qk = 576) and its first d_v = 512 columns as V.
 //
 // One CTA = (v part, KV split, query row). Heads (<= 128, zero-padded) sit on
-// the MMA M dimension; q is resident in shared memory. KV rows are gathered 32
-// at a time with 16-byte cp.async into 128-byte-swizzled tiles (double
-// buffered), used K-major for S = q K^T and MN-major for O += P V. S (32
+// the MMA M dimension; q is resident in shared memory. KV rows arrive 32 at a
+// time by TMA (tiled boxes for contiguous runs, tile::gather4 row gathers
+// otherwise) into 128-byte-swizzled tiles (double buffered), used K-major for S = q K^T and MN-major for O += P V. S (32
 // columns) and O (d_v / n_parts <= 256 columns, the fp32 accumulator) live in
 // TMEM; one thread per head runs the online softmax on its S row (lazy
 // rescaling: the running max moves only when a block raises it by > 2^8) and
@@ -40,9 +40,7 @@ struct ACfg {
   static constexpr int kPBytes = 128 * BN * 2;
   static constexpr int kSCol = kVN;
   static constexpr int kTmemCols = (kVN + BN) <= 128 ? 128 : ((kVN + BN) <= 256 ? 256 : 512);
-  static constexpr int kRowUnits = DQK / 8;
-  static constexpr int kVRowUnits = DV / 8;
-  static constexpr size_t kSmem = 1024 + kQBytes + 2 * kKVBytes + 2 * kVBytes + kPBytes + 2 * BN * 4 + 64;
+  static constexpr size_t kSmem = 1024 + kQBytes + 2 * kKVBytes + 2 * kVBytes + kPBytes + 2 * BN * 4 + 80;
 };
 
 __device__ __forceinline__ void spin_ns(unsigned long long ns) {
@@ -53,7 +51,9 @@ __device__ __forceinline__ void spin_ns(unsigned long long ns) {
 
 template <int DQK, int DV, bool SEP_V>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_kernel(const __grid_constant__ CUtensorMap tm_q, const AttnArgs a) {
+    attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kt,
+                const __grid_constant__ CUtensorMap tm_kg, const __grid_constant__ CUtensorMap tm_vt,
+                const __grid_constant__ CUtensorMap tm_vg, const AttnArgs a) {
   using C = ACfg<DQK, DV, SEP_V>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -66,7 +66,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* q_full = bars;
   uint64_t* s_full = bars + 1;
   uint64_t* pv_done = bars + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3);
+  uint64_t* kv_full = bars + 3;   // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -83,6 +84,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(q_full, 1);
     mbar_init(s_full, 1);
     mbar_init(pv_done, 1);
+    mbar_init(&kv_full[0], 1);
+    mbar_init(&kv_full[1], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -104,34 +107,53 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int c = 0; c < C::kQChunks; ++c) tma_load_2d(sQ + c * 16384, &tm_q, q_full, c * 64, r * a.Hq);
   }
 
+  // Gathers run on TMA, issued by warp 0: lane j holds entry j of the next
+  // block's indices (prefetched one block ahead). A block of 32 consecutive
+  // valid rows (the sink and window parts of a streaming index set) loads as
+  // tiled boxes; any other block as tile::gather4 row gathers (4 rows each).
+  // Invalid entries gather row 0 of the sequence (finite; masked in the softmax).
+  auto idx_at = [&](int blk) -> int {
+    const int ip = (blk0 + blk) * BN + tid;
+    int id = (blk < nblk && ip < a.k) ? __ldg(idx_row + ip) : -1;
+    return id >= a.L_max ? -1 : id;
+  };
+  int idx_reg = tid < BN ? idx_at(0) : -1;
+  constexpr uint32_t kBlockBytes = BN * (DQK + (SEP_V ? DV : 0)) * 2;
   auto load_block = [&](int blk, int buf) {
-    if (tid < BN) {
-      const int ip = (blk0 + blk) * BN + tid;
-      int id = ip < a.k ? __ldg(idx_row + ip) : -1;
-      if (id >= a.L_max) id = -1;
+    if (warp == 0) {
+      const int id = idx_reg;
       idx_s[buf * BN + tid] = id;
-    }
-    __syncthreads();
-    uint8_t* kv = sKV + buf * C::kKVBytes;
-    const long long row0 = static_cast<long long>(b) * a.L_max;
-    for (int u = tid; u < BN * C::kRowUnits; u += kThreads) {
-      const int j = u / C::kRowUnits, cu = u % C::kRowUnits;
-      const int id = idx_s[buf * BN + j];
-      uint8_t* dst = kv + (cu >> 3) * C::kChunkBytes + j * 128 + (((cu & 7) ^ (j & 7)) << 4);
-      const uint16_t* src = id >= 0 ? a.kp + (row0 + id) * a.k_stride + cu * 8 : a.kp;
-      cp_async_16(dst, src, id >= 0 ? 16u : 0u);
-    }
-    if (SEP_V) {
-      uint8_t* vv = sV + buf * C::kVBytes;
-      for (int u = tid; u < BN * C::kVRowUnits; u += kThreads) {
-        const int j = u / C::kVRowUnits, cu = u % C::kVRowUnits;
-        const int id = idx_s[buf * BN + j];
-        uint8_t* dst = vv + (cu >> 3) * C::kChunkBytes + j * 128 + (((cu & 7) ^ (j & 7)) << 4);
-        const uint16_t* src = id >= 0 ? a.vp + (row0 + id) * a.v_stride + cu * 8 : a.vp;
-        cp_async_16(dst, src, id >= 0 ? 16u : 0u);
+      idx_reg = idx_at(blk + 1);
+      const int id0 = __shfl_sync(0xffffffffu, id, 0);
+      const bool contiguous = __all_sync(0xffffffffu, id0 >= 0 && id == id0 + tid);
+      const int row0 = b * a.L_max;
+      const int y = row0 + (id >= 0 ? id : 0);
+      int ys[BN];
+#pragma unroll
+      for (int j = 0; j < BN; ++j) ys[j] = __shfl_sync(0xffffffffu, y, j);
+      if (tid == 0) {
+        mbar_arrive_expect_tx(&kv_full[buf], kBlockBytes);
+        uint8_t* kv = sKV + buf * C::kKVBytes;
+        uint8_t* vv = sV + buf * C::kVBytes;
+        if (contiguous) {
+          for (int c = 0; c < C::kQChunks; ++c) tma_load_2d(kv + c * C::kChunkBytes, &tm_kt, &kv_full[buf], c * 64, row0 + id0);
+          if (SEP_V)
+            for (int c = 0; c < DV / 64; ++c) tma_load_2d(vv + c * C::kChunkBytes, &tm_vt, &kv_full[buf], c * 64, row0 + id0);
+        } else {
+          for (int c = 0; c < C::kQChunks; ++c)
+#pragma unroll
+            for (int g = 0; g < BN / 4; ++g)
+              tma_gather4(kv + c * C::kChunkBytes + g * 512, &tm_kg, &kv_full[buf], c * 64, ys[4 * g], ys[4 * g + 1],
+                          ys[4 * g + 2], ys[4 * g + 3]);
+          if (SEP_V)
+            for (int c = 0; c < DV / 64; ++c)
+#pragma unroll
+              for (int g = 0; g < BN / 4; ++g)
+                tma_gather4(vv + c * C::kChunkBytes + g * 512, &tm_vg, &kv_full[buf], c * 64, ys[4 * g],
+                            ys[4 * g + 1], ys[4 * g + 2], ys[4 * g + 3]);
+        }
       }
     }
-    cp_async_commit();
   };
 
   const uint32_t idesc_qk = make_idesc(1, 1, 128, BN, 0, 0);
@@ -146,14 +168,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int buf = blk & 1;
     const bool pv_ok = blk >= 1 ? mbar_wait(pv_done, (blk - 1) & 1, a.status) : true;   // frees buf^1, P and O
     if (!__syncthreads_and(pv_ok)) { fail = true; break; }
-    if (blk + 1 < nblk) {
-      load_block(blk + 1, buf ^ 1);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    fence_proxy_async_smem();
-    __syncthreads();
+    if (blk + 1 < nblk) load_block(blk + 1, buf ^ 1);
+    const bool kv_ok = mbar_wait(&kv_full[buf], (blk >> 1) & 1, a.status);
+    if (!__syncthreads_and(kv_ok)) { fail = true; break; }
     if (tid == 0) {
       const bool q_ok = blk > 0 || mbar_wait(q_full, 0, a.status);
       if (!q_ok) {
@@ -316,42 +333,67 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // Merge KV-split partials: m* = max m_s; o = sum O_s 2^(m_s - m*) / sum l_s 2^(m_s - m*).
 __global__ void __launch_bounds__(128) combine_kernel(const AttnArgs a) {
+  __shared__ float s_f[64];
+  __shared__ float s_den;
   const int r = blockIdx.x, h = blockIdx.y;
-  const int c = threadIdx.x * 4;
-  if (c >= a.d_v) return;
-  const long long base = static_cast<long long>(r) * a.n_split * a.Hq + h;
-  float M = -INFINITY;
-  for (int s = 0; s < a.n_split; ++s) {
-    const long long i = base + static_cast<long long>(s) * a.Hq;
-    if (a.part_l[i] > 0.f) M = fmaxf(M, a.part_m[i]);
-  }
-  float den = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int s = 0; s < a.n_split; ++s) {
-    const long long i = base + static_cast<long long>(s) * a.Hq;
-    const float l = a.part_l[i];
-    if (l > 0.f) {
-      const float f = exp2f(a.part_m[i] - M);
-      den += l * f;
-      const float4 o = *reinterpret_cast<const float4*>(a.part_o + i * a.d_v + c);
-      acc[0] += o.x * f;
-      acc[1] += o.y * f;
-      acc[2] += o.z * f;
-      acc[3] += o.w * f;
+  const int ns = a.n_split;
+  const long long base = static_cast<long long>(r) * ns * a.Hq + h;
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    float m[2], l[2];
+    float M = -INFINITY;
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int sidx = lane + 32 * q;
+      m[q] = -INFINITY;
+      l[q] = 0.f;
+      if (sidx < ns) {
+        const long long i = base + static_cast<long long>(sidx) * a.Hq;
+        l[q] = a.part_l[i];
+        m[q] = l[q] > 0.f ? a.part_m[i] : -INFINITY;
+      }
+      M = fmaxf(M, m[q]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float den = 0.f;
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const float f = l[q] > 0.f ? exp2f(m[q] - M) : 0.f;
+      if (lane + 32 * q < 64) s_f[lane + 32 * q] = f;
+      den += l[q] * f;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    if (lane == 0) {
+      s_den = den;
+      if (a.lse) a.lse[static_cast<long long>(r) * a.Hq + h] = den > 0.f ? (M + log2f(den)) * 0.69314718055994530942f : -INFINITY;
     }
   }
-  const float inv = den > 0.f ? 1.f / den : 0.f;
+  __syncthreads();
+  const int c = threadIdx.x * 4;
+  if (c >= a.d_v) return;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+  for (int sidx = 0; sidx < ns; ++sidx) {
+    const float f = s_f[sidx];
+    const float4 o = *reinterpret_cast<const float4*>(a.part_o + (base + static_cast<long long>(sidx) * a.Hq) * a.d_v + c);
+    acc[0] = fmaf(o.x, f, acc[0]);
+    acc[1] = fmaf(o.y, f, acc[1]);
+    acc[2] = fmaf(o.z, f, acc[2]);
+    acc[3] = fmaf(o.w, f, acc[3]);
+  }
+  const float inv = s_den > 0.f ? 1.f / s_den : 0.f;
   const __nv_bfloat162 v01 = __floats2bfloat162_rn(acc[0] * inv, acc[1] * inv);
   const __nv_bfloat162 v23 = __floats2bfloat162_rn(acc[2] * inv, acc[3] * inv);
   uint2 pk;
   pk.x = *reinterpret_cast<const uint32_t*>(&v01);
   pk.y = *reinterpret_cast<const uint32_t*>(&v23);
   *reinterpret_cast<uint2*>(a.out + (static_cast<long long>(r) * a.Hq + h) * a.d_v + c) = pk;
-  if (threadIdx.x == 0 && a.lse)
-    a.lse[static_cast<long long>(r) * a.Hq + h] = den > 0.f ? (M + log2f(den)) * 0.69314718055994530942f : -INFINITY;
 }
 
 template <int DQK, int DV, bool SEP_V>
-cudaError_t launch_t(const CUtensorMap& tm_q, const AttnArgs& a, cudaStream_t stream) {
+cudaError_t launch_t(const AttnMaps& m, const AttnArgs& a, cudaStream_t stream) {
   using C = ACfg<DQK, DV, SEP_V>;
   const void* fn = reinterpret_cast<const void*>(&attn_kernel<DQK, DV, SEP_V>);
   size_t smem = C::kSmem;
@@ -359,7 +401,9 @@ cudaError_t launch_t(const CUtensorMap& tm_q, const AttnArgs& a, cudaStream_t st
   cudaError_t e = set_max_smem(fn, smem);
   if (e != cudaSuccess) return e;
   const dim3 grid(C::kNVP, a.n_split, a.B * a.T);
-  void* args[] = {const_cast<CUtensorMap*>(&tm_q), const_cast<AttnArgs*>(&a)};
+  void* args[] = {const_cast<CUtensorMap*>(&m.q), const_cast<CUtensorMap*>(&m.k_tile),
+                  const_cast<CUtensorMap*>(&m.k_rows), const_cast<CUtensorMap*>(&m.v_tile),
+                  const_cast<CUtensorMap*>(&m.v_rows), const_cast<AttnArgs*>(&a)};
   return cudaLaunchKernel(fn, grid, dim3(kThreads), args, smem, stream);
 }
 
@@ -370,21 +414,22 @@ size_t attn_smem_bytes(int d_qk, int d_v, bool sep_v) {
   return ACfg<64, 64, true>::kSmem;
 }
 
-cudaError_t launch_attn(const CUtensorMap& tm_q, const AttnArgs& a, cudaStream_t stream) {
+cudaError_t launch_attn(const AttnMaps& m, const AttnArgs& a, cudaStream_t stream) {
   if (a.d_qk == 576 && a.d_v == 512) {
     if (a.sep_v) return cudaErrorNotSupported;   // MLA keeps V inside the latent row
-    return launch_t<576, 512, false>(tm_q, a, stream);
+    return launch_t<576, 512, false>(m, a, stream);
   }
   if (a.d_qk == 64 && a.d_v == 64) {
-    if (a.sep_v) return launch_t<64, 64, true>(tm_q, a, stream);
-    return launch_t<64, 64, false>(tm_q, a, stream);
+    if (a.sep_v) return launch_t<64, 64, true>(m, a, stream);
+    return launch_t<64, 64, false>(m, a, stream);
   }
   return cudaErrorNotSupported;
 }
 
 cudaError_t launch_attn_combine(const AttnArgs& a, cudaStream_t stream) {
+  if (a.n_split > 64) return cudaErrorInvalidValue;
   const dim3 grid(a.B * a.T, a.Hq);
-  combine_kernel<<<grid, a.d_v / 4, 0, stream>>>(a);
+  combine_kernel<<<grid, a.d_v / 4 < 32 ? 32 : a.d_v / 4, 0, stream>>>(a);
   return cudaGetLastError();
 }
 

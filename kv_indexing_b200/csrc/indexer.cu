@@ -15,11 +15,12 @@
 // ReLU, the head-weighted sum and the causal mask are thread-local and the
 // [keys x heads] product never leaves the SM.
 //
-// Roles (192 threads, one CTA per SM, persistent over a contiguous item range):
+// Roles (320 threads, one CTA per SM, persistent over a contiguous tile range):
 //   warp 0      TMA producer: key tiles into an S-stage ring, query tiles into
 //               1-2 buffers (re-loaded only when the query group changes)
-//   warp 1      TMEM owner + single-thread UMMA issuer, double-buffered accumulator
-//   warps 2..5  epilogue: TMEM -> registers -> fp32 scores in global memory
+//   warp 1      TMEM owner + single-thread UMMA issuer; 2 or 4 accumulators
+//   warps 2..9  two epilogue warpgroups taking alternate tiles:
+//               TMEM -> registers -> fp32 scores in global memory
 //
 // Two tile sources: FLAT (128 consecutive key rows of one sequence) and
 // GATHER (the recalled pages of one query, 128 / P pages per tile, used by the
@@ -30,7 +31,8 @@
 namespace lsa {
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kEpiWG = 2;                      // epilogue warpgroups
+constexpr int kThreads = 64 + 128 * kEpiWG;
 constexpr int kTileM = 128;
 
 template <int DK, bool FP8>
@@ -44,98 +46,84 @@ struct Cfg {
   static_assert(kBoxes >= 1, "row must span at least one 128-byte box");
 };
 
-struct Item {
-  int b, t_or_g, j, q0;
-  long long group;
-  bool live;
-};
-
 __device__ __forceinline__ int clamp_len(const int* seq_len, int b, int L_max) {
   int L = __ldg(seq_len + b);
   return L < 0 ? 0 : (L > L_max ? L_max : L);
 }
 
-__device__ __forceinline__ Item decode_item(const IndexerArgs& a, long long item) {
-  Item it;
-  it.j = static_cast<int>(item % a.n_tiles);
-  const long long grp = item / a.n_tiles;
-  it.group = grp;
+// Per query group (FLAT: NQ queries of one sequence; GATHER: one query row).
+struct Group {
+  int b, q0, nq;      // sequence, first query, valid queries
+  int pos0;           // absolute position of query q0 (may be negative)
+  int n_live;         // tiles of this group that hold visible keys
+};
+
+__device__ __forceinline__ Group make_group(const IndexerArgs& a, long long grp) {
+  Group g;
   if (!a.gather) {
-    const int g = static_cast<int>(grp % a.G);
-    const int b = static_cast<int>(grp / a.G);
-    it.b = b;
-    it.t_or_g = g;
-    it.q0 = g * a.NQ;
-    const int Lb = clamp_len(a.seq_len, b, a.L_max);
-    const int t_last = min(a.T - 1, it.q0 + a.NQ - 1);
-    const int pos_last = Lb - a.T + t_last;
-    const int nvis = pos_last < 0 ? 0 : (pos_last + 1) / a.vis_div;
-    it.live = static_cast<long long>(kTileM) * it.j < nvis;
+    g.b = static_cast<int>(grp / a.G);
+    g.q0 = static_cast<int>(grp - static_cast<long long>(g.b) * a.G) * a.NQ;
+    g.nq = min(a.NQ, a.T - g.q0);
+    g.pos0 = clamp_len(a.seq_len, g.b, a.L_max) - a.T + g.q0;
+    const int pos_last = g.pos0 + g.nq - 1;
+    const int nvis = pos_last < 0 ? 0 : (pos_last + 1) >> a.vis_shift;
+    g.n_live = min(a.n_tiles, (nvis + kTileM - 1) / kTileM);
   } else {
     const int r = static_cast<int>(grp);
-    const int b = r / a.T, t = r % a.T;
-    it.b = b;
-    it.t_or_g = t;
-    it.q0 = t;
-    it.live = clamp_len(a.seq_len, b, a.L_max) - a.T + t >= 0;
+    g.b = r / a.T;
+    g.q0 = r - g.b * a.T;
+    g.nq = 1;
+    g.pos0 = clamp_len(a.seq_len, g.b, a.L_max) - a.T + g.q0;
+    g.n_live = g.pos0 >= 0 ? a.n_tiles : 0;
   }
-  return it;
+  return g;
 }
 
-// Write one score (or -inf) for query `qi` of the tile, key row `row`.
-template <bool FP8>
-__device__ __forceinline__ void emit_score(const IndexerArgs& a, const Item& it, int qi, int row, float score,
-                                           bool dead) {
-  if (!a.gather) {
-    const int t = it.q0 + qi;
-    if (qi >= a.NQ || t >= a.T) return;
-    const int s = kTileM * it.j + row;
-    if (s >= a.L_rows) return;
-    const int pos = clamp_len(a.seq_len, it.b, a.L_max) - a.T + t;
-    const int nvis = pos < 0 ? 0 : (pos + 1) / a.vis_div;
-    float v = -INFINITY;
-    if (!dead && s < nvis) {
-      v = score;
-      if (FP8) v *= __ldg(a.k_scale + static_cast<long long>(it.b) * a.L_rows + s);
-    }
-    a.out[(static_cast<long long>(it.b) * a.T + t) * a.out_row_stride + s] = v;
-  } else {
-    if (qi != 0) return;
-    const int slot = kTileM * it.j + row;
-    if (slot >= a.M * a.P) return;
-    const int r = it.b * a.T + it.t_or_g;
-    const int pos = clamp_len(a.seq_len, it.b, a.L_max) - a.T + it.t_or_g;
-    float v = -INFINITY;
-    if (!dead && pos >= 0) {
-      const int page = __ldg(a.pages + static_cast<long long>(r) * a.M + slot / a.P);
-      const int tok = page * a.P + slot % a.P;
-      const int sink_end = min(a.sink, pos + 1);
-      const int w_lo = max(sink_end, pos - a.window + 1);
-      // only dynamic candidates (visible, in neither the sink nor the window)
-      if (page >= 0 && tok >= sink_end && tok < w_lo) v = score;
-    }
-    a.out[static_cast<long long>(r) * a.out_row_stride + slot] = v;
+// Walks this CTA's contiguous range of (group, tile) items without divisions.
+struct TileIter {
+  long long item, end, grp;
+  int j;
+  Group g;
+  __device__ __forceinline__ void begin(const IndexerArgs& a, long long b0, long long e0) {
+    item = b0;
+    end = e0;
+    grp = b0 / a.n_tiles;
+    j = static_cast<int>(b0 - grp * a.n_tiles);
+    g = make_group(a, grp);
   }
-}
-
-__device__ __forceinline__ float relu_dot16(const float* wcol, const uint32_t (&v)[16]) {
-  float acc = 0.f;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) acc = fmaf(wcol[i], fmaxf(__uint_as_float(v[i]), 0.f), acc);
-  return acc;
-}
-
-__device__ __forceinline__ float relu_dot32(const float* wcol, const uint32_t (&v)[32]) {
-  float acc = 0.f;
-#pragma unroll
-  for (int i = 0; i < 32; ++i) acc = fmaf(wcol[i], fmaxf(__uint_as_float(v[i]), 0.f), acc);
-  return acc;
-}
+  __device__ __forceinline__ bool valid() const { return item < end; }
+  __device__ __forceinline__ bool live() const { return j < g.n_live; }
+  __device__ __forceinline__ void next(const IndexerArgs& a) {
+    ++item;
+    if (++j == a.n_tiles) {
+      j = 0;
+      ++grp;
+      if (item < end) g = make_group(a, grp);
+    }
+  }
+};
 
 __device__ __forceinline__ void spin_ns(unsigned long long ns) {
   const unsigned long long t0 = globaltimer_ns();
   while (globaltimer_ns() - t0 < ns) {
   }
+}
+
+// acc[i % 8] += w[i] * max(v[i], 0): eight independent FMA chains.
+template <int NV>
+__device__ __forceinline__ void relu_dot_acc(const float* wcol, const uint32_t (&v)[NV], float (&acc)[8]) {
+#pragma unroll
+  for (int i = 0; i < NV; i += 4) {
+    const float4 wv = *reinterpret_cast<const float4*>(wcol + i);
+    acc[(i + 0) & 7] = fmaf(wv.x, fmaxf(__uint_as_float(v[i + 0]), 0.f), acc[(i + 0) & 7]);
+    acc[(i + 1) & 7] = fmaf(wv.y, fmaxf(__uint_as_float(v[i + 1]), 0.f), acc[(i + 1) & 7]);
+    acc[(i + 2) & 7] = fmaf(wv.z, fmaxf(__uint_as_float(v[i + 2]), 0.f), acc[(i + 2) & 7]);
+    acc[(i + 3) & 7] = fmaf(wv.w, fmaxf(__uint_as_float(v[i + 3]), 0.f), acc[(i + 3) & 7]);
+  }
+}
+
+__device__ __forceinline__ float sum8(const float (&a)[8]) {
+  return ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
 }
 
 template <int DK, bool FP8>
@@ -145,17 +133,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   using C = Cfg<DK, FP8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int S = a.stages, NB = a.nbuf_b, N = a.N;
+  const int S = a.stages, NB = a.nbuf_b, N = a.N, NACC = a.n_acc;
   uint8_t* sA = base;
   uint8_t* sB = sA + static_cast<size_t>(S) * C::kATileBytes;
-  float* wcol_all = reinterpret_cast<float*>(sB + static_cast<size_t>(NB) * N * C::kRowBytes);  // [4][N]
-  uint64_t* a_full = reinterpret_cast<uint64_t*>(wcol_all + 4 * N);
+  float* wcol_all = reinterpret_cast<float*>(sB + static_cast<size_t>(NB) * N * C::kRowBytes);  // [8][N]
+  uint64_t* a_full = reinterpret_cast<uint64_t*>(wcol_all + 4 * kEpiWG * N);
   uint64_t* a_empty = a_full + S;
   uint64_t* b_full = a_empty + S;
   uint64_t* b_empty = b_full + 2;
   uint64_t* acc_full = b_empty + 2;
-  uint64_t* acc_empty = acc_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  uint64_t* acc_empty = acc_full + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -164,7 +152,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const long long it_end = it_begin + per + (blockIdx.x < rem ? 1 : 0);
 
   uint32_t tmem_cols = 32;
-  while (tmem_cols < static_cast<uint32_t>(2 * N)) tmem_cols <<= 1;
+  while (tmem_cols < static_cast<uint32_t>(NACC * N)) tmem_cols <<= 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -174,8 +162,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&b_full[i], 1);
       mbar_init(&b_empty[i], 1);
+    }
+    for (int i = 0; i < 4; ++i) {
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], 4);
+      mbar_init(&acc_empty[i], 4);    // the four warps of the epilogue warpgroup owning the slot
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -196,21 +186,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tm_q);
       const uint64_t pol = policy_evict_first();   // keys are streamed once
       long long na = 0, ng = 0, cur = -1;
-      for (long long item = it_begin; item < it_end; ++item) {
+      TileIter it;
+      for (it.begin(a, it_begin, it_end); it.valid(); it.next(a)) {
+        if (!it.live()) continue;
         if (*abort_flag) break;
-        const Item it = decode_item(a, item);
-        if (!it.live) continue;
-        if (it.group != cur) {
+        if (it.grp != cur) {
           const int bs = static_cast<int>(ng % NB);
           const uint32_t ph = static_cast<uint32_t>((ng / NB) & 1);
           if (!mbar_wait(&b_empty[bs], ph ^ 1, a.status)) { *abort_flag = 1; break; }
           mbar_arrive_expect_tx(&b_full[bs], N * C::kRowBytes);
-          const int qrow = (it.b * a.T + it.q0) * a.H;
+          const int qrow = (it.g.b * a.T + it.g.q0) * a.H;
           uint8_t* dst = sB + static_cast<size_t>(bs) * N * C::kRowBytes;
 #pragma unroll
           for (int bx = 0; bx < C::kBoxes; ++bx)
             tma_load_2d(dst + bx * N * 128, &tm_q, &b_full[bs], bx * C::kBoxElems, qrow);
-          cur = it.group;
+          cur = it.grp;
           ++ng;
         }
         const int s = static_cast<int>(na % S);
@@ -219,18 +209,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(&a_full[s], C::kATileBytes);
         uint8_t* dst = sA + static_cast<size_t>(s) * C::kATileBytes;
         if (!a.gather) {
-          const int y = it.b * a.L_rows + kTileM * it.j;
+          const int y = it.g.b * a.L_rows + kTileM * it.j;
 #pragma unroll
           for (int bx = 0; bx < C::kBoxes; ++bx)
             tma_load_2d_hint(dst + bx * kTileM * 128, &tm_k, &a_full[s], bx * C::kBoxElems, y, pol);
         } else {
           const int per_tile = kTileM / a.P;
-          const long long r = static_cast<long long>(it.b) * a.T + it.t_or_g;
+          const long long r = it.grp;
           for (int sub = 0; sub < per_tile; ++sub) {
             const int pi = it.j * per_tile + sub;
             int page = pi < a.M ? __ldg(a.pages + r * a.M + pi) : -1;
             if (page < 0) page = 0;   // masked in the epilogue
-            const int y = it.b * a.L_max + page * a.P;
+            const int y = it.g.b * a.L_max + page * a.P;
 #pragma unroll
             for (int bx = 0; bx < C::kBoxes; ++bx)
               tma_load_2d_hint(dst + bx * kTileM * 128 + sub * a.P * 128, &tm_k, &a_full[s], bx * C::kBoxElems,
@@ -246,20 +236,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc = FP8 ? make_idesc(0, 0, kTileM, N, 0, 0) : make_idesc(1, 1, kTileM, N, 0, 0);
       long long na = 0, ng = 0, nt = 0, cur = -1;
       int bs = 0;
-      for (long long item = it_begin; item < it_end; ++item) {
+      TileIter it;
+      for (it.begin(a, it_begin, it_end); it.valid(); it.next(a)) {
+        if (!it.live()) continue;
         if (*abort_flag) break;
-        const Item it = decode_item(a, item);
-        if (!it.live) continue;
-        if (it.group != cur) {
+        if (it.grp != cur) {
           if (cur >= 0) umma_commit(&b_empty[bs]);   // old query tile free once its MMAs finish
           bs = static_cast<int>(ng % NB);
           const uint32_t ph = static_cast<uint32_t>((ng / NB) & 1);
           if (!mbar_wait(&b_full[bs], ph, a.status)) { *abort_flag = 1; break; }
-          cur = it.group;
+          cur = it.grp;
           ++ng;
         }
-        const int acc = static_cast<int>(nt & 1);
-        const uint32_t aph = static_cast<uint32_t>((nt >> 1) & 1);
+        const int acc = static_cast<int>(nt % NACC);
+        const uint32_t aph = static_cast<uint32_t>((nt / NACC) & 1);
         if (!mbar_wait(&acc_empty[acc], aph ^ 1, a.status)) { *abort_flag = 1; break; }
         const int s = static_cast<int>(na % S);
         const uint32_t ph = static_cast<uint32_t>((na / S) & 1);
@@ -286,64 +276,100 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------------------------------------------------- epilogue --
+    const int ew = warp - 2;              // 0..7
+    const int wg = ew >> 2;               // epilogue warpgroup: takes live tiles with nt % 2 == wg
     const int qw = warp & 3;              // TMEM lane quarter of this warp
     const int row = qw * 32 + lane;       // key row of the tile owned by this thread
-    float* wcol = wcol_all + qw * N;      // per-warp copy: no cross-warp barrier needed
+    float* wcol = wcol_all + ew * N;      // per-warp copy: no cross-warp barrier needed
     long long nt = 0, cur = -1;
-    for (long long item = it_begin; item < it_end; ++item) {
+    int sink_end = 0, w_lo = 0;
+    TileIter it;
+    for (it.begin(a, it_begin, it_end); it.valid(); it.next(a)) {
+      const bool live = it.live();
+      const bool mine = live ? ((nt & 1) == wg) : ((it.j & 1) == wg);
+      if (!mine) {
+        nt += live ? 1 : 0;
+        continue;
+      }
       if (__any_sync(0xffffffffu, *abort_flag != 0)) break;   // warp-uniform exit
-      const Item it = decode_item(a, item);
-      if (it.group != cur) {
+      const Group& g = it.g;
+      if (it.grp != cur) {
         __syncwarp();
         for (int c = lane; c < N; c += 32) {
-          const int qi = c / a.H, h = c % a.H, t = it.q0 + qi;
+          const int qi = c / a.H, h = c - qi * a.H;
           float wv = 0.f;
-          if (qi < a.NQ && t < a.T) {
-            const long long wi = (static_cast<long long>(it.b) * a.T + t) * a.H + h;
+          if (qi < g.nq) {
+            const long long wi = (static_cast<long long>(g.b) * a.T + g.q0 + qi) * a.H + h;
             wv = __ldg(a.w + wi) * a.inv_sqrt_d;
             if (FP8) wv *= __ldg(a.q_scale + wi);
           }
           wcol[c] = wv;
         }
         __syncwarp();
-        cur = it.group;
+        if (a.gather && g.pos0 >= 0) {
+          sink_end = min(a.sink, g.pos0 + 1);
+          w_lo = max(sink_end, g.pos0 - a.window + 1);
+        }
+        cur = it.grp;
       }
-      if (!it.live) {
-        for (int qi = 0; qi < a.NQ; ++qi) emit_score<FP8>(a, it, qi, row, 0.f, true);
+      const int s = kTileM * it.j + row;                       // key row (FLAT) or slot (GATHER)
+      const long long orow = (static_cast<long long>(g.b) * a.T + g.q0) * a.out_row_stride;
+      if (!live) {
+        if (!a.gather) {
+          if (s < a.L_rows)
+            for (int qi = 0; qi < g.nq; ++qi) a.out[orow + qi * a.out_row_stride + s] = -INFINITY;
+        } else if (s < a.M * a.P) {
+          a.out[orow + s] = -INFINITY;
+        }
         continue;
       }
-      const int acc = static_cast<int>(nt & 1);
-      const uint32_t aph = static_cast<uint32_t>((nt >> 1) & 1);
+      const int acc = static_cast<int>(nt % NACC);
+      const uint32_t aph = static_cast<uint32_t>((nt / NACC) & 1);
+      ++nt;
       if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[acc], aph, a.status))) { *abort_flag = 1; break; }
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(qw * 32) << 16) + static_cast<uint32_t>(acc * N);
+      float kscale = 1.f;
+      if (FP8 && s < a.L_rows) kscale = __ldg(a.k_scale + static_cast<long long>(g.b) * a.L_rows + s);
       if (a.H >= 16) {
         for (int qi = 0; qi < a.NQ; ++qi) {
+          float acc8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
           const int c_end = (qi + 1) * a.H;
-          float sc = 0.f;
           for (int c0 = qi * a.H; c0 < c_end;) {
             if (c_end - c0 >= 64) {
               uint32_t v0[32], v1[32];
               tmem_ld32(tbase + c0, v0);
               tmem_ld32(tbase + c0 + 32, v1);
               tmem_ld_wait();
-              sc += relu_dot32(wcol + c0, v0) + relu_dot32(wcol + c0 + 32, v1);
+              relu_dot_acc<32>(wcol + c0, v0, acc8);
+              relu_dot_acc<32>(wcol + c0 + 32, v1, acc8);
               c0 += 64;
             } else if (c_end - c0 >= 32) {
               uint32_t v0[32];
               tmem_ld32(tbase + c0, v0);
               tmem_ld_wait();
-              sc += relu_dot32(wcol + c0, v0);
+              relu_dot_acc<32>(wcol + c0, v0, acc8);
               c0 += 32;
             } else {
               uint32_t v0[16];
               tmem_ld16(tbase + c0, v0);
               tmem_ld_wait();
-              sc += relu_dot16(wcol + c0, v0);
+              relu_dot_acc<16>(wcol + c0, v0, acc8);
               c0 += 16;
             }
           }
-          emit_score<FP8>(a, it, qi, row, sc, false);
+          if (qi < g.nq) {
+            const float sc = sum8(acc8);
+            if (!a.gather) {
+              const int pos = g.pos0 + qi;   // key s visible iff s < (pos + 1) >> vis_shift
+              const int nvis = pos < 0 ? 0 : (pos + 1) >> a.vis_shift;
+              if (s < a.L_rows) a.out[orow + qi * a.out_row_stride + s] = s < nvis ? sc * kscale : -INFINITY;
+            } else if (s < a.M * a.P) {
+              const int page = __ldg(a.pages + (static_cast<long long>(g.b) * a.T + g.q0) * a.M + s / a.P);
+              const int tok = page * a.P + (s & (a.P - 1));
+              a.out[orow + s] = (page >= 0 && tok >= sink_end && tok < w_lo) ? sc : -INFINITY;
+            }
+          }
         }
       } else {
         // H in {4, 8}: one 16-column load covers 16 / H queries
@@ -351,23 +377,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t v[16];
           tmem_ld16(tbase + c0, v);
           tmem_ld_wait();
-          if (a.H == 8) {
-#pragma unroll
-            for (int qq = 0; qq < 2; ++qq) {
-              float sc = 0.f;
-#pragma unroll
-              for (int i = 0; i < 8; ++i)
-                sc = fmaf(wcol[c0 + qq * 8 + i], fmaxf(__uint_as_float(v[qq * 8 + i]), 0.f), sc);
-              emit_score<FP8>(a, it, c0 / 8 + qq, row, sc, false);
-            }
-          } else {
-#pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-              float sc = 0.f;
-#pragma unroll
-              for (int i = 0; i < 4; ++i)
-                sc = fmaf(wcol[c0 + qq * 4 + i], fmaxf(__uint_as_float(v[qq * 4 + i]), 0.f), sc);
-              emit_score<FP8>(a, it, c0 / 4 + qq, row, sc, false);
+          const int per = 16 / a.H;
+          for (int qq = 0; qq < per; ++qq) {
+            float sc = 0.f;
+            for (int i = 0; i < a.H; ++i)
+              sc = fmaf(wcol[c0 + qq * a.H + i], fmaxf(__uint_as_float(v[qq * a.H + i]), 0.f), sc);
+            const int qi = c0 / a.H + qq;
+            if (qi >= g.nq) continue;
+            if (!a.gather) {
+              const int pos = g.pos0 + qi;
+              const int nvis = pos < 0 ? 0 : (pos + 1) >> a.vis_shift;
+              if (s < a.L_rows) a.out[orow + qi * a.out_row_stride + s] = s < nvis ? sc * kscale : -INFINITY;
+            } else if (s < a.M * a.P) {
+              const int page = __ldg(a.pages + (static_cast<long long>(g.b) * a.T + g.q0) * a.M + s / a.P);
+              const int tok = page * a.P + (s & (a.P - 1));
+              a.out[orow + s] = (page >= 0 && tok >= sink_end && tok < w_lo) ? sc : -INFINITY;
             }
           }
         }
@@ -375,7 +399,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[acc]);
-      ++nt;
     }
   }
 
@@ -397,22 +420,20 @@ const void* kernel_ptr() {
 
 size_t indexer_smem_bytes(int d, bool fp8, int N, int stages, int nbuf_b) {
   const size_t row = static_cast<size_t>(d) * (fp8 ? 1 : 2);
-  return 1024 + stages * 128 * row + nbuf_b * N * row + 4 * N * 4 + (2 * stages + 8) * 8 + 16;
+  return 1024 + stages * 128 * row + nbuf_b * N * row + 4 * kEpiWG * N * 4 + (2 * stages + 12) * 8 + 16;
 }
 
 void indexer_pick_pipeline(int d, bool fp8, int N, int* stages, int* nbuf_b) {
   const size_t kMax = 232448;
-  const size_t row = static_cast<size_t>(d) * (fp8 ? 1 : 2);
-  const size_t a_tile = 128 * row, b_tile = N * row;
   int nb = 2;
   if (indexer_smem_bytes(d, fp8, N, 3, 2) > kMax) nb = 1;
   int s = 8;
   while (s > 2 && indexer_smem_bytes(d, fp8, N, s, nb) > kMax) --s;
-  (void)a_tile;
-  (void)b_tile;
   *stages = s;
   *nbuf_b = nb;
 }
+
+int indexer_n_acc(int N) { return 4 * N <= 512 ? 4 : 2; }
 
 cudaError_t launch_indexer(const CUtensorMap& tm_k, const CUtensorMap& tm_q, const IndexerArgs& a, bool fp8,
                            int grid, cudaStream_t stream) {

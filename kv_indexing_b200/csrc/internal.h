@@ -18,9 +18,10 @@ struct IndexerArgs {
   int L_max;             // token capacity per sequence (seq_len clamp; gather rows)
   int NQ, N, G;          // queries per tile, MMA N (= NQ * H), query groups per sequence
   int n_tiles;           // tiles per group (FLAT) or per query row (GATHER)
-  int vis_div;           // FLAT: key s visible to pos iff s < (pos + 1) / vis_div
+  int vis_shift;         // FLAT: key s visible to pos iff s < (pos + 1) >> vis_shift (rows of 2^shift tokens)
   int gather;            // 0 = FLAT, 1 = GATHER
   int stages, nbuf_b;    // A-tile ring depth, B-tile buffers (1 or 2)
+  int n_acc;             // TMEM accumulators (2 or 4)
   long long n_items;
   const int* seq_len;
   const float* w;
@@ -37,6 +38,7 @@ struct IndexerArgs {
 
 size_t indexer_smem_bytes(int d, bool fp8, int N, int stages, int nbuf_b);
 void indexer_pick_pipeline(int d, bool fp8, int N, int* stages, int* nbuf_b);
+int indexer_n_acc(int N);
 cudaError_t launch_indexer(const CUtensorMap& tm_k, const CUtensorMap& tm_q, const IndexerArgs& a,
                            bool fp8, int grid, cudaStream_t stream);
 
@@ -56,11 +58,30 @@ struct SelectArgs {
   const int* pages;       // kSelectHierTokens: [B*T, M]
   int* out;
   int out_len;            // k (tokens) or M (pages)
-  int cap;                // keys cached in shared memory per CTA (0 = stream from global)
+  // scratch (workspace): per-CTA candidate lists and per-row arrival counters
+  uint32_t* cand_keys;    // [rows, C, cand_cap]
+  int* cand_slots;        // [rows, C, cand_cap]
+  unsigned* row_arrivals; // [rows]
+  int cand_cap;
+  int final_in_smem;
+  // grid-cooperative path: per-row coordination blocks
+  void* grid_ws;
+  size_t grid_row_bytes;
+  int* status;
 };
 
-cudaError_t launch_select(const SelectArgs& a, int cluster, cudaStream_t stream);
-int select_cluster_size(int rows, int max_dyn, int num_sms, int* cap);
+// C CTAs per row, `seg` slots each; each keeps at most `cand_cap` candidates.
+struct SelectPlan {
+  int C, seg, cand_cap;
+  bool final_in_smem;
+  bool grid;              // grid-cooperative launch (rows * C CTAs co-resident)
+};
+
+// d_bound: an upper bound on the dynamic budget of any row (k - sink - window for
+// token selection, M for page recall).
+SelectPlan select_plan(int rows, int n_slots, int d_bound, int num_sms);
+size_t select_ws_bytes(int rows, const SelectPlan& p);
+cudaError_t launch_select(const SelectArgs& a, const SelectPlan& p, void* ws, cudaStream_t stream);
 
 // ------------------------------------------------------------------ pooling --
 cudaError_t launch_pool(const uint16_t* k, const int* seq_len, int B, int L_max, int d, int P,
@@ -87,8 +108,15 @@ struct AttnArgs {
 };
 
 constexpr int kAttnBN = 32;  // KV rows per block
+
+// TMA descriptors of one attention launch: q tiles [128 heads x 64], K/V row
+// tiles [32 rows x 64] (contiguous blocks) and one-row boxes for row gathers.
+struct AttnMaps {
+  CUtensorMap q, k_tile, k_rows, v_tile, v_rows;
+};
+
 size_t attn_smem_bytes(int d_qk, int d_v, bool sep_v);
-cudaError_t launch_attn(const CUtensorMap& tm_q, const AttnArgs& a, cudaStream_t stream);
+cudaError_t launch_attn(const AttnMaps& maps, const AttnArgs& a, cudaStream_t stream);
 cudaError_t launch_attn_combine(const AttnArgs& a, cudaStream_t stream);
 
 // --------------------------------------------------------------------- misc --

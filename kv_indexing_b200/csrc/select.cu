@@ -10,28 +10,32 @@
 // Hierarchical Indexing (forced sink/window pages + the top pages of the
 // dynamic region, all ascending) and the fine token set over recalled pages.
 //
-// Algorithm: scores map to order-preserving uint32 keys (-inf -> 0 = not a
-// candidate, -0 -> +0). A cluster of C CTAs splits the row's dynamic range
-// into C contiguous segments; three radix passes (11, 11, 10 bits) build
-// per-CTA histograms, merged across the cluster through distributed shared
-// memory, that narrow down the exact key of the D-th best candidate. Every
-// candidate above that key is taken, plus the lowest-index candidates equal to
-// it; an ordered compaction (block scans, cluster-wide segment offsets) writes
-// them in ascending index order. The result does not depend on C.
-#include <cooperative_groups.h>
-
+// Algorithm (one launch, no clusters): scores map to order-preserving uint32
+// keys (-inf -> 0 = not a candidate, -0 -> +0). C CTAs split a row's dynamic
+// range into contiguous segments; each thread holds up to 16 consecutive keys
+// in registers. A CTA finds the exact key of its local D-th best candidate by
+// radix select over 13-bit digits of (key - segment min): the digits span the
+// segment's actual key range, so the counts spread over the histogram instead
+// of piling into a few exponent bins, and two passes usually resolve it. It
+// writes its local top-D (key, slot) list, in slot order, to the workspace.
+// Any element of the row's top-D is in its segment's top-D, so the last CTA of
+// the row to finish (a per-row arrival counter) runs the same exact select over
+// the concatenated lists (32 per thread) and writes the final row. Ties go to
+// the lower slot at both levels, so the result equals the definition exactly.
+// Oversized segments or merges fall back to a shared/global-memory radix select.
 #include "internal.h"
 #include "ptx.cuh"
-
-namespace cg = cooperative_groups;
 
 namespace lsa {
 namespace {
 
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
-constexpr int kBins = 2048;
-constexpr int kPerThread = 8;   // consecutive elements per thread in the compaction
+constexpr int kDigitBits = 13;   // register-path radix digit
+constexpr int kDigits = 1 << kDigitBits;
+constexpr int kPer = 8;          // consecutive elements per thread per compaction chunk (fallback)
+constexpr int kRL = 16;          // keys per thread, local phase
+constexpr int kRF = 32;          // keys per thread, merge phase
 
 __device__ __forceinline__ uint32_t score_key(float f) {
   uint32_t u = __float_as_uint(f);
@@ -102,7 +106,7 @@ __device__ __forceinline__ Plan make_plan(const SelectArgs& a, int r) {
   return p;
 }
 
-// Inclusive scan of one value per thread (thread order). Uses `tmp` [kWarps+1].
+// Inclusive scan of one value per thread (thread order). Uses `tmp` [kWarps].
 __device__ __forceinline__ uint32_t block_incl_scan(uint32_t v, uint32_t* tmp, uint32_t* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t x = v;
@@ -129,207 +133,148 @@ __device__ __forceinline__ uint32_t block_incl_scan(uint32_t v, uint32_t* tmp, u
   return res;
 }
 
-// Histogram update with warp aggregation (lanes hitting the same bin add once).
-__device__ __forceinline__ void hist_add(uint32_t* h, uint32_t bin, bool active) {
-  const uint32_t key = active ? bin : 0xFFFFFFFFu;
-  const unsigned peers = __match_any_sync(0xffffffffu, key);
-  const int leader = __ffs(peers) - 1;
-  if (active && (threadIdx.x & 31) == leader) atomicAdd(&h[bin], static_cast<uint32_t>(__popc(peers)));
+struct Thr {
+  uint32_t thr;       // exact key of the D-th best candidate
+  uint32_t need_eq;   // how many keys equal to thr are taken (lowest index first)
+  bool all;           // every candidate is taken (fewer than D of them)
+};
+
+struct Shared {
+  uint32_t hist[kDigits];
+  uint32_t tmp[32];
+  uint32_t red[3][kWarps];
+  uint32_t cnt, mn, mx;
+  int bin;
+  uint32_t above;
+  int last;
+};
+
+// Block-wide count / min / max of per-thread partials (into sh.cnt, sh.mn, sh.mx).
+__device__ __forceinline__ void block_cnt_min_max(uint32_t c, uint32_t mn, uint32_t mx, Shared& sh) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    c += __shfl_xor_sync(0xffffffffu, c, o);
+    mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  if (lane == 0) {
+    sh.red[0][warp] = c;
+    sh.red[1][warp] = mn;
+    sh.red[2][warp] = mx;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    c = lane < kWarps ? sh.red[0][lane] : 0u;
+    mn = lane < kWarps ? sh.red[1][lane] : 0xFFFFFFFFu;
+    mx = lane < kWarps ? sh.red[2][lane] : 0u;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      c += __shfl_xor_sync(0xffffffffu, c, o);
+      mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+      mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+    if (lane == 0) {
+      sh.cnt = c;
+      sh.mn = mn;
+      sh.mx = mx;
+    }
+  }
+  __syncthreads();
 }
 
-template <bool IN_SMEM>
-__device__ __forceinline__ uint32_t key_at(const uint32_t* keys, const float* row, int my_lo, int i) {
-  if (IN_SMEM) return keys[i];
-  return score_key(__ldg(row + my_lo + i));
-}
-
-template <bool IN_SMEM>
-__global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelectArgs a) {
-  cg::cluster_group cluster = cg::this_cluster();
-  const int C = static_cast<int>(cluster.num_blocks());
-  const int rank = static_cast<int>(cluster.block_rank());
-  const int r = blockIdx.y;
+// Exact threshold of the D-th best key of keys[0, n) (key 0 = not a candidate).
+__device__ Thr cta_threshold(const uint32_t* keys, int n, uint32_t D, Shared& sh) {
   const int tid = threadIdx.x;
-
-  extern __shared__ uint32_t sm[];
-  uint32_t* hist[2] = {sm, sm + kBins};
-  uint32_t* ghist = sm + 2 * kBins;
-  uint32_t* tmp = ghist + kBins;          // kWarps + 1 scan scratch
-  uint32_t* pub = tmp + 32;               // [0] = gt count, [1] = eq count (read by the cluster)
-  uint32_t* keys = pub + 32;
-  __shared__ int s_bin;
-  __shared__ uint32_t s_above;
-
-  const Plan pl = make_plan(a, r);
-  int* out = a.out + static_cast<long long>(r) * a.out_len;
-  const float* row = a.scores + static_cast<long long>(r) * a.row_stride;
-  if (!pl.valid) {
-    if (rank == 0)
-      for (int i = tid; i < a.out_len; i += kThreads) out[i] = -1;
-    return;   // every CTA of the cluster takes this branch (same row)
+  Thr r{0u, 0u, false};
+  uint32_t c = 0u;
+  for (int i = tid; i < n; i += kThreads) c += keys[i] != 0u ? 1u : 0u;
+  uint32_t total = 0u;
+  block_incl_scan(c, sh.tmp, &total);
+  if (total <= D) {
+    r.all = true;
+    return r;
   }
-
-  const int len = pl.dyn_hi - pl.dyn_lo;
-  const int seg = (len + C - 1) / C;
-  int my_lo = pl.dyn_lo + rank * seg;
-  if (my_lo > pl.dyn_hi) my_lo = pl.dyn_hi;
-  const int my_hi = min(pl.dyn_hi, my_lo + seg);
-  const int my_n = my_hi - my_lo;
-
-  // ---- pass 0: load keys (cache in shared memory) + top-digit histogram ----
-  for (int i = tid; i < kBins; i += kThreads) hist[0][i] = 0u;
-  __syncthreads();
-  for (int i0 = 0; i0 < my_n; i0 += kThreads) {
-    const int i = i0 + tid;
-    uint32_t k = 0u;
-    if (i < my_n) {
-      k = score_key(__ldg(row + my_lo + i));
-      if (IN_SMEM) keys[i] = k;
-    }
-    hist_add(hist[0], k >> 21, k != 0u);
+  if (D == 0u) {
+    r.thr = 0xFFFFFFFFu;
+    return r;
   }
-  __syncthreads();
-
-  uint32_t prefix = 0u, mask = 0u, need = static_cast<uint32_t>(pl.D);
-  uint32_t thr = 0u, need_eq = 0u;
-  bool take_all = false;
-  uint32_t n_cand = 0u;
-
-  const int shifts[3] = {21, 10, 0};
-  const int widths[3] = {11, 11, 10};
+  uint32_t prefix = 0u, mask = 0u, need = D;
   for (int pass = 0; pass < 3; ++pass) {
-    const int shift = shifts[pass];
-    const int nb = 1 << widths[pass];
+    const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+    const int nb = pass == 2 ? 1024 : 2048;
     const uint32_t dmask = static_cast<uint32_t>(nb - 1);
-    uint32_t* h = hist[pass & 1];
-    if (pass > 0) {
-      for (int i = tid; i < nb; i += kThreads) h[i] = 0u;
-      __syncthreads();
-      for (int i0 = 0; i0 < my_n; i0 += kThreads) {
-        const int i = i0 + tid;
-        const uint32_t k = i < my_n ? key_at<IN_SMEM>(keys, row, my_lo, i) : 0u;
-        const bool act = k != 0u && (k & mask) == prefix;
-        hist_add(h, (k >> shift) & dmask, act);
-      }
-      __syncthreads();
-    }
-    // merge the cluster's histograms
-    cluster.sync();
-    for (int i = tid; i < nb; i += kThreads) {
-      uint32_t s = 0u;
-      for (int c = 0; c < C; ++c) s += cluster.map_shared_rank(h, c)[i];
-      ghist[i] = s;
+    for (int i = tid; i < nb; i += kThreads) sh.hist[i] = 0u;
+    __syncthreads();
+    for (int i = tid; i < n; i += kThreads) {
+      const uint32_t k = keys[i];
+      if (k != 0u && (k & mask) == prefix) atomicAdd(&sh.hist[(k >> shift) & dmask], 1u);
     }
     __syncthreads();
-
-    const int per = nb / kThreads;             // bins per thread (4 or 2)
-    const int hi_bin = nb - per * tid;         // this thread owns bins [hi_bin - per, hi_bin)
+    const int per = nb / kThreads;             // bins per thread (4 or 2), counted from the top
+    const int hi_bin = nb - per * tid;
     uint32_t local = 0u;
-    for (int q = 1; q <= per; ++q) local += ghist[hi_bin - q];
-    uint32_t total = 0u;
-    const uint32_t incl = block_incl_scan(local, tmp, &total);
-
-    if (pass == 0) {
-      n_cand = total;
-      // fixed outputs and padding (rank 0), now that the dynamic count is known
-      if (rank == 0) {
-        const int n_sel = min(static_cast<uint32_t>(pl.D), n_cand);
-        for (int i = tid; i < pl.lead_a_n; i += kThreads) out[i] = pl.lead_a_lo + i;
-        for (int i = tid; i < pl.lead_b_n; i += kThreads) out[pl.lead_a_n + i] = pl.lead_b_lo + i;
-        const int tr0 = pl.dyn_off + n_sel;
-        for (int i = tid; i < pl.trail_n; i += kThreads) out[tr0 + i] = pl.trail_lo + i;
-        for (int i = tr0 + pl.trail_n + tid; i < a.out_len; i += kThreads) out[i] = -1;
-      }
-      if (n_cand <= need) {
-        take_all = true;
-        break;
-      }
-      if (need == 0u) break;
-    }
-
+    for (int q = 1; q <= per; ++q) local += sh.hist[hi_bin - q];
+    const uint32_t incl = block_incl_scan(local, sh.tmp, nullptr);
     const uint32_t excl = incl - local;
     if (excl < need && need <= incl) {
       uint32_t above = excl;
       for (int q = 1; q <= per; ++q) {
         const int bb = hi_bin - q;
-        if (above + ghist[bb] >= need) {
-          s_bin = bb;
-          s_above = above;
+        if (above + sh.hist[bb] >= need) {
+          sh.bin = bb;
+          sh.above = above;
           break;
         }
-        above += ghist[bb];
+        above += sh.hist[bb];
       }
     }
     __syncthreads();
-    prefix |= static_cast<uint32_t>(s_bin) << shift;
+    prefix |= static_cast<uint32_t>(sh.bin) << shift;
     mask |= dmask << shift;
-    need -= s_above;
+    need -= sh.above;
     __syncthreads();
   }
+  r.thr = prefix;
+  r.need_eq = need;
+  return r;
+}
 
-  if (take_all) {
-    thr = 0u;          // every candidate (key > 0)
-    need_eq = 0u;
-  } else if (pl.D == 0) {
-    thr = 0xFFFFFFFFu;
-    need_eq = 0u;
-  } else {
-    thr = prefix;      // exact key of the D-th best candidate
-    need_eq = need;    // how many candidates equal to it are taken (lowest index first)
+// Emit the selected elements of keys[0, n) in index order: emit(out_pos, i).
+// Returns how many were selected.
+template <class F>
+__device__ uint32_t cta_emit(const uint32_t* keys, int n, const Thr& t, Shared& sh, F&& emit) {
+  const int tid = threadIdx.x;
+  uint32_t eq_total = 0u;
+  if (!t.all) {
+    uint32_t e = 0u;
+    for (int i = tid; i < n; i += kThreads) e += (keys[i] == t.thr && keys[i] != 0u) ? 1u : 0u;
+    block_incl_scan(e, sh.tmp, &eq_total);
   }
-
-  // ---- counts per segment, published to the cluster ----
-  uint32_t gt = 0u, eq = 0u;
-  for (int i = tid; i < my_n; i += kThreads) {
-    const uint32_t k = key_at<IN_SMEM>(keys, row, my_lo, i);
-    gt += (k > thr && k != 0u) ? 1u : 0u;
-    eq += (k == thr && k != 0u) ? 1u : 0u;
-  }
-  uint32_t tgt = 0u, teq = 0u;
-  block_incl_scan(gt, tmp, &tgt);
-  block_incl_scan(eq, tmp, &teq);
-  if (tid == 0) {
-    pub[0] = tgt;
-    pub[1] = teq;
-  }
-  cluster.sync();
-  uint32_t base_sel = 0u, eq_before = 0u, my_take = 0u;
-  for (int c = 0; c < C; ++c) {
-    const uint32_t* rp = cluster.map_shared_rank(pub, c);
-    const uint32_t g_c = rp[0], e_c = rp[1];
-    const uint32_t take_c = need_eq > eq_before ? min(need_eq - eq_before, e_c) : 0u;
-    if (c < rank) base_sel += g_c + take_c;
-    if (c == rank) my_take = take_c;
-    eq_before += e_c;
-  }
-
-  // ---- ordered compaction of this segment ----
-  const int chunk = kThreads * kPerThread;
+  const bool tie_scan = !t.all && t.need_eq > 0u && t.need_eq < eq_total;
+  const bool ties_all = t.need_eq >= eq_total;
   uint32_t eq_run = 0u, sel_run = 0u;
-  int* dyn_out = out + pl.dyn_off + base_sel;
-  for (int c0 = 0; c0 < my_n; c0 += chunk) {
-    const int i0 = c0 + tid * kPerThread;
-    uint32_t kk[kPerThread];
+  for (int c0 = 0; c0 < n; c0 += kThreads * kPer) {
+    const int i0 = c0 + tid * kPer;
+    uint32_t kk[kPer];
     uint32_t ne = 0u;
 #pragma unroll
-    for (int e = 0; e < kPerThread; ++e) {
-      const int i = i0 + e;
-      kk[e] = i < my_n ? key_at<IN_SMEM>(keys, row, my_lo, i) : 0u;
-      ne += (kk[e] == thr && kk[e] != 0u) ? 1u : 0u;
+    for (int e = 0; e < kPer; ++e) {
+      kk[e] = i0 + e < n ? keys[i0 + e] : 0u;
+      ne += (kk[e] == t.thr && kk[e] != 0u) ? 1u : 0u;
     }
-    uint32_t eq_tot = 0u;
-    const uint32_t eq_ex = block_incl_scan(ne, tmp, &eq_tot) - ne + eq_run;
-    uint32_t ns = 0u, er = eq_ex;
-    uint32_t selmask = 0u;
+    uint32_t eq_tot = 0u, er = 0u;
+    if (tie_scan) er = block_incl_scan(ne, sh.tmp, &eq_tot) - ne + eq_run;
+    uint32_t selmask = 0u, ns = 0u;
 #pragma unroll
-    for (int e = 0; e < kPerThread; ++e) {
+    for (int e = 0; e < kPer; ++e) {
       const uint32_t k = kk[e];
       bool s = false;
       if (k != 0u) {
-        if (k > thr) {
+        if (t.all || k > t.thr) {
           s = true;
-        } else if (k == thr) {
-          s = er < my_take;
+        } else if (k == t.thr) {
+          s = tie_scan ? (er < t.need_eq) : ties_all;
           ++er;
         }
       }
@@ -339,59 +284,817 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelectArgs a)
       }
     }
     uint32_t sel_tot = 0u;
-    uint32_t pos_out = block_incl_scan(ns, tmp, &sel_tot) - ns + sel_run;
+    uint32_t pos = block_incl_scan(ns, sh.tmp, &sel_tot) - ns + sel_run;
 #pragma unroll
-    for (int e = 0; e < kPerThread; ++e) {
-      if (selmask & (1u << e)) {
-        const int slot = my_lo + i0 + e;
-        int tok = slot;
-        if (a.mode == kSelectHierTokens) {
-          const int page = __ldg(a.pages + static_cast<long long>(r) * a.M + slot / a.P);
-          tok = page * a.P + slot % a.P;
-        }
-        dyn_out[pos_out++] = tok;
-      }
-    }
+    for (int e = 0; e < kPer; ++e)
+      if (selmask & (1u << e)) emit(pos++, i0 + e);
     eq_run += eq_tot;
     sel_run += sel_tot;
   }
-  cluster.sync();   // peers may still read this CTA's published counts
+  return sel_run;
+}
+
+
+// Exact threshold of the D-th best key among the nonzero keys held in
+// registers (thread t holds keys[t*R .. t*R+R)).
+template <int R>
+__device__ Thr reg_threshold(const uint32_t (&k)[R], uint32_t D, Shared& sh) {
+  const int tid = threadIdx.x;
+  uint32_t c = 0u, mn = 0xFFFFFFFFu, mx = 0u;
+#pragma unroll
+  for (int j = 0; j < R; ++j)
+    if (k[j] != 0u) {
+      ++c;
+      mn = min(mn, k[j]);
+      mx = max(mx, k[j]);
+    }
+  block_cnt_min_max(c, mn, mx, sh);
+  Thr r{0u, 0u, false};
+  const uint32_t total = sh.cnt, kmin = sh.mn, kmax = sh.mx;
+  if (total <= D) {
+    r.all = true;
+    return r;
+  }
+  if (D == 0u) {
+    r.thr = 0xFFFFFFFFu;
+    return r;
+  }
+  if (kmin == kmax) {
+    r.thr = kmax;
+    r.need_eq = D;
+    return r;
+  }
+  const int bits = 32 - __clz(kmax - kmin);              // every rel = key - kmin is < 2^bits
+  int prev = bits;                                        // keys in play satisfy rel >> prev == hi
+  int shift = bits > kDigitBits ? bits - kDigitBits : 0;
+  uint32_t hi = 0u, need = D;
+  while (true) {
+    const int width = prev - shift;                       // digit bits this pass (<= 13)
+    const int nb = 1 << width;
+    const uint32_t dmask = static_cast<uint32_t>(nb - 1);
+    for (int i = tid; i < nb; i += kThreads) sh.hist[i] = 0u;
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < R; ++j) {
+      const uint32_t rel = k[j] - kmin;
+      const bool in = k[j] != 0u && (prev >= 32 || (rel >> prev) == hi);
+      if (in) atomicAdd(&sh.hist[(rel >> shift) & dmask], 1u);
+    }
+    __syncthreads();
+    const int per = (nb + kThreads - 1) / kThreads;       // bins per thread, counted from the top
+    const int top = nb - per * tid;
+    uint32_t local = 0u;
+    for (int q = 1; q <= per; ++q)
+      if (top - q >= 0) local += sh.hist[top - q];
+    const uint32_t incl = block_incl_scan(local, sh.tmp, nullptr);
+    const uint32_t excl = incl - local;
+    if (excl < need && need <= incl) {
+      uint32_t above = excl;
+      for (int q = 1; q <= per; ++q) {
+        const int bb = top - q;
+        if (bb < 0) break;
+        if (above + sh.hist[bb] >= need) {
+          sh.bin = bb;
+          sh.above = above;
+          break;
+        }
+        above += sh.hist[bb];
+      }
+    }
+    __syncthreads();
+    hi = (width >= 32 ? 0u : (hi << width)) | static_cast<uint32_t>(sh.bin);
+    need -= sh.above;
+    __syncthreads();
+    if (shift == 0) break;
+    prev = shift;
+    shift = shift > kDigitBits ? shift - kDigitBits : 0;
+  }
+  r.thr = kmin + hi;
+  r.need_eq = need;
+  return r;
+}
+
+// Emit the selected register-held keys in index order: emit(out_pos, j).
+// Layout (warp-striped): lane l of warp w holds element w*32*R + 32*j + l in
+// k[j], so index order is (warp, j, lane). Positions come from per-stripe warp
+// ballots plus one exclusive scan over the warps' counts.
+template <int R, class F>
+__device__ uint32_t reg_emit(const uint32_t (&k)[R], const Thr& t, Shared& sh, F&& emit) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t lt = (1u << lane) - 1u;
+  uint32_t gtm[R], eqm[R];
+  uint32_t n_gt = 0u, n_eq = 0u;
+#pragma unroll
+  for (int j = 0; j < R; ++j) {
+    const bool nz = k[j] != 0u;
+    gtm[j] = __ballot_sync(0xffffffffu, nz && (t.all || k[j] > t.thr));
+    eqm[j] = __ballot_sync(0xffffffffu, nz && !t.all && k[j] == t.thr);
+    n_gt += __popc(gtm[j]);
+    n_eq += __popc(eqm[j]);
+  }
+  // ties before this warp -> this warp's share of the need_eq lowest-index ties
+  if (lane == 0) sh.red[0][warp] = n_eq;
+  __syncthreads();
+  uint32_t eq_before = 0u;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) eq_before += w < warp ? sh.red[0][w] : 0u;
+  const uint32_t take = t.need_eq > eq_before ? min(t.need_eq - eq_before, n_eq) : 0u;
+  if (lane == 0) sh.red[1][warp] = n_gt + take;
+  __syncthreads();
+  uint32_t pos = 0u, total = 0u;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    const uint32_t v = sh.red[1][w];
+    pos += w < warp ? v : 0u;
+    total += v;
+  }
+  uint32_t eq_run = 0u;
+#pragma unroll
+  for (int j = 0; j < R; ++j) {
+    // ties of this stripe with warp-local rank < take are selected
+    uint32_t tk = 0u;
+    if (eqm[j]) {
+      const uint32_t rank = eq_run + __popc(eqm[j] & lt);
+      tk = __ballot_sync(0xffffffffu, ((eqm[j] >> lane) & 1u) && rank < take);
+    }
+    const uint32_t sel = gtm[j] | tk;
+    if ((sel >> lane) & 1u) emit(pos + __popc(sel & lt), j);
+    pos += __popc(sel);
+    eq_run += __popc(eqm[j]);
+  }
+  __syncthreads();   // sh.red is reused by the next call
+  return total;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelectArgs a) {
+  const int C = gridDim.x;
+  const int c = blockIdx.x;
+  const int r = blockIdx.y;
+  const int tid = threadIdx.x;
+  __shared__ Shared sh;
+  extern __shared__ uint32_t dyn[];   // keys (local phase) / keys + slots (final phase)
+
+  const Plan pl = make_plan(a, r);
+  int* out = a.out + static_cast<long long>(r) * a.out_len;
+  if (!pl.valid) {
+    if (c == 0)
+      for (int i = tid; i < a.out_len; i += kThreads) out[i] = -1;
+    return;   // every CTA of the row takes this branch; the arrival counter is untouched
+  }
+
+  // ---------------------------------------------------------- local phase --
+  const int len = pl.dyn_hi - pl.dyn_lo;
+  const int seg = (len + C - 1) / C;
+  int my_lo = pl.dyn_lo + c * seg;
+  if (my_lo > pl.dyn_hi) my_lo = pl.dyn_hi;
+  const int my_n = min(pl.dyn_hi, my_lo + seg) - my_lo;
+  const float* row = a.scores + static_cast<long long>(r) * a.row_stride + my_lo;
+  const long long cbase = (static_cast<long long>(r) * C + c) * a.cand_cap;
+  uint32_t* ck = a.cand_keys + cbase;
+  int* cs = a.cand_slots + cbase;
+  uint32_t n_loc = 0u;
+  if (my_n <= kThreads * kRL) {
+    uint32_t k[kRL];
+    const int i0 = (tid >> 5) * 32 * kRL + (tid & 31);   // element of k[j]: i0 + 32 * j
+    float v[kRL];
+#pragma unroll
+    for (int j = 0; j < kRL; ++j) v[j] = i0 + 32 * j < my_n ? __ldg(row + i0 + 32 * j) : -INFINITY;
+#pragma unroll
+    for (int j = 0; j < kRL; ++j) k[j] = score_key(v[j]);
+    const Thr tl = reg_threshold<kRL>(k, static_cast<uint32_t>(pl.D), sh);
+    n_loc = reg_emit<kRL>(k, tl, sh, [&](uint32_t p, int j) {
+      ck[p] = k[j];
+      cs[p] = my_lo + i0 + 32 * j;
+    });
+  } else {
+    uint32_t* keys = dyn;
+    for (int i0 = 0; i0 < my_n; i0 += kThreads * 8) {
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * kThreads + tid;
+        v[u] = i < my_n ? __ldg(row + i) : -INFINITY;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * kThreads + tid;
+        if (i < my_n) keys[i] = score_key(v[u]);
+      }
+    }
+    __syncthreads();
+    const Thr tl = cta_threshold(keys, my_n, static_cast<uint32_t>(pl.D), sh);
+    n_loc = cta_emit(keys, my_n, tl, sh, [&](uint32_t p, int i) {
+      ck[p] = keys[i];
+      cs[p] = my_lo + i;
+    });
+  }
+  for (int i = static_cast<int>(n_loc) + tid; i < a.cand_cap; i += kThreads) ck[i] = 0u;   // unused: no candidate
+
+  // ------------------------------------------------- last CTA of the row --
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) sh.last = atomicAdd(a.row_arrivals + r, 1u) == static_cast<unsigned>(C - 1);
+  __syncthreads();
+  if (!sh.last) return;
+  __threadfence();
+
+  const int n_all = C * a.cand_cap;
+  const uint32_t* gk = a.cand_keys + static_cast<long long>(r) * n_all;
+  const int* gs = a.cand_slots + static_cast<long long>(r) * n_all;
+  int* dyn_out = out + pl.dyn_off;
+  const int M = a.M, P = a.P;
+  const long long prow = static_cast<long long>(r) * M;
+  auto token = [&](int slot) {
+    return a.mode == kSelectHierTokens ? __ldg(a.pages + prow + slot / P) * P + slot % P : slot;
+  };
+  uint32_t n_sel = 0u;
+  if (n_all <= kThreads * kRF) {
+    uint32_t k[kRF];
+    int sl[kRF];
+    const int i0 = (tid >> 5) * 32 * kRF + (tid & 31);   // element of k[j]: i0 + 32 * j
+#pragma unroll
+    for (int j = 0; j < kRF; ++j) {
+      const bool ok = i0 + 32 * j < n_all;
+      k[j] = ok ? __ldcg(gk + i0 + 32 * j) : 0u;
+      sl[j] = ok ? __ldcg(gs + i0 + 32 * j) : 0;
+    }
+    const Thr tf = reg_threshold<kRF>(k, static_cast<uint32_t>(pl.D), sh);
+    n_sel = reg_emit<kRF>(k, tf, sh, [&](uint32_t p, int j) { dyn_out[p] = token(sl[j]); });
+  } else {
+    const Thr tf = cta_threshold(gk, n_all, static_cast<uint32_t>(pl.D), sh);
+    n_sel = cta_emit(gk, n_all, tf, sh, [&](uint32_t p, int i) { dyn_out[p] = token(__ldcg(gs + i)); });
+  }
+  for (int i = tid; i < pl.lead_a_n; i += kThreads) out[i] = pl.lead_a_lo + i;
+  for (int i = tid; i < pl.lead_b_n; i += kThreads) out[pl.lead_a_n + i] = pl.lead_b_lo + i;
+  const int tr0 = pl.dyn_off + static_cast<int>(n_sel);
+  for (int i = tid; i < pl.trail_n; i += kThreads) out[tr0 + i] = pl.trail_lo + i;
+  for (int i = tr0 + pl.trail_n + tid; i < a.out_len; i += kThreads) out[i] = -1;
+  if (tid == 0) a.row_arrivals[r] = 0u;   // ready for the next call on this workspace
+}
+
+
+// ---------------------------------------------------------------------------
+// Grid-cooperative variant (all CTAs of the launch co-resident, one CTA per SM).
+// The CTAs of a row hold their segment's keys in registers and cooperate
+// through a per-row block in the workspace: a CTA arrives on a counter, the
+// last to arrive does the row-wide step and releases the others through a flag
+// (bounded spin). Steps:
+//   S0  row max key (atomicMax).
+//   A   histogram of d = (max - key) >> 13 over 2048 bins, i.e. the two
+//       binades of key space below the max; scores of one row sit close
+//       together, so the D-th best is almost always inside. S1: the last CTA
+//       finds the bin b1 holding the D-th best and the count above it.
+//   B   each CTA lists its few keys in bin b1. S2: the last CTA resolves the
+//       exact D-th key from the lists and gives every CTA its output offset and
+//       its share of the ties (lowest index first).
+// If fewer than D candidates fall in the window, or a list overflows, the row
+// switches (uniformly) to three exact radix rounds over the full key (11/11/10
+// bits) with the same arrive/release steps. Every CTA then writes its own
+// selections in index order.
+// ---------------------------------------------------------------------------
+
+constexpr int kSubHist = 4;       // round-A sub-histograms (warp w uses w % 4)
+constexpr int kWHStride = 2052;   // sub-histogram stride (words), bank-staggered
+constexpr int kListCap = 256;     // round-B list capacity per CTA
+constexpr int kRangeShift = 13;   // round-A bin width: 2^13 key units (2048 bins = 2 binades)
+constexpr int kMaxGridC = 64;     // CTAs per row on the grid path
+
+enum : unsigned { kModeRange = 0u, kModeAll = 1u, kModeNone = 2u, kModeRadix = 3u };
+
+// Flags are 64-bit words released with their payload (bit 63 = released), so a
+// waiting CTA receives the row-wide result in the same load that releases it.
+constexpr unsigned long long kReleased = 1ull << 63;
+
+struct GridRow {                      // per row, zeroed before each launch
+  unsigned arrive[8];
+  unsigned maxkey, overflow;
+  unsigned long long flag[8];         // S0: max key; S1: mode/bin/need; radix rounds: bin/need
+  unsigned long long fl[kMaxGridC];   // per CTA: threshold | offset | ties taken
+  unsigned histA[2048];               // round A window histogram
+};
+
+// per-row, per-CTA arrays following the GridRow blocks (written before being read)
+struct GridCta {
+  unsigned* cnt;      // [C] candidates
+  unsigned* inr;      // [C] candidates inside the round-A window
+  unsigned* def;      // [C] keys above the bin / prefix (definitely selected)
+  unsigned* ln;       // [C] round-B list lengths
+  unsigned* lists;    // [C][kListCap] round-B (max - key) values
+  unsigned* h3;       // [C][1024] fallback round-3 histograms
+  unsigned* hist1;    // [2048] fallback round-1 histogram (zeroed when the fallback starts)
+  unsigned* hist2;    // [2048] fallback round-2 histogram
+};
+
+__host__ __device__ constexpr size_t grid_blocks_bytes(int rows) {
+  return (sizeof(GridRow) * static_cast<size_t>(rows) + 255) / 256 * 256;
+}
+__host__ __device__ constexpr size_t grid_row_bytes(int C) {
+  return (static_cast<size_t>(C) * (4 * 4 + kListCap * 4 + 1024 * 4) + 2 * 2048 * 4 + 255) / 256 * 256;
+}
+
+__device__ __forceinline__ GridCta grid_cta(uint8_t* base, int C) {
+  GridCta g;
+  g.cnt = reinterpret_cast<unsigned*>(base);
+  g.inr = g.cnt + C;
+  g.def = g.inr + C;
+  g.ln = g.def + C;
+  g.lists = g.ln + C;
+  g.h3 = g.lists + static_cast<size_t>(C) * kListCap;
+  g.hist1 = g.h3 + static_cast<size_t>(C) * 1024;
+  g.hist2 = g.hist1 + 2048;
+  return g;
+}
+
+__device__ __forceinline__ unsigned long long ld_acquire64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release64(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+struct GShared {
+  unsigned long long v64;
+  unsigned u[4];
+  int ok;
+};
+
+// True in every thread of the CTA that arrives last on `counter` (of `n`).
+__device__ __forceinline__ bool arrive_last(unsigned* counter, unsigned n, Shared& sh) {
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) sh.last = atomicAdd(counter, 1u) == n - 1u;
+  __syncthreads();
+  if (sh.last) __threadfence();
+  return sh.last != 0;
+}
+
+// Wait (bounded) for a released flag; every thread gets the payload. False on timeout.
+__device__ __forceinline__ bool wait64(const unsigned long long* flag, unsigned long long* val, int* status,
+                                       GShared& gs) {
+  if (threadIdx.x == 0) {
+    const unsigned long long t0 = globaltimer_ns();
+    unsigned long long v;
+    gs.ok = 1;
+    while (!((v = ld_acquire64(flag)) & kReleased)) {
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        record_timeout(status);
+        gs.ok = 0;
+        break;
+      }
+    }
+    gs.v64 = v;
+  }
+  __syncthreads();
+  *val = gs.v64;
+  const bool ok = gs.ok != 0;
+  __syncthreads();
+  return ok;
+}
+
+// Release a payload flag (after the CTA's published writes).
+__device__ __forceinline__ void release64(unsigned long long* flag, unsigned long long payload) {
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) st_release64(flag, kReleased | payload);
+}
+
+// Row-wide step: the last CTA runs `work` (returns the payload, uniform) and
+// releases; the others wait. Every thread gets the payload.
+template <class W>
+__device__ __forceinline__ bool row_step(unsigned* arrive, unsigned long long* flag, unsigned C, int* status,
+                                         Shared& sh, GShared& gs, unsigned long long* val, W&& work) {
+  if (arrive_last(arrive, C, sh)) {
+    const unsigned long long v = work();
+    release64(flag, v);
+    *val = kReleased | v;
+    return true;
+  }
+  return wait64(flag, val, status, gs);
+}
+
+__device__ __forceinline__ unsigned long long pack_cta(unsigned thr, unsigned offset, unsigned take, unsigned mode) {
+  return (static_cast<unsigned long long>(mode == kModeAll) << 62) |
+         (static_cast<unsigned long long>(mode == kModeNone) << 61) |
+         (static_cast<unsigned long long>(thr) << 28) | (static_cast<unsigned long long>(offset & 0x3FFFu) << 14) |
+         (take & 0x3FFFu);
+}
+
+// Bin where the running count over bins [0, nb) reaches `need`, scanning from
+// the top (descending keys) or from bin 0 (when bin 0 holds the largest keys).
+template <bool FROM_TOP, bool GLOBAL>
+__device__ __forceinline__ void find_bin(const unsigned* h, int nb, unsigned need, Shared& sh) {
+  const int tid = threadIdx.x;
+  const int per = nb / kThreads;
+  unsigned vals[16];
+  unsigned local = 0u;
+#pragma unroll
+  for (int q = 0; q < 16; ++q) {
+    if (q < per) {
+      const int bb = FROM_TOP ? nb - 1 - (per * tid + q) : per * tid + q;
+      vals[q] = GLOBAL ? __ldcg(h + bb) : h[bb];
+      local += vals[q];
+    }
+  }
+  const unsigned incl = block_incl_scan(local, sh.tmp, nullptr);
+  const unsigned excl = incl - local;
+  if (excl < need && need <= incl) {
+    unsigned above = excl;
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      if (q < per) {
+        if (above + vals[q] >= need) {
+          sh.bin = FROM_TOP ? nb - 1 - (per * tid + q) : per * tid + q;
+          sh.above = above;
+          break;
+        }
+        above += vals[q];
+      }
+    }
+  }
+  __syncthreads();
+}
+
+// Per-CTA offsets and tie shares from per-CTA (definite, tie) counts held by
+// threads cc < C; writes the packed per-CTA flags (released).
+__device__ __forceinline__ void publish_ctas(GridRow* G, unsigned C, unsigned def, unsigned eq, unsigned need_eq,
+                                             unsigned thr, unsigned mode, Shared& sh) {
+  const int tid = threadIdx.x;
+  const unsigned my_eq = tid < static_cast<int>(C) ? eq : 0u;
+  const unsigned eq_before = block_incl_scan(my_eq, sh.tmp, nullptr) - my_eq;
+  const unsigned tk = need_eq > eq_before ? min(need_eq - eq_before, my_eq) : 0u;
+  const unsigned n = tid < static_cast<int>(C) ? def + tk : 0u;
+  const unsigned off = block_incl_scan(n, sh.tmp, nullptr) - n;
+  __threadfence();
+  __syncthreads();
+  if (tid < static_cast<int>(C)) st_release64(&G->fl[tid], kReleased | pack_cta(thr, off, tk, mode));
+}
+
+__global__ void __launch_bounds__(kThreads, 1) select_grid_kernel(const SelectArgs a) {
+  const unsigned C = gridDim.x;
+  const int c = blockIdx.x;
+  const int r = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  __shared__ Shared sh;
+  __shared__ GShared gs;
+  __shared__ unsigned s_cnt;
+  extern __shared__ uint32_t sub[];   // [kSubHist][kWHStride] round-A histograms
+
+  const Plan pl = make_plan(a, r);
+  int* out = a.out + static_cast<long long>(r) * a.out_len;
+  if (!pl.valid) {
+    if (c == 0)
+      for (int i = tid; i < a.out_len; i += kThreads) out[i] = -1;
+    return;   // every CTA of the row returns; the row's block is untouched
+  }
+  GridRow* G = reinterpret_cast<GridRow*>(a.grid_ws) + r;
+  const GridCta X = grid_cta(reinterpret_cast<uint8_t*>(a.grid_ws) + grid_blocks_bytes(a.B * a.T) +
+                                 static_cast<size_t>(r) * a.grid_row_bytes, C);
+  const unsigned D = static_cast<unsigned>(pl.D);
+
+  // keys of this CTA's segment, warp-striped in registers
+  const int len = pl.dyn_hi - pl.dyn_lo;
+  const int seg = (len + static_cast<int>(C) - 1) / static_cast<int>(C);
+  int my_lo = pl.dyn_lo + c * seg;
+  if (my_lo > pl.dyn_hi) my_lo = pl.dyn_hi;
+  const int my_n = min(pl.dyn_hi, my_lo + seg) - my_lo;
+  const float* row = a.scores + static_cast<long long>(r) * a.row_stride + my_lo;
+  const int i0 = warp * 32 * kRL + lane;
+  uint32_t k[kRL];
+  {
+    float v[kRL];
+#pragma unroll
+    for (int j = 0; j < kRL; ++j) v[j] = i0 + 32 * j < my_n ? __ldg(row + i0 + 32 * j) : -INFINITY;
+#pragma unroll
+    for (int j = 0; j < kRL; ++j) k[j] = score_key(v[j]);
+  }
+  unsigned long long fv = 0ull;
+
+  // ---- S0: row max key and candidate counts ----
+  {
+    uint32_t nz = 0u, mx = 0u;
+#pragma unroll
+    for (int j = 0; j < kRL; ++j)
+      if (k[j] != 0u) {
+        ++nz;
+        mx = max(mx, k[j]);
+      }
+    block_cnt_min_max(nz, 0xFFFFFFFFu, mx, sh);
+    if (tid == 0) {
+      X.cnt[c] = sh.cnt;
+      if (sh.cnt) atomicMax(&G->maxkey, sh.mx);
+    }
+    uint4* z = reinterpret_cast<uint4*>(sub);
+    for (int i = tid; i < kSubHist * kWHStride / 4; i += kThreads) z[i] = make_uint4(0u, 0u, 0u, 0u);
+  }
+  if (!row_step(&G->arrive[0], &G->flag[0], C, a.status, sh, gs, &fv, [&] {
+        return static_cast<unsigned long long>(__ldcg(&G->maxkey));
+      }))
+    return;
+  const uint32_t kmax = static_cast<uint32_t>(fv);
+
+  // ---- round A: window histogram ----
+  {
+    uint32_t* h = sub + (warp % kSubHist) * kWHStride;
+    uint32_t nin = 0u;
+#pragma unroll
+    for (int j = 0; j < kRL; ++j) {
+      if (k[j] == 0u) continue;
+      const uint32_t d = (kmax - k[j]) >> kRangeShift;
+      if (d < 2048u) {
+        ++nin;
+        atomicAdd(&h[d], 1u);
+      }
+    }
+    uint32_t my_in = 0u;
+    block_incl_scan(nin, sh.tmp, &my_in);   // barrier: sub-histograms complete
+    for (int bin = tid; bin < 2048; bin += kThreads) {
+      unsigned sum = 0u;
+#pragma unroll
+      for (int w = 0; w < kSubHist; ++w) sum += sub[w * kWHStride + bin];
+      if (sum) atomicAdd(&G->histA[bin], sum);
+    }
+    if (tid == 0) X.inr[c] = my_in;
+  }
+  if (!row_step(&G->arrive[1], &G->flag[1], C, a.status, sh, gs, &fv, [&]() -> unsigned long long {
+        const unsigned cn = tid < static_cast<int>(C) ? __ldcg(X.cnt + tid) : 0u;
+        const unsigned ci = tid < static_cast<int>(C) ? __ldcg(X.inr + tid) : 0u;
+        unsigned total = 0u, total_in = 0u;
+        block_incl_scan(cn, sh.tmp, &total);
+        block_incl_scan(ci, sh.tmp, &total_in);
+        if (total <= D || D == 0u) {
+          const unsigned mode = D == 0u ? kModeNone : kModeAll;
+          publish_ctas(G, C, D == 0u ? 0u : cn, 0u, 0u, 0u, mode, sh);
+          return static_cast<unsigned long long>(mode) << 48;
+        }
+        if (total_in < D) {
+          for (int i = tid; i < 4096; i += kThreads) X.hist1[i] = 0u;   // hist1 and hist2
+          return static_cast<unsigned long long>(kModeRadix) << 48;
+        }
+        find_bin<false, true>(G->histA, 2048, D, sh);
+        return (static_cast<unsigned long long>(kModeRange) << 48) |
+               (static_cast<unsigned long long>(sh.bin) << 16) | (D - sh.above);
+      }))
+    return;
+  unsigned mode = static_cast<unsigned>(fv >> 48) & 3u;
+
+  if (mode == kModeRange) {
+    // ---- round B: list this CTA's keys in bin b1 ----
+    const unsigned b1 = static_cast<unsigned>(fv >> 16) & 0xFFFFu, need1 = static_cast<unsigned>(fv & 0xFFFFu);
+    if (tid == 0) s_cnt = 0u;
+    __syncthreads();
+    unsigned* lst = X.lists + static_cast<size_t>(c) * kListCap;
+    uint32_t nd = 0u;
+#pragma unroll
+    for (int j = 0; j < kRL; ++j) {
+      if (k[j] == 0u) continue;
+      const uint32_t rel = kmax - k[j];
+      const uint32_t d = rel >> kRangeShift;
+      if (d < b1) {
+        ++nd;
+      } else if (d == b1) {
+        const unsigned p = atomicAdd(&s_cnt, 1u);
+        if (p < kListCap) lst[p] = rel;
+      }
+    }
+    uint32_t my_def = 0u;
+    block_incl_scan(nd, sh.tmp, &my_def);
+    if (tid == 0) {
+      X.def[c] = my_def;
+      X.ln[c] = s_cnt;
+      if (s_cnt > kListCap) atomicOr(&G->overflow, 1u);
+    }
+    if (arrive_last(&G->arrive[2], C, sh)) {
+      if (__ldcg(&G->overflow)) {
+        for (int i = tid; i < 4096; i += kThreads) X.hist1[i] = 0u;
+        release64(&G->flag[2], static_cast<unsigned long long>(kModeRadix) << 48);
+      } else {
+        // exact D-th key: histogram of the listed keys' low 13 bits of (max - key)
+        for (int i = tid; i < (1 << kRangeShift); i += kThreads) sh.hist[i] = 0u;
+        __syncthreads();
+        for (unsigned cc = warp; cc < C; cc += kWarps) {
+          const unsigned n = __ldcg(X.ln + cc);
+          for (unsigned i = lane; i < n; i += 32)
+            atomicAdd(&sh.hist[__ldcg(X.lists + cc * kListCap + i) & ((1u << kRangeShift) - 1u)], 1u);
+        }
+        __syncthreads();
+        find_bin<false, false>(sh.hist, 1 << kRangeShift, need1, sh);
+        const unsigned thr_rel = (b1 << kRangeShift) | static_cast<unsigned>(sh.bin);
+        const unsigned need_eq = need1 - sh.above;
+        // per CTA: keys strictly above the threshold and ties equal to it
+        for (unsigned cc = warp; cc < C; cc += kWarps) {
+          const unsigned n = __ldcg(X.ln + cc);
+          unsigned lo = 0u, eq = 0u;
+          for (unsigned i = lane; i < n; i += 32) {
+            const unsigned rel = __ldcg(X.lists + cc * kListCap + i);
+            lo += rel < thr_rel ? 1u : 0u;
+            eq += rel == thr_rel ? 1u : 0u;
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) {
+            lo += __shfl_xor_sync(0xffffffffu, lo, o);
+            eq += __shfl_xor_sync(0xffffffffu, eq, o);
+          }
+          if (lane == 0) {
+            sh.hist[8192 - 1 - 2 * cc] = lo;
+            sh.hist[8192 - 2 - 2 * cc] = eq;
+          }
+        }
+        __syncthreads();
+        const unsigned def = tid < static_cast<int>(C) ? __ldcg(X.def + tid) + sh.hist[8192 - 1 - 2 * tid] : 0u;
+        const unsigned eq = tid < static_cast<int>(C) ? sh.hist[8192 - 2 - 2 * tid] : 0u;
+        publish_ctas(G, C, def, eq, need_eq, kmax - thr_rel, kModeRange, sh);
+        release64(&G->flag[2], static_cast<unsigned long long>(kModeRange) << 48);
+      }
+    }
+    if (!wait64(&G->flag[2], &fv, a.status, gs)) return;
+    mode = static_cast<unsigned>(fv >> 48) & 3u;
+  }
+
+  if (mode == kModeRadix) {
+    // ---- fallback: three exact radix rounds over the full key ----
+    for (int i = tid; i < 2048; i += kThreads) sh.hist[i] = 0u;
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kRL; ++j)
+      if (k[j] != 0u) atomicAdd(&sh.hist[k[j] >> 21], 1u);
+    __syncthreads();
+    for (int bin = tid; bin < 2048; bin += kThreads)
+      if (sh.hist[bin]) atomicAdd(&X.hist1[bin], sh.hist[bin]);
+    if (!row_step(&G->arrive[3], &G->flag[3], C, a.status, sh, gs, &fv, [&] {
+          find_bin<true, true>(X.hist1, 2048, D, sh);
+          return (static_cast<unsigned long long>(sh.bin) << 16) | (D - sh.above);
+        }))
+      return;
+    const unsigned b1 = static_cast<unsigned>(fv >> 16) & 0xFFFFu, need1 = static_cast<unsigned>(fv & 0xFFFFu);
+    for (int i = tid; i < 2048; i += kThreads) sh.hist[i] = 0u;
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kRL; ++j)
+      if (k[j] != 0u && (k[j] >> 21) == b1) atomicAdd(&sh.hist[(k[j] >> 10) & 2047u], 1u);
+    __syncthreads();
+    for (int bin = tid; bin < 2048; bin += kThreads)
+      if (sh.hist[bin]) atomicAdd(&X.hist2[bin], sh.hist[bin]);
+    if (!row_step(&G->arrive[4], &G->flag[4], C, a.status, sh, gs, &fv, [&] {
+          find_bin<true, true>(X.hist2, 2048, need1, sh);
+          return (static_cast<unsigned long long>(sh.bin) << 16) | (need1 - sh.above);
+        }))
+      return;
+    const unsigned p22 = (b1 << 11) | (static_cast<unsigned>(fv >> 16) & 0xFFFFu);
+    const unsigned need2 = static_cast<unsigned>(fv & 0xFFFFu);
+    unsigned* h3 = X.h3 + static_cast<size_t>(c) * 1024;
+    for (int i = tid; i < 1024; i += kThreads) sh.hist[i] = 0u;
+    __syncthreads();
+    uint32_t ngt = 0u;
+#pragma unroll
+    for (int j = 0; j < kRL; ++j) {
+      if (k[j] == 0u) continue;
+      const uint32_t hi22 = k[j] >> 10;
+      if (hi22 > p22) ++ngt;
+      else if (hi22 == p22) atomicAdd(&sh.hist[k[j] & 1023u], 1u);
+    }
+    uint32_t my_gt = 0u;
+    block_incl_scan(ngt, sh.tmp, &my_gt);
+    for (int i = tid; i < 1024; i += kThreads) h3[i] = sh.hist[i];
+    if (tid == 0) X.def[c] = my_gt;
+    if (arrive_last(&G->arrive[5], C, sh)) {
+      for (int i = tid; i < 1024; i += kThreads) {
+        unsigned sum = 0u;
+#pragma unroll 8
+        for (unsigned cc = 0; cc < C; ++cc) sum += __ldcg(X.h3 + cc * 1024 + i);
+        sh.hist[i] = sum;
+      }
+      __syncthreads();
+      find_bin<true, false>(sh.hist, 1024, need2, sh);
+      const unsigned b3 = static_cast<unsigned>(sh.bin);
+      const unsigned need_eq = need2 - sh.above;
+      for (unsigned cc = warp; cc < C; cc += kWarps) {
+        unsigned above = 0u;
+        for (int i = lane; i < 1024; i += 32)
+          if (static_cast<unsigned>(i) > b3) above += __ldcg(X.h3 + cc * 1024 + i);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) above += __shfl_xor_sync(0xffffffffu, above, o);
+        if (lane == 0) {
+          sh.hist[2048 + 2 * cc] = above + __ldcg(X.def + cc);
+          sh.hist[2048 + 2 * cc + 1] = __ldcg(X.h3 + cc * 1024 + b3);
+        }
+      }
+      __syncthreads();
+      const unsigned def = tid < static_cast<int>(C) ? sh.hist[2048 + 2 * tid] : 0u;
+      const unsigned eq = tid < static_cast<int>(C) ? sh.hist[2048 + 2 * tid + 1] : 0u;
+      publish_ctas(G, C, def, eq, need_eq, (p22 << 10) | b3, kModeRange, sh);
+    }
+    mode = kModeRange;
+  }
+
+  // ---- emit this CTA's selections in index order ----
+  if (!wait64(&G->fl[c], &fv, a.status, gs)) return;
+  Thr t{0u, 0u, false};
+  if ((fv >> 62) & 1ull) {
+    t.all = true;
+  } else if ((fv >> 61) & 1ull) {
+    t.thr = 0xFFFFFFFFu;   // nothing is taken
+  } else {
+    t.thr = static_cast<unsigned>(fv >> 28);
+  }
+  t.need_eq = static_cast<unsigned>(fv & 0x3FFFu);
+  const int base = static_cast<int>((fv >> 14) & 0x3FFFu);
+  int* dyn_out = out + pl.dyn_off + base;
+  const long long prow = static_cast<long long>(r) * a.M;
+  const uint32_t n_mine = reg_emit<kRL>(k, t, sh, [&](uint32_t p, int j) {
+    const int slot = my_lo + i0 + 32 * j;
+    dyn_out[p] = a.mode == kSelectHierTokens ? __ldg(a.pages + prow + slot / a.P) * a.P + slot % a.P : slot;
+  });
+  if (c == static_cast<int>(C) - 1) {
+    // the last segment ends the dynamic block: its end is the selected count
+    const int n_sel = base + static_cast<int>(n_mine);
+    for (int i = tid; i < pl.lead_a_n; i += kThreads) out[i] = pl.lead_a_lo + i;
+    for (int i = tid; i < pl.lead_b_n; i += kThreads) out[pl.lead_a_n + i] = pl.lead_b_lo + i;
+    const int tr0 = pl.dyn_off + n_sel;
+    for (int i = tid; i < pl.trail_n; i += kThreads) out[tr0 + i] = pl.trail_lo + i;
+    for (int i = tr0 + pl.trail_n + tid; i < a.out_len; i += kThreads) out[i] = -1;
+  }
 }
 
 }  // namespace
 
-int select_cluster_size(int rows, int max_dyn, int num_sms, int* cap) {
-  const int kCapMax = 40960;   // keys cached per CTA (160 KB)
-  int C = 1;
-  while (C < 8 && rows * C * 2 <= num_sms) C *= 2;
-  while (C < 8 && (max_dyn + C - 1) / C > kCapMax) C *= 2;
-  const int seg = (max_dyn + C - 1) / C;
-  *cap = seg <= kCapMax ? seg : 0;
-  return C;
+SelectPlan select_plan(int rows, int n_slots, int d_bound, int num_sms) {
+  const int kLocalRegs = kThreads * kRL;    // segment that fits the register path
+  const int kMergeRegs = kThreads * kRF;    // merged candidates that fit the register path
+  constexpr int kSegMax = 32768;            // fallback: keys per CTA in shared memory
+  SelectPlan p{};
+  auto seg_of = [&](int C) { return (n_slots + C - 1) / C; };
+  // grid-cooperative path: register-sized segments, one CTA per SM, all co-resident
+  const int Cg = std::max(1, (n_slots + kLocalRegs - 1) / kLocalRegs);
+  int Cgrid = Cg;
+  while (rows * Cgrid * 2 <= num_sms && seg_of(Cgrid * 2) >= 1024) Cgrid *= 2;   // more CTAs for latency
+  if (rows * Cgrid <= num_sms && Cgrid <= kMaxGridC) {
+    p.grid = true;
+    p.C = Cgrid;
+    p.seg = seg_of(Cgrid);
+    p.cand_cap = 0;
+    return p;
+  }
+  // few rows: ~2K keys per CTA for latency; rows alone fill the GPU: register-sized segments
+  int C = rows >= num_sms ? std::max(1, (n_slots + kLocalRegs - 1) / kLocalRegs)
+                          : std::max(1, std::min(64, (n_slots + 2047) / 2048));
+  while (seg_of(C) > kLocalRegs && C < 1024) C *= 2;                   // local keys in registers
+  while (C > 1 && C * std::min(d_bound, seg_of(C)) > kMergeRegs && seg_of(C / 2) <= kLocalRegs) C /= 2;
+  while (seg_of(C) > kSegMax) C *= 2;
+  p.C = C;
+  p.seg = seg_of(C);
+  p.cand_cap = std::max(1, std::min(d_bound, p.seg));
+  p.final_in_smem = false;
+  return p;
 }
 
-cudaError_t launch_select(const SelectArgs& a, int C, cudaStream_t stream) {
-  const bool in_smem = a.cap > 0;
-  const void* fn = in_smem ? reinterpret_cast<const void*>(&select_kernel<true>)
-                           : reinterpret_cast<const void*>(&select_kernel<false>);
-  const size_t smem = (3 * kBins + 64) * sizeof(uint32_t) + static_cast<size_t>(a.cap) * sizeof(uint32_t);
-  cudaError_t e = set_max_smem(fn, smem);
-  if (e != cudaSuccess) return e;
+size_t select_ws_bytes(int rows, const SelectPlan& p) {
+  if (p.grid) return grid_blocks_bytes(rows) + grid_row_bytes(p.C) * rows;
+  const size_t n = static_cast<size_t>(rows) * p.C * p.cand_cap;
+  return ((n * 8 + rows * 4 + 255) / 256) * 256;
+}
+
+cudaError_t launch_select(const SelectArgs& a0, const SelectPlan& p, void* ws, cudaStream_t stream) {
+  SelectArgs a = a0;
   const int rows = a.B * a.T;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(C, rows, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = C;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  void* args[] = {const_cast<SelectArgs*>(&a)};
-  return cudaLaunchKernelExC(&cfg, fn, args);
+  if (p.grid) {
+    a.grid_ws = ws;
+    a.grid_row_bytes = grid_row_bytes(p.C);
+    // reset the rows' coordination blocks (counters, flags, window histograms)
+    cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(GridRow) * static_cast<size_t>(rows), stream);
+    if (e != cudaSuccess) return e;
+    const size_t smem = static_cast<size_t>(kSubHist) * kWHStride * 4;
+    const void* fn = reinterpret_cast<const void*>(&select_grid_kernel);
+    e = set_max_smem(fn, smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.C, rows, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;   // all CTAs co-resident: rows wait on each other
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    void* args[] = {&a};
+    return cudaLaunchKernelExC(&cfg, fn, args);
+  }
+  const size_t n = static_cast<size_t>(rows) * p.C * p.cand_cap;
+  a.cand_cap = p.cand_cap;
+  a.final_in_smem = p.final_in_smem ? 1 : 0;
+  a.cand_keys = static_cast<uint32_t*>(ws);
+  a.cand_slots = reinterpret_cast<int*>(a.cand_keys + n);
+  a.row_arrivals = reinterpret_cast<unsigned*>(a.cand_slots + n);
+  cudaError_t e = cudaMemsetAsync(a.row_arrivals, 0, rows * sizeof(unsigned), stream);
+  if (e != cudaSuccess) return e;
+  const size_t smem = p.seg > kThreads * kRL ? static_cast<size_t>(p.seg) * 4 : 0;   // fallback keys
+  const void* fn = reinterpret_cast<const void*>(&select_kernel);
+  e = set_max_smem(fn, smem);
+  if (e != cudaSuccess) return e;
+  void* args[] = {&a};
+  return cudaLaunchKernel(fn, dim3(p.C, rows), dim3(kThreads), args, smem, stream);
 }
 
 }  // namespace lsa

@@ -1,9 +1,10 @@
 """ctypes binding of the LSA C ABI (include/lsa.h).
 
 Argument marshalling only: every step of the path runs in the CUDA kernels of
-liblsa.so. The functions carry the C names and take torch CUDA tensors (or raw
-pointers through the ``*_raw`` forms). There is no CPU fallback: if the library
-is missing or a call fails, an exception is raised.
+liblsa.so. The functions carry the C names and take torch CUDA tensors; outputs
+and workspaces are allocated with torch when the caller does not pass them.
+There is no CPU fallback: if the library is missing or a call fails, an
+exception is raised.
 """
 from __future__ import annotations
 
@@ -227,7 +228,7 @@ def lsa_index_flat(q, w, k, seq_len, budget, *, q_scale=None, k_scale=None, idx=
     return idx if with_idx else None
 
 
-def lsa_select_streaming(scores, seq_len, budget, *, idx=None, stream=None):
+def lsa_select_streaming(scores, seq_len, budget, *, idx=None, workspace=None, stream=None):
     """Streaming selection over given fp32 scores [B,T,L_max]. Returns idx [B,T,k]."""
     torch = _torch()
     lib = load()
@@ -236,8 +237,10 @@ def lsa_select_streaming(scores, seq_len, budget, *, idx=None, stream=None):
     B, T, L_max = scores.shape
     if idx is None:
         idx = torch.empty((B, T, budget[0]), dtype=torch.int32, device=scores.device)
-    _check(lib.lsa_select_streaming(_ptr(scores), _ptr(seq_len), B, T, L_max, Budget(*budget), _ptr(idx), None, 0,
-                                    _stream(stream)))
+    need = workspace_size(LSA_OP_SELECT, budget=budget, B=B, T=T, L_max=L_max)
+    ws = _workspace(need, scores.device, workspace)
+    _check(lib.lsa_select_streaming(_ptr(scores), _ptr(seq_len), B, T, L_max, Budget(*budget), _ptr(idx), _ptr(ws),
+                                    _nbytes(ws), _stream(stream)))
     return idx
 
 
