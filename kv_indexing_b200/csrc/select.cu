@@ -107,7 +107,7 @@ __device__ __forceinline__ Plan make_plan(const SelectArgs& a, int r) {
 }
 
 // Inclusive scan of one value per thread (thread order). Uses `tmp` [kWarps].
-__device__ __forceinline__ uint32_t block_incl_scan(uint32_t v, uint32_t* tmp, uint32_t* total) {
+__device__ __noinline__ uint32_t block_incl_scan(uint32_t v, uint32_t* tmp, uint32_t* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t x = v;
 #pragma unroll
@@ -150,7 +150,7 @@ struct Shared {
 };
 
 // Block-wide count / min / max of per-thread partials (into sh.cnt, sh.mn, sh.mx).
-__device__ __forceinline__ void block_cnt_min_max(uint32_t c, uint32_t mn, uint32_t mx, Shared& sh) {
+__device__ __noinline__ void block_cnt_min_max(uint32_t c, uint32_t mn, uint32_t mx, Shared& sh) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -621,7 +621,7 @@ struct GShared {
 };
 
 // True in every thread of the CTA that arrives last on `counter` (of `n`).
-__device__ __forceinline__ bool arrive_last(unsigned* counter, unsigned n, Shared& sh) {
+__device__ __noinline__ bool arrive_last(unsigned* counter, unsigned n, Shared& sh) {
   __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) sh.last = atomicAdd(counter, 1u) == n - 1u;
@@ -631,8 +631,8 @@ __device__ __forceinline__ bool arrive_last(unsigned* counter, unsigned n, Share
 }
 
 // Wait (bounded) for a released flag; every thread gets the payload. False on timeout.
-__device__ __forceinline__ bool wait64(const unsigned long long* flag, unsigned long long* val, int* status,
-                                       GShared& gs) {
+__device__ __noinline__ bool wait64(const unsigned long long* flag, unsigned long long* val, int* status,
+                                    GShared& gs) {
   if (threadIdx.x == 0) {
     const unsigned long long t0 = globaltimer_ns();
     unsigned long long v;
@@ -684,7 +684,7 @@ __device__ __forceinline__ unsigned long long pack_cta(unsigned thr, unsigned of
 // Bin where the running count over bins [0, nb) reaches `need`, scanning from
 // the top (descending keys) or from bin 0 (when bin 0 holds the largest keys).
 template <bool FROM_TOP, bool GLOBAL>
-__device__ __forceinline__ void find_bin(const unsigned* h, int nb, unsigned need, Shared& sh) {
+__device__ __noinline__ void find_bin(const unsigned* h, int nb, unsigned need, Shared& sh) {
   const int tid = threadIdx.x;
   const int per = nb / kThreads;
   unsigned vals[16];
@@ -718,8 +718,8 @@ __device__ __forceinline__ void find_bin(const unsigned* h, int nb, unsigned nee
 
 // Per-CTA offsets and tie shares from per-CTA (definite, tie) counts held by
 // threads cc < C; writes the packed per-CTA flags (released).
-__device__ __forceinline__ void publish_ctas(GridRow* G, unsigned C, unsigned def, unsigned eq, unsigned need_eq,
-                                             unsigned thr, unsigned mode, Shared& sh) {
+__device__ __noinline__ void publish_ctas(GridRow* G, unsigned C, unsigned def, unsigned eq, unsigned need_eq,
+                                          unsigned thr, unsigned mode, Shared& sh) {
   const int tid = threadIdx.x;
   const unsigned my_eq = tid < static_cast<int>(C) ? eq : 0u;
   const unsigned eq_before = block_incl_scan(my_eq, sh.tmp, nullptr) - my_eq;
@@ -731,6 +731,51 @@ __device__ __forceinline__ void publish_ctas(GridRow* G, unsigned C, unsigned de
   if (tid < static_cast<int>(C)) st_release64(&G->fl[tid], kReleased | pack_cta(thr, off, tk, mode));
 }
 
+// Ordered emission of the selected keys of this CTA (keys in shared memory,
+// warp-striped: element w*32*kRL + 32*j + lane). Two rolled passes: per-warp
+// counts, then positions from per-stripe ballots.
+template <class F>
+__device__ __forceinline__ uint32_t smem_emit(const uint32_t* keys, const Thr& t, Shared& sh, F&& emit) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t lt = (1u << lane) - 1u;
+  const int base = warp * 32 * kRL + lane;
+  uint32_t n_gt = 0u, n_eq = 0u;
+#pragma unroll 4
+  for (int j = 0; j < kRL; ++j) {
+    const uint32_t k = keys[base + 32 * j];
+    n_gt += __popc(__ballot_sync(0xffffffffu, k != 0u && (t.all || k > t.thr)));
+    n_eq += __popc(__ballot_sync(0xffffffffu, k != 0u && !t.all && k == t.thr));
+  }
+  if (lane == 0) sh.red[0][warp] = n_eq;
+  __syncthreads();
+  uint32_t eq_before = 0u;
+  for (int w = 0; w < warp; ++w) eq_before += sh.red[0][w];
+  const uint32_t take = t.need_eq > eq_before ? min(t.need_eq - eq_before, n_eq) : 0u;
+  if (lane == 0) sh.red[1][warp] = n_gt + take;
+  __syncthreads();
+  uint32_t pos = 0u, total = 0u;
+  for (int w = 0; w < kWarps; ++w) {
+    const uint32_t v = sh.red[1][w];
+    pos += w < warp ? v : 0u;
+    total += v;
+  }
+  uint32_t eq_run = 0u;
+#pragma unroll 2
+  for (int j = 0; j < kRL; ++j) {
+    const uint32_t k = keys[base + 32 * j];
+    const uint32_t gtm = __ballot_sync(0xffffffffu, k != 0u && (t.all || k > t.thr));
+    const bool is_eq = k != 0u && !t.all && k == t.thr;
+    const uint32_t eqm = __ballot_sync(0xffffffffu, is_eq);
+    const uint32_t tk = __ballot_sync(0xffffffffu, is_eq && eq_run + __popc(eqm & lt) < take);
+    const uint32_t sel = gtm | tk;
+    if ((sel >> lane) & 1u) emit(pos + __popc(sel & lt), base + 32 * j);
+    pos += __popc(sel);
+    eq_run += __popc(eqm);
+  }
+  __syncthreads();   // sh.red is reused
+  return total;
+}
+
 __global__ void __launch_bounds__(kThreads, 1) select_grid_kernel(const SelectArgs a) {
   const unsigned C = gridDim.x;
   const int c = blockIdx.x;
@@ -739,7 +784,9 @@ __global__ void __launch_bounds__(kThreads, 1) select_grid_kernel(const SelectAr
   __shared__ Shared sh;
   __shared__ GShared gs;
   __shared__ unsigned s_cnt;
-  extern __shared__ uint32_t sub[];   // [kSubHist][kWHStride] round-A histograms
+  extern __shared__ uint32_t dsm[];
+  uint32_t* keys = dsm;                                  // [kThreads * kRL] warp-striped
+  uint32_t* sub = dsm + kThreads * kRL;                  // [kSubHist][kWHStride] round-A histograms
 
   const Plan pl = make_plan(a, r);
   int* out = a.out + static_cast<long long>(r) * a.out_len;
@@ -753,40 +800,34 @@ __global__ void __launch_bounds__(kThreads, 1) select_grid_kernel(const SelectAr
                                  static_cast<size_t>(r) * a.grid_row_bytes, C);
   const unsigned D = static_cast<unsigned>(pl.D);
 
-  // keys of this CTA's segment, warp-striped in registers
+  // keys of this CTA's segment (element e at keys[e], e < kThreads * kRL)
   const int len = pl.dyn_hi - pl.dyn_lo;
   const int seg = (len + static_cast<int>(C) - 1) / static_cast<int>(C);
   int my_lo = pl.dyn_lo + c * seg;
   if (my_lo > pl.dyn_hi) my_lo = pl.dyn_hi;
   const int my_n = min(pl.dyn_hi, my_lo + seg) - my_lo;
   const float* row = a.scores + static_cast<long long>(r) * a.row_stride + my_lo;
-  const int i0 = warp * 32 * kRL + lane;
-  uint32_t k[kRL];
+  const int base = warp * 32 * kRL + lane;   // this thread's elements: base + 32 * j
+  uint32_t nz = 0u, mx = 0u;
+#pragma unroll 8
+  for (int j = 0; j < kRL; ++j) {
+    const int e = base + 32 * j;
+    const uint32_t k = score_key(e < my_n ? __ldg(row + e) : -INFINITY);
+    keys[e] = k;
+    nz += k != 0u ? 1u : 0u;
+    mx = max(mx, k);
+  }
   {
-    float v[kRL];
-#pragma unroll
-    for (int j = 0; j < kRL; ++j) v[j] = i0 + 32 * j < my_n ? __ldg(row + i0 + 32 * j) : -INFINITY;
-#pragma unroll
-    for (int j = 0; j < kRL; ++j) k[j] = score_key(v[j]);
+    uint4* z = reinterpret_cast<uint4*>(sub);
+    for (int i = tid; i < kSubHist * kWHStride / 4; i += kThreads) z[i] = make_uint4(0u, 0u, 0u, 0u);
   }
   unsigned long long fv = 0ull;
 
   // ---- S0: row max key and candidate counts ----
-  {
-    uint32_t nz = 0u, mx = 0u;
-#pragma unroll
-    for (int j = 0; j < kRL; ++j)
-      if (k[j] != 0u) {
-        ++nz;
-        mx = max(mx, k[j]);
-      }
-    block_cnt_min_max(nz, 0xFFFFFFFFu, mx, sh);
-    if (tid == 0) {
-      X.cnt[c] = sh.cnt;
-      if (sh.cnt) atomicMax(&G->maxkey, sh.mx);
-    }
-    uint4* z = reinterpret_cast<uint4*>(sub);
-    for (int i = tid; i < kSubHist * kWHStride / 4; i += kThreads) z[i] = make_uint4(0u, 0u, 0u, 0u);
+  block_cnt_min_max(nz, 0xFFFFFFFFu, mx, sh);
+  if (tid == 0) {
+    X.cnt[c] = sh.cnt;
+    if (sh.cnt) atomicMax(&G->maxkey, sh.mx);
   }
   if (!row_step(&G->arrive[0], &G->flag[0], C, a.status, sh, gs, &fv, [&] {
         return static_cast<unsigned long long>(__ldcg(&G->maxkey));
@@ -798,11 +839,11 @@ __global__ void __launch_bounds__(kThreads, 1) select_grid_kernel(const SelectAr
   {
     uint32_t* h = sub + (warp % kSubHist) * kWHStride;
     uint32_t nin = 0u;
-#pragma unroll
+#pragma unroll 4
     for (int j = 0; j < kRL; ++j) {
-      if (k[j] == 0u) continue;
-      const uint32_t d = (kmax - k[j]) >> kRangeShift;
-      if (d < 2048u) {
+      const uint32_t k = keys[base + 32 * j];
+      const uint32_t d = (kmax - k) >> kRangeShift;
+      if (k != 0u && d < 2048u) {
         ++nin;
         atomicAdd(&h[d], 1u);
       }
@@ -810,9 +851,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_grid_kernel(const SelectAr
     uint32_t my_in = 0u;
     block_incl_scan(nin, sh.tmp, &my_in);   // barrier: sub-histograms complete
     for (int bin = tid; bin < 2048; bin += kThreads) {
-      unsigned sum = 0u;
-#pragma unroll
-      for (int w = 0; w < kSubHist; ++w) sum += sub[w * kWHStride + bin];
+      const unsigned sum = sub[bin] + sub[kWHStride + bin] + sub[2 * kWHStride + bin] + sub[3 * kWHStride + bin];
       if (sum) atomicAdd(&G->histA[bin], sum);
     }
     if (tid == 0) X.inr[c] = my_in;
@@ -846,14 +885,14 @@ __global__ void __launch_bounds__(kThreads, 1) select_grid_kernel(const SelectAr
     __syncthreads();
     unsigned* lst = X.lists + static_cast<size_t>(c) * kListCap;
     uint32_t nd = 0u;
-#pragma unroll
+#pragma unroll 4
     for (int j = 0; j < kRL; ++j) {
-      if (k[j] == 0u) continue;
-      const uint32_t rel = kmax - k[j];
+      const uint32_t k = keys[base + 32 * j];
+      const uint32_t rel = kmax - k;
       const uint32_t d = rel >> kRangeShift;
-      if (d < b1) {
+      if (k != 0u && d < b1) {
         ++nd;
-      } else if (d == b1) {
+      } else if (k != 0u && d == b1) {
         const unsigned p = atomicAdd(&s_cnt, 1u);
         if (p < kListCap) lst[p] = rel;
       }
@@ -916,9 +955,10 @@ __global__ void __launch_bounds__(kThreads, 1) select_grid_kernel(const SelectAr
     // ---- fallback: three exact radix rounds over the full key ----
     for (int i = tid; i < 2048; i += kThreads) sh.hist[i] = 0u;
     __syncthreads();
-#pragma unroll
-    for (int j = 0; j < kRL; ++j)
-      if (k[j] != 0u) atomicAdd(&sh.hist[k[j] >> 21], 1u);
+    for (int j = 0; j < kRL; ++j) {
+      const uint32_t k = keys[base + 32 * j];
+      if (k != 0u) atomicAdd(&sh.hist[k >> 21], 1u);
+    }
     __syncthreads();
     for (int bin = tid; bin < 2048; bin += kThreads)
       if (sh.hist[bin]) atomicAdd(&X.hist1[bin], sh.hist[bin]);
@@ -930,9 +970,10 @@ __global__ void __launch_bounds__(kThreads, 1) select_grid_kernel(const SelectAr
     const unsigned b1 = static_cast<unsigned>(fv >> 16) & 0xFFFFu, need1 = static_cast<unsigned>(fv & 0xFFFFu);
     for (int i = tid; i < 2048; i += kThreads) sh.hist[i] = 0u;
     __syncthreads();
-#pragma unroll
-    for (int j = 0; j < kRL; ++j)
-      if (k[j] != 0u && (k[j] >> 21) == b1) atomicAdd(&sh.hist[(k[j] >> 10) & 2047u], 1u);
+    for (int j = 0; j < kRL; ++j) {
+      const uint32_t k = keys[base + 32 * j];
+      if (k != 0u && (k >> 21) == b1) atomicAdd(&sh.hist[(k >> 10) & 2047u], 1u);
+    }
     __syncthreads();
     for (int bin = tid; bin < 2048; bin += kThreads)
       if (sh.hist[bin]) atomicAdd(&X.hist2[bin], sh.hist[bin]);
@@ -947,12 +988,12 @@ __global__ void __launch_bounds__(kThreads, 1) select_grid_kernel(const SelectAr
     for (int i = tid; i < 1024; i += kThreads) sh.hist[i] = 0u;
     __syncthreads();
     uint32_t ngt = 0u;
-#pragma unroll
     for (int j = 0; j < kRL; ++j) {
-      if (k[j] == 0u) continue;
-      const uint32_t hi22 = k[j] >> 10;
+      const uint32_t k = keys[base + 32 * j];
+      if (k == 0u) continue;
+      const uint32_t hi22 = k >> 10;
       if (hi22 > p22) ++ngt;
-      else if (hi22 == p22) atomicAdd(&sh.hist[k[j] & 1023u], 1u);
+      else if (hi22 == p22) atomicAdd(&sh.hist[k & 1023u], 1u);
     }
     uint32_t my_gt = 0u;
     block_incl_scan(ngt, sh.tmp, &my_gt);
@@ -961,7 +1002,6 @@ __global__ void __launch_bounds__(kThreads, 1) select_grid_kernel(const SelectAr
     if (arrive_last(&G->arrive[5], C, sh)) {
       for (int i = tid; i < 1024; i += kThreads) {
         unsigned sum = 0u;
-#pragma unroll 8
         for (unsigned cc = 0; cc < C; ++cc) sum += __ldcg(X.h3 + cc * 1024 + i);
         sh.hist[i] = sum;
       }
@@ -985,7 +1025,6 @@ __global__ void __launch_bounds__(kThreads, 1) select_grid_kernel(const SelectAr
       const unsigned eq = tid < static_cast<int>(C) ? sh.hist[2048 + 2 * tid + 1] : 0u;
       publish_ctas(G, C, def, eq, need_eq, (p22 << 10) | b3, kModeRange, sh);
     }
-    mode = kModeRange;
   }
 
   // ---- emit this CTA's selections in index order ----
@@ -999,16 +1038,17 @@ __global__ void __launch_bounds__(kThreads, 1) select_grid_kernel(const SelectAr
     t.thr = static_cast<unsigned>(fv >> 28);
   }
   t.need_eq = static_cast<unsigned>(fv & 0x3FFFu);
-  const int base = static_cast<int>((fv >> 14) & 0x3FFFu);
-  int* dyn_out = out + pl.dyn_off + base;
+  const int off = static_cast<int>((fv >> 14) & 0x3FFFu);
+  int* dyn_out = out + pl.dyn_off + off;
   const long long prow = static_cast<long long>(r) * a.M;
-  const uint32_t n_mine = reg_emit<kRL>(k, t, sh, [&](uint32_t p, int j) {
-    const int slot = my_lo + i0 + 32 * j;
-    dyn_out[p] = a.mode == kSelectHierTokens ? __ldg(a.pages + prow + slot / a.P) * a.P + slot % a.P : slot;
+  const bool hier = a.mode == kSelectHierTokens;
+  const uint32_t n_mine = smem_emit(keys, t, sh, [&](uint32_t p, int e) {
+    const int slot = my_lo + e;
+    dyn_out[p] = hier ? __ldg(a.pages + prow + slot / a.P) * a.P + slot % a.P : slot;
   });
   if (c == static_cast<int>(C) - 1) {
     // the last segment ends the dynamic block: its end is the selected count
-    const int n_sel = base + static_cast<int>(n_mine);
+    const int n_sel = off + static_cast<int>(n_mine);
     for (int i = tid; i < pl.lead_a_n; i += kThreads) out[i] = pl.lead_a_lo + i;
     for (int i = tid; i < pl.lead_b_n; i += kThreads) out[pl.lead_a_n + i] = pl.lead_b_lo + i;
     const int tr0 = pl.dyn_off + n_sel;
@@ -1064,7 +1104,7 @@ cudaError_t launch_select(const SelectArgs& a0, const SelectPlan& p, void* ws, c
     // reset the rows' coordination blocks (counters, flags, window histograms)
     cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(GridRow) * static_cast<size_t>(rows), stream);
     if (e != cudaSuccess) return e;
-    const size_t smem = static_cast<size_t>(kSubHist) * kWHStride * 4;
+    const size_t smem = (static_cast<size_t>(kThreads) * kRL + static_cast<size_t>(kSubHist) * kWHStride) * 4;
     const void* fn = reinterpret_cast<const void*>(&select_grid_kernel);
     e = set_max_smem(fn, smem);
     if (e != cudaSuccess) return e;
