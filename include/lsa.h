@@ -163,6 +163,33 @@ lsa_status_t lsa_select_streaming(const float* scores, const int32_t* seq_len, i
                                   int32_t T, int32_t L_max, lsa_budget_t budget, int32_t* idx,
                                   void* workspace, size_t workspace_bytes, lsa_stream_t stream);
 
+/* Size of the static device scratch used by lsa_select_streaming_noalloc:
+ * 16 MiB, held on every GPU that loads this library until the process exits. */
+#define LSA_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+
+/* lsa_select_streaming without a workspace: same arguments minus the
+ * workspace, same output, same contract. No counterpart in the paper; it is
+ * for callers that cannot allocate device memory where they select (a plugin
+ * in a serving engine whose memory is pre-reserved for its KV cache, or a
+ * latency-critical path that cannot afford cudaMalloc/cudaFree, which may
+ * block the host and synchronise the device). It allocates nothing: the
+ * selection's scratch is a fixed LSA_NOALLOC_SCRATCH_BYTES buffer compiled
+ * into the library.
+ *   - Shapes whose scratch (lsa_workspace_size with LSA_OP_SELECT) exceeds
+ *     LSA_NOALLOC_SCRATCH_BYTES are rejected with LSA_ERR_WORKSPACE before
+ *     anything is launched; with k=2048, sink+window=1024 that admits e.g.
+ *     B*T=8 rows up to L_max=1M, or 148 rows up to L_max=8K.
+ *   - The first call on a device looks up the buffer's device address (which
+ *     may load the library's device code onto that device); make that first
+ *     call, per device, before any stream capture begins.
+ *   - Every call on a device shares the buffer. Calls whose kernels may
+ *     overlap on the GPU (different streams without ordering) race on it and
+ *     give undefined results: order them on one stream. Each call clears on
+ *     `stream` the parts of the buffer that must start at zero. */
+lsa_status_t lsa_select_streaming_noalloc(const float* scores, const int32_t* seq_len, int32_t B,
+                                          int32_t T, int32_t L_max, lsa_budget_t budget,
+                                          int32_t* idx, lsa_stream_t stream);
+
 /* Page pooling for Hierarchical Indexing [LSA abstract (3); CARD "HI"]:
  *   page_keys[b,p,:] = bf16_rne( (sum_{j<P} k[b, pP+j, :]) / P )
  * summed in fp32 in ascending j, for every full page (pP + P <= seq_len[b]);

@@ -17,7 +17,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "liblsa.so")
-SOURCES = ["api.cu", "indexer.cu", "select.cu", "pool.cu", "attn.cu"]
+SOURCES = ["api.cu", "indexer.cu", "select.cu", "pool.cu", "attn.cu", "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

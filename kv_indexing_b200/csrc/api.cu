@@ -368,6 +368,14 @@ lsa_status_t check_hier_params(const lsa_indexer_in_t* in, int P, int M, lsa_bud
 
 }  // namespace
 
+lsa_status_t set_error(lsa_status_t st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
 int* device_status_ptr() {
   static int* cache[64] = {nullptr};
   int dev = 0;

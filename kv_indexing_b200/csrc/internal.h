@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "lsa.h"
+
 namespace lsa {
 
 // ----------------------------------------------------------------- indexer --
@@ -121,6 +123,8 @@ cudaError_t launch_attn_combine(const AttnArgs& a, cudaStream_t stream);
 
 // --------------------------------------------------------------------- misc --
 int device_sm_count();
+// Records a one-line reason for lsa_last_error() and returns `st`.
+lsa_status_t set_error(lsa_status_t st, const char* fmt, ...);
 int* device_status_ptr();
 cudaError_t set_max_smem(const void* func, size_t bytes);
 

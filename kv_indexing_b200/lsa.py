@@ -18,10 +18,12 @@ LIB_PATH = os.path.join(HERE, "liblsa.so")
 LSA_OK, LSA_ERR_INVALID_ARG, LSA_ERR_UNSUPPORTED, LSA_ERR_WORKSPACE, LSA_ERR_CUDA, LSA_ERR_TIMEOUT = range(6)
 LSA_BF16, LSA_E4M3 = 0, 1
 LSA_OP_INDEX_FLAT, LSA_OP_INDEX_HIER, LSA_OP_SELECT, LSA_OP_SPARSE_ATTN, LSA_OP_LAYER_GROUP = range(5)
+LSA_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024   # static scratch of lsa_select_streaming_noalloc
 
 EXPORTS = [
     "lsa_status_string", "lsa_last_error", "lsa_workspace_size", "lsa_index_flat", "lsa_select_streaming",
     "lsa_pool_pages", "lsa_index_hier", "lsa_sparse_attn", "lsa_layer_group", "lsa_device_status",
+    "lsa_select_streaming_noalloc",
 ]
 
 
@@ -78,6 +80,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.lsa_index_flat.argtypes = [ctypes.POINTER(IndexerIn), Budget, vp, vp, vp, sz, vp]
     lib.lsa_select_streaming.restype = i32
     lib.lsa_select_streaming.argtypes = [vp, vp, i32, i32, i32, Budget, vp, vp, sz, vp]
+    lib.lsa_select_streaming_noalloc.restype = i32
+    lib.lsa_select_streaming_noalloc.argtypes = [vp, vp, i32, i32, i32, Budget, vp, vp]
     lib.lsa_pool_pages.restype = i32
     lib.lsa_pool_pages.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp]
     lib.lsa_index_hier.restype = i32
@@ -241,6 +245,25 @@ def lsa_select_streaming(scores, seq_len, budget, *, idx=None, workspace=None, s
     ws = _workspace(need, scores.device, workspace)
     _check(lib.lsa_select_streaming(_ptr(scores), _ptr(seq_len), B, T, L_max, Budget(*budget), _ptr(idx), _ptr(ws),
                                     _nbytes(ws), _stream(stream)))
+    return idx
+
+
+def lsa_select_streaming_noalloc(scores, seq_len, budget, *, idx=None, stream=None):
+    """lsa_select_streaming with the library's static scratch instead of a
+    workspace: the C entry point allocates nothing, for callers that cannot
+    allocate device memory where they select. Pass `idx` [B,T,k] int32 to keep
+    this call free of allocations on the Python side too. Calls on one device
+    share the scratch, so they must not overlap on the GPU."""
+    torch = _torch()
+    lib = load()
+    _need(scores, "scores", torch.float32, 3)
+    _need(seq_len, "seq_len", torch.int32, 1)
+    B, T, L_max = scores.shape
+    if idx is None:
+        idx = torch.empty((B, T, budget[0]), dtype=torch.int32, device=scores.device)
+    _need(idx, "idx", torch.int32, 3)
+    _check(lib.lsa_select_streaming_noalloc(_ptr(scores), _ptr(seq_len), B, T, L_max, Budget(*budget), _ptr(idx),
+                                            _stream(stream)))
     return idx
 
 
