@@ -326,6 +326,7 @@ lsa_status_t run_attn(const lsa_attn_in_t* at, const int* idx, int k, void* out,
   a.d_qk = at->d_qk; a.d_v = at->d_v; a.k = k;
   a.scale_log2 = at->scale * 1.4426950408889634f;
   a.idx = idx;
+  a.q = static_cast<const uint16_t*>(at->q);
   a.kp = static_cast<const uint16_t*>(at->k);
   a.vp = static_cast<const uint16_t*>(at->v);
   a.k_stride = at->k_row_stride; a.v_stride = at->v_row_stride;

@@ -331,6 +331,450 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// MLA decode (d_qk = 576, d_v = 512): one CTA pair (a cluster of 2) per (KV
+// split, query row). The pair splits the q.K contraction: CTA 0 holds q
+// columns [0, 320) and CTA 1 columns [320, 576), both in tensor memory (the A
+// operand of the score MMA, so q is never re-read from shared memory). Each
+// CTA loads five 64-column chunks of every gathered KV row (CTA 0 columns
+// [0, 320), CTA 1 columns [256, 576)), computes a partial score block, sends
+// it to its partner through distributed shared memory and adds the partner's:
+// both CTAs then hold the same scores (fp32 addition commutes), run the same
+// online softmax and each accumulates its half of the output columns
+// (O += P V over 256 of the 512 latent columns).
+//
+// Roles (192 threads):
+//   warp 0      TMA producer: index block -> validity mask, tiled boxes for
+//               contiguous runs, tile::gather4 row gathers otherwise, into a
+//               kStages-deep ring of 32-row blocks
+//   warp 1      TMEM owner; lane 0 issues QK(b) then PV(b - 1), so the score
+//               MMA of a block overlaps the softmax of the previous one
+//   warps 2..5  one thread per head: q -> TMEM, partial-score exchange,
+//               softmax (lazy rescale when the running max grows by > 2^8),
+//               P -> shared memory, output epilogue
+namespace mla {
+constexpr int kThreads = 192;
+constexpr int BN = kAttnBN;                         // KV rows per block
+constexpr int kStages = 8;
+constexpr int kChunks = 5;                          // 64-column chunks per CTA and block
+constexpr int kChunkBytes = BN * 128;
+constexpr int kStageBytes = kChunks * kChunkBytes;
+constexpr int kPBytes = 128 * BN * 2;
+constexpr int kXStride = 36;                        // floats per exchange row: 16-byte accesses conflict-free
+constexpr int kXBytes = 128 * kXStride * 4;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColO = 0, kColS = 256, kColQ = 320;
+constexpr int kOffP = kStages * kStageBytes;
+constexpr int kOffX = kOffP + 2 * kPBytes;
+constexpr int kOffMask = kOffX + 2 * kXBytes;
+constexpr int kOffBars = kOffMask + kStages * 4;
+constexpr int kNumBars = 2 * kStages + 13;
+constexpr int kOffMisc = kOffBars + kNumBars * 8;
+constexpr size_t kSmem = 1024 + kOffMisc + 16;
+static_assert(kOffBars % 8 == 0, "mbarriers need 8-byte alignment");
+static_assert(kSmem <= 227 * 1024, "shared memory budget");
+
+// Bounded wait that also gives up when another thread of the CTA has aborted.
+template <bool CLUSTER>
+__device__ __forceinline__ bool wait_ph(uint64_t* bar, uint32_t parity, int* status, volatile int* abort_flag) {
+  auto probe = [&] { return CLUSTER ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
+  if (probe()) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  while (true) {
+    for (int i = 0; i < 32; ++i)
+      if (probe()) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      record_timeout(status);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    mla_pair_kernel(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUtensorMap tm_kg,
+                    const AttnArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sStage = base;
+  uint8_t* sP = base + kOffP;
+  uint8_t* sX = base + kOffX;
+  uint32_t* mask_s = reinterpret_cast<uint32_t*>(base + kOffMask);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + kOffBars);
+  uint64_t* kv_full = bars;
+  uint64_t* kv_empty = bars + kStages;
+  uint64_t* s_full = bars + 2 * kStages;
+  uint64_t* s_free = s_full + 2;
+  uint64_t* p_full = s_free + 2;
+  uint64_t* pv_done = p_full + 2;
+  uint64_t* x_full = pv_done + 2;
+  uint64_t* x_free = x_full + 2;
+  uint64_t* q_ready = x_free + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_ctarank();
+  const uint32_t peer = rank ^ 1u;
+  const int split = blockIdx.y, r = blockIdx.z;
+  const int b = r / a.T;
+  const int chunk0 = rank ? 4 : 0;        // global 64-column chunk of local chunk 0
+  const int nq = rank ? 4 : 5;            // q chunks held (and score chunks multiplied)
+  const int qk_local0 = rank ? 1 : 0;     // local chunk of the first score chunk
+  const int q_chunk0 = rank ? 5 : 0;
+
+  const int nblk_total = (a.k + BN - 1) / BN;
+  const int blk0 = split * a.blocks_per_split;
+  const int nblk = max(0, min(a.blocks_per_split, nblk_total - blk0));
+  const int* idx_row = a.idx + static_cast<long long>(r) * a.k;
+
+  if (tid == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 128);
+      mbar_init(&p_full[i], 128);
+      mbar_init(&pv_done[i], 1);
+      mbar_init(&x_full[i], 128);
+      mbar_init(&x_free[i], 128);
+    }
+    mbar_init(q_ready, 128);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  cluster_sync_all();   // the partner's barriers are initialised before any remote arrive
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tO = tmem + kColO, tQ = tmem + kColQ;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer --
+    prefetch_tmap(&tm_kt);
+    prefetch_tmap(&tm_kg);
+    const int row0 = b * a.L_max;
+    for (int blk = 0; blk < nblk; ++blk) {
+      const int s = blk % kStages;
+      if (blk >= kStages) {
+        const bool ok = wait_ph<false>(&kv_empty[s], ((blk / kStages) - 1) & 1, a.status, abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) break;
+      }
+      const int ip = (blk0 + blk) * BN + lane;
+      int id = ip < a.k ? __ldg(idx_row + ip) : -1;
+      if (id >= a.L_max) id = -1;
+      const uint32_t valid = __ballot_sync(0xffffffffu, id >= 0);
+      const int id0 = __shfl_sync(0xffffffffu, id, 0);
+      const bool contiguous = __all_sync(0xffffffffu, id0 >= 0 && id == id0 + lane);
+      const int y = row0 + (id >= 0 ? id : 0);
+      int yg[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) yg[q] = __shfl_sync(0xffffffffu, y, (4 * lane + q) & 31);
+      if (lane == 0) {
+        mask_s[s] = valid;
+        mbar_arrive_expect_tx(&kv_full[s], kStageBytes);
+      }
+      __syncwarp();
+      uint8_t* st = sStage + s * kStageBytes;
+      if (contiguous) {
+        if (lane < kChunks) tma_load_2d(st + lane * kChunkBytes, &tm_kt, &kv_full[s], (chunk0 + lane) * 64, row0 + id0);
+      } else if (lane < BN / 4) {
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c)
+          tma_gather4(st + c * kChunkBytes + lane * 512, &tm_kg, &kv_full[s], (chunk0 + c) * 64, yg[0], yg[1], yg[2],
+                      yg[3]);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer --
+    if (lane == 0 && nblk > 0) {
+      const uint32_t idesc_qk = make_idesc(1, 1, 128, BN, 0, 0);
+      const uint32_t idesc_pv = make_idesc(1, 1, 128, 256, 0, 1);
+      auto issue_pv = [&](int pb) -> bool {
+        if (!wait_ph<false>(&p_full[pb & 1], (pb >> 1) & 1, a.status, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t pa = smem_u32(sP + (pb & 1) * kPBytes);
+        const uint32_t vb = smem_u32(sStage + (pb % kStages) * kStageBytes);
+#pragma unroll
+        for (int ks = 0; ks < BN / 16; ++ks) {
+          const uint64_t ad = make_sdesc(pa + ks * 256, 128, 512, kLayoutNone);
+          const uint64_t bd = make_sdesc(vb + ks * 2048, kChunkBytes, 1024, kLayoutSW128);
+          umma_f16(tO, ad, bd, idesc_pv, (pb > 0 || ks > 0) ? 1u : 0u);
+        }
+        umma_commit(&pv_done[pb & 1]);
+        umma_commit(&kv_empty[pb % kStages]);
+        return true;
+      };
+      bool ok = wait_ph<false>(q_ready, 0, a.status, abort_flag);
+      for (int blk = 0; ok && blk < nblk; ++blk) {
+        const int s = blk % kStages, i = blk & 1;
+        ok = wait_ph<false>(&kv_full[s], (blk / kStages) & 1, a.status, abort_flag);
+        if (ok && blk >= 2) ok = wait_ph<false>(&s_free[i], ((blk - 2) >> 1) & 1, a.status, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t kb = smem_u32(sStage + s * kStageBytes);
+        const uint32_t tS = tmem + kColS + i * BN;
+#pragma unroll 1
+        for (int j = 0; j < nq; ++j) {
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) {
+            const uint64_t bd = make_sdesc(kb + (qk_local0 + j) * kChunkBytes + ks * 32, 16, 1024, kLayoutSW128);
+            umma_f16_ts(tS, tQ + j * 32 + ks * 8, bd, idesc_qk, (j | ks) ? 1u : 0u);
+          }
+        }
+        umma_commit(&s_full[i]);
+        if (blk >= 1) ok = issue_pv(blk - 1);
+      }
+      if (ok) issue_pv(nblk - 1);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------- softmax / epilogue --
+    const int quarter = warp & 3;
+    const int h = quarter * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    bool ok = true;
+    // q row h -> TMEM columns (two bf16 per column, k ascending)
+    {
+      const uint16_t* qrow = a.q + (static_cast<long long>(r) * a.Hq + h) * 576;
+#pragma unroll 1
+      for (int j = 0; j < nq; ++j) {
+        uint32_t v[32];
+        if (h < a.Hq) {
+          const uint8_t* src = reinterpret_cast<const uint8_t*>(qrow + (q_chunk0 + j) * 64);
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            const uint4 w = ldg_nc_v4(src + 16 * t);
+            v[4 * t] = w.x;
+            v[4 * t + 1] = w.y;
+            v[4 * t + 2] = w.z;
+            v[4 * t + 3] = w.w;
+          }
+        } else {
+#pragma unroll
+          for (int t = 0; t < 32; ++t) v[t] = 0u;
+        }
+        tmem_st32(tQ + lane_base + j * 32, v);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(q_ready);
+    }
+    const uint32_t my_row = smem_u32(sX) + h * kXStride * 4;
+    const uint32_t peer_row = mapa_shared(my_row, peer);
+    const uint32_t peer_xfull = mapa_shared(smem_u32(x_full), peer);
+    const uint32_t peer_xfree = mapa_shared(smem_u32(x_free), peer);
+    float m_run = -INFINITY, l_run = 0.f;   // log2 domain
+    for (int blk = 0; blk < nblk; ++blk) {
+      const int s = blk % kStages, i = blk & 1, u = blk >> 1;
+      // partial scores of this CTA
+      ok = __all_sync(0xffffffffu, wait_ph<false>(&s_full[i], u & 1, a.status, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sv[32];
+      tmem_ld32(tmem + kColS + i * BN + lane_base, sv);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(&s_free[i]);
+      // exchange with the partner: send mine, receive theirs
+      if (u >= 1) {
+        ok = __all_sync(0xffffffffu, wait_ph<true>(&x_free[i], (u - 1) & 1, a.status, abort_flag));
+        if (!ok) break;
+      }
+      const uint32_t dst = peer_row + i * kXBytes;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) st_cluster_v4(dst + 16 * t, sv[4 * t], sv[4 * t + 1], sv[4 * t + 2], sv[4 * t + 3]);
+      mbar_arrive_cluster(peer_xfull + i * 8);
+      ok = __all_sync(0xffffffffu, wait_ph<true>(&x_full[i], u & 1, a.status, abort_flag));
+      if (!ok) break;
+      float x[32];
+      {
+        const float4* src = reinterpret_cast<const float4*>(sX + i * kXBytes + h * kXStride * 4);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const float4 w = src[t];
+          x[4 * t] = __uint_as_float(sv[4 * t]) + w.x;
+          x[4 * t + 1] = __uint_as_float(sv[4 * t + 1]) + w.y;
+          x[4 * t + 2] = __uint_as_float(sv[4 * t + 2]) + w.z;
+          x[4 * t + 3] = __uint_as_float(sv[4 * t + 3]) + w.w;
+        }
+      }
+      mbar_arrive_cluster(peer_xfree + i * 8);
+      // softmax over the valid entries of the block
+      ok = __all_sync(0xffffffffu, wait_ph<false>(&kv_full[s], (blk / kStages) & 1, a.status, abort_flag));
+      if (!ok) break;
+      const uint32_t valid = mask_s[s];
+      float mb = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        x[j] = ((valid >> j) & 1u) ? x[j] * a.scale_log2 : -INFINITY;
+        mb = fmaxf(mb, x[j]);
+      }
+      const float m_new = fmaxf(m_run, mb);
+      const bool move = m_new != -INFINITY && (m_run == -INFINITY || m_new > m_run + 8.f);
+      float corr = 1.f;
+      if (move) {
+        corr = m_run == -INFINITY ? 0.f : exp2f(m_run - m_new);
+        l_run *= corr;
+        m_run = m_new;
+      }
+      if (__any_sync(0xffffffffu, move && blk > 0)) {
+        // O holds earlier blocks: rescale it once PV(blk - 1) has landed
+        ok = __all_sync(0xffffffffu,
+                        wait_ph<false>(&pv_done[(blk - 1) & 1], ((blk - 1) >> 1) & 1, a.status, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll 1
+        for (int c0 = 0; c0 < 256; c0 += 32) {
+          uint32_t ov[32];
+          tmem_ld32(tO + lane_base + c0, ov);
+          tmem_ld_wait();
+#pragma unroll
+          for (int t = 0; t < 32; ++t) ov[t] = __float_as_uint(__uint_as_float(ov[t]) * corr);
+          tmem_st32(tO + lane_base + c0, ov);
+        }
+        tmem_st_wait();
+      }
+      float psum = 0.f;
+      uint32_t pk[16];
+#pragma unroll
+      for (int j = 0; j < 32; j += 2) {
+        const float p0 = m_run == -INFINITY ? 0.f : exp2f(x[j] - m_run);
+        const float p1 = m_run == -INFINITY ? 0.f : exp2f(x[j + 1] - m_run);
+        psum += p0 + p1;
+        const __nv_bfloat162 v2 = __floats2bfloat162_rn(p0, p1);
+        pk[j >> 1] = *reinterpret_cast<const uint32_t*>(&v2);
+      }
+      l_run += psum;
+      // P buffer i is free once PV(blk - 2) has completed
+      if (blk >= 2) {
+        ok = __all_sync(0xffffffffu, wait_ph<false>(&pv_done[i], ((blk - 2) >> 1) & 1, a.status, abort_flag));
+        if (!ok) break;
+      }
+      uint8_t* prow = sP + i * kPBytes + (h >> 3) * 512 + (h & 7) * 16;
+#pragma unroll
+      for (int kc = 0; kc < 4; ++kc)
+        *reinterpret_cast<uint4*>(prow + kc * 128) = make_uint4(pk[4 * kc], pk[4 * kc + 1], pk[4 * kc + 2], pk[4 * kc + 3]);
+      tc_fence_before();
+      fence_proxy_async_smem();
+      mbar_arrive(&p_full[i]);
+    }
+    if (ok && nblk > 0)
+      ok = __all_sync(0xffffffffu,
+                      wait_ph<false>(&pv_done[(nblk - 1) & 1], ((nblk - 1) >> 1) & 1, a.status, abort_flag));
+    // ---- epilogue: this CTA's 256 output columns, staged per warp for coalesced stores
+    if (ok) {
+      tc_fence_after();
+      const bool have = nblk > 0;
+      const bool final_out = a.n_split == 1;
+      const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+      float* tile = reinterpret_cast<float*>(sX) + quarter * 32 * kXStride;   // [32 rows][kXStride]
+#pragma unroll 1
+      for (int c0 = 0; c0 < 256; c0 += 32) {
+        uint32_t ov[32];
+        if (have) {
+          tmem_ld32(tO + lane_base + c0, ov);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int t = 0; t < 32; ++t) ov[t] = 0u;
+        }
+        const float f = final_out ? inv_l : 1.f;
+        float4* trow = reinterpret_cast<float4*>(tile + lane * kXStride);
+#pragma unroll
+        for (int t = 0; t < 8; ++t)
+          trow[t] = make_float4(__uint_as_float(ov[4 * t]) * f, __uint_as_float(ov[4 * t + 1]) * f,
+                                __uint_as_float(ov[4 * t + 2]) * f, __uint_as_float(ov[4 * t + 3]) * f);
+        __syncwarp();
+        if (final_out) {
+          // 8 rows per instruction, 64 bytes (32 bf16) per row
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const int rr = t * 8 + (lane >> 2), seg = lane & 3;
+            const int hh = quarter * 32 + rr;
+            const float4* srcp = reinterpret_cast<const float4*>(tile + rr * kXStride + seg * 8);
+            const float4 v0 = srcp[0], v1 = srcp[1];
+            const __nv_bfloat162 b0 = __floats2bfloat162_rn(v0.x, v0.y), b1 = __floats2bfloat162_rn(v0.z, v0.w);
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(v1.x, v1.y), b3 = __floats2bfloat162_rn(v1.z, v1.w);
+            if (hh < a.Hq) {
+              uint16_t* dstp = a.out + (static_cast<long long>(r) * a.Hq + hh) * 512 + rank * 256 + c0 + seg * 8;
+              *reinterpret_cast<uint4*>(dstp) =
+                  make_uint4(*reinterpret_cast<const uint32_t*>(&b0), *reinterpret_cast<const uint32_t*>(&b1),
+                             *reinterpret_cast<const uint32_t*>(&b2), *reinterpret_cast<const uint32_t*>(&b3));
+            }
+          }
+        } else {
+          // 4 rows per instruction, 128 bytes (32 fp32) per row
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            const int rr = t * 4 + (lane >> 3), seg = lane & 7;
+            const int hh = quarter * 32 + rr;
+            const float4 v = *reinterpret_cast<const float4*>(tile + rr * kXStride + seg * 4);
+            if (hh < a.Hq) {
+              const long long prow = (static_cast<long long>(r) * a.n_split + split) * a.Hq + hh;
+              *reinterpret_cast<float4*>(a.part_o + prow * 512 + rank * 256 + c0 + seg * 4) = v;
+            }
+          }
+        }
+        __syncwarp();
+      }
+      if (rank == 0 && h < a.Hq) {
+        if (final_out) {
+          if (a.lse)
+            a.lse[static_cast<long long>(r) * a.Hq + h] =
+                l_run > 0.f ? (m_run + log2f(l_run)) * 0.69314718055994530942f : -INFINITY;
+        } else {
+          const long long prow = (static_cast<long long>(r) * a.n_split + split) * a.Hq + h;
+          a.part_m[prow] = have ? m_run : -INFINITY;
+          a.part_l[prow] = have ? l_run : 0.f;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag) spin_ns(50000);   // let copies and MMAs in flight land before the exit
+  cluster_sync_all();                 // the partner has finished writing into this CTA's shared memory
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+cudaError_t launch(const AttnMaps& m, const AttnArgs& a, cudaStream_t stream) {
+  const void* fn = reinterpret_cast<const void*>(&mla_pair_kernel);
+  cudaError_t e = set_max_smem(fn, kSmem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2, a.n_split, a.B * a.T);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmem;
+  cfg.stream = stream;
+  cfg.attrs = nullptr;
+  cfg.numAttrs = 0;
+  void* args[] = {const_cast<CUtensorMap*>(&m.k_tile), const_cast<CUtensorMap*>(&m.k_rows),
+                  const_cast<AttnArgs*>(&a)};
+  return cudaLaunchKernelExC(&cfg, fn, args);
+}
+}  // namespace mla
+
 // Merge KV-split partials: m* = max m_s; o = sum O_s 2^(m_s - m*) / sum l_s 2^(m_s - m*).
 __global__ void __launch_bounds__(128) combine_kernel(const AttnArgs a) {
   __shared__ float s_f[64];
@@ -410,14 +854,14 @@ cudaError_t launch_t(const AttnMaps& m, const AttnArgs& a, cudaStream_t stream) 
 }  // namespace
 
 size_t attn_smem_bytes(int d_qk, int d_v, bool sep_v) {
-  if (d_qk == 576 && d_v == 512) return sep_v ? ACfg<576, 512, true>::kSmem : ACfg<576, 512, false>::kSmem;
+  if (d_qk == 576 && d_v == 512) return mla::kSmem;
   return ACfg<64, 64, true>::kSmem;
 }
 
 cudaError_t launch_attn(const AttnMaps& m, const AttnArgs& a, cudaStream_t stream) {
   if (a.d_qk == 576 && a.d_v == 512) {
     if (a.sep_v) return cudaErrorNotSupported;   // MLA keeps V inside the latent row
-    return launch_t<576, 512, false>(m, a, stream);
+    return mla::launch(m, a, stream);
   }
   if (a.d_qk == 64 && a.d_v == 64) {
     if (a.sep_v) return launch_t<64, 64, true>(m, a, stream);

@@ -96,6 +96,7 @@ struct AttnArgs {
   int k;                  // index row length
   float scale_log2;       // scale * log2(e)
   const int* idx;
+  const uint16_t* q;      // [rows, Hq, d_qk] bf16
   const uint16_t* kp;     // K rows
   const uint16_t* vp;     // V rows (may alias kp)
   long long k_stride, v_stride;
