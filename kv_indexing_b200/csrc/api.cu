@@ -171,7 +171,8 @@ AttnPlan attn_plan(const lsa_attn_in_t* at, int k) {
   AttnPlan p;
   const int rows = at->B * at->T;
   p.nvp = at->d_v >= 512 ? 2 : 1;
-  const int nblk = (k + kAttnBN - 1) / kAttnBN;
+  const int bn = at->d_qk == 576 ? kAttnBNMla : kAttnBN;   // KV rows per kernel block
+  const int nblk = (k + bn - 1) / bn;
   int ns = device_sm_count() / (rows * p.nvp);
   if (ns < 1) ns = 1;
   if (ns > nblk) ns = nblk;

@@ -338,41 +338,47 @@ __global__ void __launch_bounds__(kThreads, 1)
 // operand of the score MMA, so q is never re-read from shared memory). Each
 // CTA loads five 64-column chunks of every gathered KV row (CTA 0 columns
 // [0, 320), CTA 1 columns [256, 576)), computes a partial score block, sends
-// it to its partner through distributed shared memory and adds the partner's:
-// both CTAs then hold the same scores (fp32 addition commutes), run the same
-// online softmax and each accumulates its half of the output columns
-// (O += P V over 256 of the 512 latent columns).
+// it to its partner through distributed shared memory (one bulk copy per
+// block, counted on the partner's mbarrier) and adds the partner's: both CTAs
+// then hold the same
+// scores (fp32 addition commutes), run the same online softmax and each
+// accumulates its half of the output columns (O += P V over 256 of the 512
+// latent columns, with P in tensor memory as the MMA A operand).
 //
-// Roles (192 threads):
-//   warp 0      TMA producer: index block -> validity mask, tiled boxes for
-//               contiguous runs, tile::gather4 row gathers otherwise, into a
-//               kStages-deep ring of 32-row blocks
-//   warp 1      TMEM owner; lane 0 issues QK(b) then PV(b - 1), so the score
-//               MMA of a block overlaps the softmax of the previous one
-//   warps 2..5  one thread per head: q -> TMEM, partial-score exchange,
-//               softmax (lazy rescale when the running max grows by > 2^8),
-//               P -> shared memory, output epilogue
+// Roles (320 threads):
+//   warp 0      TMA producer: index entries (prefetched one ring ahead) ->
+//               validity mask, tiled boxes for contiguous runs, tile::gather4
+//               row gathers otherwise, into a kStages-deep ring of 64-row blocks
+//   warp 1      TMEM owner; lane 0 issues QK(b) then PV(b - 1)
+//   warps 2..9  softmax: two threads per head, each on 32 of a block's 64
+//               columns. Software-pipelined: the partial scores of block b + 1
+//               go to the partner before block b's softmax runs, so the
+//               exchange latency hides behind a whole iteration. The two
+//               threads of a head agree on the block max through a tagged
+//               shared-memory slot (bounded wait, no block-wide barrier).
 namespace mla {
-constexpr int kThreads = 192;
-constexpr int BN = kAttnBN;                         // KV rows per block
-constexpr int kStages = 8;
+constexpr int kThreads = 320;
+constexpr int kSoftThreads = 256;
+constexpr int BN = 64;                              // KV rows per block
+constexpr int kStages = 3;
 constexpr int kChunks = 5;                          // 64-column chunks per CTA and block
 constexpr int kChunkBytes = BN * 128;
 constexpr int kStageBytes = kChunks * kChunkBytes;
-constexpr int kPBytes = 128 * BN * 2;
-constexpr int kXStride = 36;                        // floats per exchange row: 16-byte accesses conflict-free
-constexpr int kXBytes = 128 * kXStride * 4;
+constexpr int kXBytes = 128 * BN * 4;               // exchange rows of 256 B, 16-byte units XOR-swizzled by row
+constexpr int kXTotalBytes = 128 * BN * 4;          // bytes the partner sends per block
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = 0, kColS = 256, kColQ = 320;
-constexpr int kOffP = kStages * kStageBytes;
-constexpr int kOffX = kOffP + 2 * kPBytes;
-constexpr int kOffMask = kOffX + 2 * kXBytes;
-constexpr int kOffBars = kOffMask + kStages * 4;
-constexpr int kNumBars = 2 * kStages + 13;
+constexpr uint32_t kColO = 0, kColS = 256, kColP = 320, kColQ = 352;
+constexpr int kOffX = kStages * kStageBytes;        // [2] receive buffers
+constexpr int kOffSend = kOffX + 2 * kXBytes;       // outgoing partial scores (same layout)
+constexpr int kOffTag = kOffSend + kXBytes;         // [2][2][128] u64 tagged max slots + [2][128] u64 sums
+constexpr int kOffMask = kOffTag + (4 * 128 + 2 * 128) * 8;
+constexpr int kOffBars = kOffMask + kStages * 8;
+constexpr int kNumBars = 2 * kStages + 10;
 constexpr int kOffMisc = kOffBars + kNumBars * 8;
 constexpr size_t kSmem = 1024 + kOffMisc + 16;
 static_assert(kOffBars % 8 == 0, "mbarriers need 8-byte alignment");
 static_assert(kSmem <= 227 * 1024, "shared memory budget");
+static_assert(kStageBytes % 1024 == 0, "swizzled tiles need 1024-byte alignment");
 
 // Bounded wait that also gives up when another thread of the CTA has aborted.
 template <bool CLUSTER>
@@ -392,6 +398,29 @@ __device__ __forceinline__ bool wait_ph(uint64_t* bar, uint32_t parity, int* sta
   }
 }
 
+// Publish (tag, value) in a shared slot; read the partner's slot once its tag
+// matches. Bounded like the barrier waits.
+__device__ __forceinline__ void put_tagged(volatile unsigned long long* slot, uint32_t tag, float v) {
+  *slot = (static_cast<unsigned long long>(tag) << 32) | __float_as_uint(v);
+}
+__device__ __forceinline__ bool get_tagged(const volatile unsigned long long* slot, uint32_t tag, float* v,
+                                           int* status, volatile int* abort_flag) {
+  unsigned long long x = *slot;
+  if (static_cast<uint32_t>(x >> 32) != tag) {
+    const unsigned long long t0 = globaltimer_ns();
+    while (static_cast<uint32_t>((x = *slot) >> 32) != tag) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        record_timeout(status);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+  *v = __uint_as_float(static_cast<uint32_t>(x));
+  return true;
+}
+
 __device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
   uint4 v;
   asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
@@ -406,19 +435,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sStage = base;
-  uint8_t* sP = base + kOffP;
   uint8_t* sX = base + kOffX;
-  uint32_t* mask_s = reinterpret_cast<uint32_t*>(base + kOffMask);
+  uint8_t* sSend = base + kOffSend;
+  volatile unsigned long long* tag_max = reinterpret_cast<volatile unsigned long long*>(base + kOffTag);  // [2][2][128]
+  volatile unsigned long long* tag_sum = tag_max + 4 * 128;                                              // [2][128]
+  uint32_t* mask_s = reinterpret_cast<uint32_t*>(base + kOffMask);                                       // [kStages][2]
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + kOffBars);
   uint64_t* kv_full = bars;
   uint64_t* kv_empty = bars + kStages;
   uint64_t* s_full = bars + 2 * kStages;
-  uint64_t* s_free = s_full + 2;
-  uint64_t* p_full = s_free + 2;
-  uint64_t* pv_done = p_full + 2;
-  uint64_t* x_full = pv_done + 2;
-  uint64_t* x_free = x_full + 2;
-  uint64_t* q_ready = x_free + 2;
+  uint64_t* s_free = s_full + 1;
+  uint64_t* p_full = s_free + 1;
+  uint64_t* pv_done = p_full + 1;
+  uint64_t* x_full = pv_done + 1;     // [2]
+  uint64_t* q_ready = x_full + 2;
+  uint64_t* send_full = q_ready + 1;  // the outgoing buffer is written
+  uint64_t* send_free = send_full + 1;  // the bulk copy has read it
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -442,18 +474,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 128);
-      mbar_init(&p_full[i], 128);
-      mbar_init(&pv_done[i], 1);
-      mbar_init(&x_full[i], 128);
-      mbar_init(&x_free[i], 128);
-    }
-    mbar_init(q_ready, 128);
+    mbar_init(s_full, 1);
+    mbar_init(s_free, kSoftThreads);
+    mbar_init(p_full, kSoftThreads);
+    mbar_init(pv_done, 1);
+    for (int i = 0; i < 2; ++i) mbar_init(&x_full[i], 1);   // own expect_tx arrive + the partner's copy bytes
+    mbar_init(q_ready, kSoftThreads);
+    mbar_init(send_full, kSoftThreads);
+    mbar_init(send_free, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
+  for (int i = tid; i < 6 * 128; i += kThreads) tag_max[i] = 0ull;   // tags start at 0 (never a live tag)
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
@@ -463,42 +495,76 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   tc_fence_after();
   cluster_sync_all();   // the partner's barriers are initialised before any remote arrive
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tO = tmem + kColO, tQ = tmem + kColQ;
+  const uint32_t tO = tmem + kColO, tQ = tmem + kColQ, tS = tmem + kColS, tP = tmem + kColP;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer --
     prefetch_tmap(&tm_kt);
     prefetch_tmap(&tm_kg);
     const int row0 = b * a.L_max;
-    for (int blk = 0; blk < nblk; ++blk) {
-      const int s = blk % kStages;
-      if (blk >= kStages) {
-        const bool ok = wait_ph<false>(&kv_empty[s], ((blk / kStages) - 1) & 1, a.status, abort_flag);
-        if (!__all_sync(0xffffffffu, ok)) break;
-      }
-      const int ip = (blk0 + blk) * BN + lane;
-      int id = ip < a.k ? __ldg(idx_row + ip) : -1;
-      if (id >= a.L_max) id = -1;
-      const uint32_t valid = __ballot_sync(0xffffffffu, id >= 0);
-      const int id0 = __shfl_sync(0xffffffffu, id, 0);
-      const bool contiguous = __all_sync(0xffffffffu, id0 >= 0 && id == id0 + lane);
-      const int y = row0 + (id >= 0 ? id : 0);
-      int yg[4];
+    // index entry e of block `bb`, -1 outside the split / row
+    auto load_id = [&](int bb, int e) -> int {
+      const int ip = (blk0 + bb) * BN + e;
+      int v = (bb < nblk && ip < a.k) ? __ldg(idx_row + ip) : -1;
+      return v >= a.L_max ? -1 : v;
+    };
+    int ids_lo[kStages], ids_hi[kStages];   // entries lane and lane + 32 of the next kStages blocks
 #pragma unroll
-      for (int q = 0; q < 4; ++q) yg[q] = __shfl_sync(0xffffffffu, y, (4 * lane + q) & 31);
-      if (lane == 0) {
-        mask_s[s] = valid;
-        mbar_arrive_expect_tx(&kv_full[s], kStageBytes);
-      }
-      __syncwarp();
-      uint8_t* st = sStage + s * kStageBytes;
-      if (contiguous) {
-        if (lane < kChunks) tma_load_2d(st + lane * kChunkBytes, &tm_kt, &kv_full[s], (chunk0 + lane) * 64, row0 + id0);
-      } else if (lane < BN / 4) {
+    for (int j = 0; j < kStages; ++j) {
+      ids_lo[j] = load_id(j, lane);
+      ids_hi[j] = load_id(j, lane + 32);
+    }
+    bool run = true;
+    for (int g = 0; run && g < nblk; g += kStages) {
 #pragma unroll
-        for (int c = 0; c < kChunks; ++c)
-          tma_gather4(st + c * kChunkBytes + lane * 512, &tm_kg, &kv_full[s], (chunk0 + c) * 64, yg[0], yg[1], yg[2],
-                      yg[3]);
+      for (int j = 0; j < kStages; ++j) {
+        const int blk = g + j;
+        if (blk >= nblk) {
+          run = false;
+          break;
+        }
+        if (blk >= kStages) {
+          const bool ok = wait_ph<false>(&kv_empty[j], ((blk / kStages) - 1) & 1, a.status, abort_flag);
+          if (!__all_sync(0xffffffffu, ok)) {
+            run = false;
+            break;
+          }
+        }
+        const int id_lo = ids_lo[j], id_hi = ids_hi[j];
+        ids_lo[j] = load_id(blk + kStages, lane);
+        ids_hi[j] = load_id(blk + kStages, lane + 32);
+        const uint32_t valid_lo = __ballot_sync(0xffffffffu, id_lo >= 0);
+        const uint32_t valid_hi = __ballot_sync(0xffffffffu, id_hi >= 0);
+        const int id0 = __shfl_sync(0xffffffffu, id_lo, 0);
+        const bool contiguous =
+            __all_sync(0xffffffffu, id0 >= 0 && id_lo == id0 + lane && id_hi == id0 + 32 + lane);
+        const int y_lo = row0 + (id_lo >= 0 ? id_lo : 0), y_hi = row0 + (id_hi >= 0 ? id_hi : 0);
+        int yg[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int src = (4 * lane + q) & 31;
+          const int a_lo = __shfl_sync(0xffffffffu, y_lo, src), a_hi = __shfl_sync(0xffffffffu, y_hi, src);
+          yg[q] = lane < 8 ? a_lo : a_hi;   // lane g gathers block rows 4g .. 4g + 3
+        }
+        if (lane == 0) {
+          mask_s[2 * j] = valid_lo;
+          mask_s[2 * j + 1] = valid_hi;
+          mbar_arrive_expect_tx(&kv_full[j], kStageBytes);
+        }
+        __syncwarp();
+        uint8_t* st = sStage + j * kStageBytes;
+        if (contiguous) {
+          if (lane < 2 * kChunks) {
+            const int c = lane >> 1, hrow = lane & 1;   // two 32-row boxes per chunk
+            tma_load_2d(st + c * kChunkBytes + hrow * (kChunkBytes / 2), &tm_kt, &kv_full[j], (chunk0 + c) * 64,
+                        row0 + id0 + 32 * hrow);
+          }
+        } else if (lane < BN / 4) {
+#pragma unroll
+          for (int c = 0; c < kChunks; ++c)
+            tma_gather4(st + c * kChunkBytes + lane * 512, &tm_kg, &kv_full[j], (chunk0 + c) * 64, yg[0], yg[1],
+                        yg[2], yg[3]);
+        }
       }
     }
   } else if (warp == 1) {
@@ -507,29 +573,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const uint32_t idesc_qk = make_idesc(1, 1, 128, BN, 0, 0);
       const uint32_t idesc_pv = make_idesc(1, 1, 128, 256, 0, 1);
       auto issue_pv = [&](int pb) -> bool {
-        if (!wait_ph<false>(&p_full[pb & 1], (pb >> 1) & 1, a.status, abort_flag)) return false;
+        if (!wait_ph<false>(p_full, pb & 1, a.status, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t pa = smem_u32(sP + (pb & 1) * kPBytes);
         const uint32_t vb = smem_u32(sStage + (pb % kStages) * kStageBytes);
 #pragma unroll
         for (int ks = 0; ks < BN / 16; ++ks) {
-          const uint64_t ad = make_sdesc(pa + ks * 256, 128, 512, kLayoutNone);
           const uint64_t bd = make_sdesc(vb + ks * 2048, kChunkBytes, 1024, kLayoutSW128);
-          umma_f16(tO, ad, bd, idesc_pv, (pb > 0 || ks > 0) ? 1u : 0u);
+          umma_f16_ts(tO, tP + ks * 8, bd, idesc_pv, (pb > 0 || ks > 0) ? 1u : 0u);
         }
-        umma_commit(&pv_done[pb & 1]);
+        umma_commit(pv_done);
         umma_commit(&kv_empty[pb % kStages]);
         return true;
       };
       bool ok = wait_ph<false>(q_ready, 0, a.status, abort_flag);
       for (int blk = 0; ok && blk < nblk; ++blk) {
-        const int s = blk % kStages, i = blk & 1;
+        const int s = blk % kStages;
         ok = wait_ph<false>(&kv_full[s], (blk / kStages) & 1, a.status, abort_flag);
-        if (ok && blk >= 2) ok = wait_ph<false>(&s_free[i], ((blk - 2) >> 1) & 1, a.status, abort_flag);
+        if (ok && blk >= 1) ok = wait_ph<false>(s_free, (blk - 1) & 1, a.status, abort_flag);
         if (!ok) break;
         tc_fence_after();
         const uint32_t kb = smem_u32(sStage + s * kStageBytes);
-        const uint32_t tS = tmem + kColS + i * BN;
 #pragma unroll 1
         for (int j = 0; j < nq; ++j) {
 #pragma unroll
@@ -538,7 +601,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             umma_f16_ts(tS, tQ + j * 32 + ks * 8, bd, idesc_qk, (j | ks) ? 1u : 0u);
           }
         }
-        umma_commit(&s_full[i]);
+        umma_commit(s_full);
         if (blk >= 1) ok = issue_pv(blk - 1);
       }
       if (ok) issue_pv(nblk - 1);
@@ -547,101 +610,140 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------- softmax / epilogue --
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;            // columns [32 half, 32 half + 32) of a block
     const int h = quarter * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     bool ok = true;
-    // q row h -> TMEM columns (two bf16 per column, k ascending)
+    // q row h -> TMEM columns (two bf16 per column, k ascending); the two
+    // threads of a head take alternate 64-column chunks
     {
-      const uint16_t* qrow = a.q + (static_cast<long long>(r) * a.Hq + h) * 576;
-#pragma unroll 1
-      for (int j = 0; j < nq; ++j) {
-        uint32_t v[32];
-        if (h < a.Hq) {
-          const uint8_t* src = reinterpret_cast<const uint8_t*>(qrow + (q_chunk0 + j) * 64);
+      const uint8_t* src = reinterpret_cast<const uint8_t*>(a.q + (static_cast<long long>(r) * a.Hq + h) * 576 +
+                                                            q_chunk0 * 64);
+      uint4 qv[3][8];
+#pragma unroll
+      for (int jj = 0; jj < 3; ++jj) {
+        const int j = 2 * jj + half;
+#pragma unroll
+        for (int t = 0; t < 8; ++t)
+          qv[jj][t] = (j < nq && h < a.Hq) ? ldg_nc_v4(src + j * 128 + 16 * t) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int jj = 0; jj < 3; ++jj) {
+        const int j = 2 * jj + half;
+        if (j < nq) {
+          uint32_t v[32];
 #pragma unroll
           for (int t = 0; t < 8; ++t) {
-            const uint4 w = ldg_nc_v4(src + 16 * t);
-            v[4 * t] = w.x;
-            v[4 * t + 1] = w.y;
-            v[4 * t + 2] = w.z;
-            v[4 * t + 3] = w.w;
+            v[4 * t] = qv[jj][t].x;
+            v[4 * t + 1] = qv[jj][t].y;
+            v[4 * t + 2] = qv[jj][t].z;
+            v[4 * t + 3] = qv[jj][t].w;
           }
-        } else {
-#pragma unroll
-          for (int t = 0; t < 32; ++t) v[t] = 0u;
+          tmem_st32(tQ + lane_base + j * 32, v);
         }
-        tmem_st32(tQ + lane_base + j * 32, v);
       }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(q_ready);
     }
-    const uint32_t my_row = smem_u32(sX) + h * kXStride * 4;
-    const uint32_t peer_row = mapa_shared(my_row, peer);
+    const uint32_t col_off = static_cast<uint32_t>(half * 32);
+    const int swz = h & 7;   // unit t of this thread's half-row sits at unit t ^ swz
+    const uint32_t peer_x = mapa_shared(smem_u32(sX), peer);
     const uint32_t peer_xfull = mapa_shared(smem_u32(x_full), peer);
-    const uint32_t peer_xfree = mapa_shared(smem_u32(x_free), peer);
-    float m_run = -INFINITY, l_run = 0.f;   // log2 domain
-    for (int blk = 0; blk < nblk; ++blk) {
-      const int s = blk % kStages, i = blk & 1, u = blk >> 1;
-      // partial scores of this CTA
-      ok = __all_sync(0xffffffffu, wait_ph<false>(&s_full[i], u & 1, a.status, abort_flag));
-      if (!ok) break;
+    const bool leader = h == 0 && half == 0;
+    uint4* send_row = reinterpret_cast<uint4*>(sSend + h * (BN * 4) + half * 128);
+    // Partial scores of block bb: TMEM -> registers, free S, stage them in the
+    // outgoing buffer; the leader ships the whole block with one bulk copy.
+    auto fetch_send = [&](int bb, uint32_t (&sv)[32]) -> bool {
+      if (!__all_sync(0xffffffffu, wait_ph<false>(s_full, bb & 1, a.status, abort_flag))) return false;
       tc_fence_after();
-      uint32_t sv[32];
-      tmem_ld32(tmem + kColS + i * BN + lane_base, sv);
+      tmem_ld32(tS + lane_base + col_off, sv);
       tmem_ld_wait();
       tc_fence_before();
-      mbar_arrive(&s_free[i]);
-      // exchange with the partner: send mine, receive theirs
-      if (u >= 1) {
-        ok = __all_sync(0xffffffffu, wait_ph<true>(&x_free[i], (u - 1) & 1, a.status, abort_flag));
+      mbar_arrive(s_free);
+      if (bb >= 1) {
+        if (leader) {
+          bulk_wait_read();   // the previous block's copy has read the outgoing buffer
+          mbar_arrive(send_free);
+        }
+        if (!__all_sync(0xffffffffu, wait_ph<false>(send_free, (bb - 1) & 1, a.status, abort_flag))) return false;
+      }
+#pragma unroll
+      for (int t = 0; t < 8; ++t) send_row[t ^ swz] = make_uint4(sv[4 * t], sv[4 * t + 1], sv[4 * t + 2], sv[4 * t + 3]);
+      fence_proxy_async_smem();
+      mbar_arrive(send_full);
+      const int i = bb & 1;
+      bool lok = true;
+      if (leader) {
+        mbar_arrive_expect_tx(&x_full[i], kXTotalBytes);
+        lok = wait_ph<false>(send_full, bb & 1, a.status, abort_flag);
+        if (lok) {
+          bulk_copy_to_peer(peer_x + i * kXBytes, sSend, kXBytes, peer_xfull + i * 8);
+          bulk_commit();
+        }
+      }
+      return __all_sync(0xffffffffu, lok);   // warp-uniform outcome
+    };
+    float m_run = -INFINITY, l_part = 0.f;   // log2 domain; l_part: this thread's columns
+    uint32_t sv_cur[32], sv_nxt[32];
+    if (nblk > 0) ok = fetch_send(0, sv_cur);
+    for (int blk = 0; ok && blk < nblk; ++blk) {
+      const int s = blk % kStages, i = blk & 1;
+      // Block blk + 1's partial leaves before block blk's softmax: the
+      // partner's reply then has a whole iteration to arrive. The partner has
+      // finished reading its buffer (blk + 1) & 1 (block blk - 1) before it
+      // sent block blk, which this thread receives below only after sending:
+      // ordering comes from the previous iteration's receive.
+      if (blk + 1 < nblk) {
+        ok = fetch_send(blk + 1, sv_nxt);
         if (!ok) break;
       }
-      const uint32_t dst = peer_row + i * kXBytes;
-#pragma unroll
-      for (int t = 0; t < 8; ++t) st_cluster_v4(dst + 16 * t, sv[4 * t], sv[4 * t + 1], sv[4 * t + 2], sv[4 * t + 3]);
-      mbar_arrive_cluster(peer_xfull + i * 8);
-      ok = __all_sync(0xffffffffu, wait_ph<true>(&x_full[i], u & 1, a.status, abort_flag));
+      ok = __all_sync(0xffffffffu, wait_ph<true>(&x_full[i], (blk >> 1) & 1, a.status, abort_flag));
       if (!ok) break;
       float x[32];
       {
-        const float4* src = reinterpret_cast<const float4*>(sX + i * kXBytes + h * kXStride * 4);
+        const float4* src = reinterpret_cast<const float4*>(sX + i * kXBytes + h * (BN * 4) + half * 128);
 #pragma unroll
         for (int t = 0; t < 8; ++t) {
-          const float4 w = src[t];
-          x[4 * t] = __uint_as_float(sv[4 * t]) + w.x;
-          x[4 * t + 1] = __uint_as_float(sv[4 * t + 1]) + w.y;
-          x[4 * t + 2] = __uint_as_float(sv[4 * t + 2]) + w.z;
-          x[4 * t + 3] = __uint_as_float(sv[4 * t + 3]) + w.w;
+          const float4 w = src[t ^ swz];
+          x[4 * t] = __uint_as_float(sv_cur[4 * t]) + w.x;
+          x[4 * t + 1] = __uint_as_float(sv_cur[4 * t + 1]) + w.y;
+          x[4 * t + 2] = __uint_as_float(sv_cur[4 * t + 2]) + w.z;
+          x[4 * t + 3] = __uint_as_float(sv_cur[4 * t + 3]) + w.w;
         }
       }
-      mbar_arrive_cluster(peer_xfree + i * 8);
-      // softmax over the valid entries of the block
       ok = __all_sync(0xffffffffu, wait_ph<false>(&kv_full[s], (blk / kStages) & 1, a.status, abort_flag));
       if (!ok) break;
-      const uint32_t valid = mask_s[s];
-      float mb = -INFINITY;
+      const uint32_t valid = mask_s[2 * s + half];
+      float mloc[8];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        x[j] = ((valid >> j) & 1u) ? x[j] * a.scale_log2 : -INFINITY;
-        mb = fmaxf(mb, x[j]);
-      }
+      for (int j = 0; j < 32; ++j) x[j] = ((valid >> j) & 1u) ? x[j] * a.scale_log2 : -INFINITY;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) mloc[t] = fmaxf(fmaxf(x[4 * t], x[4 * t + 1]), fmaxf(x[4 * t + 2], x[4 * t + 3]));
+      const float mb_mine = fmaxf(fmaxf(fmaxf(mloc[0], mloc[1]), fmaxf(mloc[2], mloc[3])),
+                                  fmaxf(fmaxf(mloc[4], mloc[5]), fmaxf(mloc[6], mloc[7])));
+      // the other half of the row's block max (tag = block + 1)
+      put_tagged(tag_max + (i * 2 + half) * 128 + h, static_cast<uint32_t>(blk + 1), mb_mine);
+      float mb_other;
+      ok = __all_sync(0xffffffffu, get_tagged(tag_max + (i * 2 + (half ^ 1)) * 128 + h, static_cast<uint32_t>(blk + 1),
+                                              &mb_other, a.status, abort_flag));
+      if (!ok) break;
+      const float mb = fmaxf(mb_mine, mb_other);
       const float m_new = fmaxf(m_run, mb);
       const bool move = m_new != -INFINITY && (m_run == -INFINITY || m_new > m_run + 8.f);
       float corr = 1.f;
       if (move) {
         corr = m_run == -INFINITY ? 0.f : exp2f(m_run - m_new);
-        l_run *= corr;
+        l_part *= corr;
         m_run = m_new;
       }
       if (__any_sync(0xffffffffu, move && blk > 0)) {
-        // O holds earlier blocks: rescale it once PV(blk - 1) has landed
-        ok = __all_sync(0xffffffffu,
-                        wait_ph<false>(&pv_done[(blk - 1) & 1], ((blk - 1) >> 1) & 1, a.status, abort_flag));
+        // O holds earlier blocks: rescale this thread's 128 columns once PV(blk - 1) has landed
+        ok = __all_sync(0xffffffffu, wait_ph<false>(pv_done, (blk - 1) & 1, a.status, abort_flag));
         if (!ok) break;
         tc_fence_after();
 #pragma unroll 1
-        for (int c0 = 0; c0 < 256; c0 += 32) {
+        for (int c0 = half * 128; c0 < half * 128 + 128; c0 += 32) {
           uint32_t ov[32];
           tmem_ld32(tO + lane_base + c0, ov);
           tmem_ld_wait();
@@ -651,42 +753,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         tmem_st_wait();
       }
-      float psum = 0.f;
+      float ps[4] = {0.f, 0.f, 0.f, 0.f};
       uint32_t pk[16];
 #pragma unroll
       for (int j = 0; j < 32; j += 2) {
         const float p0 = m_run == -INFINITY ? 0.f : exp2f(x[j] - m_run);
         const float p1 = m_run == -INFINITY ? 0.f : exp2f(x[j + 1] - m_run);
-        psum += p0 + p1;
+        ps[(j >> 1) & 3] += p0 + p1;
         const __nv_bfloat162 v2 = __floats2bfloat162_rn(p0, p1);
         pk[j >> 1] = *reinterpret_cast<const uint32_t*>(&v2);
       }
-      l_run += psum;
-      // P buffer i is free once PV(blk - 2) has completed
-      if (blk >= 2) {
-        ok = __all_sync(0xffffffffu, wait_ph<false>(&pv_done[i], ((blk - 2) >> 1) & 1, a.status, abort_flag));
+      l_part += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+      // P lives in TMEM (one block): free once PV(blk - 1) has completed
+      if (blk >= 1) {
+        ok = __all_sync(0xffffffffu, wait_ph<false>(pv_done, (blk - 1) & 1, a.status, abort_flag));
         if (!ok) break;
       }
-      uint8_t* prow = sP + i * kPBytes + (h >> 3) * 512 + (h & 7) * 16;
-#pragma unroll
-      for (int kc = 0; kc < 4; ++kc)
-        *reinterpret_cast<uint4*>(prow + kc * 128) = make_uint4(pk[4 * kc], pk[4 * kc + 1], pk[4 * kc + 2], pk[4 * kc + 3]);
+      tc_fence_after();
+      tmem_st16(tP + lane_base + half * 16, pk);   // keys [32 half, 32 half + 32) of row h
+      tmem_st_wait();
       tc_fence_before();
-      fence_proxy_async_smem();
-      mbar_arrive(&p_full[i]);
+      mbar_arrive(p_full);
+#pragma unroll
+      for (int t = 0; t < 32; ++t) sv_cur[t] = sv_nxt[t];
     }
     if (ok && nblk > 0)
-      ok = __all_sync(0xffffffffu,
-                      wait_ph<false>(&pv_done[(nblk - 1) & 1], ((nblk - 1) >> 1) & 1, a.status, abort_flag));
-    // ---- epilogue: this CTA's 256 output columns, staged per warp for coalesced stores
+      ok = __all_sync(0xffffffffu, wait_ph<false>(pv_done, (nblk - 1) & 1, a.status, abort_flag));
+    // row sum over both halves (fixed order: both threads get the same value)
+    float l_run = 0.f;
+    if (ok) {
+      put_tagged(tag_sum + half * 128 + h, 0xFFFFFFFFu, l_part);
+      float l_other;
+      ok = __all_sync(0xffffffffu, get_tagged(tag_sum + (half ^ 1) * 128 + h, 0xFFFFFFFFu, &l_other, a.status,
+                                              abort_flag));
+      l_run = half == 0 ? l_part + l_other : l_other + l_part;
+    }
+    // ---- epilogue: this thread's 128 output columns, staged per warp for coalesced stores
     if (ok) {
       tc_fence_after();
       const bool have = nblk > 0;
       const bool final_out = a.n_split == 1;
       const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
-      float* tile = reinterpret_cast<float*>(sX) + quarter * 32 * kXStride;   // [32 rows][kXStride]
+      float* tile = reinterpret_cast<float*>(sX) + (warp - 2) * 32 * 36;   // [32 rows][36]
 #pragma unroll 1
-      for (int c0 = 0; c0 < 256; c0 += 32) {
+      for (int c0 = half * 128; c0 < half * 128 + 128; c0 += 32) {
         uint32_t ov[32];
         if (have) {
           tmem_ld32(tO + lane_base + c0, ov);
@@ -696,7 +806,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           for (int t = 0; t < 32; ++t) ov[t] = 0u;
         }
         const float f = final_out ? inv_l : 1.f;
-        float4* trow = reinterpret_cast<float4*>(tile + lane * kXStride);
+        float4* trow = reinterpret_cast<float4*>(tile + lane * 36);
 #pragma unroll
         for (int t = 0; t < 8; ++t)
           trow[t] = make_float4(__uint_as_float(ov[4 * t]) * f, __uint_as_float(ov[4 * t + 1]) * f,
@@ -708,7 +818,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           for (int t = 0; t < 4; ++t) {
             const int rr = t * 8 + (lane >> 2), seg = lane & 3;
             const int hh = quarter * 32 + rr;
-            const float4* srcp = reinterpret_cast<const float4*>(tile + rr * kXStride + seg * 8);
+            const float4* srcp = reinterpret_cast<const float4*>(tile + rr * 36 + seg * 8);
             const float4 v0 = srcp[0], v1 = srcp[1];
             const __nv_bfloat162 b0 = __floats2bfloat162_rn(v0.x, v0.y), b1 = __floats2bfloat162_rn(v0.z, v0.w);
             const __nv_bfloat162 b2 = __floats2bfloat162_rn(v1.x, v1.y), b3 = __floats2bfloat162_rn(v1.z, v1.w);
@@ -725,7 +835,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           for (int t = 0; t < 8; ++t) {
             const int rr = t * 4 + (lane >> 3), seg = lane & 7;
             const int hh = quarter * 32 + rr;
-            const float4 v = *reinterpret_cast<const float4*>(tile + rr * kXStride + seg * 4);
+            const float4 v = *reinterpret_cast<const float4*>(tile + rr * 36 + seg * 4);
             if (hh < a.Hq) {
               const long long prow = (static_cast<long long>(r) * a.n_split + split) * a.Hq + hh;
               *reinterpret_cast<float4*>(a.part_o + prow * 512 + rank * 256 + c0 + seg * 4) = v;
@@ -734,7 +844,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
       }
-      if (rank == 0 && h < a.Hq) {
+      if (rank == 0 && half == 0 && h < a.Hq) {
         if (final_out) {
           if (a.lse)
             a.lse[static_cast<long long>(r) * a.Hq + h] =

@@ -110,7 +110,8 @@ struct AttnArgs {
   int* status;            // per-device status word
 };
 
-constexpr int kAttnBN = 32;  // KV rows per block
+constexpr int kAttnBN = 32;  // KV rows per block (d_qk = 64)
+constexpr int kAttnBNMla = 64;  // KV rows per block (MLA, d_qk = 576)
 
 // TMA descriptors of one attention launch: q tiles [128 heads x 64], K/V row
 // tiles [32 rows x 64] (contiguous blocks) and one-row boxes for row gathers.
