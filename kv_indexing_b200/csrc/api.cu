@@ -187,7 +187,7 @@ size_t attn_ws_bytes(const lsa_attn_in_t* at, int k) {
   if (p.n_split <= 1) return 0;
   const size_t rows = static_cast<size_t>(at->B) * at->T;
   const size_t nm = rows * p.n_split * at->Hq;
-  return align_up(nm * at->d_v * 4, 256) + 2 * align_up(nm * 4, 256);
+  return align_up(nm * at->d_v * 2, 256) + 2 * align_up(nm * 4, 256);
 }
 
 SelectPlan token_select_plan(int rows, int n_slots, lsa_budget_t bu) {
@@ -339,8 +339,8 @@ lsa_status_t run_attn(const lsa_attn_in_t* at, const int* idx, int k, void* out,
   if (p.n_split > 1) {
     const size_t nm = static_cast<size_t>(at->B) * at->T * p.n_split * at->Hq;
     uint8_t* w = static_cast<uint8_t*>(ws);
-    a.part_o = reinterpret_cast<float*>(w);
-    w += align_up(nm * at->d_v * 4, 256);
+    a.part_o = reinterpret_cast<uint16_t*>(w);
+    w += align_up(nm * at->d_v * 2, 256);
     a.part_m = reinterpret_cast<float*>(w);
     w += align_up(nm * 4, 256);
     a.part_l = reinterpret_cast<float*>(w);

@@ -299,7 +299,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           l_run > 0.f ? (m_run + log2f(l_run)) * 0.69314718055994530942f : -INFINITY;
   } else {
     const long long prow = (static_cast<long long>(r) * a.n_split + split) * a.Hq + h;
-    float* po = a.part_o + prow * DV + vp * C::kVN;
+    uint16_t* po = a.part_o + prow * DV + vp * C::kVN;
+    const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
 #pragma unroll 1
     for (int c0 = 0; c0 < C::kVN; c0 += 32) {
       uint32_t ov[32];
@@ -308,12 +309,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_wait();
       }
       if (write_row) {
-        float4* dst = reinterpret_cast<float4*>(po + c0);
+        uint32_t pkd[16];
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-          dst[q] = have ? make_float4(__uint_as_float(ov[4 * q]), __uint_as_float(ov[4 * q + 1]),
-                                      __uint_as_float(ov[4 * q + 2]), __uint_as_float(ov[4 * q + 3]))
-                        : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int i = 0; i < 32; i += 2) {
+          const float o0 = have ? __uint_as_float(ov[i]) * inv_l : 0.f;
+          const float o1 = have ? __uint_as_float(ov[i + 1]) * inv_l : 0.f;
+          const __nv_bfloat162 v2 = __floats2bfloat162_rn(o0, o1);
+          pkd[i >> 1] = *reinterpret_cast<const uint32_t*>(&v2);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(po + c0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) dst[q] = make_uint4(pkd[4 * q], pkd[4 * q + 1], pkd[4 * q + 2], pkd[4 * q + 3]);
       }
     }
     if (vp == 0 && write_row) {
@@ -373,7 +379,7 @@ constexpr int kOffSend = kOffX + 2 * kXBytes;       // outgoing partial scores (
 constexpr int kOffTag = kOffSend + kXBytes;         // [2][2][128] u64 tagged max slots + [2][128] u64 sums
 constexpr int kOffMask = kOffTag + (4 * 128 + 2 * 128) * 8;
 constexpr int kOffBars = kOffMask + kStages * 8;
-constexpr int kNumBars = 2 * kStages + 10;
+constexpr int kNumBars = 2 * kStages + 11;
 constexpr int kOffMisc = kOffBars + kNumBars * 8;
 constexpr size_t kSmem = 1024 + kOffMisc + 16;
 static_assert(kOffBars % 8 == 0, "mbarriers need 8-byte alignment");
@@ -421,17 +427,9 @@ __device__ __forceinline__ bool get_tagged(const volatile unsigned long long* sl
   return true;
 }
 
-__device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
-
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mla_pair_kernel(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUtensorMap tm_kg,
-                    const AttnArgs a) {
+                    const __grid_constant__ CUtensorMap tm_q, const AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sStage = base;
@@ -451,6 +449,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   uint64_t* q_ready = x_full + 2;
   uint64_t* send_full = q_ready + 1;  // the outgoing buffer is written
   uint64_t* send_free = send_full + 1;  // the bulk copy has read it
+  uint64_t* q_full = send_free + 1;     // q chunks staged in shared memory
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -482,6 +481,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mbar_init(q_ready, kSoftThreads);
     mbar_init(send_full, kSoftThreads);
     mbar_init(send_free, 1);
+    mbar_init(q_full, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -494,11 +494,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   cluster_sync_all();   // the partner's barriers are initialised before any remote arrive
+  // Second cluster phase: q is staged in the exchange buffers, so the partner
+  // may copy scores into them only after this CTA has moved q into TMEM. The
+  // softmax threads arrive after that move and wait before their first send;
+  // the other warps never touch those buffers and arrive right away.
   const uint32_t tmem = *tmem_slot;
   const uint32_t tO = tmem + kColO, tQ = tmem + kColQ, tS = tmem + kColS, tP = tmem + kColP;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer --
+    if (lane == 0) {
+      // q rows [r Hq, r Hq + 128) x this CTA's chunks, 128-byte swizzled, into the exchange buffers
+      mbar_arrive_expect_tx(q_full, nq * 16384);
+      for (int j = 0; j < nq; ++j) tma_load_2d(sX + j * 16384, &tm_q, q_full, (q_chunk0 + j) * 64, r * a.Hq);
+    }
+    __syncwarp();
+    cluster_arrive_release();
     prefetch_tmap(&tm_kt);
     prefetch_tmap(&tm_kg);
     const int row0 = b * a.L_max;
@@ -567,7 +578,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
       }
     }
+    cluster_wait_acquire();
   } else if (warp == 1) {
+    cluster_arrive_release();
     // ---------------------------------------------------------- MMA issuer --
     if (lane == 0 && nblk > 0) {
       const uint32_t idesc_qk = make_idesc(1, 1, 128, BN, 0, 0);
@@ -607,6 +620,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (ok) issue_pv(nblk - 1);
     }
     __syncwarp();
+    cluster_wait_acquire();
   } else {
     // ------------------------------------------------- softmax / epilogue --
     const int quarter = warp & 3;
@@ -614,30 +628,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int h = quarter * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     bool ok = true;
-    // q row h -> TMEM columns (two bf16 per column, k ascending); the two
-    // threads of a head take alternate 64-column chunks
-    {
-      const uint8_t* src = reinterpret_cast<const uint8_t*>(a.q + (static_cast<long long>(r) * a.Hq + h) * 576 +
-                                                            q_chunk0 * 64);
-      uint4 qv[3][8];
-#pragma unroll
-      for (int jj = 0; jj < 3; ++jj) {
-        const int j = 2 * jj + half;
-#pragma unroll
-        for (int t = 0; t < 8; ++t)
-          qv[jj][t] = (j < nq && h < a.Hq) ? ldg_nc_v4(src + j * 128 + 16 * t) : make_uint4(0u, 0u, 0u, 0u);
-      }
+    // q row h -> TMEM columns (two bf16 per column, k ascending) from the
+    // swizzled staging tiles; the two threads of a head take alternate chunks.
+    // Rows h >= Hq hold finite values of other rows (or zeros) and are never written out.
+    ok = __all_sync(0xffffffffu, wait_ph<false>(q_full, 0, a.status, abort_flag));
+    if (ok) {
 #pragma unroll
       for (int jj = 0; jj < 3; ++jj) {
         const int j = 2 * jj + half;
         if (j < nq) {
+          const uint4* row = reinterpret_cast<const uint4*>(sX + j * 16384 + h * 128);
           uint32_t v[32];
 #pragma unroll
           for (int t = 0; t < 8; ++t) {
-            v[4 * t] = qv[jj][t].x;
-            v[4 * t + 1] = qv[jj][t].y;
-            v[4 * t + 2] = qv[jj][t].z;
-            v[4 * t + 3] = qv[jj][t].w;
+            const uint4 w = row[t ^ (h & 7)];
+            v[4 * t] = w.x;
+            v[4 * t + 1] = w.y;
+            v[4 * t + 2] = w.z;
+            v[4 * t + 3] = w.w;
           }
           tmem_st32(tQ + lane_base + j * 32, v);
         }
@@ -646,6 +654,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(q_ready);
     }
+    cluster_arrive_release();   // this CTA's exchange buffers are free
+    cluster_wait_acquire();     // and so are the partner's
     const uint32_t col_off = static_cast<uint32_t>(half * 32);
     const int swz = h & 7;   // unit t of this thread's half-row sits at unit t ^ swz
     const uint32_t peer_x = mapa_shared(smem_u32(sX), peer);
@@ -686,7 +696,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     };
     float m_run = -INFINITY, l_part = 0.f;   // log2 domain; l_part: this thread's columns
     uint32_t sv_cur[32], sv_nxt[32];
-    if (nblk > 0) ok = fetch_send(0, sv_cur);
+    if (ok && nblk > 0) ok = fetch_send(0, sv_cur);
     for (int blk = 0; ok && blk < nblk; ++blk) {
       const int s = blk % kStages, i = blk & 1;
       // Block blk + 1's partial leaves before block blk's softmax: the
@@ -805,41 +815,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int t = 0; t < 32; ++t) ov[t] = 0u;
         }
-        const float f = final_out ? inv_l : 1.f;
+        const float f = inv_l;   // final output and split partials are both normalised
         float4* trow = reinterpret_cast<float4*>(tile + lane * 36);
 #pragma unroll
         for (int t = 0; t < 8; ++t)
           trow[t] = make_float4(__uint_as_float(ov[4 * t]) * f, __uint_as_float(ov[4 * t + 1]) * f,
                                 __uint_as_float(ov[4 * t + 2]) * f, __uint_as_float(ov[4 * t + 3]) * f);
         __syncwarp();
-        if (final_out) {
-          // 8 rows per instruction, 64 bytes (32 bf16) per row
+        // 8 rows per instruction, 64 bytes (32 bf16) per row
 #pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            const int rr = t * 8 + (lane >> 2), seg = lane & 3;
-            const int hh = quarter * 32 + rr;
-            const float4* srcp = reinterpret_cast<const float4*>(tile + rr * 36 + seg * 8);
-            const float4 v0 = srcp[0], v1 = srcp[1];
-            const __nv_bfloat162 b0 = __floats2bfloat162_rn(v0.x, v0.y), b1 = __floats2bfloat162_rn(v0.z, v0.w);
-            const __nv_bfloat162 b2 = __floats2bfloat162_rn(v1.x, v1.y), b3 = __floats2bfloat162_rn(v1.z, v1.w);
-            if (hh < a.Hq) {
-              uint16_t* dstp = a.out + (static_cast<long long>(r) * a.Hq + hh) * 512 + rank * 256 + c0 + seg * 8;
-              *reinterpret_cast<uint4*>(dstp) =
-                  make_uint4(*reinterpret_cast<const uint32_t*>(&b0), *reinterpret_cast<const uint32_t*>(&b1),
-                             *reinterpret_cast<const uint32_t*>(&b2), *reinterpret_cast<const uint32_t*>(&b3));
-            }
-          }
-        } else {
-          // 4 rows per instruction, 128 bytes (32 fp32) per row
-#pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            const int rr = t * 4 + (lane >> 3), seg = lane & 7;
-            const int hh = quarter * 32 + rr;
-            const float4 v = *reinterpret_cast<const float4*>(tile + rr * 36 + seg * 4);
-            if (hh < a.Hq) {
-              const long long prow = (static_cast<long long>(r) * a.n_split + split) * a.Hq + hh;
-              *reinterpret_cast<float4*>(a.part_o + prow * 512 + rank * 256 + c0 + seg * 4) = v;
-            }
+        for (int t = 0; t < 4; ++t) {
+          const int rr = t * 8 + (lane >> 2), seg = lane & 3;
+          const int hh = quarter * 32 + rr;
+          const float4* srcp = reinterpret_cast<const float4*>(tile + rr * 36 + seg * 8);
+          const float4 v0 = srcp[0], v1 = srcp[1];
+          const __nv_bfloat162 b0 = __floats2bfloat162_rn(v0.x, v0.y), b1 = __floats2bfloat162_rn(v0.z, v0.w);
+          const __nv_bfloat162 b2 = __floats2bfloat162_rn(v1.x, v1.y), b3 = __floats2bfloat162_rn(v1.z, v1.w);
+          if (hh < a.Hq) {
+            const long long orow = final_out ? static_cast<long long>(r) * a.Hq + hh
+                                             : (static_cast<long long>(r) * a.n_split + split) * a.Hq + hh;
+            uint16_t* dstp = (final_out ? a.out : a.part_o) + orow * 512 + rank * 256 + c0 + seg * 8;
+            *reinterpret_cast<uint4*>(dstp) =
+                make_uint4(*reinterpret_cast<const uint32_t*>(&b0), *reinterpret_cast<const uint32_t*>(&b1),
+                           *reinterpret_cast<const uint32_t*>(&b2), *reinterpret_cast<const uint32_t*>(&b3));
           }
         }
         __syncwarp();
@@ -880,12 +878,13 @@ cudaError_t launch(const AttnMaps& m, const AttnArgs& a, cudaStream_t stream) {
   cfg.attrs = nullptr;
   cfg.numAttrs = 0;
   void* args[] = {const_cast<CUtensorMap*>(&m.k_tile), const_cast<CUtensorMap*>(&m.k_rows),
-                  const_cast<AttnArgs*>(&a)};
+                  const_cast<CUtensorMap*>(&m.q), const_cast<AttnArgs*>(&a)};
   return cudaLaunchKernelExC(&cfg, fn, args);
 }
 }  // namespace mla
 
-// Merge KV-split partials: m* = max m_s; o = sum O_s 2^(m_s - m*) / sum l_s 2^(m_s - m*).
+// Merge KV-split partials (o_s = O_s / l_s in bf16, with m_s and l_s):
+//   f_s = l_s 2^(m_s - m*),  m* = max m_s;  o = sum f_s o_s / sum f_s.
 __global__ void __launch_bounds__(128) combine_kernel(const AttnArgs a) {
   __shared__ float s_f[64];
   __shared__ float s_den;
@@ -913,9 +912,9 @@ __global__ void __launch_bounds__(128) combine_kernel(const AttnArgs a) {
     float den = 0.f;
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
-      const float f = l[q] > 0.f ? exp2f(m[q] - M) : 0.f;
+      const float f = l[q] > 0.f ? l[q] * exp2f(m[q] - M) : 0.f;
       if (lane + 32 * q < 64) s_f[lane + 32 * q] = f;
-      den += l[q] * f;
+      den += f;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
@@ -931,11 +930,11 @@ __global__ void __launch_bounds__(128) combine_kernel(const AttnArgs a) {
 #pragma unroll 4
   for (int sidx = 0; sidx < ns; ++sidx) {
     const float f = s_f[sidx];
-    const float4 o = *reinterpret_cast<const float4*>(a.part_o + (base + static_cast<long long>(sidx) * a.Hq) * a.d_v + c);
-    acc[0] = fmaf(o.x, f, acc[0]);
-    acc[1] = fmaf(o.y, f, acc[1]);
-    acc[2] = fmaf(o.z, f, acc[2]);
-    acc[3] = fmaf(o.w, f, acc[3]);
+    const uint2 o = *reinterpret_cast<const uint2*>(a.part_o + (base + static_cast<long long>(sidx) * a.Hq) * a.d_v + c);
+    acc[0] = fmaf(__uint_as_float(o.x << 16), f, acc[0]);
+    acc[1] = fmaf(__uint_as_float(o.x & 0xFFFF0000u), f, acc[1]);
+    acc[2] = fmaf(__uint_as_float(o.y << 16), f, acc[2]);
+    acc[3] = fmaf(__uint_as_float(o.y & 0xFFFF0000u), f, acc[3]);
   }
   const float inv = s_den > 0.f ? 1.f / s_den : 0.f;
   const __nv_bfloat162 v01 = __floats2bfloat162_rn(acc[0] * inv, acc[1] * inv);

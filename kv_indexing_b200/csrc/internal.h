@@ -104,7 +104,7 @@ struct AttnArgs {
   int n_split, blocks_per_split;
   uint16_t* out;          // [rows, Hq, d_v] bf16
   float* lse;             // [rows, Hq] or null
-  float* part_o;          // [rows, n_split, Hq, d_v]
+  uint16_t* part_o;       // [rows, n_split, Hq, d_v] bf16, each split normalised by its own sum
   float* part_m;          // [rows, n_split, Hq]
   float* part_l;          // [rows, n_split, Hq]
   int* status;            // per-device status word
