@@ -153,6 +153,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   uint32_t tmem_cols = 32;
   while (tmem_cols < static_cast<uint32_t>(NACC * N)) tmem_cols <<= 1;
+  if (threadIdx.x == 0 && it_begin < it_end) {
+    // the first group's sequence length gates the first key load: start fetching it now
+    const long long grp0 = it_begin / a.n_tiles;
+    const int b0 = a.gather ? static_cast<int>(grp0 / a.T) : static_cast<int>(grp0 / a.G);
+    asm volatile("prefetch.global.L1 [%0];" ::"l"(a.seq_len + b0));
+  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -423,14 +429,20 @@ size_t indexer_smem_bytes(int d, bool fp8, int N, int stages, int nbuf_b) {
   return 1024 + stages * 128 * row + nbuf_b * N * row + 4 * kEpiWG * N * 4 + (2 * stages + 12) * 8 + 16;
 }
 
+// The key ring is what keeps HBM busy (bytes in flight per SM); a second
+// query buffer only hides the reload at a query-group change, so it is kept
+// only when it costs no key stage.
 void indexer_pick_pipeline(int d, bool fp8, int N, int* stages, int* nbuf_b) {
   const size_t kMax = 232448;
-  int nb = 2;
-  if (indexer_smem_bytes(d, fp8, N, 3, 2) > kMax) nb = 1;
-  int s = 8;
-  while (s > 2 && indexer_smem_bytes(d, fp8, N, s, nb) > kMax) --s;
-  *stages = s;
-  *nbuf_b = nb;
+  const int kMaxStages = 4;   // measured: deeper key rings only add queueing latency at the HBM read ceiling
+  auto fit = [&](int nb) {
+    int s = kMaxStages;
+    while (s > 2 && indexer_smem_bytes(d, fp8, N, s, nb) > kMax) --s;
+    return s;
+  };
+  const int s2 = fit(2), s1 = fit(1);
+  *nbuf_b = s2 >= s1 ? 2 : 1;
+  *stages = s2 >= s1 ? s2 : s1;
 }
 
 int indexer_n_acc(int N) { return 4 * N <= 512 ? 4 : 2; }
