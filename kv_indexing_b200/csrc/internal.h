@@ -77,6 +77,7 @@ struct SelectPlan {
   int C, seg, cand_cap;
   bool final_in_smem;
   bool grid;              // grid-cooperative launch (rows * C CTAs co-resident)
+  bool cluster;           // one thread-block cluster of C CTAs per row (no workspace)
 };
 
 // d_bound: an upper bound on the dynamic budget of any row (k - sink - window for

@@ -6,23 +6,21 @@
 // Per query row: sink tokens [0, min(S, pos+1)), the window (the W most recent
 // visible tokens not already in the sink), then the top D = k - |sink| - |window|
 // dynamic candidates by (score descending, index ascending), written in
-// ascending index order, then -1 padding. The same kernel selects pages for
+// ascending index order, then -1 padding. The same kernels select pages for
 // Hierarchical Indexing (forced sink/window pages + the top pages of the
 // dynamic region, all ascending) and the fine token set over recalled pages.
 //
-// Algorithm (one launch, no clusters): scores map to order-preserving uint32
-// keys (-inf -> 0 = not a candidate, -0 -> +0). C CTAs split a row's dynamic
-// range into contiguous segments; each thread holds up to 16 consecutive keys
-// in registers. A CTA finds the exact key of its local D-th best candidate by
-// radix select over 13-bit digits of (key - segment min): the digits span the
-// segment's actual key range, so the counts spread over the histogram instead
-// of piling into a few exponent bins, and two passes usually resolve it. It
-// writes its local top-D (key, slot) list, in slot order, to the workspace.
-// Any element of the row's top-D is in its segment's top-D, so the last CTA of
-// the row to finish (a per-row arrival counter) runs the same exact select over
-// the concatenated lists (32 per thread) and writes the final row. Ties go to
-// the lower slot at both levels, so the result equals the definition exactly.
-// Oversized segments or merges fall back to a shared/global-memory radix select.
+// Scores map to order-preserving uint32 keys (-inf -> 0 = not a candidate,
+// -0 -> +0); ties go to the lower slot, so every path equals the definition
+// exactly. Three launch shapes, chosen by select_plan:
+//   cluster  rows of <= 8 x 16384 dynamic slots: one thread-block cluster per
+//            row, keys in shared memory, agreement through DSMEM and cluster
+//            barriers (select_cluster_kernel; no workspace)
+//   grid     longer rows when rows x CTAs fit the GPU at once: one cooperative
+//            launch, agreement through per-row blocks in global memory
+//            (select_grid_kernel)
+//   two-level otherwise: each CTA keeps its segment's local top-D candidates,
+//            the last CTA of the row merges them (select_kernel)
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -734,14 +732,14 @@ __device__ __noinline__ void publish_ctas(GridRow* G, unsigned C, unsigned def, 
 // Ordered emission of the selected keys of this CTA (keys in shared memory,
 // warp-striped: element w*32*kRL + 32*j + lane). Two rolled passes: per-warp
 // counts, then positions from per-stripe ballots.
-template <class F>
+template <int R, class F>
 __device__ __forceinline__ uint32_t smem_emit(const uint32_t* keys, const Thr& t, Shared& sh, F&& emit) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const uint32_t lt = (1u << lane) - 1u;
-  const int base = warp * 32 * kRL + lane;
+  const int base = warp * 32 * R + lane;
   uint32_t n_gt = 0u, n_eq = 0u;
 #pragma unroll 4
-  for (int j = 0; j < kRL; ++j) {
+  for (int j = 0; j < R; ++j) {
     const uint32_t k = keys[base + 32 * j];
     n_gt += __popc(__ballot_sync(0xffffffffu, k != 0u && (t.all || k > t.thr)));
     n_eq += __popc(__ballot_sync(0xffffffffu, k != 0u && !t.all && k == t.thr));
@@ -761,7 +759,7 @@ __device__ __forceinline__ uint32_t smem_emit(const uint32_t* keys, const Thr& t
   }
   uint32_t eq_run = 0u;
 #pragma unroll 2
-  for (int j = 0; j < kRL; ++j) {
+  for (int j = 0; j < R; ++j) {
     const uint32_t k = keys[base + 32 * j];
     const uint32_t gtm = __ballot_sync(0xffffffffu, k != 0u && (t.all || k > t.thr));
     const bool is_eq = k != 0u && !t.all && k == t.thr;
@@ -1042,7 +1040,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_grid_kernel(const SelectAr
   int* dyn_out = out + pl.dyn_off + off;
   const long long prow = static_cast<long long>(r) * a.M;
   const bool hier = a.mode == kSelectHierTokens;
-  const uint32_t n_mine = smem_emit(keys, t, sh, [&](uint32_t p, int e) {
+  const uint32_t n_mine = smem_emit<kRL>(keys, t, sh, [&](uint32_t p, int e) {
     const int slot = my_lo + e;
     dyn_out[p] = hier ? __ldg(a.pages + prow + slot / a.P) * a.P + slot % a.P : slot;
   });
@@ -1057,6 +1055,425 @@ __global__ void __launch_bounds__(kThreads, 1) select_grid_kernel(const SelectAr
   }
 }
 
+
+// ------------------------------------------------------------ cluster path --
+// One thread-block cluster of C <= 8 CTAs per row, each holding up to 16384
+// consecutive dynamic slots' keys in shared memory. The CTAs agree on the
+// exact D-th key through distributed shared memory and hardware cluster
+// barriers: (1) every CTA broadcasts its max key and candidate count into
+// every CTA's slots; (2) each builds a 2048-bin histogram of
+// (max - key) >> 13 and every CTA sums the cluster's histograms to find the
+// boundary bin; (3) each lists its keys in that bin and every CTA resolves the
+// exact key (and the tie count) from all lists, then the per-CTA output
+// offsets; (4) each CTA writes its selections in index order. If the window
+// of the histogram holds fewer than D keys, or a boundary list overflows, all
+// CTAs take three exact radix rounds over the full key instead (the decision
+// is made from the same cluster-wide data in every CTA, so the barriers stay
+// uniform). No global workspace and no spin waits: only barriers.
+constexpr int kClusterMax = 8;
+constexpr int kRC = 32;                         // keys per thread
+constexpr int kCtaKeys = kThreads * kRC;        // 16384 slots per CTA
+constexpr int kListCapC = 512;                  // boundary-bin keys per CTA
+enum { kXMax = 0, kXCnt = 1, kXIn = 2, kXDef = 3, kXLen = 4, kXGt = 5, kXEq = 6, kXSlots = 7 };
+
+__device__ __forceinline__ uint4 ld_cluster_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+// Thread t < C writes v into slot [kind][c] of cluster CTA t.
+__device__ __forceinline__ void cluster_broadcast(uint32_t* xs, int kind, int c, int C, uint32_t v) {
+  if (static_cast<int>(threadIdx.x) < C)
+    st_cluster_u32(mapa_shared(smem_u32(xs + kind * kClusterMax + c), threadIdx.x), v);
+}
+
+// Sum over the cluster of h[0, nb) (each CTA's copy; nb <= 4 * kThreads) into
+// the local dst: one 16-byte load per CTA per thread, all in flight together.
+__device__ __forceinline__ void cluster_sum(const uint32_t* h, int nb, int C, uint32_t* dst) {
+  const int i = threadIdx.x * 4;
+  if (i >= nb) return;
+  const uint32_t a0 = smem_u32(h) + 4u * i;
+  uint4 v[kClusterMax];
+#pragma unroll
+  for (int cc = 0; cc < kClusterMax; ++cc)
+    v[cc] = cc < C ? ld_cluster_v4(mapa_shared(a0, cc)) : make_uint4(0u, 0u, 0u, 0u);
+  uint4 sum = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+  for (int cc = 0; cc < kClusterMax; ++cc) {
+    sum.x += v[cc].x;
+    sum.y += v[cc].y;
+    sum.z += v[cc].z;
+    sum.w += v[cc].w;
+  }
+  *reinterpret_cast<uint4*>(dst + i) = sum;
+}
+
+// Per-CTA output offsets and tie shares from per-CTA (greater, equal) counts:
+// CTA cc takes gt[cc] + take[cc] where ties go to the lower CTAs first.
+__device__ __forceinline__ void cluster_offsets(const uint32_t* gt, const uint32_t* eq, int C, uint32_t need_eq,
+                                                int c, uint32_t* off, uint32_t* take, uint32_t* total) {
+  uint32_t run = 0u, eq_before = 0u;
+  for (int cc = 0; cc < C; ++cc) {
+    const uint32_t tk = need_eq > eq_before ? min(need_eq - eq_before, eq[cc]) : 0u;
+    if (cc == c) {
+      *off = run;
+      *take = tk;
+    }
+    run += gt[cc] + tk;
+    eq_before += eq[cc];
+  }
+  *total = run;
+}
+
+// Inclusive scan of one value per thread, inlined (cluster path).
+__device__ __noinline__ uint32_t scan_incl(uint32_t v, uint32_t* tmp, uint32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) tmp[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t w = lane < kWarps ? tmp[lane] : 0u;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    if (lane < kWarps) tmp[lane] = w;
+  }
+  __syncthreads();
+  const uint32_t res = x + (warp > 0 ? tmp[warp - 1] : 0u);
+  if (total) *total = tmp[kWarps - 1];
+  __syncthreads();
+  return res;
+}
+
+// Bin of a local histogram h[0, PER * kThreads) where the running count from
+// bin 0 (FROM_TOP = false) or from the last bin reaches `need`: *bin and the
+// count strictly before it (*above). Uniform result in every thread.
+template <int PER, bool FROM_TOP>
+__device__ __noinline__ void find_bin_c(const uint32_t* h, uint32_t need, Shared& sh, uint32_t* bin,
+                                           uint32_t* above) {
+  constexpr int nb = PER * kThreads;
+  const int tid = threadIdx.x;
+  uint32_t vals[PER];
+  uint32_t local = 0u;
+#pragma unroll
+  for (int q = 0; q < PER; ++q) {
+    const int bb = FROM_TOP ? nb - 1 - (PER * tid + q) : PER * tid + q;
+    vals[q] = h[bb];
+    local += vals[q];
+  }
+  const uint32_t incl = scan_incl(local, sh.tmp, nullptr);
+  const uint32_t excl = incl - local;
+  if (excl < need && need <= incl) {
+    uint32_t run = excl;
+    bool done = false;
+#pragma unroll
+    for (int q = 0; q < PER; ++q) {
+      if (!done && run + vals[q] >= need) {
+        sh.bin = FROM_TOP ? nb - 1 - (PER * tid + q) : PER * tid + q;
+        sh.above = run;
+        done = true;
+      }
+      run += vals[q];
+    }
+  }
+  __syncthreads();
+  *bin = static_cast<uint32_t>(sh.bin);
+  *above = sh.above;
+  __syncthreads();
+}
+
+// Element e of a CTA's segment sits at keys[e + (e >> 5)]: thread t owns the
+// 32 consecutive elements [32 t, 32 t + 32) at keys[33 t .. 33 t + 31], so both
+// the warp-coalesced fill and the per-thread passes are free of bank conflicts.
+__device__ __forceinline__ int skew(int e) { return e + (e >> 5); }
+
+__global__ void __launch_bounds__(kThreads, 1) select_cluster_kernel(const SelectArgs a) {
+  const int C = static_cast<int>(gridDim.x);
+  const int c = static_cast<int>(cluster_ctarank());
+  const int r = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  __shared__ Shared sh;
+  __shared__ unsigned s_cnt;
+  extern __shared__ uint32_t dsm[];
+  uint32_t* keys = dsm;                              // [kCtaKeys + kCtaKeys / 32] skewed
+  uint32_t* histA = keys + kCtaKeys + kCtaKeys / 32; // [2048]  read by the cluster
+  uint32_t* fbh = histA + 2048;                      // [2048]  fallback rounds, read by the cluster
+  uint32_t* list = fbh + 2048;                       // [kListCapC] read by the cluster
+  uint32_t* xs = list + kListCapC;                   // [kXSlots][kClusterMax] broadcast slots
+  uint32_t* sub = xs + kXSlots * kClusterMax;        // [kSubHist][kWHStride] local
+  uint32_t* lists = sub + kSubHist * kWHStride;      // [kClusterMax][kListCapC] local copies of every list
+
+  const Plan pl = make_plan(a, r);                   // identical in every CTA of the cluster
+  int* out = a.out + static_cast<long long>(r) * a.out_len;
+  if (!pl.valid) {
+    if (c == 0)
+      for (int i = tid; i < a.out_len; i += kThreads) out[i] = -1;
+    return;   // the whole cluster returns before touching shared memory of another CTA
+  }
+  cluster_arrive_release();   // this CTA has started: its shared memory may be written by the others
+  const uint32_t D = static_cast<uint32_t>(pl.D);
+  const int len = pl.dyn_hi - pl.dyn_lo;
+  const int seg = (len + C - 1) / C;
+  int my_lo = pl.dyn_lo + c * seg;
+  if (my_lo > pl.dyn_hi) my_lo = pl.dyn_hi;
+  const int my_n = min(pl.dyn_hi, my_lo + seg) - my_lo;
+  const float* row = a.scores + static_cast<long long>(r) * a.row_stride + my_lo;
+
+  // ---- (1) keys (coalesced fill), local max and count; broadcast
+  uint32_t nz = 0u, mx = 0u;
+  {
+    const int e0 = warp * 32 * kRC + lane;
+    float f[kRC];
+#pragma unroll
+    for (int j = 0; j < kRC; ++j) f[j] = e0 + 32 * j < my_n ? __ldg(row + e0 + 32 * j) : -INFINITY;
+#pragma unroll
+    for (int j = 0; j < kRC; ++j) {
+      const uint32_t k = score_key(f[j]);
+      keys[skew(e0 + 32 * j)] = k;
+      nz += k != 0u ? 1u : 0u;
+      mx = max(mx, k);
+    }
+  }
+  {
+    uint4* z = reinterpret_cast<uint4*>(sub);
+    for (int i = tid; i < kSubHist * kWHStride / 4; i += kThreads) z[i] = make_uint4(0u, 0u, 0u, 0u);
+  }
+  block_cnt_min_max(nz, 0xFFFFFFFFu, mx, sh);        // also orders the fill before the per-thread passes
+  cluster_wait_acquire();     // every CTA of the cluster has started
+  cluster_broadcast(xs, kXMax, c, C, sh.mx);
+  cluster_broadcast(xs, kXCnt, c, C, sh.cnt);
+  cluster_sync_all();
+
+  const uint32_t* kv = keys + 33 * tid;   // this thread's 32 consecutive elements
+
+  uint32_t kmax = 0u, total = 0u;
+  for (int cc = 0; cc < C; ++cc) {
+    kmax = max(kmax, xs[kXMax * kClusterMax + cc]);
+    total += xs[kXCnt * kClusterMax + cc];
+  }
+  Thr t{0u, 0u, false};
+  uint32_t my_off = 0u;
+  if (total <= D || D == 0u) {
+    // every candidate is taken (or none): offsets are candidate-count prefixes
+    t.all = D != 0u;
+    if (!t.all) t.thr = 0xFFFFFFFFu;
+    for (int cc = 0; cc < c && t.all; ++cc) my_off += xs[kXCnt * kClusterMax + cc];
+  } else {
+    bool radix = false;
+    // ---- (2) window histogram of (max - key) >> 13: bin 0 holds the largest keys
+    {
+      uint32_t* h = sub + (warp % kSubHist) * kWHStride;
+      uint32_t nin = 0u;
+#pragma unroll 4
+      for (int j = 0; j < kRC; ++j) {
+        const uint32_t d = (kmax - kv[j]) >> kRangeShift;
+        if (kv[j] != 0u && d < 2048u) {
+          ++nin;
+          atomicAdd(&h[d], 1u);
+        }
+      }
+      uint32_t my_in = 0u;
+      scan_incl(nin, sh.tmp, &my_in);                // barrier: sub-histograms complete
+      for (int bin = tid; bin < 2048; bin += kThreads)
+        histA[bin] = sub[bin] + sub[kWHStride + bin] + sub[2 * kWHStride + bin] + sub[3 * kWHStride + bin];
+      cluster_broadcast(xs, kXIn, c, C, my_in);
+    }
+    cluster_sync_all();
+    uint32_t total_in = 0u;
+    for (int cc = 0; cc < C; ++cc) total_in += xs[kXIn * kClusterMax + cc];
+    radix = total_in < D;
+    uint32_t b1 = 0u, need1 = 0u;
+    if (!radix) {
+      cluster_sum(histA, 2048, C, sh.hist);
+      __syncthreads();
+      uint32_t above = 0u;
+      find_bin_c<2048 / kThreads, false>(sh.hist, D, sh, &b1, &above);
+      need1 = D - above;
+      // ---- (3) list this CTA's keys in the boundary bin (as max - key)
+      if (tid == 0) s_cnt = 0u;
+      __syncthreads();
+      uint32_t nd = 0u;
+#pragma unroll 4
+      for (int j = 0; j < kRC; ++j) {
+        const uint32_t rel = kmax - kv[j];
+        const uint32_t d = rel >> kRangeShift;
+        if (kv[j] != 0u && d <= b1) {
+          if (d < b1) {
+            ++nd;
+          } else {
+            const unsigned p = atomicAdd(&s_cnt, 1u);
+            if (p < kListCapC) list[p] = rel;
+          }
+        }
+      }
+      uint32_t my_def = 0u;
+      scan_incl(nd, sh.tmp, &my_def);
+      cluster_broadcast(xs, kXDef, c, C, my_def);
+      cluster_broadcast(xs, kXLen, c, C, s_cnt);
+    }
+    cluster_sync_all();
+    if (!radix)
+      for (int cc = 0; cc < C; ++cc) radix = radix || xs[kXLen * kClusterMax + cc] > static_cast<uint32_t>(kListCapC);
+    if (!radix) {
+      // copy every CTA's list here (16-byte loads, all in flight), then the
+      // exact key: histogram of the low 13 bits of (max - key)
+      {
+        constexpr int kV = kListCapC / 4;                    // uint4 per list
+        const uint32_t l0 = smem_u32(list);
+        uint4 v[kClusterMax * kV / kThreads];
+#pragma unroll
+        for (int q = 0; q < kClusterMax * kV / kThreads; ++q) {
+          const int g = tid + q * kThreads, cc = g / kV, u = g % kV;
+          v[q] = (cc < C && 4u * u < xs[kXLen * kClusterMax + cc]) ? ld_cluster_v4(mapa_shared(l0 + 16u * u, cc))
+                                                                  : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int q = 0; q < kClusterMax * kV / kThreads; ++q)
+          reinterpret_cast<uint4*>(lists)[tid + q * kThreads] = v[q];
+      }
+      {
+        uint4* z = reinterpret_cast<uint4*>(sh.hist);
+        for (int i = tid; i < (1 << kRangeShift) / 4; i += kThreads) z[i] = make_uint4(0u, 0u, 0u, 0u);
+      }
+      __syncthreads();
+      for (int cc = 0; cc < C; ++cc) {
+        const uint32_t n = xs[kXLen * kClusterMax + cc];
+        for (uint32_t i = tid; i < n; i += kThreads)
+          atomicAdd(&sh.hist[lists[cc * kListCapC + i] & ((1u << kRangeShift) - 1u)], 1u);
+      }
+      __syncthreads();
+      uint32_t b2 = 0u, above2 = 0u;
+      find_bin_c<(1 << kRangeShift) / kThreads, false>(sh.hist, need1, sh, &b2, &above2);
+      const uint32_t thr_rel = (b1 << kRangeShift) | b2;
+      const uint32_t need_eq = need1 - above2;
+      // per CTA: keys strictly above the exact key, and ties equal to it
+      if (warp < C) {
+        const uint32_t n = xs[kXLen * kClusterMax + warp];
+        uint32_t lo = 0u, eq = 0u;
+        for (uint32_t i = lane; i < n; i += 32) {
+          const uint32_t rel = lists[warp * kListCapC + i];
+          lo += rel < thr_rel ? 1u : 0u;
+          eq += rel == thr_rel ? 1u : 0u;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          lo += __shfl_xor_sync(0xffffffffu, lo, o);
+          eq += __shfl_xor_sync(0xffffffffu, eq, o);
+        }
+        if (lane == 0) {
+          sh.red[0][warp] = xs[kXDef * kClusterMax + warp] + lo;
+          sh.red[1][warp] = eq;
+        }
+      }
+      __syncthreads();
+      uint32_t tot = 0u;
+      cluster_offsets(sh.red[0], sh.red[1], C, need_eq, c, &my_off, &t.need_eq, &tot);
+      t.thr = kmax - thr_rel;
+    } else {
+      // ---- fallback: three exact radix rounds over the full key
+      uint32_t prefix = 0u, mask = 0u, need = D;
+      for (int pass = 0; pass < 3; ++pass) {
+        const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+        const int nb = pass == 2 ? 1024 : 2048;
+        const uint32_t dmask = static_cast<uint32_t>(nb - 1);
+        if (pass > 0) cluster_sync_all();           // the previous round's histogram has been read
+        for (int i = tid; i < nb; i += kThreads) fbh[i] = 0u;
+        __syncthreads();
+#pragma unroll 4
+        for (int j = 0; j < kRC; ++j)
+          if (kv[j] != 0u && (kv[j] & mask) == prefix) atomicAdd(&fbh[(kv[j] >> shift) & dmask], 1u);
+        cluster_sync_all();
+        cluster_sum(fbh, nb, C, sh.hist);
+        __syncthreads();
+        uint32_t bin = 0u, above = 0u;
+        if (nb == 2048)
+          find_bin_c<2048 / kThreads, true>(sh.hist, need, sh, &bin, &above);
+        else
+          find_bin_c<1024 / kThreads, true>(sh.hist, need, sh, &bin, &above);
+        prefix |= bin << shift;
+        mask |= dmask << shift;
+        need -= above;
+      }
+      uint32_t gt = 0u, eq = 0u;
+#pragma unroll 4
+      for (int j = 0; j < kRC; ++j) {
+        gt += (kv[j] != 0u && kv[j] > prefix) ? 1u : 0u;
+        eq += (kv[j] != 0u && kv[j] == prefix) ? 1u : 0u;
+      }
+      uint32_t my_gt = 0u, my_eq = 0u;
+      scan_incl(gt, sh.tmp, &my_gt);
+      scan_incl(eq, sh.tmp, &my_eq);
+      cluster_broadcast(xs, kXGt, c, C, my_gt);
+      cluster_broadcast(xs, kXEq, c, C, my_eq);
+      cluster_sync_all();
+      uint32_t tot = 0u;
+      cluster_offsets(xs + kXGt * kClusterMax, xs + kXEq * kClusterMax, C, need, c, &my_off, &t.need_eq, &tot);
+      t.thr = prefix;
+    }
+  }
+
+  // ---- (4) this CTA's selections in index order: per-thread counts, two scans
+  uint32_t n_gt = 0u, n_eq = 0u;
+#pragma unroll 4
+  for (int j = 0; j < kRC; ++j) {
+    const bool cand = kv[j] != 0u;
+    n_gt += (cand && (t.all || kv[j] > t.thr)) ? 1u : 0u;
+    n_eq += (cand && !t.all && kv[j] == t.thr) ? 1u : 0u;
+  }
+  uint32_t eq_tot = 0u;
+  const uint32_t eq_before = scan_incl(n_eq, sh.tmp, &eq_tot) - n_eq;      // ties in lower elements of this CTA
+  const uint32_t take = t.need_eq > eq_before ? min(t.need_eq - eq_before, n_eq) : 0u;
+  uint32_t n_mine = 0u;
+  uint32_t pos = scan_incl(n_gt + take, sh.tmp, &n_mine) - (n_gt + take);
+  int* dyn_out = out + pl.dyn_off + my_off;
+  const long long prow = static_cast<long long>(r) * a.M;
+  const bool hier = a.mode == kSelectHierTokens;
+  if (n_gt + take > 0u) {
+    uint32_t taken = 0u;
+#pragma unroll 4
+    for (int j = 0; j < kRC; ++j) {
+      const uint32_t k = kv[j];
+      bool s = false;
+      if (k != 0u) {
+        if (t.all || k > t.thr) {
+          s = true;
+        } else if (k == t.thr && taken < take) {
+          s = true;
+          ++taken;
+        }
+      }
+      if (s) {
+        const int slot = my_lo + 32 * tid + j;
+        dyn_out[pos++] = hier ? __ldg(a.pages + prow + slot / a.P) * a.P + slot % a.P : slot;
+      }
+    }
+  }
+  if (c == C - 1) {
+    // the last segment ends the dynamic block: its end is the selected count
+    const int n_sel = static_cast<int>(my_off + n_mine);
+    for (int i = tid; i < pl.lead_a_n; i += kThreads) out[i] = pl.lead_a_lo + i;
+    for (int i = tid; i < pl.lead_b_n; i += kThreads) out[pl.lead_a_n + i] = pl.lead_b_lo + i;
+    const int tr0 = pl.dyn_off + n_sel;
+    for (int i = tid; i < pl.trail_n; i += kThreads) out[tr0 + i] = pl.trail_lo + i;
+    for (int i = tr0 + pl.trail_n + tid; i < a.out_len; i += kThreads) out[i] = -1;
+  }
+  cluster_sync_all();   // no CTA leaves while another may still read its lists or histograms
+}
+
 }  // namespace
 
 SelectPlan select_plan(int rows, int n_slots, int d_bound, int num_sms) {
@@ -1065,6 +1482,13 @@ SelectPlan select_plan(int rows, int n_slots, int d_bound, int num_sms) {
   constexpr int kSegMax = 32768;            // fallback: keys per CTA in shared memory
   SelectPlan p{};
   auto seg_of = [&](int C) { return (n_slots + C - 1) / C; };
+  // cluster path: one cluster of up to 8 CTAs per row, any number of rows
+  if (n_slots <= kClusterMax * kCtaKeys) {
+    p.cluster = true;
+    p.C = std::max(1, (n_slots + kCtaKeys - 1) / kCtaKeys);
+    p.seg = seg_of(p.C);
+    return p;
+  }
   // grid-cooperative path: register-sized segments, one CTA per SM, all co-resident
   const int Cg = std::max(1, (n_slots + kLocalRegs - 1) / kLocalRegs);
   int Cgrid = Cg;
@@ -1090,6 +1514,7 @@ SelectPlan select_plan(int rows, int n_slots, int d_bound, int num_sms) {
 }
 
 size_t select_ws_bytes(int rows, const SelectPlan& p) {
+  if (p.cluster) return 0;
   if (p.grid) return grid_blocks_bytes(rows) + grid_row_bytes(p.C) * rows;
   const size_t n = static_cast<size_t>(rows) * p.C * p.cand_cap;
   return ((n * 8 + rows * 4 + 255) / 256) * 256;
@@ -1098,6 +1523,27 @@ size_t select_ws_bytes(int rows, const SelectPlan& p) {
 cudaError_t launch_select(const SelectArgs& a0, const SelectPlan& p, void* ws, cudaStream_t stream) {
   SelectArgs a = a0;
   const int rows = a.B * a.T;
+  if (p.cluster) {
+    const size_t smem = static_cast<size_t>(kCtaKeys + kCtaKeys / 32 + 2048 + 2048 + kListCapC +
+                                            kXSlots * kClusterMax + kSubHist * kWHStride + kClusterMax * kListCapC) * 4;
+    const void* fn = reinterpret_cast<const void*>(&select_cluster_kernel);
+    cudaError_t e = set_max_smem(fn, smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.C, rows, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = p.C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    void* args[] = {&a};
+    return cudaLaunchKernelExC(&cfg, fn, args);
+  }
   if (p.grid) {
     a.grid_ws = ws;
     a.grid_row_bytes = grid_row_bytes(p.C);

@@ -86,14 +86,17 @@ def test_workspace_checks_and_sizes():
     n_ext = L.workspace_size(L.LSA_OP_INDEX_FLAT, indexer=ii, budget=(2048, 64, 960), scores_external=True)
     assert n - n_ext == 8 * 131072 * 4                     # the score buffer moves out of the workspace
     sel = L.workspace_size(L.LSA_OP_SELECT, budget=(2048, 64, 960), B=8, T=1, L_max=131072)
-    assert sel == n_ext > 0                                # the rest is selection scratch
+    assert sel == n_ext == 0                               # rows of <= 128K keys select in cluster shared memory
     st = lib.lsa_index_flat(ctypes.byref(ii), L.Budget(2048, 64, 960), 16, None, 256, n - 1, None)
     assert st == L.LSA_ERR_WORKSPACE
-    st = lib.lsa_select_streaming(16, 16, 8, 1, 131072, L.Budget(2048, 64, 960), 16, 256, sel - 1, None)
+    big = L.workspace_size(L.LSA_OP_SELECT, budget=(2048, 64, 960), B=2, T=1, L_max=1 << 20)
+    assert big > 0                                         # longer rows need selection scratch
+    st = lib.lsa_select_streaming(16, 16, 2, 1, 1 << 20, L.Budget(2048, 64, 960), 16, 256, big - 1, None)
     assert st == L.LSA_ERR_WORKSPACE
     hi = L.workspace_size(L.LSA_OP_INDEX_HIER, indexer=_indexer(B=2, L_max=1 << 20), budget=(2048, 64, 960),
                           P=64, M=256)
-    assert hi > 2 * (1 << 14) * 4 + 2 * 256 * 4 + 2 * 256 * 64 * 4
+    # page scores + recalled pages + fine scores; 16K-candidate selections need no scratch
+    assert hi == 2 * (1 << 14) * 4 + 2 * 256 * 4 + 2 * 256 * 64 * 4
 
 
 def test_hier_parameter_validation():

@@ -63,9 +63,10 @@ def test_select_negative_scores_and_empty_rows():
     assert (got[0, 0] == -1).all() and (got[0, 1] == -1).all()
 
 
-@pytest.mark.parametrize("B,L_max", [(8, 131072), (2, 1 << 20)])
-def test_select_long_rows_cluster_paths(B, L_max):
-    # 128K rows use the shared-memory-cached path, 1M rows the streaming path
+@pytest.mark.parametrize("B,L_max", [(8, 131072), (3, 393216), (2, 1 << 20)])
+def test_select_long_rows_all_launch_paths(B, L_max):
+    # 128K rows: one cluster per row; 384K rows: the grid-cooperative launch
+    # (rows x CTAs fit the GPU at once); 1M rows: per-segment candidates + merge
     rng = np.random.default_rng(L_max)
     sc = rng.standard_normal((B, 1, L_max)).astype(np.float32)
     sc = np.abs(sc) + np.float32(3.0)
