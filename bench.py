@@ -9,7 +9,15 @@ unless --workload says otherwise. Inputs are seeded synthetic data resident in
 HBM; L2 is flushed (256 MiB write) between timed steps, outside the timed events.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME]
+                    [--workload NAME] [--fp8]
+
+Workloads (kv_indexing_b200.inputs.WORKLOADS): flat_decode_128k (default, the
+headline), hier_decode_1m (hierarchical indexing at 1M tokens; page pooling
+timed once, outside the step), cli_group_256k / cli_group_256k_flat (one
+indexing pass feeding two layers), prefill_64k (4096 causal queries; --fp8 for
+e4m3 indexer inputs). Long KV caches for timing are drawn on the device with
+torch's seeded generator; the indexer inputs come from the seeded host
+generator (needles included).
 
 Prints one JSON line (rank 0). Under torchrun each rank runs its own batch
 (weak scaling, no data-path collective); times are device times, max over ranks.
@@ -44,6 +52,7 @@ def parse():
     p.add_argument("--seed", type=int, default=1)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--fp8", action="store_true", help="prefill: e4m3 indexer keys and queries")
     return p.parse_args()
 
 
@@ -91,6 +100,27 @@ def kernel_traffic(name: str):
     except OSError:
         return None
     return ent["dram_bytes_per_launch"] if sha == ent["source_sha256"] else None
+
+
+# ---------------------------------------------------------------------------
+# multi-rank plumbing (one process per GPU; weak scaling, no data-path collective)
+# ---------------------------------------------------------------------------
+
+
+def rank_seed(seed: int, rank: int) -> int:
+    """Each rank times its own independent batch."""
+    return seed + 1000 * rank
+
+
+def max_over_ranks(x: float, dev, pg) -> float:
+    """Whole-job time = the slowest rank's device time."""
+    if not pg:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], device=dev, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
 
 
 # ---------------------------------------------------------------------------
@@ -226,6 +256,203 @@ def workload_config(w, **extra):
 
 
 # ---------------------------------------------------------------------------
+# other workloads: a generic stage timer over one CUDA graph per step
+# ---------------------------------------------------------------------------
+
+
+def time_stages(torch, stages, K, warmup, flush, dev, pg):
+    """stages: [(name, fn(stream))]. One graph per step with external events
+    between the stages; L2 flushed between steps, outside the events."""
+    import torch.distributed as dist
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(max(3, warmup)):
+        flush()
+        for _, fn in stages:
+            fn(stream)
+    torch.cuda.synchronize()
+    n = len(stages)
+    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n + 1)]
+    g = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(stream)
+    with torch.cuda.graph(g, stream=cap, capture_error_mode="relaxed"):
+        s = torch.cuda.current_stream(dev)
+        ev[0].record(s)
+        for i, (_, fn) in enumerate(stages):
+            fn(s)
+            ev[i + 1].record(s)
+    torch.cuda.synchronize()
+    for _ in range(3):
+        flush()
+        g.replay()
+    torch.cuda.synchronize()
+    per = [[] for _ in range(n)]
+    tot = []
+    if pg:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(str(torch.cuda.get_device_properties(dev).uuid)) as clk:
+        for _ in range(K):
+            flush()
+            g.replay()
+            torch.cuda.synchronize()
+            for i in range(n):
+                per[i].append(ev[i].elapsed_time(ev[i + 1]))
+            tot.append(ev[0].elapsed_time(ev[n]))
+    torch.cuda.synchronize()
+    if pg:
+        dist.barrier()
+    total_ms = max_over_ranks(float(sum(tot)), dev, pg)
+    del g
+    return {name: 1000 * sum(per[i]) / K for i, (name, _) in enumerate(stages)}, total_ms / K, clk.summary()
+
+
+def device_bf16_normal(torch, shape, seed, dev):
+    """Seeded N(0,1) bf16 drawn on the device (timing inputs for long KV caches)."""
+    g = torch.Generator(device=dev)
+    g.manual_seed(int(seed))
+    return torch.randn(shape, generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+
+
+def run_workload(args, w, rank, world, dev, pg):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from kv_indexing_b200 import inputs as I
+    from kv_indexing_b200 import lsa as L
+
+    seed = rank_seed(args.seed, rank)
+    x = I.make_indexer_inputs(w, seed)
+
+    def up(arr, kind):
+        t = torch.from_numpy(np.ascontiguousarray(arr).view(np.int16) if kind == "bf16" else arr)
+        t = t.view(torch.bfloat16) if kind == "bf16" else t
+        return t.to(dev)
+
+    q, k, wt, sl = up(x["q_idx"], "bf16"), up(x["k_idx"], "bf16"), up(x["w"], "f32"), up(x["seq_len"], "i32")
+    B, T = w.B, w.T
+    budget = (w.k, w.sink, w.window)
+    layers = []
+    for li in range(w.n_layers):
+        qa = device_bf16_normal(torch, (B, T, w.Hq, w.d_qk), 7919 * seed + 2 * li, dev)
+        kv = device_bf16_normal(torch, (B, w.L, w.d_qk), 7919 * seed + 2 * li + 1, dev)
+        layers.append({"q": qa, "kv": kv, "scale": w.scale, "d_v": w.d_v})
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def flush():
+        flush_buf.random_(0, 255)
+
+    peaks, peak_src = measured_peaks()
+    idx = torch.empty((B, T, w.k), dtype=torch.int32, device=dev)
+    outs = [torch.empty((B, T, w.Hq, w.d_v), dtype=torch.bfloat16, device=dev) for _ in range(w.n_layers)]
+    extra = {}
+    ai = L.attn_in(layers[0]["q"], sl, w.scale, kv=layers[0]["kv"], d_v=w.d_v)
+    attn_ws = torch.empty(max(256, L.workspace_size(L.LSA_OP_SPARSE_ATTN, attn=ai, budget=(w.k, 0, 0))),
+                          dtype=torch.uint8, device=dev)
+
+    def attn_stage(li):
+        lay = layers[li]
+        return lambda s: L.lsa_sparse_attn(lay["q"], idx, sl, w.scale, kv=lay["kv"], d_v=w.d_v, out=outs[li],
+                                           workspace=attn_ws, stream=s)
+
+    if w.T > 1:
+        kind = "prefill"
+        qk = dict(q=q, k=k)
+        if args.fp8:
+            if "k_idx_fp8" not in x:
+                raise SystemExit(f"workload {w.name} has no e4m3 indexer inputs")
+            qk = dict(q=up(x["q_idx_fp8"], "u8").view(torch.float8_e4m3fn),
+                      k=up(x["k_idx_fp8"], "u8").view(torch.float8_e4m3fn),
+                      q_scale=up(x["q_scale"], "f32"), k_scale=up(x["k_scale"], "f32"))
+        ii = L.indexer_in(qk["q"], wt, qk["k"], sl, qk.get("q_scale"), qk.get("k_scale"))
+        ws = torch.empty(max(256, L.workspace_size(L.LSA_OP_INDEX_FLAT, indexer=ii, budget=budget)),
+                         dtype=torch.uint8, device=dev)
+        stages = [("indexer+select", lambda s: L.lsa_index_flat(qk["q"], wt, qk["k"], sl, budget,
+                                                                 q_scale=qk.get("q_scale"), k_scale=qk.get("k_scale"),
+                                                                 idx=idx, workspace=ws, stream=s)),
+                  ("attention", attn_stage(0))]
+    elif w.n_layers > 1:
+        kind = "group"
+        page_keys = L.lsa_pool_pages(k, sl, w.P) if w.P else None
+        ii = L.indexer_in(q, wt, k, sl)
+        ais = [L.attn_in(l["q"], sl, w.scale, kv=l["kv"], d_v=w.d_v) for l in layers]
+        ws = torch.empty(max(256, L.workspace_size(L.LSA_OP_LAYER_GROUP, indexer=ii, attn=ais, budget=budget,
+                                                   P=w.P, M=w.M, n_layers=w.n_layers)), dtype=torch.uint8, device=dev)
+        stages = [("group", lambda s: L.lsa_layer_group(q, wt, k, sl, budget, layers, P=w.P, M=w.M,
+                                                        page_keys=page_keys, outs=outs, idx=idx, workspace=ws,
+                                                        stream=s))]
+    else:
+        kind = "hier"
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        page_keys = torch.zeros((B, w.L // w.P, w.d), dtype=torch.bfloat16, device=dev)
+        e0.record()
+        L.lsa_pool_pages(k, sl, w.P, page_keys=page_keys)
+        e1.record()
+        torch.cuda.synchronize()
+        extra["page_pooling_once_us"] = 1000 * e0.elapsed_time(e1)
+        ii = L.indexer_in(q, wt, k, sl)
+        ws = torch.empty(max(256, L.workspace_size(L.LSA_OP_INDEX_HIER, indexer=ii, budget=budget, P=w.P, M=w.M)),
+                         dtype=torch.uint8, device=dev)
+        stages = [("hier_index", lambda s: L.lsa_index_hier(q, wt, k, sl, page_keys, w.P, w.M, budget, idx=idx,
+                                                            workspace=ws, stream=s)),
+                  ("attention", attn_stage(0))]
+
+    br, ms_per_step, clocks = time_stages(torch, stages, args.steps, args.warmup, flush, dev, pg)
+    L.lsa_device_status()
+    units = B * T * world
+    value = units / (ms_per_step / 1000.0)
+
+    # roofline of the dominant stage
+    if kind == "prefill":
+        pos = np.arange(w.L - w.T, w.L, dtype=np.float64)
+        flops = 2.0 * w.H * w.d * float(np.sum(pos + 1)) * B
+        us = br["indexer+select"]
+        peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * (2.0 if args.fp8 else 1.0)
+        roof = {"bound": "tensor", "kernel": "indexer+select call (tcgen05 score GEMM, causal tiles; top-k)",
+                "achieved": flops / (us * 1e-6) / 1e12, "peak": peak, "unit": "TFLOP/s",
+                "frac": flops / (us * 1e-6) / 1e12 / peak, "traffic": None, "algorithmic_flops_per_launch": flops,
+                "launch_us": us, "peak_source": peak_src + (" bf16 sustained x 2 (e4m3 nominal ratio)" if args.fp8
+                                                             else " bf16 sustained")}
+    elif kind == "group":
+        if w.P:
+            ib = (w.L // w.P) * w.d * 2 + w.M * w.P * w.d * 2
+        else:
+            ib = indexer_bytes_per_query(w)
+        byts = (ib + w.n_layers * attention_bytes_per_query(w)) * B * T
+        us = br["group"]
+        roof = {"bound": "hbm", "kernel": "layer-group call (one indexing pass + %d attention layers)" % w.n_layers,
+                "achieved": byts / (us * 1e-6) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": byts / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], "traffic": None,
+                "algorithmic_bytes_per_launch": byts, "launch_us": us, "peak_source": peak_src}
+    else:
+        byts = ((w.L // w.P) * w.d * 2 + w.M * w.P * w.d * 2) * B * T
+        us = br["hier_index"]
+        roof = {"bound": "hbm", "kernel": "hierarchical indexing call (page scores, recall, fine scores, top-k)",
+                "achieved": byts / (us * 1e-6) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": byts / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], "traffic": None,
+                "algorithmic_bytes_per_launch": byts, "launch_us": us, "peak_source": peak_src}
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "e4m3" if args.fp8 else "bf16",
+            "data": "synthetic (seeded N(0,1) bf16 indexer inputs with 1% needles from the host generator; "
+                    "latent KV and attention queries drawn on the device with a seeded generator)",
+            "config": workload_config(w, parallelism=f"replicas x{world} (independent batches)",
+                                      fp8_indexer=bool(args.fp8)),
+            "roofline": roof, "cpu_baseline": None, "e2e": None, "breakdown_us": br, **extra,
+            "tokens_scanned_per_s": value * w.L, "clocks": clocks,
+            "note": "extra workload line; the headline, e2e and CPU baseline are on flat_decode_128k",
+        }
+        print(json.dumps(line), flush=True)
+    if pg:
+        dist.destroy_process_group()
+    return 0
+
+
+# ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
 
@@ -254,9 +481,9 @@ def main():
         pg = True
     L.load()
     w = I.WORKLOADS[args.workload]
-    if w.P or w.n_layers > 1 or w.T > 1:
-        raise SystemExit(f"bench.py times the flat decode step; workload {w.name} is covered by the tests")
-    seed = args.seed + 1000 * rank                       # each rank its own batch
+    if w.P or w.n_layers > 1 or w.T > 1 or args.fp8:
+        return run_workload(args, w, rank, world, dev, pg)
+    seed = rank_seed(args.seed, rank)                   # each rank its own batch
     x = I.make_indexer_inputs(w, seed)
     a = I.make_attn_inputs(w, seed)
 
@@ -339,11 +566,7 @@ def main():
     if pg:
         dist.barrier()
     L.lsa_device_status()
-    total_ms = float(sum(t_step))
-    if pg:
-        tt = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(float(sum(t_step)), dev, pg)
     ms_per_step = total_ms / K
     units = B * T * world
     value = units / (ms_per_step / 1000.0)
@@ -373,11 +596,7 @@ def main():
             torch.cuda.synchronize()
             if i >= 3:
                 e2e_ms.append(e0.elapsed_time(e1))
-        em = sum(e2e_ms) / len(e2e_ms)
-        if pg:
-            tt = torch.tensor([em], device=dev, dtype=torch.float64)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            em = float(tt.item())
+        em = max_over_ranks(sum(e2e_ms) / len(e2e_ms), dev, pg)
         e2e = {"value": units / (em / 1000.0), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "ms_per_step": em,
                "note": "KV and indexer-key caches resident; per step the new queries go in and o, idx come out"}

@@ -86,6 +86,10 @@ WORKLOADS: Dict[str, Workload] = {
     "cli_group_256k": Workload(
         name="cli_group_256k", B=4, L=262144, T=1, H=64, d=128, k=2048, sink=64,
         window=960, needle_frac=0.01, P=64, M=256, n_layers=2),
+    # The same group with flat indexing (hierarchy off).
+    "cli_group_256k_flat": Workload(
+        name="cli_group_256k_flat", B=4, L=262144, T=1, H=64, d=128, k=2048, sink=64,
+        window=960, needle_frac=0.01, n_layers=2),
 }
 
 
