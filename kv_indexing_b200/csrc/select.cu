@@ -1076,14 +1076,6 @@ constexpr int kCtaKeys = kThreads * kRC;        // 16384 slots per CTA
 constexpr int kListCapC = 512;                  // boundary-bin keys per CTA
 enum { kXMax = 0, kXCnt = 1, kXIn = 2, kXDef = 3, kXLen = 4, kXGt = 5, kXEq = 6, kXSlots = 7 };
 
-__device__ __forceinline__ uint4 ld_cluster_v4(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "r"(addr)
-               : "memory");
-  return v;
-}
 __device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
