@@ -70,6 +70,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
+  pdl_trigger();
   const int tid = threadIdx.x, warp = tid >> 5;
   const int vp = blockIdx.x, split = blockIdx.y, r = blockIdx.z;
   const int b = r / a.T;
@@ -96,6 +97,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_wait();   // inputs may come from the previous kernel in the stream
   const uint32_t tmem = *tmem_slot;
   const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
   const uint32_t tO = tmem;
@@ -453,6 +455,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
+  pdl_trigger();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_ctarank();
   const uint32_t peer = rank ^ 1u;
@@ -494,6 +497,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   cluster_sync_all();   // the partner's barriers are initialised before any remote arrive
+  pdl_wait();           // q, indices and KV may come from the previous kernel in the stream
   // Second cluster phase: q is staged in the exchange buffers, so the partner
   // may copy scores into them only after this CTA has moved q into TMEM. The
   // softmax threads arrive after that move and wait before their first send;
@@ -875,17 +879,17 @@ cudaError_t launch(const AttnMaps& m, const AttnArgs& a, cudaStream_t stream) {
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = kSmem;
   cfg.stream = stream;
-  cfg.attrs = nullptr;
-  cfg.numAttrs = 0;
   void* args[] = {const_cast<CUtensorMap*>(&m.k_tile), const_cast<CUtensorMap*>(&m.k_rows),
                   const_cast<CUtensorMap*>(&m.q), const_cast<AttnArgs*>(&a)};
-  return cudaLaunchKernelExC(&cfg, fn, args);
+  return launch_pdl(fn, cfg.gridDim, cfg.blockDim, cfg.dynamicSmemBytes, stream, args);
 }
 }  // namespace mla
 
 // Merge KV-split partials (o_s = O_s / l_s in bf16, with m_s and l_s):
 //   f_s = l_s 2^(m_s - m*),  m* = max m_s;  o = sum f_s o_s / sum f_s.
 __global__ void __launch_bounds__(128) combine_kernel(const AttnArgs a) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float s_f[64];
   __shared__ float s_den;
   const int r = blockIdx.x, h = blockIdx.y;
@@ -957,7 +961,7 @@ cudaError_t launch_t(const AttnMaps& m, const AttnArgs& a, cudaStream_t stream) 
   void* args[] = {const_cast<CUtensorMap*>(&m.q), const_cast<CUtensorMap*>(&m.k_tile),
                   const_cast<CUtensorMap*>(&m.k_rows), const_cast<CUtensorMap*>(&m.v_tile),
                   const_cast<CUtensorMap*>(&m.v_rows), const_cast<AttnArgs*>(&a)};
-  return cudaLaunchKernel(fn, grid, dim3(kThreads), args, smem, stream);
+  return launch_pdl(fn, grid, dim3(kThreads), smem, stream, args);
 }
 
 }  // namespace
@@ -982,8 +986,9 @@ cudaError_t launch_attn(const AttnMaps& m, const AttnArgs& a, cudaStream_t strea
 cudaError_t launch_attn_combine(const AttnArgs& a, cudaStream_t stream) {
   if (a.n_split > 64) return cudaErrorInvalidValue;
   const dim3 grid(a.B * a.T, a.Hq);
-  combine_kernel<<<grid, a.d_v / 4 < 32 ? 32 : a.d_v / 4, 0, stream>>>(a);
-  return cudaGetLastError();
+  void* args[] = {const_cast<AttnArgs*>(&a)};
+  return launch_pdl(reinterpret_cast<const void*>(&combine_kernel), grid, dim3(a.d_v / 4 < 32 ? 32 : a.d_v / 4),
+                    0, stream, args);
 }
 
 }  // namespace lsa

@@ -146,6 +146,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
+  pdl_trigger();
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const long long per = a.n_items / gridDim.x, rem = a.n_items % gridDim.x;
   const long long it_begin = blockIdx.x * per + min(static_cast<long long>(blockIdx.x), rem);
@@ -153,12 +154,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   uint32_t tmem_cols = 32;
   while (tmem_cols < static_cast<uint32_t>(NACC * N)) tmem_cols <<= 1;
-  if (threadIdx.x == 0 && it_begin < it_end) {
-    // the first group's sequence length gates the first key load: start fetching it now
-    const long long grp0 = it_begin / a.n_tiles;
-    const int b0 = a.gather ? static_cast<int>(grp0 / a.T) : static_cast<int>(grp0 / a.G);
-    asm volatile("prefetch.global.L1 [%0];" ::"l"(a.seq_len + b0));
-  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -184,6 +179,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();   // inputs may come from the previous kernel in the stream
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
@@ -461,7 +457,7 @@ cudaError_t launch_indexer(const CUtensorMap& tm_k, const CUtensorMap& tm_q, con
   cudaError_t e = set_max_smem(fn, smem);
   if (e != cudaSuccess) return e;
   void* args[] = {const_cast<CUtensorMap*>(&tm_k), const_cast<CUtensorMap*>(&tm_q), const_cast<IndexerArgs*>(&a)};
-  return cudaLaunchKernel(fn, dim3(grid), dim3(kThreads), args, smem, stream);
+  return launch_pdl(fn, dim3(grid), dim3(kThreads), smem, stream, args);
 }
 
 }  // namespace lsa

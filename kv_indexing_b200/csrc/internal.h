@@ -130,5 +130,10 @@ int device_sm_count();
 lsa_status_t set_error(lsa_status_t st, const char* fmt, ...);
 int* device_status_ptr();
 cudaError_t set_max_smem(const void* func, size_t bytes);
+// Launch with programmatic stream serialization (plus up to two extra launch
+// attributes): the kernel may start while the previous kernel in the stream
+// finishes, and orders itself with pdl_wait before reading shared inputs.
+cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, size_t smem, cudaStream_t stream, void** args,
+                       const cudaLaunchAttribute* extra = nullptr, int n_extra = 0);
 
 }  // namespace lsa

@@ -10,12 +10,15 @@
 #include <cuda_bf16.h>
 
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace lsa {
 namespace {
 
 __global__ void __launch_bounds__(256) pool_kernel(const uint16_t* __restrict__ k, const int* __restrict__ seq_len,
                                                    int L_max, int d, int P, uint16_t* __restrict__ pk) {
+  pdl_trigger();
+  pdl_wait();
   const int b = blockIdx.y;
   const int vec_per_row = d / 8;   // 16-byte vectors per key row
   const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -56,8 +59,8 @@ cudaError_t launch_pool(const uint16_t* k, const int* seq_len, int B, int L_max,
   const long long n = static_cast<long long>(L_max / P) * (d / 8);
   const int threads = 256;
   const dim3 grid(static_cast<unsigned>((n + threads - 1) / threads), B);
-  pool_kernel<<<grid, threads, 0, stream>>>(k, seq_len, L_max, d, P, page_keys);
-  return cudaGetLastError();
+  void* args[] = {(void*)&k, (void*)&seq_len, &L_max, &d, &P, &page_keys};
+  return launch_pdl(reinterpret_cast<const void*>(&pool_kernel), grid, dim3(threads), 0, stream, args);
 }
 
 }  // namespace lsa

@@ -29,6 +29,16 @@ __device__ __forceinline__ void record_timeout(int* status) {
   if (status) atomicOr(status, kStatusTimeout);
 }
 
+// ------------------------------------------------- programmatic launch --
+// Kernels are launched with programmatic stream serialization: each one lets
+// its dependent grid launch as soon as all of its CTAs have started
+// (pdl_trigger at entry) and waits for the preceding grid to complete and
+// flush its memory (pdl_wait) before its first read of global data another
+// kernel may have written. Without a programmatic predecessor pdl_wait returns
+// at once.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---------------------------------------------------------------- mbarrier --
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");

@@ -425,6 +425,8 @@ __device__ uint32_t reg_emit(const uint32_t (&k)[R], const Thr& t, Shared& sh, F
 }
 
 __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelectArgs a) {
+  pdl_trigger();
+  pdl_wait();
   const int C = gridDim.x;
   const int c = blockIdx.x;
   const int r = blockIdx.y;
@@ -775,6 +777,8 @@ __device__ __forceinline__ uint32_t smem_emit(const uint32_t* keys, const Thr& t
 }
 
 __global__ void __launch_bounds__(kThreads, 1) select_grid_kernel(const SelectArgs a) {
+  pdl_trigger();
+  pdl_wait();
   const unsigned C = gridDim.x;
   const int c = blockIdx.x;
   const int r = blockIdx.y;
@@ -1194,6 +1198,8 @@ __device__ __noinline__ void find_bin_c(const uint32_t* h, uint32_t need, Shared
 __device__ __forceinline__ int skew(int e) { return e + (e >> 5); }
 
 __global__ void __launch_bounds__(kThreads, 1) select_cluster_kernel(const SelectArgs a) {
+  pdl_trigger();
+  pdl_wait();
   const int C = static_cast<int>(gridDim.x);
   const int c = static_cast<int>(cluster_ctarank());
   const int r = blockIdx.y;
@@ -1521,20 +1527,13 @@ cudaError_t launch_select(const SelectArgs& a0, const SelectPlan& p, void* ws, c
     const void* fn = reinterpret_cast<const void*>(&select_cluster_kernel);
     cudaError_t e = set_max_smem(fn, smem);
     if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(p.C, rows, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = p.C;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
     void* args[] = {&a};
-    return cudaLaunchKernelExC(&cfg, fn, args);
+    return launch_pdl(fn, dim3(p.C, rows, 1), dim3(kThreads, 1, 1), smem, stream, args, attr, 1);
   }
   if (p.grid) {
     a.grid_ws = ws;
@@ -1572,7 +1571,7 @@ cudaError_t launch_select(const SelectArgs& a0, const SelectPlan& p, void* ws, c
   e = set_max_smem(fn, smem);
   if (e != cudaSuccess) return e;
   void* args[] = {&a};
-  return cudaLaunchKernel(fn, dim3(p.C, rows), dim3(kThreads), args, smem, stream);
+  return launch_pdl(fn, dim3(p.C, rows), dim3(kThreads), smem, stream, args);
 }
 
 }  // namespace lsa
