@@ -520,7 +520,8 @@ def main():
         L.lsa_select_streaming(scores, sl, budget, idx=idx, workspace=sel_ws, stream=stream)
 
     def k_attn():
-        L.lsa_sparse_attn(qa, idx, sl, w.scale, kv=kv, d_v=w.d_v, out=out, workspace=attn_ws, stream=stream)
+        L.lsa_sparse_attn(qa, idx, sl, w.scale, kv=kv, d_v=w.d_v, out=out, workspace=attn_ws, stream=stream,
+                          stream_budget=budget)
 
     def flush():
         flush_buf.random_(0, 255)   # touch 256 MiB (> 126 MB L2)
@@ -549,7 +550,8 @@ def main():
             L.lsa_select_streaming(scores, sl, budget, idx=idx, workspace=sel_ws, stream=s)
             if stage_events:
                 ev[2].record(s)
-            L.lsa_sparse_attn(qa, idx, sl, w.scale, kv=kv, d_v=w.d_v, out=out, workspace=attn_ws, stream=s)
+            L.lsa_sparse_attn(qa, idx, sl, w.scale, kv=kv, d_v=w.d_v, out=out, workspace=attn_ws, stream=s,
+                              stream_budget=budget)
             ev[3].record(s)
         torch.cuda.synchronize()
         for _ in range(3):
@@ -608,7 +610,8 @@ def main():
             e0.record(stream)
             dq.copy_(hq, non_blocking=True); dw.copy_(hw, non_blocking=True); dqa.copy_(hqa, non_blocking=True)
             ix = L.lsa_index_flat(dq, dw, k, sl, budget, idx=idx, workspace=flat_ws, stream=stream)
-            L.lsa_sparse_attn(dqa, ix, sl, w.scale, kv=kv, d_v=w.d_v, out=out, workspace=attn_ws, stream=stream)
+            L.lsa_sparse_attn(dqa, ix, sl, w.scale, kv=kv, d_v=w.d_v, out=out, workspace=attn_ws, stream=stream,
+                              stream_budget=budget)
             ho.copy_(out, non_blocking=True); hi.copy_(idx, non_blocking=True)
             e1.record(stream)
             torch.cuda.synchronize()

@@ -114,6 +114,15 @@ typedef struct lsa_attn_in {
   const void* v;
   int64_t k_row_stride;
   int64_t v_row_stride;
+  /* Optional layout promise (0 / 0 or -1 / -1 = none): every index row starts
+   * with the streaming prefix lsa_select_streaming writes for this sink and
+   * window -- the sink tokens [0, min(sink, pos+1)) ascending, then the window
+   * tokens up to pos ascending (LSA abstract (1), SI). The MLA kernel then
+   * computes those entries instead of reading them, and its work on them may
+   * overlap the kernel in the same stream that writes the rest of idx: that
+   * kernel must not read or write this call's workspace or outputs. A row
+   * that breaks the promise gives undefined results. */
+  int32_t stream_sink, stream_window;
 } lsa_attn_in_t;
 
 typedef enum lsa_op {

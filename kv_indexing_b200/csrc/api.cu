@@ -141,6 +141,14 @@ lsa_status_t check_attn(const lsa_attn_in_t* at, int k) {
   if (mla && !alias) return fail(LSA_ERR_UNSUPPORTED, "d_qk=576/d_v=512 requires v == k (MLA latent rows)");
   if (!(at->scale > 0.f) || !std::isfinite(at->scale)) return fail(LSA_ERR_INVALID_ARG, "scale must be finite and > 0");
   if (k < 1 || k > 8192) return fail(LSA_ERR_UNSUPPORTED, "index row length %d outside [1, 8192]", k);
+  if (at->stream_sink < -1 || at->stream_window < -1)
+    return fail(LSA_ERR_INVALID_ARG, "stream_sink / stream_window below -1");
+  if (at->stream_sink > 0 || at->stream_window > 0) {
+    if (at->stream_sink < 0 || at->stream_window < 0 ||
+        static_cast<long long>(at->stream_sink) + at->stream_window > k)
+      return fail(LSA_ERR_INVALID_ARG, "streaming prefix (sink %d + window %d) must fit the index row of %d",
+                  at->stream_sink, at->stream_window, k);
+  }
   if (static_cast<long long>(at->B) * at->T * at->Hq >= (1ll << 31))
     return fail(LSA_ERR_UNSUPPORTED, "too many query rows");
   return LSA_OK;
@@ -333,6 +341,9 @@ lsa_status_t run_attn(const lsa_attn_in_t* at, const int* idx, int k, void* out,
   a.k_stride = at->k_row_stride; a.v_stride = at->v_row_stride;
   a.sep_v = !(at->v == at->k && at->v_row_stride == at->k_row_stride);
   a.n_split = p.n_split; a.blocks_per_split = p.bps;
+  a.stream_sink = at->stream_sink > 0 ? at->stream_sink : 0;
+  a.stream_window = at->stream_window > 0 ? at->stream_window : 0;
+  a.seq_len = at->seq_len;
   a.out = static_cast<uint16_t*>(out);
   a.lse = lse;
   a.status = device_status_ptr();
@@ -486,7 +497,9 @@ lsa_status_t lsa_workspace_size(lsa_op_t op, const lsa_op_args_t* args, size_t* 
         if ((s = check_attn(&args->attn[i], args->budget.k)) != LSA_OK) return s;
         at = std::max(at, attn_ws_bytes(&args->attn[i], args->budget.k));
       }
-      *bytes = idx_bytes + std::max(ix, at);
+      // the attention's region is separate: with the streaming prefix promise its
+      // first splits may run while the group's selection still reads its scratch
+      *bytes = idx_bytes + ix + at;
       return LSA_OK;
     }
   }
@@ -600,6 +613,7 @@ lsa_status_t lsa_layer_group(const lsa_indexer_in_t* in, const void* page_keys, 
   uint8_t* w = static_cast<uint8_t*>(workspace);
   int32_t* idx_buf = idx ? idx : reinterpret_cast<int32_t*>(w);
   w += align_up(static_cast<size_t>(in->B) * in->T * budget.k * 4, 256);
+  uint8_t* attn_ws = w + (P ? hier_ws_bytes(in, P, M, budget, false) : flat_ws_bytes(in, budget, false));
   if (P) {
     if ((s = run_hier(in, page_keys, P, M, budget, idx_buf, nullptr, w, st)) != LSA_OK) return s;
   } else {
@@ -612,7 +626,10 @@ lsa_status_t lsa_layer_group(const lsa_indexer_in_t* in, const void* page_keys, 
   }
   for (int i = 0; i < n_layers; ++i) {
     float* lse = lse_outs ? lse_outs[i] : nullptr;
-    if ((s = run_attn(&layers[i], idx_buf, budget.k, outs[i], lse, w, st)) != LSA_OK) return s;
+    lsa_attn_in_t lay = layers[i];   // the group's own selection wrote idx: its streaming prefix is known
+    lay.stream_sink = budget.sink;
+    lay.stream_window = budget.window;
+    if ((s = run_attn(&lay, idx_buf, budget.k, outs[i], lse, attn_ws, st)) != LSA_OK) return s;
   }
   return LSA_OK;
 }

@@ -70,7 +70,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-  pdl_trigger();
   const int tid = threadIdx.x, warp = tid >> 5;
   const int vp = blockIdx.x, split = blockIdx.y, r = blockIdx.z;
   const int b = r / a.T;
@@ -98,6 +97,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   pdl_wait();   // inputs may come from the previous kernel in the stream
+  pdl_trigger();
   const uint32_t tmem = *tmem_slot;
   const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
   const uint32_t tO = tmem;
@@ -455,11 +455,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-  pdl_trigger();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_ctarank();
   const uint32_t peer = rank ^ 1u;
-  const int split = blockIdx.y, r = blockIdx.z;
+  const int r = blockIdx.y, split = blockIdx.z;   // splits outermost: the streaming-prefix splits launch first
   const int b = r / a.T;
   const int chunk0 = rank ? 4 : 0;        // global 64-column chunk of local chunk 0
   const int nq = rank ? 4 : 5;            // q chunks held (and score chunks multiplied)
@@ -470,6 +469,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int blk0 = split * a.blocks_per_split;
   const int nblk = max(0, min(a.blocks_per_split, nblk_total - blk0));
   const int* idx_row = a.idx + static_cast<long long>(r) * a.k;
+  // Streaming prefix: with the layout promise, a split whose entries all lie
+  // in the row's sink + window prefix computes them (sink s at entry s, window
+  // token w_lo + j at entry sink_end + j) and never reads idx, so it need not
+  // wait for the kernel that writes the rest of the row.
+  bool fixed = false;
+  int f_sink_end = 0, f_wlo = 0;
+  if (a.stream_sink + a.stream_window > 0 && nblk > 0) {
+    int L = __ldg(a.seq_len + b);
+    L = L < 0 ? 0 : (L > a.L_max ? a.L_max : L);
+    const int pos = L - a.T + (r - b * a.T);
+    if (pos >= 0) {
+      f_sink_end = min(a.stream_sink, pos + 1);
+      f_wlo = max(f_sink_end, pos - a.stream_window + 1);
+      const int n_fixed = f_sink_end + (pos + 1 - f_wlo);
+      fixed = min(a.k, (blk0 + nblk) * BN) <= n_fixed;
+    }
+  }
 
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) {
@@ -497,7 +513,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   cluster_sync_all();   // the partner's barriers are initialised before any remote arrive
-  pdl_wait();           // q, indices and KV may come from the previous kernel in the stream
+  if (!fixed) pdl_wait();   // the index rows come from the previous kernel in the stream
+  pdl_trigger();
   // Second cluster phase: q is staged in the exchange buffers, so the partner
   // may copy scores into them only after this CTA has moved q into TMEM. The
   // softmax threads arrive after that move and wait before their first send;
@@ -520,7 +537,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // index entry e of block `bb`, -1 outside the split / row
     auto load_id = [&](int bb, int e) -> int {
       const int ip = (blk0 + bb) * BN + e;
-      int v = (bb < nblk && ip < a.k) ? __ldg(idx_row + ip) : -1;
+      if (bb >= nblk || ip >= a.k) return -1;
+      if (fixed) return ip < f_sink_end ? ip : f_wlo + (ip - f_sink_end);
+      const int v = __ldg(idx_row + ip);
       return v >= a.L_max ? -1 : v;
     };
     int ids_lo[kStages], ids_hi[kStages];   // entries lane and lane + 32 of the next kStages blocks
@@ -875,7 +894,7 @@ cudaError_t launch(const AttnMaps& m, const AttnArgs& a, cudaStream_t stream) {
   cudaError_t e = set_max_smem(fn, kSmem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2, a.n_split, a.B * a.T);
+  cfg.gridDim = dim3(2, a.B * a.T, a.n_split);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = kSmem;
   cfg.stream = stream;
@@ -888,8 +907,8 @@ cudaError_t launch(const AttnMaps& m, const AttnArgs& a, cudaStream_t stream) {
 // Merge KV-split partials (o_s = O_s / l_s in bf16, with m_s and l_s):
 //   f_s = l_s 2^(m_s - m*),  m* = max m_s;  o = sum f_s o_s / sum f_s.
 __global__ void __launch_bounds__(128) combine_kernel(const AttnArgs a) {
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
   __shared__ float s_f[64];
   __shared__ float s_den;
   const int r = blockIdx.x, h = blockIdx.y;

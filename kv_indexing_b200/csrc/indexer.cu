@@ -146,7 +146,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-  pdl_trigger();
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const long long per = a.n_items / gridDim.x, rem = a.n_items % gridDim.x;
   const long long it_begin = blockIdx.x * per + min(static_cast<long long>(blockIdx.x), rem);
@@ -180,6 +179,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   pdl_wait();   // inputs may come from the previous kernel in the stream
+  pdl_trigger();
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --

@@ -103,6 +103,8 @@ struct AttnArgs {
   long long k_stride, v_stride;
   int sep_v;              // V rows loaded separately (not a prefix of the K row)
   int n_split, blocks_per_split;
+  int stream_sink, stream_window;   // > 0: index rows start with this streaming prefix (computed, not read)
+  const int* seq_len;               // [B] (streaming prefix only)
   uint16_t* out;          // [rows, Hq, d_v] bf16
   float* lse;             // [rows, Hq] or null
   uint16_t* part_o;       // [rows, n_split, Hq, d_v] bf16, each split normalised by its own sum

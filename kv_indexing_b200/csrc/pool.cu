@@ -17,8 +17,8 @@ namespace {
 
 __global__ void __launch_bounds__(256) pool_kernel(const uint16_t* __restrict__ k, const int* __restrict__ seq_len,
                                                    int L_max, int d, int P, uint16_t* __restrict__ pk) {
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
   const int b = blockIdx.y;
   const int vec_per_row = d / 8;   // 16-byte vectors per key row
   const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;

@@ -30,12 +30,13 @@ __device__ __forceinline__ void record_timeout(int* status) {
 }
 
 // ------------------------------------------------- programmatic launch --
-// Kernels are launched with programmatic stream serialization: each one lets
-// its dependent grid launch as soon as all of its CTAs have started
-// (pdl_trigger at entry) and waits for the preceding grid to complete and
-// flush its memory (pdl_wait) before its first read of global data another
-// kernel may have written. Without a programmatic predecessor pdl_wait returns
-// at once.
+// Kernels are launched with programmatic stream serialization. Each waits for
+// the preceding grid to complete and flush its memory (pdl_wait) before its
+// first read of data that grid may have written, and only then lets its own
+// dependent grid launch (pdl_trigger). So when a kernel starts, everything
+// launched two or more kernels before it has completed: only the immediate
+// predecessor's outputs need the wait. Without a programmatic predecessor
+// pdl_wait returns at once.
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 

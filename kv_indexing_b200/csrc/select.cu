@@ -425,8 +425,8 @@ __device__ uint32_t reg_emit(const uint32_t (&k)[R], const Thr& t, Shared& sh, F
 }
 
 __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelectArgs a) {
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
   const int C = gridDim.x;
   const int c = blockIdx.x;
   const int r = blockIdx.y;
@@ -777,8 +777,8 @@ __device__ __forceinline__ uint32_t smem_emit(const uint32_t* keys, const Thr& t
 }
 
 __global__ void __launch_bounds__(kThreads, 1) select_grid_kernel(const SelectArgs a) {
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
   const unsigned C = gridDim.x;
   const int c = blockIdx.x;
   const int r = blockIdx.y;
@@ -1198,8 +1198,8 @@ __device__ __noinline__ void find_bin_c(const uint32_t* h, uint32_t need, Shared
 __device__ __forceinline__ int skew(int e) { return e + (e >> 5); }
 
 __global__ void __launch_bounds__(kThreads, 1) select_cluster_kernel(const SelectArgs a) {
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
   const int C = static_cast<int>(gridDim.x);
   const int c = static_cast<int>(cluster_ctarank());
   const int r = blockIdx.y;

@@ -48,7 +48,8 @@ class AttnIn(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("T", ctypes.c_int32), ("Hq", ctypes.c_int32), ("d_qk", ctypes.c_int32),
                 ("d_v", ctypes.c_int32), ("L_max", ctypes.c_int32), ("scale", ctypes.c_float),
                 ("seq_len", ctypes.c_void_p), ("q", ctypes.c_void_p), ("k", ctypes.c_void_p),
-                ("v", ctypes.c_void_p), ("k_row_stride", ctypes.c_int64), ("v_row_stride", ctypes.c_int64)]
+                ("v", ctypes.c_void_p), ("k_row_stride", ctypes.c_int64), ("v_row_stride", ctypes.c_int64),
+                ("stream_sink", ctypes.c_int32), ("stream_window", ctypes.c_int32)]
 
 
 class OpArgs(ctypes.Structure):
@@ -156,22 +157,24 @@ def indexer_in(q, w, k, seq_len, q_scale=None, k_scale=None) -> IndexerIn:
                      _ptr(q_scale) if fp8 else None, _ptr(w), _ptr(k), _ptr(k_scale) if fp8 else None)
 
 
-def attn_in(q, seq_len, scale, *, kv=None, k=None, v=None, d_v=None) -> AttnIn:
+def attn_in(q, seq_len, scale, *, kv=None, k=None, v=None, d_v=None, stream_budget=None) -> AttnIn:
     """Describe attention tensors: q [B,T,Hq,d_qk]; MLA kv [B,L_max,d_qk] (V = first d_v
-    columns) or separate k [B,L_max,d_qk], v [B,L_max,d_v]; all bf16."""
+    columns) or separate k [B,L_max,d_qk], v [B,L_max,d_v]; all bf16. stream_budget
+    (k, sink, window) promises the index rows start with that streaming prefix."""
     torch = _torch()
     _need(q, "q", torch.bfloat16, 4)
     _need(seq_len, "seq_len", torch.int32, 1)
     B, T, Hq, d_qk = q.shape
+    ss, sw = (-1, -1) if stream_budget is None else (int(stream_budget[1]), int(stream_budget[2]))
     if kv is not None:
         _need(kv, "kv", torch.bfloat16, 3)
         dv = d_v if d_v is not None else (512 if d_qk == 576 else d_qk)
         return AttnIn(B, T, Hq, d_qk, dv, kv.shape[1], float(scale), _ptr(seq_len), _ptr(q), _ptr(kv), _ptr(kv),
-                      kv.shape[2], kv.shape[2])
+                      kv.shape[2], kv.shape[2], ss, sw)
     _need(k, "k", torch.bfloat16, 3)
     _need(v, "v", torch.bfloat16, 3)
     return AttnIn(B, T, Hq, d_qk, v.shape[2], k.shape[1], float(scale), _ptr(seq_len), _ptr(q), _ptr(k), _ptr(v),
-                  k.shape[2], v.shape[2])
+                  k.shape[2], v.shape[2], ss, sw)
 
 
 def workspace_size(op: int, *, indexer: Optional[IndexerIn] = None, attn=None, budget=(1, 0, 0), P=0, M=0,
@@ -298,11 +301,13 @@ def lsa_index_hier(q, w, k, seq_len, page_keys, P, M, budget, *, idx=None, pages
 
 
 def lsa_sparse_attn(q, idx, seq_len, scale, *, kv=None, k=None, v=None, d_v=None, out=None, lse=None,
-                    workspace=None, stream=None):
-    """Sparse attention over idx [B,T,k]. Returns (out [B,T,Hq,d_v] bf16, lse or None)."""
+                    workspace=None, stream=None, stream_budget=None):
+    """Sparse attention over idx [B,T,k]. Returns (out [B,T,Hq,d_v] bf16, lse or None).
+    stream_budget (k, sink, window): idx rows come from the streaming selection with
+    that budget, so their sink/window prefix may be computed instead of read."""
     torch = _torch()
     lib = load()
-    ai = attn_in(q, seq_len, scale, kv=kv, k=k, v=v, d_v=d_v)
+    ai = attn_in(q, seq_len, scale, kv=kv, k=k, v=v, d_v=d_v, stream_budget=stream_budget)
     _need(idx, "idx", torch.int32, 3)
     if out is None:
         out = torch.empty((ai.B, ai.T, ai.Hq, ai.d_v), dtype=torch.bfloat16, device=q.device)

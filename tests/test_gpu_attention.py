@@ -100,3 +100,27 @@ def test_attention_select_all_equals_dense():
         mask[t, :256 - 8 + t + 1] = True
     ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask, scale=0.125)
     assert_attention_close(g[0], ref.permute(1, 0, 2).numpy())
+
+
+def test_attention_streaming_prefix_promise_matches_reading_idx():
+    # Index rows from the streaming selection; the attention computes their sink
+    # and window prefix itself when promised. Same indices -> identical bytes.
+    w = I.scaled(I.WORKLOADS["flat_decode_128k"], B=3, L=8192)
+    x = I.make_attn_inputs(w, 11)
+    sl = np.array([8192, 5000, 900], np.int32)
+    rng = np.random.default_rng(12)
+    sc = rng.standard_normal((3, 1, 8192)).astype(np.float32)
+    for b in range(3):
+        sc[b, 0, sl[b]:] = -np.inf
+    budget = (w.k, w.sink, w.window)
+    sl_d, q, kv = dev(sl, "i32"), dev(x["qa"], "bf16"), dev(x["kv"], "bf16")
+    idx = L.lsa_select_streaming(dev(sc, "f32"), sl_d, budget)
+    lse1 = torch.empty((3, 1, w.Hq), dtype=torch.float32, device="cuda")
+    lse2 = torch.empty_like(lse1)
+    o1, _ = L.lsa_sparse_attn(q, idx, sl_d, w.scale, kv=kv, d_v=w.d_v, lse=lse1)
+    o2, _ = L.lsa_sparse_attn(q, idx, sl_d, w.scale, kv=kv, d_v=w.d_v, lse=lse2, stream_budget=budget)
+    torch.cuda.synchronize()
+    L.lsa_device_status()
+    assert torch.equal(o1, o2) and torch.equal(lse1, lse2)
+    o, ol = oracle_attn(w, x, host(idx), sl)
+    assert_attention_close(O.bf16_to_f64(host(o2)), o)
