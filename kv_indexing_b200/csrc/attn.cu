@@ -985,11 +985,6 @@ cudaError_t launch_t(const AttnMaps& m, const AttnArgs& a, cudaStream_t stream) 
 
 }  // namespace
 
-size_t attn_smem_bytes(int d_qk, int d_v, bool sep_v) {
-  if (d_qk == 576 && d_v == 512) return mla::kSmem;
-  return ACfg<64, 64, true>::kSmem;
-}
-
 cudaError_t launch_attn(const AttnMaps& m, const AttnArgs& a, cudaStream_t stream) {
   if (a.d_qk == 576 && a.d_v == 512) {
     if (a.sep_v) return cudaErrorNotSupported;   // MLA keeps V inside the latent row

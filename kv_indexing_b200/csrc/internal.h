@@ -122,7 +122,6 @@ struct AttnMaps {
   CUtensorMap q, k_tile, k_rows, v_tile, v_rows;
 };
 
-size_t attn_smem_bytes(int d_qk, int d_v, bool sep_v);
 cudaError_t launch_attn(const AttnMaps& maps, const AttnArgs& a, cudaStream_t stream);
 cudaError_t launch_attn_combine(const AttnArgs& a, cudaStream_t stream);
 
