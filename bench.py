@@ -503,7 +503,7 @@ def main():
     scores = torch.empty((B, T, w.L), dtype=torch.float32, device=dev)
     idx = torch.empty((B, T, w.k), dtype=torch.int32, device=dev)
     out = torch.empty((B, T, w.Hq, w.d_v), dtype=torch.bfloat16, device=dev)
-    ai = L.attn_in(qa, sl, w.scale, kv=kv, d_v=w.d_v)
+    ai = L.attn_in(qa, sl, w.scale, kv=kv, d_v=w.d_v, stream_budget=budget)
     attn_ws_n = L.workspace_size(L.LSA_OP_SPARSE_ATTN, attn=ai, budget=(w.k, 0, 0))
     attn_ws = torch.empty(max(attn_ws_n, 256), dtype=torch.uint8, device=dev)
     flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)

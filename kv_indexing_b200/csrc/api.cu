@@ -173,6 +173,7 @@ FlatPlan flat_plan(int T, int H, int L_rows) {
 
 struct AttnPlan {
   int n_split, bps, nvp;
+  int fixed_blocks, fixed_splits, bps_fixed;   // streaming-prefix blocks and their own splits
 };
 
 AttnPlan attn_plan(const lsa_attn_in_t* at, int k) {
@@ -187,6 +188,24 @@ AttnPlan attn_plan(const lsa_attn_in_t* at, int k) {
   if (ns > 64) ns = 64;   // the split combine merges at most 64 partials
   p.bps = (nblk + ns - 1) / ns;
   p.n_split = (nblk + p.bps - 1) / p.bps;
+  p.fixed_blocks = p.fixed_splits = p.bps_fixed = 0;
+  // MLA with the streaming-prefix promise: the prefix splits run while the top-k
+  // still works, so the rest of the row is the critical path -- give it splits of
+  // half the size (the prefix keeps the plain size).
+  const int prefix = (at->stream_sink > 0 ? at->stream_sink : 0) + (at->stream_window > 0 ? at->stream_window : 0);
+  if (at->d_qk == 576 && prefix / bn >= 2 && p.bps >= 2) {
+    const int F = std::min(nblk, prefix / bn);
+    const int bps_d = p.bps / 2;
+    const int fs = (F + p.bps - 1) / p.bps;
+    const int ds = (nblk - F + bps_d - 1) / bps_d;
+    if (fs + ds <= 64) {
+      p.fixed_blocks = F;
+      p.fixed_splits = fs;
+      p.bps_fixed = p.bps;
+      p.bps = bps_d;
+      p.n_split = fs + ds;
+    }
+  }
   return p;
 }
 
@@ -341,6 +360,7 @@ lsa_status_t run_attn(const lsa_attn_in_t* at, const int* idx, int k, void* out,
   a.k_stride = at->k_row_stride; a.v_stride = at->v_row_stride;
   a.sep_v = !(at->v == at->k && at->v_row_stride == at->k_row_stride);
   a.n_split = p.n_split; a.blocks_per_split = p.bps;
+  a.fixed_blocks = p.fixed_blocks; a.fixed_splits = p.fixed_splits; a.bps_fixed = p.bps_fixed;
   a.stream_sink = at->stream_sink > 0 ? at->stream_sink : 0;
   a.stream_window = at->stream_window > 0 ? at->stream_window : 0;
   a.seq_len = at->seq_len;
@@ -495,7 +515,10 @@ lsa_status_t lsa_workspace_size(lsa_op_t op, const lsa_op_args_t* args, size_t* 
       size_t at = 0;
       for (int i = 0; i < args->n_layers; ++i) {
         if ((s = check_attn(&args->attn[i], args->budget.k)) != LSA_OK) return s;
-        at = std::max(at, attn_ws_bytes(&args->attn[i], args->budget.k));
+        lsa_attn_in_t lay = args->attn[i];   // as launched: with the group's streaming prefix
+        lay.stream_sink = args->budget.sink;
+        lay.stream_window = args->budget.window;
+        at = std::max(at, attn_ws_bytes(&lay, args->budget.k));
       }
       // the attention's region is separate: with the streaming prefix promise its
       // first splits may run while the group's selection still reads its scratch

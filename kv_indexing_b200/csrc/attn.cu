@@ -466,8 +466,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int q_chunk0 = rank ? 5 : 0;
 
   const int nblk_total = (a.k + BN - 1) / BN;
-  const int blk0 = split * a.blocks_per_split;
-  const int nblk = max(0, min(a.blocks_per_split, nblk_total - blk0));
+  const bool prefix_split = split < a.fixed_splits;
+  const int blk0 = prefix_split ? split * a.bps_fixed
+                                : a.fixed_blocks + (split - a.fixed_splits) * a.blocks_per_split;
+  const int nblk = max(0, prefix_split ? min(a.bps_fixed, a.fixed_blocks - blk0)
+                                       : min(a.blocks_per_split, nblk_total - blk0));
   const int* idx_row = a.idx + static_cast<long long>(r) * a.k;
   // Streaming prefix: with the layout promise, a split whose entries all lie
   // in the row's sink + window prefix computes them (sink s at entry s, window

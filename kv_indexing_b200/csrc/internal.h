@@ -103,6 +103,8 @@ struct AttnArgs {
   long long k_stride, v_stride;
   int sep_v;              // V rows loaded separately (not a prefix of the K row)
   int n_split, blocks_per_split;
+  int fixed_blocks, fixed_splits, bps_fixed;   // splits [0, fixed_splits) cover blocks [0, fixed_blocks) in
+                                               // bps_fixed-block pieces; the others blocks_per_split each
   int stream_sink, stream_window;   // > 0: index rows start with this streaming prefix (computed, not read)
   const int* seq_len;               // [B] (streaming prefix only)
   uint16_t* out;          // [rows, Hq, d_v] bf16

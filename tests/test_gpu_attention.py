@@ -104,7 +104,8 @@ def test_attention_select_all_equals_dense():
 
 def test_attention_streaming_prefix_promise_matches_reading_idx():
     # Index rows from the streaming selection; the attention computes their sink
-    # and window prefix itself when promised. Same indices -> identical bytes.
+    # and window prefix itself when promised (and splits the row differently), so
+    # both paths must match the oracle within the attention tolerance.
     w = I.scaled(I.WORKLOADS["flat_decode_128k"], B=3, L=8192)
     x = I.make_attn_inputs(w, 11)
     sl = np.array([8192, 5000, 900], np.int32)
@@ -121,6 +122,8 @@ def test_attention_streaming_prefix_promise_matches_reading_idx():
     o2, _ = L.lsa_sparse_attn(q, idx, sl_d, w.scale, kv=kv, d_v=w.d_v, lse=lse2, stream_budget=budget)
     torch.cuda.synchronize()
     L.lsa_device_status()
-    assert torch.equal(o1, o2) and torch.equal(lse1, lse2)
     o, ol = oracle_attn(w, x, host(idx), sl)
+    assert_attention_close(O.bf16_to_f64(host(o1)), o)
     assert_attention_close(O.bf16_to_f64(host(o2)), o)
+    assert np.allclose(host(lse2), ol, atol=1e-3, rtol=1e-3)
+    assert np.allclose(host(lse1), host(lse2), atol=1e-3, rtol=1e-3)
