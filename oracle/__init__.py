@@ -8,5 +8,5 @@ from .lsa_oracle import (  # noqa: F401
     bf16_to_f64, f32_to_bf16_rne, e4m3_to_f64, indexer_scores_row, indexer_scores,
     streaming_regions, top_by_score, select_streaming_row, select_streaming,
     index_flat, pool_pages, page_sets, index_hier_row, index_hier,
-    sparse_attention_row, sparse_attention, layer_group,
+    sparse_attention_row, sparse_attention, layer_group, entry_position, index_compressed,
 )

@@ -48,6 +48,13 @@ R8  Sparse attention: o[h] = sum_j softmax_j(scale * qa[h].K[idx_j]) V[idx_j]
 R9  Cross-layer indexing: one index set per query, computed once from the
     group's indexer inputs, feeds every layer of the group.
 R10 FP8 keys/queries: the value of an e4m3 code times its float32 row scale.
+R11 Compressed entries (the DSA article's "Technical Evolution": the indexer
+    picks top-k entries of compressed historical representations): entry e
+    stands for tokens [e m, e m + m) and exists once all m are cached, so the
+    query at pos sees entries e < (pos + 1) // m. Its key is given (the pages
+    name no compressor). Scores are R1 on the entry keys; the selection is
+    R3-R5 over entries, at entry position (pos + 1) // m - 1, with budget, sink
+    and window counted in entries. m = 1 is flat indexing.
 """
 from __future__ import annotations
 
@@ -346,6 +353,41 @@ def index_hier(q, w, k, page_keys, seq_len, *, P: int, M: int, budget: int,
                 bf16_to_f64(q[b, t]), np.asarray(w[b, t], np.float64), kd, pk,
                 pos, P, M, budget, sink, window)
     return idx, pages
+
+
+# ---------------------------------------------------------------------------
+# Compressed-entry indexing (DSA article, "Technical Evolution and
+# Applications": top-k over compressed historical entries; R11)
+# ---------------------------------------------------------------------------
+
+
+def entry_position(pos: int, m: int) -> int:
+    """Position of the query at token ``pos`` among entries of ``m`` tokens: the
+    last complete entry, -1 if none is complete yet (R11)."""
+    return (pos + 1) // m - 1
+
+
+def index_compressed(q, w, entry_keys, seq_len, *, m: int, budget: int, sink: int,
+                     window: int, q_scale=None, k_scale=None, fp8: bool = False):
+    """Indexing over compressed entries. entry_keys [B, L_max // m, d] (bf16 or
+    e4m3 codes); seq_len in tokens. Returns (idx [B,T,budget] entry ids, scores
+    float32 [B,T,L_max // m] with -inf at entries not yet complete)."""
+    B, T = q.shape[0], q.shape[1]
+    n_e = entry_keys.shape[1]
+    L_max = n_e * m
+    scores = np.full((B, T, n_e), NEG_INF32, dtype=np.float32)
+    idx = np.full((B, T, budget), -1, dtype=np.int32)
+    for b in range(B):
+        L = int(min(max(int(seq_len[b]), 0), L_max))
+        kd = _decode_k(entry_keys[b], None if k_scale is None else k_scale[b], fp8)
+        for t in range(T):
+            pe = entry_position(L - T + t, m)
+            if pe < 0:
+                continue
+            qd = _decode_q(q[b, t], None if q_scale is None else q_scale[b, t], fp8)
+            scores[b, t] = indexer_scores_row(qd, np.asarray(w[b, t], np.float64), kd, pe + 1)
+            idx[b, t] = select_streaming_row(scores[b, t], pe, budget, sink, window)
+    return idx, scores
 
 
 # ---------------------------------------------------------------------------

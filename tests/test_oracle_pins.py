@@ -484,3 +484,67 @@ def test_input_needles_are_planted_in_dynamic_region():
     npos = npos[npos >= 0]
     assert npos.size == w.n_needles
     assert (npos >= w.sink).all() and (npos <= w.L - 1 - w.window).all()
+
+
+# ---------------------------------------------------------------------------
+# compressed-entry indexing
+# ---------------------------------------------------------------------------
+
+
+def test_compressed_entry_one_token_equals_flat():
+    rng = np.random.default_rng(21)
+    B, T, H, d, L = 2, 3, 4, 16, 96
+    q = I.normal_bf16((B, T, H, d), rng)
+    k = I.normal_bf16((B, L, d), rng)
+    w = rng.random((B, T, H)).astype(np.float32)
+    sl = np.array([L, 70], np.int32)
+    gi, gs = O.index_compressed(q, w, k, sl, m=1, budget=24, sink=4, window=6)
+    fi, fs = O.index_flat(q, w, k, sl, budget=24, sink=4, window=6)
+    assert np.array_equal(gi, fi)
+    assert np.array_equal(gs, fs)
+
+
+def test_compressed_entry_visibility_by_membership():
+    """An entry is scored iff every token it stands for is visible."""
+    rng = np.random.default_rng(22)
+    B, T, H, d, m, n_e = 1, 9, 2, 8, 4, 12
+    q = I.normal_bf16((B, T, H, d), rng)
+    ek = I.normal_bf16((B, n_e, d), rng)
+    w = rng.random((B, T, H)).astype(np.float32)
+    sl = np.array([37], np.int32)                    # queries at tokens 28 .. 36
+    _, sc = O.index_compressed(q, w, ek, sl, m=m, budget=8, sink=1, window=2)
+    for t in range(T):
+        pos = 37 - T + t
+        for e in range(n_e):
+            complete = all(tok <= pos for tok in range(e * m, e * m + m))
+            assert np.isfinite(sc[0, t, e]) == complete, (pos, e)
+
+
+def test_compressed_entry_closed_form():
+    """Entry keys (e, 0), q = (1, 0), w = 1: score = e / sqrt(2), so the
+    dynamic block takes the highest complete entries. m = 4, token 41: entries
+    0..9 are complete; sink {0, 1}, window {7, 8, 9}, D = 2 -> {5, 6}."""
+    n_e, m = 12, 4
+    ek = np.zeros((1, n_e, 2), np.float32)
+    ek[0, :, 0] = np.arange(n_e)
+    q = np.array([[[[1.0, 0.0]]]], np.float32)
+    w = np.ones((1, 1, 1), np.float32)
+    idx, sc = O.index_compressed(bf16(q), w, bf16(ek), np.array([42], np.int32), m=m, budget=7, sink=2,
+                                 window=3)
+    assert idx[0, 0].tolist() == [0, 1, 7, 8, 9, 5, 6]
+    assert np.allclose(sc[0, 0, :10], np.arange(10) / math.sqrt(2.0), rtol=1e-6)
+    assert np.isneginf(sc[0, 0, 10:]).all()
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_compressed_entry_select_brute_force(seed):
+    rng = np.random.default_rng(300 + seed)
+    B, T, H, d, m, n_e = 1, 6, 1, 4, 8, 40
+    q = bf16(np.ones((B, T, H, d)))
+    ek = bf16(rng.integers(0, 3, size=(B, n_e, d)).astype(np.float32) * 0.5)   # many tied scores
+    w = np.ones((B, T, H), np.float32)
+    sl = np.array([n_e * m - 5], np.int32)
+    idx, sc = O.index_compressed(q, w, ek, sl, m=m, budget=12, sink=2, window=3)
+    for t in range(T):
+        pe = (int(sl[0]) - T + t + 1) // m - 1
+        assert idx[0, t].tolist() == _brute_select(sc[0, t].tolist(), pe, 12, 2, 3)
