@@ -130,18 +130,20 @@ typedef enum lsa_op {
   LSA_OP_INDEX_HIER = 1,
   LSA_OP_SELECT = 2,
   LSA_OP_SPARSE_ATTN = 3,
-  LSA_OP_LAYER_GROUP = 4
+  LSA_OP_LAYER_GROUP = 4,
+  LSA_OP_INDEX_COMPRESSED = 5
 } lsa_op_t;
 
 /* Arguments of lsa_workspace_size; fill the members the op uses. */
 typedef struct lsa_op_args {
-  const lsa_indexer_in_t* indexer; /* INDEX_FLAT, INDEX_HIER, LAYER_GROUP */
+  const lsa_indexer_in_t* indexer; /* INDEX_FLAT, INDEX_HIER, LAYER_GROUP, INDEX_COMPRESSED */
   const lsa_attn_in_t* attn;       /* SPARSE_ATTN; LAYER_GROUP: n_layers entries */
   lsa_budget_t budget;             /* INDEX_*, SELECT, LAYER_GROUP; SPARSE_ATTN uses k */
   int32_t P, M;                    /* INDEX_HIER; LAYER_GROUP (P = 0: flat) */
   int32_t n_layers;                /* LAYER_GROUP */
   int32_t B, T, L_max;             /* SELECT */
-  int32_t scores_external;         /* INDEX_FLAT: 1 if the caller passes scores_out */
+  int32_t scores_external;         /* INDEX_FLAT, INDEX_COMPRESSED: 1 if the caller passes scores_out */
+  int32_t m;                       /* INDEX_COMPRESSED: tokens per entry */
 } lsa_op_args_t;
 
 /* One-line description of a status code (static storage). */
@@ -164,6 +166,28 @@ lsa_status_t lsa_workspace_size(lsa_op_t op, const lsa_op_args_t* args, size_t* 
 lsa_status_t lsa_index_flat(const lsa_indexer_in_t* in, lsa_budget_t budget, int32_t* idx,
                             float* scores_out, void* workspace, size_t workspace_bytes,
                             lsa_stream_t stream);
+
+/* Indexing over compressed entries [DSA article, "Technical Evolution and
+ * Applications": the indexer picks the top-k of compressed historical
+ * entries]. in->k holds one key per entry, [B, L_max/m, d] (bf16, or e4m3
+ * with k_scale [B, L_max/m]); entry e stands for tokens [e m, e m + m) and
+ * the query at pos sees it once all of them are cached: (e + 1) m <= pos + 1.
+ * in->L_max and seq_len count tokens. Scores are lsa_index_flat's on the entry
+ * keys; the streaming selection runs over entries, at the query's last
+ * complete entry, with budget.k, sink and window counted in entries. The
+ * pages name no compressor: the entry keys are inputs.
+ *   m          tokens per entry: a power of 2 in [1, 128] (m = 1 is
+ *              lsa_index_flat); L_max % 128 == 0 as for every indexer call
+ *   idx        [B,T,k] int32 entry ids out, laid out as lsa_index_flat's (a
+ *              query with no complete entry gets -1 everywhere). May be NULL
+ *              (scores only; scores_out required).
+ *   scores_out [B,T,L_max/m] fp32 out, optional (-inf at entries not yet
+ *              complete); else kept in the workspace.
+ * Attention over the chosen entries is lsa_sparse_attn on the compressed KV
+ * rows [B, L_max/m, d_qk] with these idx. */
+lsa_status_t lsa_index_compressed(const lsa_indexer_in_t* in, int32_t m, lsa_budget_t budget,
+                                  int32_t* idx, float* scores_out, void* workspace,
+                                  size_t workspace_bytes, lsa_stream_t stream);
 
 /* Streaming selection alone [DSA "Dynamic Token Selector"; LSA abstract (1)]
  * over given scores [B,T,L_max] fp32 (-inf = not a candidate; NaN unsupported;
@@ -234,7 +258,14 @@ lsa_status_t lsa_sparse_attn(const lsa_attn_in_t* in, const int32_t* idx, int32_
  *   layers [n_layers] attention inputs (own q and KV per layer, same B, T,
  *          L_max and seq_len as the indexer); outs[i] [B,T,Hq,d_v] bf16;
  *   lse_outs NULL or n_layers pointers (each may be NULL);
- *   idx [B,T,k] int32 out, optional (else kept in the workspace). */
+ *   idx [B,T,k] int32 out, optional (else kept in the workspace).
+ * Consecutive MLA layers (d_qk=576, d_v=512) with the same Hq run as one
+ * attention launch (up to 4 layers each), so their work overlaps; the
+ * attention of every layer starts on its streaming-prefix entries while the
+ * selection still runs. Hence the layers' outputs must not overlap one
+ * another or idx (LSA_ERR_INVALID_ARG, checked for outs and idx). The split
+ * plan of a shared launch differs from a single lsa_sparse_attn call's, so the
+ * outputs agree with that call within rounding, not bit for bit. */
 lsa_status_t lsa_layer_group(const lsa_indexer_in_t* in, const void* page_keys, int32_t P,
                              int32_t M, lsa_budget_t budget, int32_t n_layers,
                              const lsa_attn_in_t* layers, void* const* outs,

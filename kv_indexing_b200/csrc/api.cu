@@ -176,13 +176,14 @@ struct AttnPlan {
   int fixed_blocks, fixed_splits, bps_fixed;   // streaming-prefix blocks and their own splits
 };
 
-AttnPlan attn_plan(const lsa_attn_in_t* at, int k) {
+// `layers`: layers that share the launch (their CTAs split the GPU between them).
+AttnPlan attn_plan(const lsa_attn_in_t* at, int k, int layers = 1) {
   AttnPlan p;
   const int rows = at->B * at->T;
   p.nvp = at->d_v >= 512 ? 2 : 1;
   const int bn = at->d_qk == 576 ? kAttnBNMla : kAttnBN;   // KV rows per kernel block
   const int nblk = (k + bn - 1) / bn;
-  int ns = device_sm_count() / (rows * p.nvp);
+  int ns = device_sm_count() / (rows * layers * p.nvp);
   if (ns < 1) ns = 1;
   if (ns > nblk) ns = nblk;
   if (ns > 64) ns = 64;   // the split combine merges at most 64 partials
@@ -209,12 +210,33 @@ AttnPlan attn_plan(const lsa_attn_in_t* at, int k) {
   return p;
 }
 
-size_t attn_ws_bytes(const lsa_attn_in_t* at, int k) {
-  const AttnPlan p = attn_plan(at, k);
+size_t attn_ws_bytes(const lsa_attn_in_t* at, int k, int layers = 1) {
+  const AttnPlan p = attn_plan(at, k, layers);
   if (p.n_split <= 1) return 0;
   const size_t rows = static_cast<size_t>(at->B) * at->T;
   const size_t nm = rows * p.n_split * at->Hq;
   return align_up(nm * at->d_v * 2, 256) + 2 * align_up(nm * 4, 256);
+}
+
+// Layers [i, i + n) of a group that go into one attention launch: consecutive
+// MLA layers with the same head count, at most kMaxLaunchLayers.
+int group_launch_layers(const lsa_attn_in_t* layers, int i, int n_layers) {
+  const lsa_attn_in_t& f = layers[i];
+  if (!(f.d_qk == 576 && f.d_v == 512)) return 1;
+  int n = 1;
+  while (n < kMaxLaunchLayers && i + n < n_layers && layers[i + n].d_qk == 576 && layers[i + n].d_v == 512 &&
+         layers[i + n].Hq == f.Hq)
+    ++n;
+  return n;
+}
+
+// The group's layer i as launched: its own selection wrote the index rows, so
+// their streaming prefix is known.
+lsa_attn_in_t group_layer(const lsa_attn_in_t* layers, int i, lsa_budget_t bu) {
+  lsa_attn_in_t lay = layers[i];
+  lay.stream_sink = bu.sink;
+  lay.stream_window = bu.window;
+  return lay;
 }
 
 SelectPlan token_select_plan(int rows, int n_slots, lsa_budget_t bu) {
@@ -231,6 +253,20 @@ size_t hier_ws_bytes(const lsa_indexer_in_t* in, int P, int M, lsa_budget_t bu, 
   s += std::max(select_ws_bytes(rows, page_select_plan(rows, in->L_max / P, M)),
                 select_ws_bytes(rows, token_select_plan(rows, M * P, bu)));      // selection scratch
   return s;
+}
+
+// Entries of m tokens per sequence, and the selection's entry shift log2(m).
+int entry_shift_of(int m) {
+  int sh = 0;
+  while ((1 << sh) < m) ++sh;
+  return sh;
+}
+
+size_t compressed_ws_bytes(const lsa_indexer_in_t* in, int m, lsa_budget_t bu, bool scores_external) {
+  const int rows = in->B * in->T;
+  const int n_e = in->L_max / m;
+  size_t s = scores_external ? 0 : align_up(static_cast<size_t>(rows) * n_e * 4, 256);
+  return s + select_ws_bytes(rows, token_select_plan(rows, n_e, bu));
 }
 
 size_t flat_ws_bytes(const lsa_indexer_in_t* in, lsa_budget_t bu, bool scores_external) {
@@ -270,9 +306,10 @@ lsa_status_t run_flat_scores(const lsa_indexer_in_t* in, const void* keys, int L
 
 lsa_status_t run_select(int mode, int B, int T, int L_max, const int* seq_len, const float* scores,
                         long long row_stride, int n_slots, lsa_budget_t bu, int P, int M, const int* pages,
-                        int* out, int out_len, void* sws, cudaStream_t st) {
+                        int* out, int out_len, void* sws, cudaStream_t st, int entry_shift = 0) {
   SelectArgs a{};
   a.mode = mode; a.B = B; a.T = T; a.L_max = L_max; a.seq_len = seq_len;
+  a.entry_shift = entry_shift;
   a.scores = scores; a.row_stride = row_stride; a.n_slots = n_slots;
   a.k = bu.k; a.sink = bu.sink; a.window = bu.window; a.P = P; a.M = M; a.pages = pages;
   a.out = out; a.out_len = out_len;
@@ -338,46 +375,55 @@ lsa_status_t run_hier(const lsa_indexer_in_t* in, const void* page_keys, int P, 
                     M * P, bu, P, M, pages, idx, bu.k, sws, st);
 }
 
-lsa_status_t run_attn(const lsa_attn_in_t* at, const int* idx, int k, void* out, float* lse, void* ws,
-                      cudaStream_t st) {
-  const AttnPlan p = attn_plan(at, k);
-  AttnMaps maps;
-  lsa_status_t s = make_tmap(&maps.q, at->q, false, at->d_qk, static_cast<uint64_t>(at->B) * at->T * at->Hq, 64, 128);
-  if (s != LSA_OK) return s;
-  const uint64_t kv_rows = static_cast<uint64_t>(at->B) * at->L_max;
-  if ((s = make_tmap_strided(&maps.k_tile, at->k, at->d_qk, kv_rows, at->k_row_stride, 64, kAttnBN)) != LSA_OK) return s;
-  if ((s = make_tmap_strided(&maps.k_rows, at->k, at->d_qk, kv_rows, at->k_row_stride, 64, 1)) != LSA_OK) return s;
-  if ((s = make_tmap_strided(&maps.v_tile, at->v, at->d_v, kv_rows, at->v_row_stride, 64, kAttnBN)) != LSA_OK) return s;
-  if ((s = make_tmap_strided(&maps.v_rows, at->v, at->d_v, kv_rows, at->v_row_stride, 64, 1)) != LSA_OK) return s;
-  AttnArgs a{};
-  a.B = at->B; a.T = at->T; a.Hq = at->Hq; a.L_max = at->L_max;
-  a.d_qk = at->d_qk; a.d_v = at->d_v; a.k = k;
-  a.scale_log2 = at->scale * 1.4426950408889634f;
-  a.idx = idx;
-  a.q = static_cast<const uint16_t*>(at->q);
-  a.kp = static_cast<const uint16_t*>(at->k);
-  a.vp = static_cast<const uint16_t*>(at->v);
-  a.k_stride = at->k_row_stride; a.v_stride = at->v_row_stride;
-  a.sep_v = !(at->v == at->k && at->v_row_stride == at->k_row_stride);
-  a.n_split = p.n_split; a.blocks_per_split = p.bps;
-  a.fixed_blocks = p.fixed_blocks; a.fixed_splits = p.fixed_splits; a.bps_fixed = p.bps_fixed;
-  a.stream_sink = at->stream_sink > 0 ? at->stream_sink : 0;
-  a.stream_window = at->stream_window > 0 ? at->stream_window : 0;
-  a.seq_len = at->seq_len;
-  a.out = static_cast<uint16_t*>(out);
-  a.lse = lse;
-  a.status = device_status_ptr();
-  if (p.n_split > 1) {
-    const size_t nm = static_cast<size_t>(at->B) * at->T * p.n_split * at->Hq;
-    uint8_t* w = static_cast<uint8_t*>(ws);
-    a.part_o = reinterpret_cast<uint16_t*>(w);
-    w += align_up(nm * at->d_v * 2, 256);
-    a.part_m = reinterpret_cast<float*>(w);
-    w += align_up(nm * 4, 256);
-    a.part_l = reinterpret_cast<float*>(w);
+// Attention of n layers (1 <= n <= kMaxLaunchLayers) over the same index rows
+// in one launch; layer i writes outs[i] / lses[i] and keeps its split
+// partials in wss[i] (attn_ws_bytes(&ats[i], k, n) bytes each).
+lsa_status_t run_attn(const lsa_attn_in_t* ats, int n, const int* idx, int k, void* const* outs, float* const* lses,
+                      uint8_t* const* wss, cudaStream_t st) {
+  const AttnPlan p = attn_plan(&ats[0], k, n);
+  AttnMaps maps[kMaxLaunchLayers];
+  AttnArgs args[kMaxLaunchLayers];
+  for (int i = 0; i < n; ++i) {
+    const lsa_attn_in_t* at = &ats[i];
+    AttnMaps& m = maps[i];
+    lsa_status_t s = make_tmap(&m.q, at->q, false, at->d_qk, static_cast<uint64_t>(at->B) * at->T * at->Hq, 64, 128);
+    if (s != LSA_OK) return s;
+    const uint64_t kv_rows = static_cast<uint64_t>(at->B) * at->L_max;
+    if ((s = make_tmap_strided(&m.k_tile, at->k, at->d_qk, kv_rows, at->k_row_stride, 64, kAttnBN)) != LSA_OK) return s;
+    if ((s = make_tmap_strided(&m.k_rows, at->k, at->d_qk, kv_rows, at->k_row_stride, 64, 1)) != LSA_OK) return s;
+    if ((s = make_tmap_strided(&m.v_tile, at->v, at->d_v, kv_rows, at->v_row_stride, 64, kAttnBN)) != LSA_OK) return s;
+    if ((s = make_tmap_strided(&m.v_rows, at->v, at->d_v, kv_rows, at->v_row_stride, 64, 1)) != LSA_OK) return s;
+    AttnArgs& a = args[i];
+    a = AttnArgs{};
+    a.B = at->B; a.T = at->T; a.Hq = at->Hq; a.L_max = at->L_max;
+    a.d_qk = at->d_qk; a.d_v = at->d_v; a.k = k;
+    a.scale_log2 = at->scale * 1.4426950408889634f;
+    a.idx = idx;
+    a.q = static_cast<const uint16_t*>(at->q);
+    a.kp = static_cast<const uint16_t*>(at->k);
+    a.vp = static_cast<const uint16_t*>(at->v);
+    a.k_stride = at->k_row_stride; a.v_stride = at->v_row_stride;
+    a.sep_v = !(at->v == at->k && at->v_row_stride == at->k_row_stride);
+    a.n_split = p.n_split; a.blocks_per_split = p.bps;
+    a.fixed_blocks = p.fixed_blocks; a.fixed_splits = p.fixed_splits; a.bps_fixed = p.bps_fixed;
+    a.stream_sink = at->stream_sink > 0 ? at->stream_sink : 0;
+    a.stream_window = at->stream_window > 0 ? at->stream_window : 0;
+    a.seq_len = at->seq_len;
+    a.out = static_cast<uint16_t*>(outs[i]);
+    a.lse = lses ? lses[i] : nullptr;
+    a.status = device_status_ptr();
+    if (p.n_split > 1) {
+      const size_t nm = static_cast<size_t>(at->B) * at->T * p.n_split * at->Hq;
+      uint8_t* w = wss[i];
+      a.part_o = reinterpret_cast<uint16_t*>(w);
+      w += align_up(nm * at->d_v * 2, 256);
+      a.part_m = reinterpret_cast<float*>(w);
+      w += align_up(nm * 4, 256);
+      a.part_l = reinterpret_cast<float*>(w);
+    }
   }
-  LSA_CHECK_CUDA(launch_attn(maps, a, st), "attention launch");
-  if (p.n_split > 1) LSA_CHECK_CUDA(launch_attn_combine(a, st), "attention combine launch");
+  LSA_CHECK_CUDA(launch_attn(maps, args, n, st), "attention launch");
+  if (p.n_split > 1) LSA_CHECK_CUDA(launch_attn_combine(args, n, st), "attention combine launch");
   return LSA_OK;
 }
 
@@ -385,6 +431,12 @@ lsa_status_t check_ws(void* ws, size_t have, size_t need) {
   if (have < need) return fail(LSA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", have, need);
   if (need > 0 && (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)))
     return fail(LSA_ERR_INVALID_ARG, "workspace must be non-null and 256-byte aligned");
+  return LSA_OK;
+}
+
+lsa_status_t check_entry_size(const lsa_indexer_in_t* in, int m) {
+  if (!is_pow2_in(m, 1, 128)) return fail(LSA_ERR_UNSUPPORTED, "entry size m=%d not a power of 2 in [1, 128]", m);
+  if (in->L_max % m) return fail(LSA_ERR_INVALID_ARG, "L_max must be a multiple of m");
   return LSA_OK;
 }
 
@@ -485,6 +537,12 @@ lsa_status_t lsa_workspace_size(lsa_op_t op, const lsa_op_args_t* args, size_t* 
       if ((s = check_budget(args->budget)) != LSA_OK) return s;
       *bytes = flat_ws_bytes(args->indexer, args->budget, args->scores_external != 0);
       return LSA_OK;
+    case LSA_OP_INDEX_COMPRESSED:
+      if ((s = check_indexer(args->indexer, true)) != LSA_OK) return s;
+      if ((s = check_entry_size(args->indexer, args->m)) != LSA_OK) return s;
+      if ((s = check_budget(args->budget)) != LSA_OK) return s;
+      *bytes = compressed_ws_bytes(args->indexer, args->m, args->budget, args->scores_external != 0);
+      return LSA_OK;
     case LSA_OP_INDEX_HIER:
       if ((s = check_indexer(args->indexer, false)) != LSA_OK) return s;
       if ((s = check_hier_params(args->indexer, args->P, args->M, args->budget)) != LSA_OK) return s;
@@ -512,16 +570,21 @@ lsa_status_t lsa_workspace_size(lsa_op_t op, const lsa_op_args_t* args, size_t* 
       } else {
         ix = flat_ws_bytes(in, args->budget, false);
       }
-      size_t at = 0;
-      for (int i = 0; i < args->n_layers; ++i) {
+      for (int i = 0; i < args->n_layers; ++i)
         if ((s = check_attn(&args->attn[i], args->budget.k)) != LSA_OK) return s;
-        lsa_attn_in_t lay = args->attn[i];   // as launched: with the group's streaming prefix
-        lay.stream_sink = args->budget.sink;
-        lay.stream_window = args->budget.window;
-        at = std::max(at, attn_ws_bytes(&lay, args->budget.k));
+      // Every layer keeps its split partials in a region of its own, apart from
+      // the selection's scratch: with the streaming-prefix promise a launch's
+      // first splits may run while the kernel before it (the selection, or the
+      // previous launch's combine) still reads its own buffers.
+      size_t at = 0;
+      for (int i = 0; i < args->n_layers;) {
+        const int n = group_launch_layers(args->attn, i, args->n_layers);
+        for (int j = i; j < i + n; ++j) {
+          const lsa_attn_in_t lay = group_layer(args->attn, j, args->budget);
+          at += attn_ws_bytes(&lay, args->budget.k, n);
+        }
+        i += n;
       }
-      // the attention's region is separate: with the streaming prefix promise its
-      // first splits may run while the group's selection still reads its scratch
       *bytes = idx_bytes + ix + at;
       return LSA_OK;
     }
@@ -550,6 +613,33 @@ lsa_status_t lsa_index_flat(const lsa_indexer_in_t* in, lsa_budget_t budget, int
   if (idx)
     return run_select(kSelectTokens, in->B, in->T, in->L_max, in->seq_len, scores, in->L_max, in->L_max, budget, 0,
                       0, nullptr, idx, budget.k, w, st);
+  return LSA_OK;
+}
+
+lsa_status_t lsa_index_compressed(const lsa_indexer_in_t* in, int32_t m, lsa_budget_t budget, int32_t* idx,
+                                  float* scores_out, void* workspace, size_t workspace_bytes, lsa_stream_t stream) {
+  lsa_status_t s;
+  if ((s = check_indexer(in, true)) != LSA_OK) return s;
+  if ((s = check_entry_size(in, m)) != LSA_OK) return s;
+  if ((s = check_budget(budget)) != LSA_OK) return s;
+  if (!idx && !scores_out) return fail(LSA_ERR_INVALID_ARG, "need idx or scores_out");
+  if ((idx && !aligned16(idx)) || (scores_out && !aligned16(scores_out)))
+    return fail(LSA_ERR_INVALID_ARG, "outputs must be 16-byte aligned");
+  const size_t need = compressed_ws_bytes(in, m, budget, scores_out != nullptr);
+  if ((s = check_ws(workspace, workspace_bytes, need)) != LSA_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int n_e = in->L_max / m;
+  const int shift = entry_shift_of(m);
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  float* scores = scores_out;
+  if (!scores) {
+    scores = reinterpret_cast<float*>(w);
+    w += align_up(static_cast<size_t>(in->B) * in->T * n_e * 4, 256);
+  }
+  if ((s = run_flat_scores(in, in->k, n_e, shift, scores, st)) != LSA_OK) return s;
+  if (idx)
+    return run_select(kSelectTokens, in->B, in->T, in->L_max, in->seq_len, scores, n_e, n_e, budget, 0, 0, nullptr,
+                      idx, budget.k, w, st, shift);
   return LSA_OK;
 }
 
@@ -605,7 +695,8 @@ lsa_status_t lsa_sparse_attn(const lsa_attn_in_t* in, const int32_t* idx, int32_
   if (!aligned16(out) || (lse && !aligned16(lse))) return fail(LSA_ERR_INVALID_ARG, "outputs must be 16-byte aligned");
   if (static_cast<long long>(in->B) * in->T > 65535) return fail(LSA_ERR_UNSUPPORTED, "at most 65535 query rows per call");
   if ((s = check_ws(workspace, workspace_bytes, attn_ws_bytes(in, k))) != LSA_OK) return s;
-  return run_attn(in, idx, k, out, lse, workspace, reinterpret_cast<cudaStream_t>(stream));
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  return run_attn(in, 1, idx, k, &out, &lse, &ws, reinterpret_cast<cudaStream_t>(stream));
 }
 
 lsa_status_t lsa_layer_group(const lsa_indexer_in_t* in, const void* page_keys, int32_t P, int32_t M,
@@ -627,6 +718,27 @@ lsa_status_t lsa_layer_group(const lsa_indexer_in_t* in, const void* page_keys, 
       return fail(LSA_ERR_INVALID_ARG, "layer %d shapes differ from the indexer's", i);
     if (!outs[i] || !aligned16(outs[i])) return fail(LSA_ERR_INVALID_ARG, "layer %d output null or unaligned", i);
   }
+  // Layers' outputs may be written concurrently (one launch, or a launch whose
+  // streaming-prefix splits start before the previous one ends): no overlaps,
+  // and none with the index rows the selection writes meanwhile.
+  auto span = [&](int i, uintptr_t* lo, uintptr_t* hi) {
+    *lo = reinterpret_cast<uintptr_t>(outs[i]);
+    *hi = *lo + static_cast<uintptr_t>(layers[i].B) * layers[i].T * layers[i].Hq * layers[i].d_v * 2;
+  };
+  for (int i = 0; i < n_layers; ++i) {
+    uintptr_t a0, a1;
+    span(i, &a0, &a1);
+    for (int j = i + 1; j < n_layers; ++j) {
+      uintptr_t b0, b1;
+      span(j, &b0, &b1);
+      if (a0 < b1 && b0 < a1) return fail(LSA_ERR_INVALID_ARG, "outputs of layers %d and %d overlap", i, j);
+    }
+    if (idx) {
+      const uintptr_t i0 = reinterpret_cast<uintptr_t>(idx);
+      const uintptr_t i1 = i0 + static_cast<uintptr_t>(in->B) * in->T * budget.k * 4;
+      if (a0 < i1 && i0 < a1) return fail(LSA_ERR_INVALID_ARG, "output of layer %d overlaps idx", i);
+    }
+  }
   lsa_op_args_t wa{};
   wa.indexer = in; wa.attn = layers; wa.budget = budget; wa.P = P; wa.M = M; wa.n_layers = n_layers;
   size_t need = 0;
@@ -647,12 +759,19 @@ lsa_status_t lsa_layer_group(const lsa_indexer_in_t* in, const void* page_keys, 
                         0, 0, nullptr, idx_buf, budget.k, sws, st)) != LSA_OK)
       return s;
   }
-  for (int i = 0; i < n_layers; ++i) {
-    float* lse = lse_outs ? lse_outs[i] : nullptr;
-    lsa_attn_in_t lay = layers[i];   // the group's own selection wrote idx: its streaming prefix is known
-    lay.stream_sink = budget.sink;
-    lay.stream_window = budget.window;
-    if ((s = run_attn(&lay, idx_buf, budget.k, outs[i], lse, attn_ws, st)) != LSA_OK) return s;
+  for (int i = 0; i < n_layers;) {
+    const int n = group_launch_layers(layers, i, n_layers);
+    lsa_attn_in_t lays[kMaxLaunchLayers];
+    float* lses[kMaxLaunchLayers];
+    uint8_t* wss[kMaxLaunchLayers];
+    for (int j = 0; j < n; ++j) {
+      lays[j] = group_layer(layers, i + j, budget);
+      lses[j] = lse_outs ? lse_outs[i + j] : nullptr;
+      wss[j] = attn_ws;
+      attn_ws += attn_ws_bytes(&lays[j], budget.k, n);
+    }
+    if ((s = run_attn(lays, n, idx_buf, budget.k, outs + i, lses, wss, st)) != LSA_OK) return s;
+    i += n;
   }
   return LSA_OK;
 }

@@ -25,6 +25,28 @@
 namespace lsa {
 namespace {
 
+// Outputs of one layer of a launch (see launch_attn).
+struct LayerOut {
+  uint16_t* out;          // [rows, Hq, d_v] bf16
+  float* lse;             // [rows, Hq] or null
+  uint16_t* part_o;       // [rows, n_split, Hq, d_v] bf16 split partials
+  float* part_m;          // [rows, n_split, Hq]
+  float* part_l;          // [rows, n_split, Hq]
+  float scale_log2;       // the layer's softmax scale * log2(e)
+};
+struct LayerOuts {
+  LayerOut l[kMaxLaunchLayers];
+  int n;
+};
+
+LayerOuts layer_outs(const AttnArgs* args, int n) {
+  LayerOuts lo{};
+  lo.n = n;
+  for (int i = 0; i < n; ++i)
+    lo.l[i] = LayerOut{args[i].out, args[i].lse, args[i].part_o, args[i].part_m, args[i].part_l, args[i].scale_log2};
+  return lo;
+}
+
 constexpr int kThreads = 128;
 constexpr int BN = kAttnBN;
 
@@ -429,9 +451,13 @@ __device__ __forceinline__ bool get_tagged(const volatile unsigned long long* sl
   return true;
 }
 
+// K/V tile and row-gather maps and q maps of every layer of a launch.
+struct MapSet {
+  CUtensorMap kt[kMaxLaunchLayers], kg[kMaxLaunchLayers], q[kMaxLaunchLayers];
+};
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    mla_pair_kernel(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUtensorMap tm_kg,
-                    const __grid_constant__ CUtensorMap tm_q, const AttnArgs a) {
+    mla_pair_kernel(const __grid_constant__ MapSet maps, const __grid_constant__ LayerOuts lo, const AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sStage = base;
@@ -458,7 +484,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_ctarank();
   const uint32_t peer = rank ^ 1u;
-  const int r = blockIdx.y, split = blockIdx.z;   // splits outermost: the streaming-prefix splits launch first
+  // z = split * layers + layer: splits outermost, so the streaming-prefix splits of all layers launch first
+  const int layer = static_cast<int>(blockIdx.z) % lo.n;
+  const int r = blockIdx.y, split = static_cast<int>(blockIdx.z) / lo.n;
+  const LayerOut& Lo = lo.l[layer];
+  const CUtensorMap* tm_kt = &maps.kt[layer];
+  const CUtensorMap* tm_kg = &maps.kg[layer];
+  const CUtensorMap* tm_q = &maps.q[layer];
   const int b = r / a.T;
   const int chunk0 = rank ? 4 : 0;        // global 64-column chunk of local chunk 0
   const int nq = rank ? 4 : 5;            // q chunks held (and score chunks multiplied)
@@ -516,7 +548,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   cluster_sync_all();   // the partner's barriers are initialised before any remote arrive
-  if (!fixed) pdl_wait();   // the index rows come from the previous kernel in the stream
+  // The index rows come from the previous kernel in the stream. The last cluster
+  // waits in any case, so this grid never completes before that kernel does.
+  if (!fixed || (blockIdx.y == gridDim.y - 1 && blockIdx.z == gridDim.z - 1)) pdl_wait();
   pdl_trigger();
   // Second cluster phase: q is staged in the exchange buffers, so the partner
   // may copy scores into them only after this CTA has moved q into TMEM. The
@@ -530,12 +564,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       // q rows [r Hq, r Hq + 128) x this CTA's chunks, 128-byte swizzled, into the exchange buffers
       mbar_arrive_expect_tx(q_full, nq * 16384);
-      for (int j = 0; j < nq; ++j) tma_load_2d(sX + j * 16384, &tm_q, q_full, (q_chunk0 + j) * 64, r * a.Hq);
+      for (int j = 0; j < nq; ++j) tma_load_2d(sX + j * 16384, tm_q, q_full, (q_chunk0 + j) * 64, r * a.Hq);
     }
     __syncwarp();
     cluster_arrive_release();
-    prefetch_tmap(&tm_kt);
-    prefetch_tmap(&tm_kg);
+    prefetch_tmap(tm_kt);
+    prefetch_tmap(tm_kg);
     const int row0 = b * a.L_max;
     // index entry e of block `bb`, -1 outside the split / row
     auto load_id = [&](int bb, int e) -> int {
@@ -593,13 +627,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (contiguous) {
           if (lane < 2 * kChunks) {
             const int c = lane >> 1, hrow = lane & 1;   // two 32-row boxes per chunk
-            tma_load_2d(st + c * kChunkBytes + hrow * (kChunkBytes / 2), &tm_kt, &kv_full[j], (chunk0 + c) * 64,
+            tma_load_2d(st + c * kChunkBytes + hrow * (kChunkBytes / 2), tm_kt, &kv_full[j], (chunk0 + c) * 64,
                         row0 + id0 + 32 * hrow);
           }
         } else if (lane < BN / 4) {
 #pragma unroll
           for (int c = 0; c < kChunks; ++c)
-            tma_gather4(st + c * kChunkBytes + lane * 512, &tm_kg, &kv_full[j], (chunk0 + c) * 64, yg[0], yg[1],
+            tma_gather4(st + c * kChunkBytes + lane * 512, tm_kg, &kv_full[j], (chunk0 + c) * 64, yg[0], yg[1],
                         yg[2], yg[3]);
         }
       }
@@ -753,7 +787,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const uint32_t valid = mask_s[2 * s + half];
       float mloc[8];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) x[j] = ((valid >> j) & 1u) ? x[j] * a.scale_log2 : -INFINITY;
+      for (int j = 0; j < 32; ++j) x[j] = ((valid >> j) & 1u) ? x[j] * Lo.scale_log2 : -INFINITY;
 #pragma unroll
       for (int t = 0; t < 8; ++t) mloc[t] = fmaxf(fmaxf(x[4 * t], x[4 * t + 1]), fmaxf(x[4 * t + 2], x[4 * t + 3]));
       const float mb_mine = fmaxf(fmaxf(fmaxf(mloc[0], mloc[1]), fmaxf(mloc[2], mloc[3])),
@@ -860,7 +894,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           if (hh < a.Hq) {
             const long long orow = final_out ? static_cast<long long>(r) * a.Hq + hh
                                              : (static_cast<long long>(r) * a.n_split + split) * a.Hq + hh;
-            uint16_t* dstp = (final_out ? a.out : a.part_o) + orow * 512 + rank * 256 + c0 + seg * 8;
+            uint16_t* dstp = (final_out ? Lo.out : Lo.part_o) + orow * 512 + rank * 256 + c0 + seg * 8;
             *reinterpret_cast<uint4*>(dstp) =
                 make_uint4(*reinterpret_cast<const uint32_t*>(&b0), *reinterpret_cast<const uint32_t*>(&b1),
                            *reinterpret_cast<const uint32_t*>(&b2), *reinterpret_cast<const uint32_t*>(&b3));
@@ -870,13 +904,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       if (rank == 0 && half == 0 && h < a.Hq) {
         if (final_out) {
-          if (a.lse)
-            a.lse[static_cast<long long>(r) * a.Hq + h] =
+          if (Lo.lse)
+            Lo.lse[static_cast<long long>(r) * a.Hq + h] =
                 l_run > 0.f ? (m_run + log2f(l_run)) * 0.69314718055994530942f : -INFINITY;
         } else {
           const long long prow = (static_cast<long long>(r) * a.n_split + split) * a.Hq + h;
-          a.part_m[prow] = have ? m_run : -INFINITY;
-          a.part_l[prow] = have ? l_run : 0.f;
+          Lo.part_m[prow] = have ? m_run : -INFINITY;
+          Lo.part_l[prow] = have ? l_run : 0.f;
         }
       }
     }
@@ -892,29 +926,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   }
 }
 
-cudaError_t launch(const AttnMaps& m, const AttnArgs& a, cudaStream_t stream) {
+cudaError_t launch(const AttnMaps* m, const AttnArgs* a, int n, cudaStream_t stream) {
   const void* fn = reinterpret_cast<const void*>(&mla_pair_kernel);
   cudaError_t e = set_max_smem(fn, kSmem);
   if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2, a.B * a.T, a.n_split);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = kSmem;
-  cfg.stream = stream;
-  void* args[] = {const_cast<CUtensorMap*>(&m.k_tile), const_cast<CUtensorMap*>(&m.k_rows),
-                  const_cast<CUtensorMap*>(&m.q), const_cast<AttnArgs*>(&a)};
-  return launch_pdl(fn, cfg.gridDim, cfg.blockDim, cfg.dynamicSmemBytes, stream, args);
+  MapSet maps{};
+  for (int i = 0; i < n; ++i) {
+    maps.kt[i] = m[i].k_tile;
+    maps.kg[i] = m[i].k_rows;
+    maps.q[i] = m[i].q;
+  }
+  LayerOuts lo = layer_outs(a, n);
+  AttnArgs shared = a[0];
+  void* args[] = {&maps, &lo, &shared};
+  return launch_pdl(fn, dim3(2, a[0].B * a[0].T, a[0].n_split * n), dim3(kThreads, 1, 1), kSmem, stream, args);
 }
 }  // namespace mla
 
 // Merge KV-split partials (o_s = O_s / l_s in bf16, with m_s and l_s):
 //   f_s = l_s 2^(m_s - m*),  m* = max m_s;  o = sum f_s o_s / sum f_s.
-__global__ void __launch_bounds__(128) combine_kernel(const AttnArgs a) {
+__global__ void __launch_bounds__(128) combine_kernel(const __grid_constant__ LayerOuts lo, const AttnArgs a) {
   pdl_wait();
   pdl_trigger();
   __shared__ float s_f[64];
   __shared__ float s_den;
   const int r = blockIdx.x, h = blockIdx.y;
+  const LayerOut& Lo = lo.l[blockIdx.z];
   const int ns = a.n_split;
   const long long base = static_cast<long long>(r) * ns * a.Hq + h;
   if (threadIdx.x < 32) {
@@ -928,8 +965,8 @@ __global__ void __launch_bounds__(128) combine_kernel(const AttnArgs a) {
       l[q] = 0.f;
       if (sidx < ns) {
         const long long i = base + static_cast<long long>(sidx) * a.Hq;
-        l[q] = a.part_l[i];
-        m[q] = l[q] > 0.f ? a.part_m[i] : -INFINITY;
+        l[q] = Lo.part_l[i];
+        m[q] = l[q] > 0.f ? Lo.part_m[i] : -INFINITY;
       }
       M = fmaxf(M, m[q]);
     }
@@ -946,7 +983,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const AttnArgs a) {
     for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
     if (lane == 0) {
       s_den = den;
-      if (a.lse) a.lse[static_cast<long long>(r) * a.Hq + h] = den > 0.f ? (M + log2f(den)) * 0.69314718055994530942f : -INFINITY;
+      if (Lo.lse) Lo.lse[static_cast<long long>(r) * a.Hq + h] = den > 0.f ? (M + log2f(den)) * 0.69314718055994530942f : -INFINITY;
     }
   }
   __syncthreads();
@@ -956,7 +993,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const AttnArgs a) {
 #pragma unroll 4
   for (int sidx = 0; sidx < ns; ++sidx) {
     const float f = s_f[sidx];
-    const uint2 o = *reinterpret_cast<const uint2*>(a.part_o + (base + static_cast<long long>(sidx) * a.Hq) * a.d_v + c);
+    const uint2 o = *reinterpret_cast<const uint2*>(Lo.part_o + (base + static_cast<long long>(sidx) * a.Hq) * a.d_v + c);
     acc[0] = fmaf(__uint_as_float(o.x << 16), f, acc[0]);
     acc[1] = fmaf(__uint_as_float(o.x & 0xFFFF0000u), f, acc[1]);
     acc[2] = fmaf(__uint_as_float(o.y << 16), f, acc[2]);
@@ -968,7 +1005,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const AttnArgs a) {
   uint2 pk;
   pk.x = *reinterpret_cast<const uint32_t*>(&v01);
   pk.y = *reinterpret_cast<const uint32_t*>(&v23);
-  *reinterpret_cast<uint2*>(a.out + (static_cast<long long>(r) * a.Hq + h) * a.d_v + c) = pk;
+  *reinterpret_cast<uint2*>(Lo.out + (static_cast<long long>(r) * a.Hq + h) * a.d_v + c) = pk;
 }
 
 template <int DQK, int DV, bool SEP_V>
@@ -988,24 +1025,31 @@ cudaError_t launch_t(const AttnMaps& m, const AttnArgs& a, cudaStream_t stream) 
 
 }  // namespace
 
-cudaError_t launch_attn(const AttnMaps& m, const AttnArgs& a, cudaStream_t stream) {
+cudaError_t launch_attn(const AttnMaps* m, const AttnArgs* args, int n, cudaStream_t stream) {
+  if (n < 1 || n > kMaxLaunchLayers) return cudaErrorInvalidValue;
+  const AttnArgs& a = args[0];
   if (a.d_qk == 576 && a.d_v == 512) {
-    if (a.sep_v) return cudaErrorNotSupported;   // MLA keeps V inside the latent row
-    return mla::launch(m, a, stream);
+    for (int i = 0; i < n; ++i)
+      if (args[i].sep_v) return cudaErrorNotSupported;   // MLA keeps V inside the latent row
+    return mla::launch(m, args, n, stream);
   }
+  if (n != 1) return cudaErrorNotSupported;
   if (a.d_qk == 64 && a.d_v == 64) {
-    if (a.sep_v) return launch_t<64, 64, true>(m, a, stream);
-    return launch_t<64, 64, false>(m, a, stream);
+    if (a.sep_v) return launch_t<64, 64, true>(m[0], a, stream);
+    return launch_t<64, 64, false>(m[0], a, stream);
   }
   return cudaErrorNotSupported;
 }
 
-cudaError_t launch_attn_combine(const AttnArgs& a, cudaStream_t stream) {
-  if (a.n_split > 64) return cudaErrorInvalidValue;
-  const dim3 grid(a.B * a.T, a.Hq);
-  void* args[] = {const_cast<AttnArgs*>(&a)};
+cudaError_t launch_attn_combine(const AttnArgs* args, int n, cudaStream_t stream) {
+  const AttnArgs& a = args[0];
+  if (a.n_split > 64 || n < 1 || n > kMaxLaunchLayers) return cudaErrorInvalidValue;
+  LayerOuts lo = layer_outs(args, n);
+  AttnArgs shared = a;
+  const dim3 grid(a.B * a.T, a.Hq, n);
+  void* kargs[] = {&lo, &shared};
   return launch_pdl(reinterpret_cast<const void*>(&combine_kernel), grid, dim3(a.d_v / 4 < 32 ? 32 : a.d_v / 4),
-                    0, stream, args);
+                    0, stream, kargs);
 }
 
 }  // namespace lsa

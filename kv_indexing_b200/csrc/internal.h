@@ -57,6 +57,8 @@ struct SelectArgs {
   int n_slots;            // slots per row
   int k, sink, window;    // token budget
   int P, M;               // pages / hier
+  int entry_shift;        // > 0: slots are entries of 2^shift tokens (kSelectTokens); the
+                          // query's slot position is its last complete entry
   const int* pages;       // kSelectHierTokens: [B*T, M]
   int* out;
   int out_len;            // k (tokens) or M (pages)
@@ -124,8 +126,13 @@ struct AttnMaps {
   CUtensorMap q, k_tile, k_rows, v_tile, v_rows;
 };
 
-cudaError_t launch_attn(const AttnMaps& maps, const AttnArgs& a, cudaStream_t stream);
-cudaError_t launch_attn_combine(const AttnArgs& a, cudaStream_t stream);
+// One launch may cover several layers of a cross-layer group that share the
+// index rows, B, T, L_max, Hq, the head dims and the split plan; each layer has
+// its own q, latent rows, scale, outputs and split partials. maps[i] / args[i]
+// describe layer i (the shared fields of args[0] are used). MLA only when n > 1.
+constexpr int kMaxLaunchLayers = 4;
+cudaError_t launch_attn(const AttnMaps* maps, const AttnArgs* args, int n, cudaStream_t stream);
+cudaError_t launch_attn_combine(const AttnArgs* args, int n, cudaStream_t stream);
 
 // --------------------------------------------------------------------- misc --
 int device_sm_count();
