@@ -15,7 +15,9 @@ Workloads (kv_indexing_b200.inputs.WORKLOADS): flat_decode_128k (default, the
 headline), hier_decode_1m (hierarchical indexing at 1M tokens; page pooling
 timed once, outside the step), cli_group_256k / cli_group_256k_flat (one
 indexing pass feeding two layers), prefill_64k (4096 causal queries; --fp8 for
-e4m3 indexer inputs). Long KV caches for timing are drawn on the device with
+e4m3 indexer inputs), compressed_decode_1m (indexing over 262144 entries of 4
+tokens each, then attention over the 2048 chosen compressed latent entries;
+--fp8 for e4m3 entry keys). Long KV caches for timing are drawn on the device with
 torch's seeded generator; the indexer inputs come from the seeded host
 generator (needles included).
 
@@ -250,7 +252,8 @@ def run_reference(args, rank: int, world: int):
 def workload_config(w, **extra):
     c = {"workload": w.name, "B": w.B, "L": w.L, "T": w.T, "H_I": w.H, "d_I": w.d, "k": w.k, "sink": w.sink,
          "window": w.window, "Hq": w.Hq, "d_qk": w.d_qk, "d_v": w.d_v, "P": w.P, "M": w.M,
-         "n_layers": w.n_layers, "l2": "flushed between timed steps (256 MiB write, outside the timed events)"}
+         "n_layers": w.n_layers, "entry_tokens_m": w.m,
+         "l2": "flushed between timed steps (256 MiB write, outside the timed events)"}
     c.update(extra)
     return c
 
@@ -323,7 +326,15 @@ def run_workload(args, w, rank, world, dev, pg):
     from kv_indexing_b200 import lsa as L
 
     seed = rank_seed(args.seed, rank)
-    x = I.make_indexer_inputs(w, seed)
+    if w.m:
+        # compressed entries: the indexer's keys are the entry keys [B, L/m, d]
+        x = I.make_compressed_inputs(w, seed)
+        x["k_idx"] = x.pop("entry_keys")
+        if "entry_keys_fp8" in x:
+            x["k_idx_fp8"] = x.pop("entry_keys_fp8")
+    else:
+        x = I.make_indexer_inputs(w, seed)
+    kv_rows = w.L // w.m if w.m else w.L
 
     def up(arr, kind):
         t = torch.from_numpy(np.ascontiguousarray(arr).view(np.int16) if kind == "bf16" else arr)
@@ -336,7 +347,7 @@ def run_workload(args, w, rank, world, dev, pg):
     layers = []
     for li in range(w.n_layers):
         qa = device_bf16_normal(torch, (B, T, w.Hq, w.d_qk), 7919 * seed + 2 * li, dev)
-        kv = device_bf16_normal(torch, (B, w.L, w.d_qk), 7919 * seed + 2 * li + 1, dev)
+        kv = device_bf16_normal(torch, (B, kv_rows, w.d_qk), 7919 * seed + 2 * li + 1, dev)
         layers.append({"q": qa, "kv": kv, "scale": w.scale, "d_v": w.d_v})
     flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
@@ -356,7 +367,29 @@ def run_workload(args, w, rank, world, dev, pg):
         return lambda s: L.lsa_sparse_attn(lay["q"], idx, sl, w.scale, kv=lay["kv"], d_v=w.d_v, out=outs[li],
                                            workspace=attn_ws, stream=s)
 
-    if w.T > 1:
+    if w.m:
+        kind = "compressed"
+        qk = dict(q=q, k=k)
+        if args.fp8:
+            qk = dict(q=up(x["q_idx_fp8"], "u8").view(torch.float8_e4m3fn),
+                      k=up(x["k_idx_fp8"], "u8").view(torch.float8_e4m3fn),
+                      q_scale=up(x["q_scale"], "f32"), k_scale=up(x["k_scale"], "f32"))
+        ii = L.indexer_in(qk["q"], wt, qk["k"], sl, qk.get("q_scale"), qk.get("k_scale"), m=w.m)
+        cws = torch.empty(max(256, L.workspace_size(L.LSA_OP_INDEX_COMPRESSED, indexer=ii, budget=budget, m=w.m)),
+                          dtype=torch.uint8, device=dev)
+        # one query per sequence (decode): its entry position is seq_len // m - 1
+        sl_e = torch.div(sl, w.m, rounding_mode="floor").to(torch.int32)
+        lay = layers[0]
+        ai_c = L.attn_in(lay["q"], sl_e, w.scale, kv=lay["kv"], d_v=w.d_v, stream_budget=budget)
+        cattn_ws = torch.empty(max(256, L.workspace_size(L.LSA_OP_SPARSE_ATTN, attn=ai_c, budget=(w.k, 0, 0))),
+                               dtype=torch.uint8, device=dev)
+        stages = [("index_compressed", lambda s: L.lsa_index_compressed(
+                      qk["q"], wt, qk["k"], sl, w.m, budget, q_scale=qk.get("q_scale"), k_scale=qk.get("k_scale"),
+                      idx=idx, workspace=cws, stream=s)),
+                  ("attention", lambda s: L.lsa_sparse_attn(lay["q"], idx, sl_e, w.scale, kv=lay["kv"], d_v=w.d_v,
+                                                            out=outs[0], workspace=cattn_ws, stream_budget=budget,
+                                                            stream=s))]
+    elif w.T > 1:
         kind = "prefill"
         qk = dict(q=q, k=k)
         if args.fp8:
@@ -418,6 +451,14 @@ def run_workload(args, w, rank, world, dev, pg):
                 "frac": flops / (us * 1e-6) / 1e12 / peak, "traffic": None, "algorithmic_flops_per_launch": flops,
                 "launch_us": us, "peak_source": peak_src + (" bf16 sustained x 2 (e4m3 nominal ratio)" if args.fp8
                                                              else " bf16 sustained")}
+    elif kind == "compressed":
+        n_e = w.L // w.m
+        byts = (n_e * w.d * (1 if args.fp8 else 2) + (n_e * 4 if args.fp8 else 0) + w.H * w.d * 2 + w.H * 4) * B * T
+        us = br["index_compressed"]
+        roof = {"bound": "hbm", "kernel": "compressed-entry indexing call (entry scores, streaming top-k)",
+                "achieved": byts / (us * 1e-6) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": byts / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], "traffic": None,
+                "algorithmic_bytes_per_launch": byts, "launch_us": us, "peak_source": peak_src}
     elif kind == "group":
         if w.P:
             ib = (w.L // w.P) * w.d * 2 + w.M * w.P * w.d * 2
@@ -484,7 +525,7 @@ def main():
         pg = True
     L.load()
     w = I.WORKLOADS[args.workload]
-    if w.P or w.n_layers > 1 or w.T > 1 or args.fp8:
+    if w.P or w.m or w.n_layers > 1 or w.T > 1 or args.fp8:
         return run_workload(args, w, rank, world, dev, pg)
     seed = rank_seed(args.seed, rank)                   # each rank its own batch
     x = I.make_indexer_inputs(w, seed)

@@ -54,7 +54,8 @@ __device__ __forceinline__ Plan make_plan(const SelectArgs& a, int r) {
   const int b = r / a.T, t = r % a.T;
   int L = __ldg(a.seq_len + b);
   L = L < 0 ? 0 : (L > a.L_max ? a.L_max : L);
-  const int pos = L - a.T + t;
+  int pos = L - a.T + t;
+  if (a.entry_shift > 0) pos = ((pos + 1) >> a.entry_shift) - 1;   // last complete entry
   p.valid = pos >= 0;
   if (!p.valid) return p;
   const int sink_end = min(a.sink, pos + 1);

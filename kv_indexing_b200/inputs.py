@@ -57,6 +57,7 @@ class Workload:
     mla: bool = True           # V = first d_v columns of the latent K row
     scale: float = 1.0 / math.sqrt(576.0)
     fp8: bool = False          # also provide FP8-e4m3 indexer keys / queries
+    m: int = 0                 # > 0: index compressed entries of m tokens (budget, sink, window in entries)
 
     @property
     def n_needles(self) -> int:
@@ -90,6 +91,12 @@ WORKLOADS: Dict[str, Workload] = {
     "cli_group_256k_flat": Workload(
         name="cli_group_256k_flat", B=4, L=262144, T=1, H=64, d=128, k=2048, sink=64,
         window=960, needle_frac=0.01, n_layers=2),
+    # Compressed-entry decode: 1M tokens as 262144 entries of 4 tokens; 2048
+    # entries chosen (16 sink + 240 window entries, the token budget's 64 / 960
+    # in entries); attention over the chosen compressed latent entries.
+    "compressed_decode_1m": Workload(
+        name="compressed_decode_1m", B=4, L=1048576, T=1, H=64, d=128, k=2048, sink=16,
+        window=240, needle_frac=0.01, m=4, fp8=True),
 }
 
 
@@ -188,6 +195,27 @@ def normal_bf16(shape, rng: np.random.Generator, chunk: int = 1 << 26) -> np.nda
 def positions(L: int, T: int) -> np.ndarray:
     """Absolute position of each of the T queries of a length-L sequence."""
     return np.arange(L - T, L, dtype=np.int64)
+
+
+def entry_workload(w: Workload) -> Workload:
+    """The workload seen over compressed entries: L // m entries, no compression."""
+    return dataclasses.replace(w, L=w.L // w.m, m=0)
+
+
+def make_compressed_inputs(w: Workload, seed: int) -> dict:
+    """Indexer inputs over compressed entries of ``w.m`` tokens.
+
+    The pages name no compressor, so the entry keys are drawn like token keys
+    (N(0,1) bf16, with needles planted in the entries of the dynamic region; see
+    make_indexer_inputs), as ``entry_keys`` [B, L/m, d] (plus e4m3 codes and
+    per-entry scales when ``w.fp8``). seq_len counts tokens (L).
+    """
+    x = make_indexer_inputs(entry_workload(w), seed)
+    x["entry_keys"] = x.pop("k_idx")
+    if "k_idx_fp8" in x:
+        x["entry_keys_fp8"] = x.pop("k_idx_fp8")
+    x["seq_len"] = np.full((w.B,), w.L, dtype=np.int32)
+    return x
 
 
 def make_indexer_inputs(w: Workload, seed: int, with_needles: bool = True) -> dict:

@@ -17,13 +17,14 @@ LIB_PATH = os.path.join(HERE, "liblsa.so")
 
 LSA_OK, LSA_ERR_INVALID_ARG, LSA_ERR_UNSUPPORTED, LSA_ERR_WORKSPACE, LSA_ERR_CUDA, LSA_ERR_TIMEOUT = range(6)
 LSA_BF16, LSA_E4M3 = 0, 1
-LSA_OP_INDEX_FLAT, LSA_OP_INDEX_HIER, LSA_OP_SELECT, LSA_OP_SPARSE_ATTN, LSA_OP_LAYER_GROUP = range(5)
+(LSA_OP_INDEX_FLAT, LSA_OP_INDEX_HIER, LSA_OP_SELECT, LSA_OP_SPARSE_ATTN, LSA_OP_LAYER_GROUP,
+ LSA_OP_INDEX_COMPRESSED) = range(6)
 LSA_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024   # static scratch of lsa_select_streaming_noalloc
 
 EXPORTS = [
     "lsa_status_string", "lsa_last_error", "lsa_workspace_size", "lsa_index_flat", "lsa_select_streaming",
     "lsa_pool_pages", "lsa_index_hier", "lsa_sparse_attn", "lsa_layer_group", "lsa_device_status",
-    "lsa_select_streaming_noalloc",
+    "lsa_select_streaming_noalloc", "lsa_index_compressed",
 ]
 
 
@@ -56,7 +57,7 @@ class OpArgs(ctypes.Structure):
     _fields_ = [("indexer", ctypes.POINTER(IndexerIn)), ("attn", ctypes.POINTER(AttnIn)), ("budget", Budget),
                 ("P", ctypes.c_int32), ("M", ctypes.c_int32), ("n_layers", ctypes.c_int32),
                 ("B", ctypes.c_int32), ("T", ctypes.c_int32), ("L_max", ctypes.c_int32),
-                ("scores_external", ctypes.c_int32)]
+                ("scores_external", ctypes.c_int32), ("m", ctypes.c_int32)]
 
 
 _lib = None
@@ -79,6 +80,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.lsa_workspace_size.argtypes = [i32, ctypes.POINTER(OpArgs), ctypes.POINTER(sz)]
     lib.lsa_index_flat.restype = i32
     lib.lsa_index_flat.argtypes = [ctypes.POINTER(IndexerIn), Budget, vp, vp, vp, sz, vp]
+    lib.lsa_index_compressed.restype = i32
+    lib.lsa_index_compressed.argtypes = [ctypes.POINTER(IndexerIn), i32, Budget, vp, vp, vp, sz, vp]
     lib.lsa_select_streaming.restype = i32
     lib.lsa_select_streaming.argtypes = [vp, vp, i32, i32, i32, Budget, vp, vp, sz, vp]
     lib.lsa_select_streaming_noalloc.restype = i32
@@ -141,8 +144,9 @@ def _need(t, name, dtype=None, dim=None):
     return t
 
 
-def indexer_in(q, w, k, seq_len, q_scale=None, k_scale=None) -> IndexerIn:
-    """Describe indexer tensors: q [B,T,H,d], w [B,T,H] f32, k [B,L_max,d], seq_len [B] i32."""
+def indexer_in(q, w, k, seq_len, q_scale=None, k_scale=None, m=1) -> IndexerIn:
+    """Describe indexer tensors: q [B,T,H,d], w [B,T,H] f32, k [B,L_max,d], seq_len [B] i32.
+    With m > 1, k holds one key per entry of m tokens: [B,L_max/m,d]."""
     torch = _torch()
     fp8 = q.dtype in (torch.float8_e4m3fn, torch.uint8)
     _need(q, "q", (torch.float8_e4m3fn, torch.uint8) if fp8 else torch.bfloat16, 4)
@@ -153,7 +157,7 @@ def indexer_in(q, w, k, seq_len, q_scale=None, k_scale=None) -> IndexerIn:
     if fp8:
         _need(q_scale, "q_scale", torch.float32, 3)
         _need(k_scale, "k_scale", torch.float32, 2)
-    return IndexerIn(B, T, H, d, k.shape[1], LSA_E4M3 if fp8 else LSA_BF16, _ptr(seq_len), _ptr(q),
+    return IndexerIn(B, T, H, d, k.shape[1] * m, LSA_E4M3 if fp8 else LSA_BF16, _ptr(seq_len), _ptr(q),
                      _ptr(q_scale) if fp8 else None, _ptr(w), _ptr(k), _ptr(k_scale) if fp8 else None)
 
 
@@ -178,7 +182,7 @@ def attn_in(q, seq_len, scale, *, kv=None, k=None, v=None, d_v=None, stream_budg
 
 
 def workspace_size(op: int, *, indexer: Optional[IndexerIn] = None, attn=None, budget=(1, 0, 0), P=0, M=0,
-                   n_layers=0, B=0, T=0, L_max=0, scores_external=False) -> int:
+                   n_layers=0, B=0, T=0, L_max=0, scores_external=False, m=0) -> int:
     lib = load()
     a = OpArgs()
     keep = []
@@ -194,6 +198,7 @@ def workspace_size(op: int, *, indexer: Optional[IndexerIn] = None, attn=None, b
     a.budget = Budget(*budget)
     a.P, a.M, a.n_layers, a.B, a.T, a.L_max = P, M, n_layers, B, T, L_max
     a.scores_external = int(bool(scores_external))
+    a.m = m
     out = ctypes.c_size_t(0)
     _check(lib.lsa_workspace_size(op, ctypes.byref(a), ctypes.byref(out)))
     return out.value
@@ -232,6 +237,25 @@ def lsa_index_flat(q, w, k, seq_len, budget, *, q_scale=None, k_scale=None, idx=
     ws = _workspace(need, q.device, workspace)
     _check(lib.lsa_index_flat(ctypes.byref(ii), Budget(*budget), _ptr(idx) if with_idx else None, _ptr(scores_out),
                               _ptr(ws), _nbytes(ws), _stream(stream)))
+    return idx if with_idx else None
+
+
+def lsa_index_compressed(q, w, entry_keys, seq_len, m, budget, *, q_scale=None, k_scale=None, idx=None,
+                         scores_out=None, with_idx=True, workspace=None, stream=None):
+    """Indexing over compressed entries of m tokens: entry_keys [B,L_max/m,d]
+    (seq_len in tokens; budget in entries). Returns idx [B,T,k] entry ids (or
+    None when with_idx is False)."""
+    torch = _torch()
+    lib = load()
+    ii = indexer_in(q, w, entry_keys, seq_len, q_scale, k_scale, m=m)
+    B, T = q.shape[0], q.shape[1]
+    if with_idx and idx is None:
+        idx = torch.empty((B, T, budget[0]), dtype=torch.int32, device=q.device)
+    need = workspace_size(LSA_OP_INDEX_COMPRESSED, indexer=ii, budget=budget, m=m,
+                          scores_external=scores_out is not None)
+    ws = _workspace(need, q.device, workspace)
+    _check(lib.lsa_index_compressed(ctypes.byref(ii), m, Budget(*budget), _ptr(idx) if with_idx else None,
+                                    _ptr(scores_out), _ptr(ws), _nbytes(ws), _stream(stream)))
     return idx if with_idx else None
 
 
