@@ -80,6 +80,7 @@ struct SelectPlan {
   bool final_in_smem;
   bool grid;              // grid-cooperative launch (rows * C CTAs co-resident)
   bool cluster;           // one thread-block cluster of C CTAs per row (no workspace)
+  int cluster_rc;         // cluster path: keys per thread (32 or 64)
 };
 
 // d_bound: an upper bound on the dynamic budget of any row (k - sink - window for

@@ -1076,8 +1076,6 @@ __global__ void __launch_bounds__(kThreads, 1) select_grid_kernel(const SelectAr
 // is made from the same cluster-wide data in every CTA, so the barriers stay
 // uniform). No global workspace and no spin waits: only barriers.
 constexpr int kClusterMax = 8;
-constexpr int kRC = 32;                         // keys per thread
-constexpr int kCtaKeys = kThreads * kRC;        // 16384 slots per CTA
 constexpr int kListCapC = 512;                  // boundary-bin keys per CTA
 enum { kXMax = 0, kXCnt = 1, kXIn = 2, kXDef = 3, kXLen = 4, kXGt = 5, kXEq = 6, kXSlots = 7 };
 
@@ -1193,12 +1191,24 @@ __device__ __noinline__ void find_bin_c(const uint32_t* h, uint32_t need, Shared
   __syncthreads();
 }
 
-// Element e of a CTA's segment sits at keys[e + (e >> 5)]: thread t owns the
-// 32 consecutive elements [32 t, 32 t + 32) at keys[33 t .. 33 t + 31], so both
-// the warp-coalesced fill and the per-thread passes are free of bank conflicts.
-__device__ __forceinline__ int skew(int e) { return e + (e >> 5); }
+// Element e of a CTA's segment sits at keys[e + e / RC]: thread t owns the RC
+// consecutive elements [RC t, RC t + RC) at keys[(RC + 1) t ...], an odd stride,
+// so both the warp-coalesced fill and the per-thread passes are free of bank
+// conflicts.
+//
+// Dynamic shared memory of a CTA holding RC keys per thread: the keys,
+// two histograms, the outgoing list, the broadcast slots and the round-A
+// sub-histograms (whose space the copies of every CTA's list reuse later).
+constexpr size_t cluster_smem_words(int RC) {
+  return static_cast<size_t>(kThreads) * (RC + 1) + 2048 + 2048 + kListCapC +
+         kXSlots * kClusterMax + kSubHist * kWHStride;
+}
+static_assert(kClusterMax * kListCapC <= kSubHist * kWHStride, "list copies fit the sub-histogram space");
 
+// RC keys per thread: 32 (16384 slots per CTA) or 64 (32768).
+template <int RC>
 __global__ void __launch_bounds__(kThreads, 1) select_cluster_kernel(const SelectArgs a) {
+  static_assert(RC == 32 || RC == 64, "keys per thread");
   pdl_wait();
   pdl_trigger();
   const int C = static_cast<int>(gridDim.x);
@@ -1208,13 +1218,13 @@ __global__ void __launch_bounds__(kThreads, 1) select_cluster_kernel(const Selec
   __shared__ Shared sh;
   __shared__ unsigned s_cnt;
   extern __shared__ uint32_t dsm[];
-  uint32_t* keys = dsm;                              // [kCtaKeys + kCtaKeys / 32] skewed
-  uint32_t* histA = keys + kCtaKeys + kCtaKeys / 32; // [2048]  read by the cluster
+  uint32_t* keys = dsm;                              // [kThreads][RC + 1]: each thread's run, then a pad word
+  uint32_t* histA = keys + kThreads * (RC + 1);      // [2048]  read by the cluster
   uint32_t* fbh = histA + 2048;                      // [2048]  fallback rounds, read by the cluster
   uint32_t* list = fbh + 2048;                       // [kListCapC] read by the cluster
   uint32_t* xs = list + kListCapC;                   // [kXSlots][kClusterMax] broadcast slots
-  uint32_t* sub = xs + kXSlots * kClusterMax;        // [kSubHist][kWHStride] local
-  uint32_t* lists = sub + kSubHist * kWHStride;      // [kClusterMax][kListCapC] local copies of every list
+  uint32_t* sub = xs + kXSlots * kClusterMax;        // [kSubHist][kWHStride] local, round A only
+  uint32_t* lists = sub;                             // [kClusterMax][kListCapC] local copies of every list (after round A)
 
   const Plan pl = make_plan(a, r);                   // identical in every CTA of the cluster
   int* out = a.out + static_cast<long long>(r) * a.out_len;
@@ -1234,15 +1244,17 @@ __global__ void __launch_bounds__(kThreads, 1) select_cluster_kernel(const Selec
 
   // ---- (1) keys (coalesced fill), local max and count; broadcast
   uint32_t nz = 0u, mx = 0u;
-  {
-    const int e0 = warp * 32 * kRC + lane;
-    float f[kRC];
+#pragma unroll 1
+  for (int h = 0; h < RC / 32; ++h) {   // 32 loads in flight per thread at a time
+    const int e0 = warp * 32 * RC + lane + 1024 * h;
+    float f[32];
 #pragma unroll
-    for (int j = 0; j < kRC; ++j) f[j] = e0 + 32 * j < my_n ? __ldg(row + e0 + 32 * j) : -INFINITY;
+    for (int j = 0; j < 32; ++j) f[j] = e0 + 32 * j < my_n ? __ldg(row + e0 + 32 * j) : -INFINITY;
 #pragma unroll
-    for (int j = 0; j < kRC; ++j) {
+    for (int j = 0; j < 32; ++j) {
       const uint32_t k = score_key(f[j]);
-      keys[skew(e0 + 32 * j)] = k;
+      const int e = e0 + 32 * j;
+      keys[e + e / RC] = k;   // one pad word per thread's run: both the fill and the per-thread passes are conflict-free
       nz += k != 0u ? 1u : 0u;
       mx = max(mx, k);
     }
@@ -1257,7 +1269,9 @@ __global__ void __launch_bounds__(kThreads, 1) select_cluster_kernel(const Selec
   cluster_broadcast(xs, kXCnt, c, C, sh.cnt);
   cluster_sync_all();
 
-  const uint32_t* kv = keys + 33 * tid;   // this thread's 32 consecutive elements
+  // this thread's RC consecutive elements, followed by one pad word
+  const uint32_t* kvb = keys + (RC + 1) * tid;
+  auto kv = [kvb](int j) { return kvb[j]; };
 
   uint32_t kmax = 0u, total = 0u;
   for (int cc = 0; cc < C; ++cc) {
@@ -1278,9 +1292,9 @@ __global__ void __launch_bounds__(kThreads, 1) select_cluster_kernel(const Selec
       uint32_t* h = sub + (warp % kSubHist) * kWHStride;
       uint32_t nin = 0u;
 #pragma unroll 4
-      for (int j = 0; j < kRC; ++j) {
-        const uint32_t d = (kmax - kv[j]) >> kRangeShift;
-        if (kv[j] != 0u && d < 2048u) {
+      for (int j = 0; j < RC; ++j) {
+        const uint32_t d = (kmax - kv(j)) >> kRangeShift;
+        if (kv(j) != 0u && d < 2048u) {
           ++nin;
           atomicAdd(&h[d], 1u);
         }
@@ -1307,10 +1321,10 @@ __global__ void __launch_bounds__(kThreads, 1) select_cluster_kernel(const Selec
       __syncthreads();
       uint32_t nd = 0u;
 #pragma unroll 4
-      for (int j = 0; j < kRC; ++j) {
-        const uint32_t rel = kmax - kv[j];
+      for (int j = 0; j < RC; ++j) {
+        const uint32_t rel = kmax - kv(j);
         const uint32_t d = rel >> kRangeShift;
-        if (kv[j] != 0u && d <= b1) {
+        if (kv(j) != 0u && d <= b1) {
           if (d < b1) {
             ++nd;
           } else {
@@ -1393,8 +1407,8 @@ __global__ void __launch_bounds__(kThreads, 1) select_cluster_kernel(const Selec
         for (int i = tid; i < nb; i += kThreads) fbh[i] = 0u;
         __syncthreads();
 #pragma unroll 4
-        for (int j = 0; j < kRC; ++j)
-          if (kv[j] != 0u && (kv[j] & mask) == prefix) atomicAdd(&fbh[(kv[j] >> shift) & dmask], 1u);
+        for (int j = 0; j < RC; ++j)
+          if (kv(j) != 0u && (kv(j) & mask) == prefix) atomicAdd(&fbh[(kv(j) >> shift) & dmask], 1u);
         cluster_sync_all();
         cluster_sum(fbh, nb, C, sh.hist);
         __syncthreads();
@@ -1409,9 +1423,9 @@ __global__ void __launch_bounds__(kThreads, 1) select_cluster_kernel(const Selec
       }
       uint32_t gt = 0u, eq = 0u;
 #pragma unroll 4
-      for (int j = 0; j < kRC; ++j) {
-        gt += (kv[j] != 0u && kv[j] > prefix) ? 1u : 0u;
-        eq += (kv[j] != 0u && kv[j] == prefix) ? 1u : 0u;
+      for (int j = 0; j < RC; ++j) {
+        gt += (kv(j) != 0u && kv(j) > prefix) ? 1u : 0u;
+        eq += (kv(j) != 0u && kv(j) == prefix) ? 1u : 0u;
       }
       uint32_t my_gt = 0u, my_eq = 0u;
       scan_incl(gt, sh.tmp, &my_gt);
@@ -1428,10 +1442,10 @@ __global__ void __launch_bounds__(kThreads, 1) select_cluster_kernel(const Selec
   // ---- (4) this CTA's selections in index order: per-thread counts, two scans
   uint32_t n_gt = 0u, n_eq = 0u;
 #pragma unroll 4
-  for (int j = 0; j < kRC; ++j) {
-    const bool cand = kv[j] != 0u;
-    n_gt += (cand && (t.all || kv[j] > t.thr)) ? 1u : 0u;
-    n_eq += (cand && !t.all && kv[j] == t.thr) ? 1u : 0u;
+  for (int j = 0; j < RC; ++j) {
+    const bool cand = kv(j) != 0u;
+    n_gt += (cand && (t.all || kv(j) > t.thr)) ? 1u : 0u;
+    n_eq += (cand && !t.all && kv(j) == t.thr) ? 1u : 0u;
   }
   uint32_t eq_tot = 0u;
   const uint32_t eq_before = scan_incl(n_eq, sh.tmp, &eq_tot) - n_eq;      // ties in lower elements of this CTA
@@ -1444,8 +1458,8 @@ __global__ void __launch_bounds__(kThreads, 1) select_cluster_kernel(const Selec
   if (n_gt + take > 0u) {
     uint32_t taken = 0u;
 #pragma unroll 4
-    for (int j = 0; j < kRC; ++j) {
-      const uint32_t k = kv[j];
+    for (int j = 0; j < RC; ++j) {
+      const uint32_t k = kv(j);
       bool s = false;
       if (k != 0u) {
         if (t.all || k > t.thr) {
@@ -1456,7 +1470,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_cluster_kernel(const Selec
         }
       }
       if (s) {
-        const int slot = my_lo + 32 * tid + j;
+        const int slot = my_lo + RC * tid + j;
         dyn_out[pos++] = hier ? __ldg(a.pages + prow + slot / a.P) * a.P + slot % a.P : slot;
       }
     }
@@ -1481,12 +1495,17 @@ SelectPlan select_plan(int rows, int n_slots, int d_bound, int num_sms) {
   constexpr int kSegMax = 32768;            // fallback: keys per CTA in shared memory
   SelectPlan p{};
   auto seg_of = [&](int C) { return (n_slots + C - 1) / C; };
-  // cluster path: one cluster of up to 8 CTAs per row, any number of rows
-  if (n_slots <= kClusterMax * kCtaKeys) {
-    p.cluster = true;
-    p.C = std::max(1, (n_slots + kCtaKeys - 1) / kCtaKeys);
-    p.seg = seg_of(p.C);
-    return p;
+  // cluster path: one cluster of up to 8 CTAs per row, any number of rows;
+  // 32 keys per thread up to 131072 slots, 64 up to 262144
+  for (const int rc : {32, 64}) {
+    const int cta_keys = kThreads * rc;
+    if (n_slots <= kClusterMax * cta_keys) {
+      p.cluster = true;
+      p.cluster_rc = rc;
+      p.C = std::max(1, (n_slots + cta_keys - 1) / cta_keys);
+      p.seg = seg_of(p.C);
+      return p;
+    }
   }
   // grid-cooperative path: register-sized segments, one CTA per SM, all co-resident
   const int Cg = std::max(1, (n_slots + kLocalRegs - 1) / kLocalRegs);
@@ -1523,9 +1542,9 @@ cudaError_t launch_select(const SelectArgs& a0, const SelectPlan& p, void* ws, c
   SelectArgs a = a0;
   const int rows = a.B * a.T;
   if (p.cluster) {
-    const size_t smem = static_cast<size_t>(kCtaKeys + kCtaKeys / 32 + 2048 + 2048 + kListCapC +
-                                            kXSlots * kClusterMax + kSubHist * kWHStride + kClusterMax * kListCapC) * 4;
-    const void* fn = reinterpret_cast<const void*>(&select_cluster_kernel);
+    const size_t smem = cluster_smem_words(p.cluster_rc) * 4;
+    const void* fn = p.cluster_rc == 64 ? reinterpret_cast<const void*>(&select_cluster_kernel<64>)
+                                        : reinterpret_cast<const void*>(&select_cluster_kernel<32>);
     cudaError_t e = set_max_smem(fn, smem);
     if (e != cudaSuccess) return e;
     cudaLaunchAttribute attr[1];

@@ -63,14 +63,19 @@ def test_select_negative_scores_and_empty_rows():
     assert (got[0, 0] == -1).all() and (got[0, 1] == -1).all()
 
 
-@pytest.mark.parametrize("B,L_max", [(8, 131072), (3, 393216), (2, 1 << 20)])
-def test_select_long_rows_all_launch_paths(B, L_max):
-    # 128K rows: one cluster per row; 384K rows: the grid-cooperative launch
-    # (rows x CTAs fit the GPU at once); 1M rows: per-segment candidates + merge
+@pytest.mark.parametrize("B,L_max,ties", [(8, 131072, True), (3, 150001, True), (4, 262144, True),
+                                          (2, 262144, False), (3, 393216, True), (2, 1 << 20, True)])
+def test_select_long_rows_all_launch_paths(B, L_max, ties):
+    # up to 128K slots: one cluster per row, 32 keys per thread; up to 256K: 64
+    # keys per thread; 384K rows: the grid-cooperative launch (rows x CTAs fit
+    # the GPU at once); 1M rows: per-segment candidates + merge. The tie block
+    # overflows the boundary lists (exact radix rounds); without it the
+    # window histogram decides.
     rng = np.random.default_rng(L_max)
     sc = rng.standard_normal((B, 1, L_max)).astype(np.float32)
     sc = np.abs(sc) + np.float32(3.0)
-    sc[:, :, rng.integers(0, L_max, size=4000)] = np.float32(9.5)     # a block of exact ties
+    if ties:
+        sc[:, :, rng.integers(0, L_max, size=4000)] = np.float32(9.5)     # a block of exact ties
     sl = np.full((B,), L_max, np.int32)
     got = run_select(sc, sl, 1, (2048, 64, 960))
     ref = O.select_streaming(sc, sl, 1, 2048, 64, 960)
