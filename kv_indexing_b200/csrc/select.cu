@@ -1191,16 +1191,30 @@ __device__ __noinline__ void find_bin_c(const uint32_t* h, uint32_t need, Shared
   __syncthreads();
 }
 
-// Element e of a CTA's segment sits at keys[e + e / RC]: thread t owns the RC
-// consecutive elements [RC t, RC t + RC) at keys[(RC + 1) t ...], an odd stride,
-// so both the warp-coalesced fill and the per-thread passes are free of bank
-// conflicts.
+// Element e of a CTA's segment sits at keys[e + 4 (e / RC)]: thread t owns the
+// RC consecutive elements [RC t, RC t + RC) at keys[(RC + 4) t ...]. The
+// warp-coalesced fill writes 32 consecutive words; the per-thread passes read
+// 16 bytes at a time, and with a stride of 4 (mod 32) words the eight threads
+// of each quarter-warp phase hit distinct bank quads: no conflicts either way.
+template <int RC, int UNROLL, class F>
+__device__ __forceinline__ void for_keys(const uint32_t* run, F&& f) {
+  const uint4* p = reinterpret_cast<const uint4*>(run);
+#pragma unroll UNROLL
+  for (int j4 = 0; j4 < RC / 4; ++j4) {
+    const uint4 v = p[j4];
+    f(v.x, 4 * j4);
+    f(v.y, 4 * j4 + 1);
+    f(v.z, 4 * j4 + 2);
+    f(v.w, 4 * j4 + 3);
+  }
+}
+
 //
 // Dynamic shared memory of a CTA holding RC keys per thread: the keys,
 // two histograms, the outgoing list, the broadcast slots and the round-A
 // sub-histograms (whose space the copies of every CTA's list reuse later).
 constexpr size_t cluster_smem_words(int RC) {
-  return static_cast<size_t>(kThreads) * (RC + 1) + 2048 + 2048 + kListCapC +
+  return static_cast<size_t>(kThreads) * (RC + 4) + 2048 + 2048 + kListCapC +
          kXSlots * kClusterMax + kSubHist * kWHStride;
 }
 static_assert(kClusterMax * kListCapC <= kSubHist * kWHStride, "list copies fit the sub-histogram space");
@@ -1217,9 +1231,10 @@ __global__ void __launch_bounds__(kThreads, 1) select_cluster_kernel(const Selec
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   __shared__ Shared sh;
   __shared__ unsigned s_cnt;
-  extern __shared__ uint32_t dsm[];
-  uint32_t* keys = dsm;                              // [kThreads][RC + 1]: each thread's run, then a pad word
-  uint32_t* histA = keys + kThreads * (RC + 1);      // [2048]  read by the cluster
+  extern __shared__ __align__(16) uint32_t cluster_dsm[];   // 16-byte loads and DSMEM copies
+  uint32_t* dsm = cluster_dsm;
+  uint32_t* keys = dsm;                              // [kThreads][RC + 4]: each thread's run, then 4 pad words
+  uint32_t* histA = keys + kThreads * (RC + 4);      // [2048]  read by the cluster
   uint32_t* fbh = histA + 2048;                      // [2048]  fallback rounds, read by the cluster
   uint32_t* list = fbh + 2048;                       // [kListCapC] read by the cluster
   uint32_t* xs = list + kListCapC;                   // [kXSlots][kClusterMax] broadcast slots
@@ -1254,7 +1269,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_cluster_kernel(const Selec
     for (int j = 0; j < 32; ++j) {
       const uint32_t k = score_key(f[j]);
       const int e = e0 + 32 * j;
-      keys[e + e / RC] = k;   // one pad word per thread's run: both the fill and the per-thread passes are conflict-free
+      keys[e + 4 * (e / RC)] = k;
       nz += k != 0u ? 1u : 0u;
       mx = max(mx, k);
     }
@@ -1269,9 +1284,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_cluster_kernel(const Selec
   cluster_broadcast(xs, kXCnt, c, C, sh.cnt);
   cluster_sync_all();
 
-  // this thread's RC consecutive elements, followed by one pad word
-  const uint32_t* kvb = keys + (RC + 1) * tid;
-  auto kv = [kvb](int j) { return kvb[j]; };
+  const uint32_t* kvb = keys + (RC + 4) * tid;   // this thread's RC consecutive elements (16-byte aligned)
 
   uint32_t kmax = 0u, total = 0u;
   for (int cc = 0; cc < C; ++cc) {
@@ -1291,14 +1304,13 @@ __global__ void __launch_bounds__(kThreads, 1) select_cluster_kernel(const Selec
     {
       uint32_t* h = sub + (warp % kSubHist) * kWHStride;
       uint32_t nin = 0u;
-#pragma unroll 4
-      for (int j = 0; j < RC; ++j) {
-        const uint32_t d = (kmax - kv(j)) >> kRangeShift;
-        if (kv(j) != 0u && d < 2048u) {
+      for_keys<RC, 2>(kvb, [&](uint32_t k, int) {
+        const uint32_t d = (kmax - k) >> kRangeShift;
+        if (k != 0u && d < 2048u) {
           ++nin;
           atomicAdd(&h[d], 1u);
         }
-      }
+      });
       uint32_t my_in = 0u;
       scan_incl(nin, sh.tmp, &my_in);                // barrier: sub-histograms complete
       for (int bin = tid; bin < 2048; bin += kThreads)
@@ -1320,11 +1332,10 @@ __global__ void __launch_bounds__(kThreads, 1) select_cluster_kernel(const Selec
       if (tid == 0) s_cnt = 0u;
       __syncthreads();
       uint32_t nd = 0u;
-#pragma unroll 4
-      for (int j = 0; j < RC; ++j) {
-        const uint32_t rel = kmax - kv(j);
+      for_keys<RC, 2>(kvb, [&](uint32_t k, int) {
+        const uint32_t rel = kmax - k;
         const uint32_t d = rel >> kRangeShift;
-        if (kv(j) != 0u && d <= b1) {
+        if (k != 0u && d <= b1) {
           if (d < b1) {
             ++nd;
           } else {
@@ -1332,7 +1343,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_cluster_kernel(const Selec
             if (p < kListCapC) list[p] = rel;
           }
         }
-      }
+      });
       uint32_t my_def = 0u;
       scan_incl(nd, sh.tmp, &my_def);
       cluster_broadcast(xs, kXDef, c, C, my_def);
@@ -1406,9 +1417,9 @@ __global__ void __launch_bounds__(kThreads, 1) select_cluster_kernel(const Selec
         if (pass > 0) cluster_sync_all();           // the previous round's histogram has been read
         for (int i = tid; i < nb; i += kThreads) fbh[i] = 0u;
         __syncthreads();
-#pragma unroll 4
-        for (int j = 0; j < RC; ++j)
-          if (kv(j) != 0u && (kv(j) & mask) == prefix) atomicAdd(&fbh[(kv(j) >> shift) & dmask], 1u);
+        for_keys<RC, 1>(kvb, [&](uint32_t k, int) {
+          if (k != 0u && (k & mask) == prefix) atomicAdd(&fbh[(k >> shift) & dmask], 1u);
+        });
         cluster_sync_all();
         cluster_sum(fbh, nb, C, sh.hist);
         __syncthreads();
@@ -1422,11 +1433,10 @@ __global__ void __launch_bounds__(kThreads, 1) select_cluster_kernel(const Selec
         need -= above;
       }
       uint32_t gt = 0u, eq = 0u;
-#pragma unroll 4
-      for (int j = 0; j < RC; ++j) {
-        gt += (kv(j) != 0u && kv(j) > prefix) ? 1u : 0u;
-        eq += (kv(j) != 0u && kv(j) == prefix) ? 1u : 0u;
-      }
+      for_keys<RC, 1>(kvb, [&](uint32_t k, int) {
+        gt += (k != 0u && k > prefix) ? 1u : 0u;
+        eq += (k != 0u && k == prefix) ? 1u : 0u;
+      });
       uint32_t my_gt = 0u, my_eq = 0u;
       scan_incl(gt, sh.tmp, &my_gt);
       scan_incl(eq, sh.tmp, &my_eq);
@@ -1441,12 +1451,11 @@ __global__ void __launch_bounds__(kThreads, 1) select_cluster_kernel(const Selec
 
   // ---- (4) this CTA's selections in index order: per-thread counts, two scans
   uint32_t n_gt = 0u, n_eq = 0u;
-#pragma unroll 4
-  for (int j = 0; j < RC; ++j) {
-    const bool cand = kv(j) != 0u;
-    n_gt += (cand && (t.all || kv(j) > t.thr)) ? 1u : 0u;
-    n_eq += (cand && !t.all && kv(j) == t.thr) ? 1u : 0u;
-  }
+  for_keys<RC, 2>(kvb, [&](uint32_t k, int) {
+    const bool cand = k != 0u;
+    n_gt += (cand && (t.all || k > t.thr)) ? 1u : 0u;
+    n_eq += (cand && !t.all && k == t.thr) ? 1u : 0u;
+  });
   uint32_t eq_tot = 0u;
   const uint32_t eq_before = scan_incl(n_eq, sh.tmp, &eq_tot) - n_eq;      // ties in lower elements of this CTA
   const uint32_t take = t.need_eq > eq_before ? min(t.need_eq - eq_before, n_eq) : 0u;
@@ -1457,9 +1466,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_cluster_kernel(const Selec
   const bool hier = a.mode == kSelectHierTokens;
   if (n_gt + take > 0u) {
     uint32_t taken = 0u;
-#pragma unroll 4
-    for (int j = 0; j < RC; ++j) {
-      const uint32_t k = kv(j);
+    for_keys<RC, 1>(kvb, [&](uint32_t k, int j) {
       bool s = false;
       if (k != 0u) {
         if (t.all || k > t.thr) {
@@ -1473,7 +1480,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_cluster_kernel(const Selec
         const int slot = my_lo + RC * tid + j;
         dyn_out[pos++] = hier ? __ldg(a.pages + prow + slot / a.P) * a.P + slot % a.P : slot;
       }
-    }
+    });
   }
   if (c == C - 1) {
     // the last segment ends the dynamic block: its end is the selected count
