@@ -120,7 +120,8 @@ typedef struct lsa_attn_in {
    * tokens up to pos ascending (LSA abstract (1), SI). The MLA kernel then
    * computes those entries instead of reading them, and its work on them may
    * overlap the kernel in the same stream that writes the rest of idx: that
-   * kernel must not read or write this call's workspace or outputs. A row
+   * kernel may write idx only, and must not read or write this call's
+   * workspace or outputs (q, k, v and seq_len are read before it ends). A row
    * that breaks the promise gives undefined results. */
   int32_t stream_sink, stream_window;
 } lsa_attn_in_t;
