@@ -112,3 +112,47 @@ def test_pool_and_select_validation():
     assert lib.lsa_pool_pages(16, 16, 1, 4096, 128, 24, 16, None) == L.LSA_ERR_UNSUPPORTED
     assert lib.lsa_pool_pages(16, 16, 1, 4000, 128, 64, 16, None) == L.LSA_ERR_INVALID_ARG
     assert lib.lsa_select_streaming(None, 16, 1, 1, 128, L.Budget(8, 2, 2), 16, None, 0, None) == L.LSA_ERR_INVALID_ARG
+
+
+def test_compressed_entry_validation_and_sizes():
+    lib = L.load()
+    bu = L.Budget(2048, 16, 240)
+    for m in (3, 256, 0):
+        ii = _indexer(L_max=4096)
+        assert lib.lsa_index_compressed(ctypes.byref(ii), m, bu, 16, None, None, 0, None) == L.LSA_ERR_UNSUPPORTED
+    ii = _indexer(L_max=4096)
+    assert lib.lsa_index_compressed(ctypes.byref(ii), 4, bu, None, None, None, 0, None) == L.LSA_ERR_INVALID_ARG
+    big = _indexer(B=4, L_max=1 << 20)
+    n = L.workspace_size(L.LSA_OP_INDEX_COMPRESSED, indexer=big, budget=(2048, 16, 240), m=4)
+    assert n == 4 * (1 << 18) * 4          # entry scores only: 262144-entry rows select in cluster shared memory
+    assert L.workspace_size(L.LSA_OP_INDEX_COMPRESSED, indexer=big, budget=(2048, 16, 240), m=4,
+                            scores_external=True) == 0
+    st = lib.lsa_index_compressed(ctypes.byref(big), 4, bu, 16, None, 256, n - 1, None)
+    assert st == L.LSA_ERR_WORKSPACE
+
+
+def test_cluster_selection_covers_rows_up_to_262144_slots():
+    assert L.workspace_size(L.LSA_OP_SELECT, budget=(2048, 64, 960), B=4, T=1, L_max=262144) == 0
+    assert L.workspace_size(L.LSA_OP_SELECT, budget=(2048, 64, 960), B=4, T=1, L_max=262144 + 64 + 960 + 1) > 0
+
+
+def _mla_layer(q, kv, B=1, T=1, L_max=1024, Hq=128):
+    return L.AttnIn(B, T, Hq, 576, 512, L_max, 0.04, 16, q, kv, kv, 576, 576, -1, -1)
+
+
+def test_layer_group_rejects_overlapping_outputs_on_host():
+    lib = L.load()
+    ii = _indexer(L_max=1024)
+    layers = (L.AttnIn * 2)(_mla_layer(1 << 20, 2 << 20), _mla_layer(3 << 20, 4 << 20))
+    bu = L.Budget(256, 16, 64)
+    out_bytes = 1 * 1 * 128 * 512 * 2
+    base = 64 << 20
+    for o1 in (base, base + out_bytes - 256):        # the same buffer, then a partial overlap
+        outs = (ctypes.c_void_p * 2)(base, o1)
+        st = lib.lsa_layer_group(ctypes.byref(ii), None, 0, 0, bu, 2, layers, outs, None, None, None, 0, None)
+        assert st == L.LSA_ERR_INVALID_ARG, lib.lsa_last_error()
+        assert b"overlap" in lib.lsa_last_error()
+    outs = (ctypes.c_void_p * 2)(base, base + out_bytes)
+    idx_over = base + out_bytes + 512                  # idx inside the second layer's output
+    st = lib.lsa_layer_group(ctypes.byref(ii), None, 0, 0, bu, 2, layers, outs, None, idx_over, None, 0, None)
+    assert st == L.LSA_ERR_INVALID_ARG and b"idx" in lib.lsa_last_error()
