@@ -548,3 +548,21 @@ def test_compressed_entry_select_brute_force(seed):
     for t in range(T):
         pe = (int(sl[0]) - T + t + 1) // m - 1
         assert idx[0, t].tolist() == _brute_select(sc[0, t].tolist(), pe, 12, 2, 3)
+
+
+def test_compressed_inputs_plant_needles_in_dynamic_entries():
+    """Entry needles sit in the decode query's dynamic entries (between the sink
+    entries and the window entries of its last complete entry), and every index
+    the oracle picks there is a complete, visible entry."""
+    w = I.scaled(I.WORKLOADS["compressed_decode_1m"], B=1, L=32768, needle_frac=0.0, needles=12)
+    x = I.make_compressed_inputs(w, seed=2)
+    n_e = w.L // w.m
+    assert x["entry_keys"].shape == (1, n_e, w.d) and int(x["seq_len"][0]) == w.L
+    npos = x["needle_pos"][0]
+    npos = npos[npos >= 0]
+    pe = O.entry_position(w.L - 1, w.m)
+    assert npos.size == 12 and (npos >= w.sink).all() and (npos <= pe - w.window).all()
+    idx, _ = O.index_compressed(x["q_idx"], x["w"], x["entry_keys"], x["seq_len"], m=w.m, budget=w.k,
+                                sink=w.sink, window=w.window)
+    sel = idx[0, 0][idx[0, 0] >= 0]
+    assert sel.size == w.k and (sel <= pe).all() and np.unique(sel).size == sel.size
