@@ -5,6 +5,7 @@
 // synchronises the stream (except lsa_device_status, which exists to do so).
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -461,29 +462,38 @@ lsa_status_t set_error(lsa_status_t st, const char* fmt, ...) {
   return st;
 }
 
+// Per-device caches, filled on first use; safe under concurrent calls from several
+// host threads (both racers store the same value). Devices beyond the table are
+// looked up on every call.
+constexpr int kCachedDevices = 64;
+
 int* device_status_ptr() {
-  static int* cache[64] = {nullptr};
+  static std::atomic<int*> cache[kCachedDevices] = {};
   int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64) dev = 0;
-  if (!cache[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_device_status) == cudaSuccess) cache[dev] = static_cast<int*>(p);
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;   // kernels skip the status word if null
+  const bool cached = dev >= 0 && dev < kCachedDevices;
+  if (cached) {
+    if (int* c = cache[dev].load(std::memory_order_acquire)) return c;
   }
-  return cache[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+  if (cached) cache[dev].store(static_cast<int*>(p), std::memory_order_release);
+  return static_cast<int*>(p);
 }
 
 int device_sm_count() {
-  static int cache[64] = {0};
+  static std::atomic<int> cache[kCachedDevices] = {};
   int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64) dev = 0;
-  if (!cache[dev]) {
-    int n = 0;
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    cache[dev] = n > 0 ? n : 148;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;   // no device: plans are only sized (workspace queries)
+  const bool cached = dev >= 0 && dev < kCachedDevices;
+  if (cached) {
+    if (const int c = cache[dev].load(std::memory_order_relaxed)) return c;
   }
-  return cache[dev];
+  int n = 0;
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  if (n <= 0) n = 148;
+  if (cached) cache[dev].store(n, std::memory_order_relaxed);
+  return n;
 }
 
 cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, size_t smem, cudaStream_t stream, void** args,
