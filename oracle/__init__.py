@@ -9,4 +9,5 @@ from .lsa_oracle import (  # noqa: F401
     streaming_regions, top_by_score, select_streaming_row, select_streaming,
     index_flat, pool_pages, page_sets, index_hier_row, index_hier,
     sparse_attention_row, sparse_attention, layer_group, entry_position, index_compressed,
+    f64_to_e4m3_rne, pool_pages_e4m3, index_hier_e4m3,
 )

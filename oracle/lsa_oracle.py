@@ -55,6 +55,12 @@ R11 Compressed entries (the DSA article's "Technical Evolution": the indexer
     name no compressor). Scores are R1 on the entry keys; the selection is
     R3-R5 over entries, at entry position (pos + 1) // m - 1, with budget, sink
     and window counted in entries. m = 1 is flat indexing.
+R12 FP8 hierarchical indexing (the survey's next item; the pages only name
+    "quantized computation"): token keys and queries as R10. A page key is the
+    float32 mean of its tokens' dequantized keys (R6's order and division),
+    stored as e4m3 with a float32 page scale amax / 448 (round to nearest even,
+    saturating), like the token keys. Page and fine scores are R1 on the
+    dequantized values; recall and selection as R7.
 """
 from __future__ import annotations
 
@@ -90,6 +96,28 @@ def f32_to_bf16_rne(x: np.ndarray) -> np.ndarray:
     is_nan = (u & np.uint64(0x7FFFFFFF)) > np.uint64(0x7F800000)
     r = np.where(is_nan, upper | np.uint64(0x0040), r)
     return r.astype(np.uint16)
+
+
+def _e4m3_table():
+    """The 127 non-negative finite e4m3 values, ascending, and their codes."""
+    codes = np.arange(0x7F, dtype=np.uint8)
+    return e4m3_to_f64(codes), codes
+
+
+def f64_to_e4m3_rne(x: np.ndarray) -> np.ndarray:
+    """Real value -> e4m3 code: the nearest finite e4m3 value, ties to the even
+    code, magnitudes beyond 448 saturating to 448; the sign bit follows x (-0
+    included). Written as a search over the value table, not bit arithmetic."""
+    vals, codes = _e4m3_table()
+    x = np.asarray(x, dtype=np.float64)
+    a = np.minimum(np.abs(x), vals[-1])
+    hi = np.clip(np.searchsorted(vals, a, side="left"), 0, vals.size - 1)
+    lo = np.maximum(hi - 1, 0)
+    d_lo, d_hi = a - vals[lo], vals[hi] - a
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & ((codes[hi] & 1) == 0))
+    c = np.where(pick_hi, codes[hi], codes[lo]).astype(np.uint8)
+    c = np.where(a == vals[hi], codes[hi], c).astype(np.uint8)
+    return (c | np.where(np.signbit(x), 0x80, 0).astype(np.uint8)).astype(np.uint8)
 
 
 def e4m3_to_f64(codes: np.ndarray) -> np.ndarray:
@@ -352,6 +380,52 @@ def index_hier(q, w, k, page_keys, seq_len, *, P: int, M: int, budget: int,
             idx[b, t], pages[b, t] = index_hier_row(
                 bf16_to_f64(q[b, t]), np.asarray(w[b, t], np.float64), kd, pk,
                 pos, P, M, budget, sink, window)
+    return idx, pages
+
+
+def pool_pages_e4m3(k8: np.ndarray, k_scale: np.ndarray, seq_len: np.ndarray, P: int):
+    """Page keys from e4m3 token keys (R12): k8 [B, L_max, d] codes with
+    k_scale [B, L_max] -> (page codes [B, L_max // P, d], page scales [B, L_max // P]).
+    Pages that are not full are returned as code 0 with scale 1."""
+    B, L_max, d = k8.shape
+    n_pages = L_max // P
+    codes = np.zeros((B, n_pages, d), dtype=np.uint8)
+    scales = np.ones((B, n_pages), dtype=np.float32)
+    for b in range(B):
+        L = int(min(max(int(seq_len[b]), 0), L_max))
+        n_full = L // P
+        if n_full == 0:
+            continue
+        x = (e4m3_to_f64(k8[b, :n_full * P]).astype(np.float32) *
+             np.asarray(k_scale[b, :n_full * P], np.float32)[:, None]).astype(np.float32)
+        x = x.reshape(n_full, P, d)
+        acc = np.zeros((n_full, d), dtype=np.float32)
+        for j in range(P):                      # float32 adds, ascending row order
+            acc = (acc + x[:, j, :]).astype(np.float32)
+        mean = (acc / np.float32(P)).astype(np.float32)
+        amax = np.max(np.abs(mean), axis=1)
+        sc = np.where(amax > 0, amax / np.float32(448.0), np.float32(1.0)).astype(np.float32)
+        codes[b, :n_full] = f64_to_e4m3_rne((mean / sc[:, None]).astype(np.float32))
+        scales[b, :n_full] = sc
+    return codes, scales
+
+
+def index_hier_e4m3(q8, q_scale, w, k8, k_scale, page_codes, page_scales, seq_len, *, P: int,
+                    M: int, budget: int, sink: int, window: int):
+    """FP8 hierarchical indexing (R12): R7 on dequantized queries, token keys and
+    page keys. Returns (idx [B,T,k], pages [B,T,M])."""
+    B, T = q8.shape[0], q8.shape[1]
+    L_max = k8.shape[1]
+    idx = np.full((B, T, budget), -1, dtype=np.int32)
+    pages = np.full((B, T, M), -1, dtype=np.int32)
+    for b in range(B):
+        L = int(min(max(int(seq_len[b]), 0), L_max))
+        kd = _decode_k(k8[b, :L], k_scale[b, :L], True)
+        pk = _decode_k(page_codes[b, :L // P], page_scales[b, :L // P], True)
+        for t in range(T):
+            idx[b, t], pages[b, t] = index_hier_row(
+                _decode_q(q8[b, t], q_scale[b, t], True), np.asarray(w[b, t], np.float64), kd, pk,
+                L - T + t, P, M, budget, sink, window)
     return idx, pages
 
 

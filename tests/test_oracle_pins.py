@@ -566,3 +566,73 @@ def test_compressed_inputs_plant_needles_in_dynamic_entries():
                                 sink=w.sink, window=w.window)
     sel = idx[0, 0][idx[0, 0] >= 0]
     assert sel.size == w.k and (sel <= pe).all() and np.unique(sel).size == sel.size
+
+
+# ---------------------------------------------------------------------------
+# FP8 hierarchical indexing (oracle only; no kernel path yet)
+# ---------------------------------------------------------------------------
+
+
+def test_oracle_e4m3_encoder_matches_torch():
+    rng = np.random.default_rng(31)
+    x = np.concatenate([rng.standard_normal(40000) * 50, rng.standard_normal(4000) * 0.01,
+                        [0.0, -0.0, 448.0, -448.0, 2.0 ** -9, 3 * 2.0 ** -10, 5 * 2.0 ** -10, 17.0, 19.0, 240.0]])
+    x = np.clip(x, -448.0, 448.0).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(O.f64_to_e4m3_rne(x), ref)
+    assert O.f64_to_e4m3_rne(np.array([500.0, -1e6]))[0] == 0x7E           # saturating
+    assert O.f64_to_e4m3_rne(np.array([-1e6]))[0] == 0xFE
+
+
+def test_pool_pages_e4m3_closed_form():
+    # one full page of P = 4 identical tokens [1, 2, 0.5, -1] (scale 1): the mean is
+    # the same row, amax 2 -> page scale 2/448, codes of 224, 448, 112, -224
+    row = O.f64_to_e4m3_rne(np.array([1.0, 2.0, 0.5, -1.0]))
+    k8 = np.tile(row, (1, 6, 1)).astype(np.uint8)                              # 6 tokens: page 1 is partial
+    ks = np.ones((1, 6), np.float32)
+    codes, scales = O.pool_pages_e4m3(k8, ks, np.array([6], np.int32), 4)
+    assert codes.shape == (1, 1, 4) and scales[0, 0] == np.float32(2.0) / np.float32(448.0)
+    assert O.e4m3_to_f64(codes[0, 0]).tolist() == [224.0, 448.0, 112.0, -224.0]
+    # token scales act before the mean: halving every token's scale halves the page scale only
+    codes2, scales2 = O.pool_pages_e4m3(k8, ks * np.float32(0.5), np.array([6], np.int32), 4)
+    assert np.array_equal(codes2, codes) and scales2[0, 0] == scales[0, 0] * np.float32(0.5)
+    # a page whose tokens differ: the mean of the dequantized rows, then quantized
+    k8b = O.f64_to_e4m3_rne(np.array([[[1.0, 0.0]], [[3.0, 0.0]], [[2.0, 4.0]], [[2.0, 0.0]]]).reshape(1, 4, 2))
+    cb, sb = O.pool_pages_e4m3(k8b, np.ones((1, 4), np.float32), np.array([4], np.int32), 4)
+    assert sb[0, 0] == np.float32(2.0) / np.float32(448.0)                     # mean row (2, 1): amax 2
+    assert O.e4m3_to_f64(cb[0, 0]).tolist() == [448.0, 224.0]
+
+
+@pytest.mark.parametrize("P,L", [(4, 128), (16, 512)])
+def test_hier_e4m3_full_recall_equals_flat_e4m3(P, L):
+    rng = np.random.default_rng(7 * P + L)
+    B, T, H, d = 2, 3, 4, 32
+    q8, qs = I.quantize_e4m3_rows(rng.standard_normal((B, T, H, d)).astype(np.float32))
+    k8, ks = I.quantize_e4m3_rows(rng.standard_normal((B, L, d)).astype(np.float32))
+    w = rng.random((B, T, H)).astype(np.float32)
+    sl = np.array([L, L - 9], np.int32)
+    kk, S, W = 48, 4, 12
+    pc, ps = O.pool_pages_e4m3(k8, ks, sl, P)
+    M = -(-L // P) + 2                                                         # M * P >= L: every page recalled
+    idx_f, _ = O.index_flat(q8, w, k8, sl, budget=kk, sink=S, window=W, q_scale=qs, k_scale=ks, fp8=True)
+    idx_h, pages = O.index_hier_e4m3(q8, qs, w, k8, ks, pc, ps, sl, P=P, M=M, budget=kk, sink=S, window=W)
+    assert np.array_equal(idx_f, idx_h)
+
+
+def test_hier_e4m3_recalls_a_planted_page():
+    """A page whose P tokens all copy one query head's vector scores highest among
+    the eligible pages for that query, so a recall of one dynamic page takes it."""
+    rng = np.random.default_rng(41)
+    B, T, H, d, L, P = 1, 1, 2, 32, 512, 16
+    qf = rng.standard_normal((B, T, H, d)).astype(np.float32)
+    kf = rng.standard_normal((B, L, d)).astype(np.float32) * 0.3
+    kf[0, 10 * P:11 * P] = qf[0, 0, 0] * 2.0                                     # page 10
+    q8, qs = I.quantize_e4m3_rows(qf)
+    k8, ks = I.quantize_e4m3_rows(kf)
+    w = np.array([[[1.0, 0.0]]], np.float32)                                    # only head 0 counts
+    sl = np.array([L], np.int32)
+    pc, ps = O.pool_pages_e4m3(k8, ks, sl, P)
+    S, W = 16, 16                                                               # forced pages: 0 and 31
+    idx, pages = O.index_hier_e4m3(q8, qs, w, k8, ks, pc, ps, sl, P=P, M=3, budget=64, sink=S, window=W)
+    assert pages[0, 0].tolist() == [0, 10, 31]
+    assert set(range(10 * P, 11 * P)) <= set(idx[0, 0].tolist())
