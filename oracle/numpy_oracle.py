@@ -1,4 +1,9 @@
-"""CPU oracle for the LSA hot path: indexer -> streaming top-k -> sparse attention.
+"""A second restatement of the LSA oracle in numpy/BLAS, kept as a cross-check.
+
+The oracle of record is the plain C++ in ``oracle/lsa_oracle.cpp`` (loaded by
+``oracle/__init__.py``). This module computes the same definitions
+independently, through numpy and BLAS, and ``tests/test_oracle_cross_check.py``
+holds the two to each other function by function.
 
 TEST INFRASTRUCTURE ONLY. Only ``tests/``, ``__graft_entry__.smoke()`` and the
 CPU-baseline / reference legs of ``bench.py`` may import or run this module. The
