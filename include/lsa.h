@@ -211,10 +211,12 @@ lsa_status_t lsa_select_streaming(const float* scores, const int32_t* seq_len, i
  * into the library.
  *   - Shapes whose scratch (lsa_workspace_size with LSA_OP_SELECT) exceeds
  *     LSA_NOALLOC_SCRATCH_BYTES are rejected with LSA_ERR_WORKSPACE before
- *     anything is launched; with k=2048, sink+window=1024 that admits e.g.
- *     B*T=8 rows up to L_max=1M, or 148 rows up to L_max=8K.
- *   - The first call on a device looks up the buffer's device address (which
- *     may load the library's device code onto that device); make that first
+ *     anything is launched. Rows of up to 262144 score slots need no
+ *     scratch at all (any number of rows); longer rows do: with k=2048 and
+ *     sink+window=1024 on a 148-SM B200, L_max=1M admits up to 15 rows.
+ *   - The first call on a device (and the first after its context changes,
+ *     e.g. after cudaDeviceReset) looks up the buffer's device address, which
+ *     may load the library's device code onto that device; make that first
  *     call, per device, before any stream capture begins.
  *   - Every call on a device shares the buffer. Calls whose kernels may
  *     overlap on the GPU (different streams without ordering) race on it and

@@ -462,24 +462,65 @@ lsa_status_t set_error(lsa_status_t st, const char* fmt, ...) {
   return st;
 }
 
-// Per-device caches, filled on first use; safe under concurrent calls from several
-// host threads (both racers store the same value). Devices beyond the table are
-// looked up on every call.
-constexpr int kCachedDevices = 64;
+// Identity of the CUDA context current on this host thread, 0 if there is none
+// yet (or the driver cannot say). The device address of a __device__ symbol is
+// valid only in the context that loaded this library's module, so per-device
+// caches of such addresses are keyed by it: after cudaDeviceReset (or any other
+// new context) the address is looked up again.
+unsigned long long current_context_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  if (!get_current || !get_id) return 0;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+  unsigned long long id = 0;
+  return get_id(ctx, &id) == CUDA_SUCCESS ? id : 0;
+}
+
+void* symbol_address_cached(SymbolCache* cache, const void* symbol, cudaError_t* err) {
+  *err = cudaSuccess;
+  int dev = 0;
+  if ((*err = cudaGetDevice(&dev)) != cudaSuccess) return nullptr;
+  const unsigned long long ctx = current_context_id();
+  std::lock_guard<std::mutex> lock(cache->mu);
+  if (dev >= 0 && dev < SymbolCache::kDevices && ctx != 0 && cache->ctx[dev] == ctx) return cache->ptr[dev];
+  void* p = nullptr;
+  if ((*err = cudaGetSymbolAddress(&p, symbol)) != cudaSuccess) return nullptr;
+  if (!p) {
+    *err = cudaErrorInvalidSymbol;
+    return nullptr;
+  }
+  // the lookup made the device's primary context current if none was
+  const unsigned long long now = ctx != 0 ? ctx : current_context_id();
+  if (dev >= 0 && dev < SymbolCache::kDevices && now != 0) {
+    cache->ctx[dev] = now;
+    cache->ptr[dev] = p;
+  }
+  return p;
+}
 
 int* device_status_ptr() {
-  static std::atomic<int*> cache[kCachedDevices] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;   // kernels skip the status word if null
-  const bool cached = dev >= 0 && dev < kCachedDevices;
-  if (cached) {
-    if (int* c = cache[dev].load(std::memory_order_acquire)) return c;
-  }
-  void* p = nullptr;
-  if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
-  if (cached) cache[dev].store(static_cast<int*>(p), std::memory_order_release);
-  return static_cast<int*>(p);
+  static SymbolCache cache;
+  cudaError_t e;
+  return static_cast<int*>(symbol_address_cached(&cache, &g_device_status, &e));   // kernels skip a null word
 }
+
+// SM counts per device ordinal, filled on first use; safe under concurrent calls
+// (both racers store the same value). Ordinals beyond the table are looked up
+// on every call.
+constexpr int kCachedDevices = 64;
 
 int device_sm_count() {
   static std::atomic<int> cache[kCachedDevices] = {};

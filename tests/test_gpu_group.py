@@ -6,9 +6,25 @@ import torch
 import oracle as O
 from kv_indexing_b200 import inputs as I
 from kv_indexing_b200 import lsa as L
-from tests.parity import assert_attention_close, check_index_row, dev, host, lead_count
+from tests.parity import assert_attention_close, check_hier_rows, check_index_row, dev, host, same_rows
 
 pytestmark = pytest.mark.gpu
+
+
+def check_layer_outputs(gi, oi, specs, outs, lses=None):
+    """Each layer's GPU output against the oracle's attention over the oracle's
+    own index set, on the rows whose GPU index row equals it (the others are
+    near-tie swaps judged by the index checks). specs: (inputs, scale, d_v, mla)."""
+    rows = same_rows(gi, oi)
+    assert len(rows) * 2 >= gi.shape[0] * gi.shape[1], "too few index rows equal the oracle's"
+    for i, ((l, scale, d_v, mla), out) in enumerate(zip(specs, outs)):
+        kw = dict(kv=l["kv"]) if mla else dict(k=l["k"], v=l["v"])
+        o_ref, l_ref = O.sparse_attention_rows(l["qa"], oi, rows, scale=scale, d_v=d_v, **kw)
+        g = O.bf16_to_f64(host(out))
+        assert_attention_close(np.stack([g[b, t] for b, t in rows]), o_ref)
+        if lses is not None:
+            gl = host(lses[i])
+            assert np.allclose(np.stack([gl[b, t] for b, t in rows]), l_ref, atol=1e-3, rtol=1e-3)
 
 
 @pytest.mark.parametrize("hier", [False, True])
@@ -28,22 +44,23 @@ def test_group_two_layers(hier):
     L.lsa_device_status()
     gi = host(idx)
     # the group's index set equals the single indexing call's, bit for bit
+    rows = [(b, 0) for b in range(w.B)]
     if hier:
-        ref_i, _ = L.lsa_index_hier(q, ww, k, sl, pk, P, M, budget)
+        pages = torch.empty((w.B, 1, M), dtype=torch.int32, device="cuda")
+        ref_i, _ = L.lsa_index_hier(q, ww, k, sl, pk, P, M, budget, pages_out=pages)
+        torch.cuda.synchronize()
+        oi = check_hier_rows(x, x["seq_len"], P, M, budget, gi, host(pages), rows)
     else:
         ref_i = L.lsa_index_flat(q, ww, k, sl, budget)
-    torch.cuda.synchronize()
-    assert np.array_equal(gi, host(ref_i))
-    # and every layer's output is attention over that set (both layers share one
-    # launch, whose split plan differs from a single-layer call's)
-    for lnp, out in zip(layers_np, outs):
-        o_ref, _ = O.sparse_attention(lnp["qa"], gi, x["seq_len"], scale=w.scale, d_v=w.d_v, kv=lnp["kv"])
-        assert_attention_close(O.bf16_to_f64(host(out)), o_ref)
-    if not hier:
+        torch.cuda.synchronize()
         os_ = O.indexer_scores(x["q_idx"], x["w"], x["k_idx"], x["seq_len"])
         oi = O.select_streaming(os_, x["seq_len"], 1, *budget)
         for b in range(w.B):
-            check_index_row(gi[b, 0], oi[b, 0], os_[b, 0], lead_count(w.L - 1, w.sink, w.window))
+            check_index_row(gi[b, 0], oi[b, 0], os_[b, 0], w.L - 1, w.sink, w.window)
+    assert np.array_equal(gi, host(ref_i))
+    # every layer's output is attention over that set (both layers share one
+    # launch, whose split plan differs from a single-layer call's)
+    check_layer_outputs(gi, oi, [(lnp, w.scale, w.d_v, True) for lnp in layers_np], outs)
 
 
 def test_group_mixed_layers_and_launch_chunks():
@@ -74,14 +91,8 @@ def test_group_mixed_layers_and_launch_chunks():
     os_ = O.indexer_scores(x["q_idx"], x["w"], x["k_idx"], sl_np)
     oi = O.select_streaming(os_, sl_np, 1, *budget)
     for b in range(w.B):
-        check_index_row(gi[b, 0], oi[b, 0], os_[b, 0], lead_count(int(sl_np[b]) - 1, w.sink, w.window))
-    for s_, l, out, lse in zip(specs, lnps, outs, lses):
-        if s_.mla:
-            o_ref, l_ref = O.sparse_attention(l["qa"], gi, sl_np, scale=s_.scale, d_v=s_.d_v, kv=l["kv"])
-        else:
-            o_ref, l_ref = O.sparse_attention(l["qa"], gi, sl_np, scale=s_.scale, d_v=s_.d_v, k=l["k"], v=l["v"])
-        assert_attention_close(O.bf16_to_f64(host(out)), o_ref)
-        assert np.allclose(host(lse), l_ref, atol=1e-3, rtol=1e-3)
+        check_index_row(gi[b, 0], oi[b, 0], os_[b, 0], int(sl_np[b]) - 1, w.sink, w.window)
+    check_layer_outputs(gi, oi, [(l, s_.scale, s_.d_v, s_.mla) for s_, l in zip(specs, lnps)], outs, lses)
 
 
 def test_group_five_mla_layers():
@@ -98,9 +109,10 @@ def test_group_five_mla_layers():
     torch.cuda.synchronize()
     L.lsa_device_status()
     gi = host(idx)
-    for l, sc, out in zip(lnps, scales, outs):
-        o_ref, _ = O.sparse_attention(l["qa"], gi, x["seq_len"], scale=sc, d_v=w.d_v, kv=l["kv"])
-        assert_attention_close(O.bf16_to_f64(host(out)), o_ref)
+    oi, os_ = O.index_flat(x["q_idx"], x["w"], x["k_idx"], x["seq_len"], budget=w.k, sink=w.sink, window=w.window)
+    for t in range(w.T):
+        check_index_row(gi[0, t], oi[0, t], os_[0, t], w.L - w.T + t, w.sink, w.window)
+    check_layer_outputs(gi, oi, [(l, sc, w.d_v, True) for l, sc in zip(lnps, scales)], outs)
 
 
 def test_group_rejects_overlapping_outputs():

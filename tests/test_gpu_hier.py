@@ -7,7 +7,7 @@ import torch
 import oracle as O
 from kv_indexing_b200 import inputs as I
 from kv_indexing_b200 import lsa as L
-from tests.parity import check_index_row, dev, host, lead_count
+from tests.parity import check_hier_rows, dev, host
 
 pytestmark = pytest.mark.gpu
 
@@ -27,12 +27,6 @@ def test_pool_pages_bit_exact(P):
         assert (got[b, nf:] == 0).all()                          # untouched (zero-initialised)
 
 
-def page_scores_oracle(x, pk, b, t, pos, P):
-    n = (pos + 1) // P
-    return O.indexer_scores_row(O.bf16_to_f64(x["q_idx"][b, t]), x["w"][b, t].astype(np.float64),
-                                O.bf16_to_f64(pk[b, :n]), n)
-
-
 def check_hier(w, x, seq_len, P, M, budget):
     q, k = dev(x["q_idx"], "bf16"), dev(x["k_idx"], "bf16")
     sl = dev(seq_len, "i32")
@@ -43,38 +37,9 @@ def check_hier(w, x, seq_len, P, M, budget):
     torch.cuda.synchronize()
     L.lsa_device_status()
     gi, gp = host(idx), host(pages)
-    pk_o = O.pool_pages(x["k_idx"], seq_len, P)
-    assert np.array_equal(host(pk)[:, :int(seq_len.min()) // P], pk_o[:, :int(seq_len.min()) // P])
-    oi, op = O.index_hier(x["q_idx"], x["w"], x["k_idx"], pk_o, seq_len, P=P, M=M, budget=budget[0],
-                          sink=budget[1], window=budget[2])
-    kd = None
-    for b in range(B):
-        for t in range(T):
-            pos = int(seq_len[b]) - T + t
-            forced, E = O.page_sets(pos, P, budget[1], budget[2])
-            psc = np.full(pk_o.shape[1], -np.inf, np.float32)
-            psc[:(pos + 1) // P] = page_scores_oracle(x, pk_o, b, t, pos, P)
-            g_pages = gp[b, t][gp[b, t] >= 0]
-            o_pages = op[b, t][op[b, t] >= 0]
-            assert set(forced) <= set(g_pages.tolist())
-            gd = np.setdiff1d(g_pages, forced)
-            od = np.setdiff1d(o_pages, forced)
-            if gd.size and not np.array_equal(gd, od):
-                tau = float(psc[od].min())
-                for pgi in np.setdiff1d(np.union1d(gd, od), np.intersect1d(gd, od)):
-                    assert abs(float(psc[pgi]) - tau) <= 1e-3 * abs(tau), "page recall differs beyond near-ties"
-            # token level: valid top-D over the GPU's recalled pages, by oracle scores
-            if kd is None or kd[0] != b:
-                kd = (b, O.bf16_to_f64(x["k_idx"][b, :int(seq_len[b])]))
-            _, _, c_rng = O.streaming_regions(pos, budget[1], budget[2])
-            cands = np.arange(c_rng.start, c_rng.stop)
-            cands = cands[np.isin(cands // P, g_pages)]
-            tsc = np.full(int(seq_len[b]), -np.inf, np.float32)
-            if cands.size:
-                tsc[cands] = O.indexer_scores_row(O.bf16_to_f64(x["q_idx"][b, t]), x["w"][b, t].astype(np.float64),
-                                                  kd[1][cands], cands.size)
-            ref = oi[b, t] if np.array_equal(gd, od) else O.select_streaming_row(tsc, pos, *budget)
-            check_index_row(gi[b, t], ref, tsc, lead_count(pos, budget[1], budget[2]))
+    n_full = int(seq_len.min()) // P
+    assert np.array_equal(host(pk)[:, :n_full], O.pool_pages(x["k_idx"], seq_len, P)[:, :n_full])
+    check_hier_rows(x, seq_len, P, M, budget, gi, gp, [(b, t) for b in range(B) for t in range(T)])
     return gi, gp
 
 

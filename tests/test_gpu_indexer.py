@@ -7,8 +7,7 @@ import torch
 import oracle as O
 from kv_indexing_b200 import inputs as I
 from kv_indexing_b200 import lsa as L
-from tests.parity import (accumulation_scale, assert_scores_close, check_index_row, dev, host,
-                          lead_count)
+from tests.parity import (accumulation_scale, assert_scores_close, check_index_row, dev, host)
 
 pytestmark = pytest.mark.gpu
 
@@ -46,7 +45,7 @@ def check_flat(x, budget, fp8=False):
     for b in range(B):
         for t in range(T):
             pos = int(x["seq_len"][b]) - T + t
-            swaps += check_index_row(gi[b, t], oi[b, t], os_[b, t], lead_count(pos, budget[1], budget[2]))
+            swaps += check_index_row(gi[b, t], oi[b, t], os_[b, t], pos, budget[1], budget[2])
     return worst, swaps
 
 

@@ -5,8 +5,9 @@ It exists for callers that cannot allocate device memory where they select: a
 plugin inside a serving engine that has reserved its GPU memory up front for
 its own KV cache, or a latency-critical decode path that cannot afford
 cudaMalloc/cudaFree (which may block the host and synchronise the device).
-Its output must equal lsa_select_streaming's exactly (index work is compared
-bit for bit), call after call, although every call reuses the same scratch.
+Its output must equal the oracle's and lsa_select_streaming's exactly (index
+work is compared bit for bit), call after call, although every call reuses the
+same scratch.
 
 This file is collected last so that a run stopping at its first failure has
 run every other test before it."""
@@ -16,6 +17,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle as O
 from kv_indexing_b200 import lsa as L
 from tests.parity import dev, host
 
@@ -54,26 +56,43 @@ def _scores(seed, B, T, L_max, seq_len, ties=False):
     return sc
 
 
-# (seed, B, T, L_max, seq_len, budget, ties): a decode batch at 128K keys, the
-# same shape again with new scores (leftover scratch must not leak into it),
-# then 160 ragged query rows with heavy ties (more rows than SMs: the other
-# launch shape).
+# Consecutive calls on the two launch shapes that keep scratch in the static
+# buffer. Rows longer than 262144 slots go to the grid-cooperative launch while
+# rows x CTAs fit the GPU at once (4 rows of 300000 slots: about 1 MiB of
+# per-row coordination blocks, counters and flags); otherwise to per-segment
+# candidate lists merged by the last CTA of each row (15 rows of 1M slots: about
+# 15.7 MiB, just under the limit). Each shape runs twice with new scores and
+# interleaved with the other, so leftovers of one call sit in the scratch when
+# the next starts.
+GRID = (4, 1, 300000, (2048, 64, 960))
+TWO_LEVEL = (15, 1, 1 << 20, (2048, 64, 960))
 CALLS = [
-    (11, 8, 1, 131072, [131072, 131072, 100000, 131072, 65536, 131072, 3000, 131072], (2048, 64, 960), False),
-    (12, 8, 1, 131072, [131072, 77777, 131072, 131072, 131072, 20000, 131072, 131072], (2048, 64, 960), False),
-    (13, 4, 40, 20000, [20000, 9000, 30, 15000], (512, 16, 100), True),
+    (21, GRID, [300000, 300000, 123457, 299999], True),
+    (22, TWO_LEVEL, [1 << 20] * 12 + [700001, 5000, 1 << 20], False),
+    (23, GRID, [299000, 300000, 300000, 65536], False),
+    (24, TWO_LEVEL, [1 << 20, 999999] + [1 << 20] * 13, True),
 ]
 
 
+def test_noalloc_shapes_use_the_static_scratch():
+    # guard: if a plan change stopped these shapes from using scratch, the GPU
+    # test below would no longer reach the static buffer
+    for B, T, L_max, budget in (GRID, TWO_LEVEL):
+        need = L.workspace_size(L.LSA_OP_SELECT, budget=budget, B=B, T=T, L_max=L_max)
+        assert 0 < need <= L.LSA_NOALLOC_SCRATCH_BYTES, (B, L_max, need)
+
+
 @pytest.mark.gpu
-def test_noalloc_select_matches_workspace_select_on_consecutive_calls():
-    for seed, B, T, L_max, seq_len, budget, ties in CALLS:
+def test_noalloc_select_matches_oracle_and_workspace_select_on_consecutive_calls():
+    for seed, (B, T, L_max, budget), seq_len, ties in CALLS:
         sl = np.array(seq_len, np.int32)
-        sc_d = dev(_scores(seed, B, T, L_max, sl, ties), "f32")
-        sl_d = dev(sl, "i32")
+        sc = _scores(seed, B, T, L_max, sl, ties)
+        sc_d, sl_d = dev(sc, "f32"), dev(sl, "i32")
         idx = torch.full((B, T, budget[0]), -7, dtype=torch.int32, device="cuda")
         L.lsa_select_streaming_noalloc(sc_d, sl_d, budget, idx=idx)
         ref = L.lsa_select_streaming(sc_d, sl_d, budget)
         torch.cuda.synchronize()
         assert L.lsa_device_status() == L.LSA_OK
-        assert np.array_equal(host(idx), host(ref)), (seed, B, T, L_max)
+        got = host(idx)
+        assert np.array_equal(got, O.select_streaming(sc, sl, T, *budget)), (seed, B, L_max)
+        assert np.array_equal(got, host(ref)), (seed, B, L_max)
