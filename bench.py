@@ -1,25 +1,31 @@
 #!/usr/bin/env python
-"""Benchmark of the LSA decode hot path on B200.
+"""Benchmark of the LSA hot path on B200.
 
 One step = one pass of the whole path over one batch: lightning-indexer scores
-(tcgen05) -> streaming top-k -> sparse MLA attention (+ split combine), on the
-flat-decode workload (8 sequences x 131072 cached tokens, one query each, top-k
-2048 = sink 64 + window 960 + 1024 dynamic; 128 query heads, d_qk 576 / d_v 512)
-unless --workload says otherwise. Inputs are seeded synthetic data resident in
-HBM; L2 is flushed (256 MiB write) between timed steps, outside the timed events.
+(tcgen05) -> streaming top-k -> sparse MLA attention (+ split combine). The
+default workload is flat decode (8 sequences x 131072 cached tokens, one query
+each, top-k 2048 = sink 64 + window 960 + 1024 dynamic; 128 query heads,
+d_qk 576 / d_v 512). Inputs are seeded synthetic data resident in HBM; L2 is
+flushed (256 MiB write) between timed steps, outside the timed events.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME] [--fp8]
 
-Workloads (kv_indexing_b200.inputs.WORKLOADS): flat_decode_128k (default, the
-headline), hier_decode_1m (hierarchical indexing at 1M tokens; page pooling
-timed once, outside the step), cli_group_256k / cli_group_256k_flat (one
-indexing pass feeding two layers), prefill_64k (4096 causal queries; --fp8 for
-e4m3 indexer inputs), compressed_decode_1m (indexing over 262144 entries of 4
-tokens each, then attention over the 2048 chosen compressed latent entries;
---fp8 for e4m3 entry keys). Long KV caches for timing are drawn on the device with
-torch's seeded generator; the indexer inputs come from the seeded host
-generator (needles included).
+Workloads (kv_indexing_b200.inputs.WORKLOADS): flat_decode_128k (default),
+flat_decode_1m and hier_decode_1m (the same 2 x 1M inputs, hierarchy off / on;
+page pooling timed once, outside the step), cli_group_256k(_flat) (one indexing
+pass feeding two layers), prefill_64k (4096 causal queries; --fp8 for e4m3
+indexer inputs), compressed_decode_1m (262144 entries of 4 tokens; --fp8 for
+e4m3 entry keys), and hier_sweep: flat against hierarchical indexing on the
+same inputs at L = 64K, 256K, 512K and 1M (B=2).
+
+Each line carries: the device-timed step (one CUDA graph per step, no events
+inside) and its per-stage breakdown (a second graph with events between the
+stages), the same step as plain stream launches, the roofline of the dominant
+kernel, `e2e` (the public API with the step's queries copied in from pinned
+host memory and o, idx copied out, split into copy, compute and host-issue
+time; also with the user's calls captured in a CUDA graph), and `cpu_baseline`
+(the C++ oracle on the host cores: all cores over the rows, and one thread).
 
 Prints one JSON line (rank 0). Under torchrun each rank runs its own batch
 (weak scaling, no data-path collective); times are device times, max over ranks.
@@ -42,6 +48,7 @@ if ROOT not in sys.path:
 
 METRIC = "decode queries/s (indexer+top-k+sparse attn) at 128K-1M; % of HBM/TC roofline"
 UNIT = "queries/s"
+SWEEP_L = (65536, 262144, 524288, 1048576)
 
 
 def parse():
@@ -54,7 +61,7 @@ def parse():
     p.add_argument("--seed", type=int, default=1)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
-    p.add_argument("--fp8", action="store_true", help="prefill: e4m3 indexer keys and queries")
+    p.add_argument("--fp8", action="store_true", help="e4m3 indexer keys and queries (prefill, compressed)")
     return p.parse_args()
 
 
@@ -63,9 +70,17 @@ def parse():
 # ---------------------------------------------------------------------------
 
 
-def indexer_bytes_per_query(w) -> int:
-    """Keys streamed once + the query's indexer vectors and head weights."""
-    return w.L * w.d * 2 + w.H * w.d * 2 + w.H * 4
+def indexer_bytes_per_query(w, fp8=False, n_keys=None) -> int:
+    """Keys streamed once (+ their e4m3 scales) + the query's vectors and head weights."""
+    n = w.L if n_keys is None else n_keys
+    if fp8:
+        return n * w.d + n * 4 + w.H * w.d + w.H * 4 + w.H * 4
+    return n * w.d * 2 + w.H * w.d * 2 + w.H * 4
+
+
+def hier_index_bytes_per_query(w) -> int:
+    """Page keys of the whole sequence + the recalled pages' token keys + q, w."""
+    return (w.L // w.P) * w.d * 2 + w.M * w.P * w.d * 2 + w.H * w.d * 2 + w.H * 4
 
 
 def attention_bytes_per_query(w) -> int:
@@ -73,8 +88,9 @@ def attention_bytes_per_query(w) -> int:
     return w.k * w.d_qk * 2 + w.Hq * w.d_qk * 2 + w.Hq * w.d_v * 2
 
 
-def step_bytes_per_query(w) -> int:
-    return indexer_bytes_per_query(w) + attention_bytes_per_query(w) + w.k * 4
+def prefill_indexer_flops(w) -> float:
+    """2 H d per visible (query, key) pair, causal."""
+    return 2.0 * w.H * w.d * sum(p + 1 for p in range(w.L - w.T, w.L)) * w.B
 
 
 def measured_peaks():
@@ -82,7 +98,7 @@ def measured_peaks():
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             return json.load(f), "measured"
     except OSError:
-        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}, "fallback"
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
 def kernel_traffic(name: str):
@@ -96,9 +112,8 @@ def kernel_traffic(name: str):
     ent = tab.get(name)
     if not ent:
         return None
-    src = os.path.join(ROOT, ent["source_file"])
     try:
-        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        sha = hashlib.sha256(open(os.path.join(ROOT, ent["source_file"]), "rb").read()).hexdigest()
     except OSError:
         return None
     return ent["dram_bytes_per_launch"] if sha == ent["source_sha256"] else None
@@ -180,75 +195,6 @@ class ClockSampler:
                 "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
-# ---------------------------------------------------------------------------
-# oracle timing (CPU baseline and the reference arm)
-# ---------------------------------------------------------------------------
-
-
-def blas_threads() -> int:
-    try:
-        from threadpoolctl import threadpool_info
-        n = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
-        return int(max(n)) if n else 1
-    except Exception:
-        return os.cpu_count() or 1
-
-
-def oracle_query(O, w, x, a, b):
-    """The whole path for query (b, 0) on the CPU oracle."""
-    rows = [(b, 0)]
-    sc = O.indexer_scores(x["q_idx"], x["w"], x["k_idx"], x["seq_len"], rows=rows)
-    pos = int(x["seq_len"][b]) - 1
-    idx = O.select_streaming_row(sc[b, 0], pos, w.k, w.sink, w.window)
-    ii = idx[None, None, :]
-    qa = a["qa"][b:b + 1]
-    kv = a["kv"][b:b + 1]
-    O.sparse_attention(qa, ii, x["seq_len"][b:b + 1], scale=w.scale, d_v=w.d_v, kv=kv)
-
-
-def time_oracle(w, x, a, budget_s: float = 12.0, max_queries=None):
-    import oracle as O
-    n, t0 = 0, time.perf_counter()
-    total = w.B * w.T if max_queries is None else max_queries
-    while n < total:
-        oracle_query(O, w, x, a, n % w.B)
-        n += 1
-        if time.perf_counter() - t0 > budget_s:
-            break
-    dt = time.perf_counter() - t0
-    return n / dt, n, dt
-
-
-def run_reference(args, rank: int, world: int):
-    """The oracle as it stands on the host cores: one query per step."""
-    if rank != 0:
-        return 0
-    from kv_indexing_b200 import inputs as I
-    import oracle as O
-    w = I.WORKLOADS[args.workload]
-    x = I.make_indexer_inputs(w, args.seed)
-    a = I.make_attn_inputs(w, args.seed)
-    for i in range(args.warmup):
-        oracle_query(O, w, x, a, i % w.B)
-    t0 = time.perf_counter()
-    for i in range(args.steps):
-        oracle_query(O, w, x, a, i % w.B)
-    dt = time.perf_counter() - t0
-    v = args.steps / dt
-    cores = blas_threads()
-    line = {
-        "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": 1000 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(w, sampled="one query of the batch per step"),
-        "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": f"{args.steps} single-query steps of the {w.B}-query batch"},
-        "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-    }
-    print(json.dumps(line), flush=True)
-    return 0
-
-
 def workload_config(w, **extra):
     c = {"workload": w.name, "B": w.B, "L": w.L, "T": w.T, "H_I": w.H, "d_I": w.d, "k": w.k, "sink": w.sink,
          "window": w.window, "Hq": w.Hq, "d_qk": w.d_qk, "d_v": w.d_v, "P": w.P, "M": w.M,
@@ -258,24 +204,215 @@ def workload_config(w, **extra):
     return c
 
 
+def kind_of(w) -> str:
+    if w.m:
+        return "compressed"
+    if w.n_layers > 1:
+        return "group"
+    if w.P:
+        return "hier"
+    return "prefill" if w.T > 1 else "flat"
+
+
+def host_inputs(w, seed):
+    """Indexer inputs from the seeded host generator (needles included); for
+    compressed entries the entry keys take the place of the token keys."""
+    from kv_indexing_b200 import inputs as I
+    if w.m:
+        x = I.make_compressed_inputs(w, seed)
+        x["k_idx"] = x.pop("entry_keys")
+        if "entry_keys_fp8" in x:
+            x["k_idx_fp8"] = x.pop("entry_keys_fp8")
+        return x
+    return I.make_indexer_inputs(w, seed)
+
+
 # ---------------------------------------------------------------------------
-# other workloads: a generic stage timer over one CUDA graph per step
+# the path of one workload on the device: stages of a step, the public-API
+# step a user calls, and what the roofline measures
 # ---------------------------------------------------------------------------
 
 
-def time_stages(torch, stages, K, warmup, flush, dev, pg):
-    """stages: [(name, fn(stream))]. One graph per step with external events
-    between the stages; L2 flushed between steps, outside the events."""
-    import torch.distributed as dist
-    stream = torch.cuda.current_stream(dev)
-    for _ in range(max(3, warmup)):
-        flush()
-        for _, fn in stages:
-            fn(stream)
-    torch.cuda.synchronize()
+class Path:
+    def __init__(self, torch, L, w, x, dev, seed, fp8, layers=None):
+        import numpy as np
+        self.torch, self.L, self.w, self.x, self.dev, self.fp8 = torch, L, w, x, dev, fp8
+        self.kind = kind_of(w)
+        B, T = w.B, w.T
+        self.budget = (w.k, w.sink, w.window)
+
+        def up(arr, kind):
+            t = torch.from_numpy(np.ascontiguousarray(arr).view(np.int16) if kind == "bf16" else
+                                 np.ascontiguousarray(arr))
+            t = t.view(torch.bfloat16) if kind == "bf16" else t
+            return t.to(dev)
+
+        self.up = up
+        self.q, self.k, self.wt, self.sl = up(x["q_idx"], "bf16"), up(x["k_idx"], "bf16"), up(x["w"], "f32"), \
+            up(x["seq_len"], "i32")
+        self.qs = self.ks = None
+        if fp8:
+            if "k_idx_fp8" not in x:
+                raise SystemExit(f"workload {w.name} has no e4m3 indexer inputs")
+            self.q = up(x["q_idx_fp8"], "u8").view(torch.float8_e4m3fn)
+            self.k = up(x["k_idx_fp8"], "u8").view(torch.float8_e4m3fn)
+            self.qs, self.ks = up(x["q_scale"], "f32"), up(x["k_scale"], "f32")
+        kv_rows = w.L // w.m if w.m else w.L
+        self.layers = layers if layers is not None else []
+        for li in range(0 if layers is not None else w.n_layers):
+            qa = device_bf16_normal(torch, (B, T, w.Hq, w.d_qk), 7919 * seed + 2 * li, dev)
+            kv = device_bf16_normal(torch, (B, kv_rows, w.d_qk), 7919 * seed + 2 * li + 1, dev)
+            self.layers.append({"q": qa, "kv": kv, "scale": w.scale, "d_v": w.d_v})
+        self.idx = torch.empty((B, T, w.k), dtype=torch.int32, device=dev)
+        self.outs = [torch.empty((B, T, w.Hq, w.d_v), dtype=torch.bfloat16, device=dev) for _ in range(w.n_layers)]
+        self.extra = {}
+        self._build()
+
+    def _ws(self, n):
+        return self.torch.empty(max(256, n), dtype=self.torch.uint8, device=self.dev)
+
+    def _build(self):
+        torch, L, w = self.torch, self.L, self.w
+        B, T, budget = w.B, w.T, self.budget
+        q, k, wt, sl, qs, ks = self.q, self.k, self.wt, self.sl, self.qs, self.ks
+        lay0 = self.layers[0]
+        # attention rows: entries for compressed indexing (decode: the query's entry
+        # position is seq_len // m - 1), tokens otherwise
+        self.sl_attn = torch.div(sl, w.m, rounding_mode="floor").to(torch.int32) if w.m else sl
+        ai = L.attn_in(lay0["q"], self.sl_attn, w.scale, kv=lay0["kv"], d_v=w.d_v, stream_budget=budget)
+        self.attn_ws = self._ws(L.workspace_size(L.LSA_OP_SPARSE_ATTN, attn=ai, budget=(w.k, 0, 0)))
+
+        def attn(li, idx=None):
+            lay = self.layers[li]
+            return lambda s: L.lsa_sparse_attn(lay["q"], self.idx if idx is None else idx, self.sl_attn, w.scale,
+                                               kv=lay["kv"], d_v=w.d_v, out=self.outs[li], workspace=self.attn_ws,
+                                               stream_budget=budget, stream=s)
+
+        kind = self.kind
+        if kind in ("flat", "prefill", "compressed"):
+            n_slots = w.L // w.m if w.m else w.L
+            self.scores = torch.empty((B, T, n_slots), dtype=torch.float32, device=self.dev)
+            sl_sel = self.sl_attn
+            self.sel_ws = self._ws(L.workspace_size(L.LSA_OP_SELECT, budget=budget, B=B, T=T, L_max=n_slots))
+            if w.m:
+                ii = L.indexer_in(q, wt, k, sl, qs, ks, m=w.m)
+                self.api_ws = self._ws(L.workspace_size(L.LSA_OP_INDEX_COMPRESSED, indexer=ii, budget=budget, m=w.m))
+                index_scores = lambda s: L.lsa_index_compressed(q, wt, k, sl, w.m, budget, q_scale=qs, k_scale=ks,
+                                                                 scores_out=self.scores, with_idx=False, stream=s)
+            else:
+                ii = L.indexer_in(q, wt, k, sl, qs, ks)
+                self.api_ws = self._ws(L.workspace_size(L.LSA_OP_INDEX_FLAT, indexer=ii, budget=budget))
+                index_scores = lambda s: L.lsa_index_flat(q, wt, k, sl, budget, q_scale=qs, k_scale=ks,
+                                                          scores_out=self.scores, with_idx=False, stream=s)
+            self.stages = [("indexer", index_scores),
+                           ("select", lambda s: L.lsa_select_streaming(self.scores, sl_sel, budget, idx=self.idx,
+                                                                       workspace=self.sel_ws, stream=s)),
+                           ("attention", attn(0))]
+            self.dominant = "indexer"
+            if kind == "prefill":
+                self.roof_kernel = "indexer (tcgen05 score GEMM over causal tiles, fused epilogue)"
+                self.roof_flops = prefill_indexer_flops(w)
+            else:
+                n_keys = w.L // w.m if w.m else w.L
+                self.roof_kernel = ("entry " if w.m else "") + "indexer (tcgen05 score GEMM + fused epilogue)"
+                self.roof_bytes = indexer_bytes_per_query(w, self.fp8, n_keys) * B * T
+        elif kind == "hier":
+            self._pool_once()
+            ii = L.indexer_in(q, wt, k, sl)
+            self.api_ws = self._ws(L.workspace_size(L.LSA_OP_INDEX_HIER, indexer=ii, budget=budget, P=w.P, M=w.M))
+            self.stages = [("hier_index", lambda s: L.lsa_index_hier(q, wt, k, sl, self.page_keys, w.P, w.M, budget,
+                                                                     idx=self.idx, workspace=self.api_ws, stream=s)),
+                           ("attention", attn(0))]
+            self.dominant = "hier_index"
+            self.roof_kernel = "hierarchical indexing call (page scores, page recall, fine scores, token top-k)"
+            self.roof_bytes = hier_index_bytes_per_query(w) * B * T
+        else:   # group
+            if w.P:
+                self._pool_once()
+            ii = L.indexer_in(q, wt, k, sl)
+            ais = [L.attn_in(l["q"], sl, w.scale, kv=l["kv"], d_v=w.d_v) for l in self.layers]
+            self.api_ws = self._ws(L.workspace_size(L.LSA_OP_LAYER_GROUP, indexer=ii, attn=ais, budget=budget,
+                                                    P=w.P, M=w.M, n_layers=w.n_layers))
+            pk = self.page_keys if w.P else None
+            self.stages = [("group", lambda s: L.lsa_layer_group(q, wt, k, sl, budget, self.layers, P=w.P, M=w.M,
+                                                                 page_keys=pk, outs=self.outs, idx=self.idx,
+                                                                 workspace=self.api_ws, stream=s))]
+            # the indexing pass alone (timed beside the step: its cost over the N layers
+            # is the per-layer amortised indexer cost)
+            self.idx_only = torch.empty_like(self.idx)
+            if w.P:
+                hws = self._ws(L.workspace_size(L.LSA_OP_INDEX_HIER, indexer=ii, budget=budget, P=w.P, M=w.M))
+                self.index_alone = [("index_alone", lambda s: L.lsa_index_hier(
+                    q, wt, k, sl, pk, w.P, w.M, budget, idx=self.idx_only, workspace=hws, stream=s))]
+            else:
+                fws = self._ws(L.workspace_size(L.LSA_OP_INDEX_FLAT, indexer=ii, budget=budget))
+                self.index_alone = [("index_alone", lambda s: L.lsa_index_flat(
+                    q, wt, k, sl, budget, idx=self.idx_only, workspace=fws, stream=s))]
+            self.dominant = "group"
+            self.roof_kernel = f"layer-group call (one indexing pass + {w.n_layers} attention layers)"
+            ib = hier_index_bytes_per_query(w) if w.P else indexer_bytes_per_query(w)
+            self.roof_bytes = (ib + w.n_layers * attention_bytes_per_query(w)) * B * T
+
+    def _pool_once(self):
+        torch, L, w = self.torch, self.L, self.w
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        self.page_keys = torch.zeros((w.B, w.L // w.P, w.d), dtype=torch.bfloat16, device=self.dev)
+        e0.record()
+        L.lsa_pool_pages(self.k, self.sl, w.P, page_keys=self.page_keys)
+        e1.record()
+        torch.cuda.synchronize()
+        self.extra["page_pooling_once_us"] = 1000 * e0.elapsed_time(e1)
+
+    # -- the public-API step a user calls, on given device inputs ------------
+    def api_step(self, s, q, wt, qas):
+        """The path through the library's public calls (what an application
+        issues per decode step), reading the queries from q, wt and qas."""
+        L, w, budget = self.L, self.w, self.budget
+        k, sl, qs, ks = self.k, self.sl, self.qs, self.ks
+        if self.kind == "group":
+            layers = [dict(l, q=qa) for l, qa in zip(self.layers, qas)]
+            L.lsa_layer_group(q, wt, k, sl, budget, layers, P=w.P, M=w.M,
+                              page_keys=self.page_keys if w.P else None, outs=self.outs, idx=self.idx,
+                              workspace=self.api_ws, stream=s)
+            return
+        if self.kind == "hier":
+            L.lsa_index_hier(q, wt, k, sl, self.page_keys, w.P, w.M, budget, idx=self.idx, workspace=self.api_ws,
+                             stream=s)
+        elif self.kind == "compressed":
+            L.lsa_index_compressed(q, wt, k, sl, w.m, budget, q_scale=qs, k_scale=ks, idx=self.idx,
+                                   workspace=self.api_ws, stream=s)
+        else:
+            L.lsa_index_flat(q, wt, k, sl, budget, q_scale=qs, k_scale=ks, idx=self.idx, workspace=self.api_ws,
+                             stream=s)
+        lay = self.layers[0]
+        L.lsa_sparse_attn(qas[0], self.idx, self.sl_attn, w.scale, kv=lay["kv"], d_v=w.d_v, out=self.outs[0],
+                          workspace=self.attn_ws, stream_budget=budget, stream=s)
+
+
+def device_bf16_normal(torch, shape, seed, dev):
+    """Seeded N(0,1) bf16 drawn on the device (latent KV caches and attention
+    queries; the long caches would take minutes on the host generator)."""
+    g = torch.Generator(device=dev)
+    g.manual_seed(int(seed))
+    out = torch.empty(shape, dtype=torch.bfloat16, device=dev)
+    flat = out.view(-1)
+    step = 1 << 28
+    for lo in range(0, flat.numel(), step):          # bounded float32 temporaries
+        n = min(step, flat.numel() - lo)
+        flat[lo:lo + n] = torch.randn((n,), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    return out
+
+
+# ---------------------------------------------------------------------------
+# device timing
+# ---------------------------------------------------------------------------
+
+
+def capture(torch, stages, dev, stream, inner_events, keep_graph=False):
     n = len(stages)
     ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n + 1)]
-    g = torch.cuda.CUDAGraph()
+    g = torch.cuda.CUDAGraph(keep_graph=keep_graph)
     cap = torch.cuda.Stream(dev)
     cap.wait_stream(stream)
     with torch.cuda.graph(g, stream=cap, capture_error_mode="relaxed"):
@@ -283,14 +420,56 @@ def time_stages(torch, stages, K, warmup, flush, dev, pg):
         ev[0].record(s)
         for i, (_, fn) in enumerate(stages):
             fn(s)
-            ev[i + 1].record(s)
+            if inner_events or i == n - 1:
+                ev[i + 1].record(s)
     torch.cuda.synchronize()
+    launches = None
+    if keep_graph:
+        launches = graph_kernel_count(g)
+        g.instantiate()
+    return g, ev, launches
+
+
+def graph_kernel_count(g):
+    """Kernel nodes of a captured graph (our launches per step), or None."""
+    try:
+        from cuda.bindings import runtime as rt
+    except Exception:
+        try:
+            from cuda import cudart as rt
+        except Exception:
+            return None
+    try:
+        raw = g.raw_cuda_graph()
+        graph = rt.cudaGraph_t(init_value=raw) if hasattr(rt, "cudaGraph_t") else raw
+        err, _, n = rt.cudaGraphGetNodes(graph, 0)
+        err, nodes, n = rt.cudaGraphGetNodes(graph, n)
+        kinds = [rt.cudaGraphNodeGetType(nd)[1] for nd in nodes]
+        return sum(1 for t in kinds if t == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel)
+    except Exception:
+        return None
+
+
+def time_device(torch, stages, K, warmup, flush, dev, pg):
+    """Whole step as one graph (events only around it), per-stage breakdown from
+    a second graph, and the same step as plain launches. Returns a dict."""
+    import torch.distributed as dist
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(max(3, warmup)):
+        flush()
+        for _, fn in stages:
+            fn(stream)
+    torch.cuda.synchronize()
+    g, ev, launches = capture(torch, stages, dev, stream, inner_events=False, keep_graph=True)
+    gb, evb, _ = capture(torch, stages, dev, stream, inner_events=True)
+    n = len(stages)
     for _ in range(3):
         flush()
         g.replay()
+        flush()
+        gb.replay()
     torch.cuda.synchronize()
-    per = [[] for _ in range(n)]
-    tot = []
+    step = []
     if pg:
         dist.barrier()
     torch.cuda.synchronize()
@@ -299,206 +478,419 @@ def time_stages(torch, stages, K, warmup, flush, dev, pg):
             flush()
             g.replay()
             torch.cuda.synchronize()
-            for i in range(n):
-                per[i].append(ev[i].elapsed_time(ev[i + 1]))
-            tot.append(ev[0].elapsed_time(ev[n]))
+            step.append(ev[0].elapsed_time(ev[n]))
     torch.cuda.synchronize()
     if pg:
         dist.barrier()
-    total_ms = max_over_ranks(float(sum(tot)), dev, pg)
+    per = [[] for _ in range(n)]
+    for _ in range(K):
+        flush()
+        gb.replay()
+        torch.cuda.synchronize()
+        for i in range(n):
+            per[i].append(evb[i].elapsed_time(evb[i + 1]))
+    # plain launches: the same calls issued on the stream, no graph
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    plain = []
+    for _ in range(K):
+        flush()
+        e0.record(stream)
+        for _, fn in stages:
+            fn(stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        plain.append(e0.elapsed_time(e1))
+    del g, gb
+    return {
+        "ms_per_step": max_over_ranks(float(sum(step)) / K, dev, pg),
+        "step_ms_median": statistics.median(step),
+        "breakdown_us": {name: 1000 * sum(per[i]) / K for i, (name, _) in enumerate(stages)},
+        "plain_ms_per_step": max_over_ranks(float(sum(plain)) / K, dev, pg),
+        "clocks": clk.summary(),
+        "launches_per_step": launches,
+    }
+
+
+def time_e2e(torch, path, K, flush, dev, pg):
+    """End to end through the public API: per step the step's queries go in
+    from pinned host memory (indexer q [+ q scales], head weights, attention q of
+    every layer) and o of every layer and idx come back; timed with events on
+    the stream (copies, compute, copies), plus the host time spent issuing the
+    calls. Also the same with the user's calls captured in a CUDA graph."""
+    stream = torch.cuda.current_stream(dev)
+    srcs = [path.q, path.wt] + ([path.qs] if path.qs is not None else []) + [l["q"] for l in path.layers]
+    hins = [t.cpu().pin_memory() for t in srcs]
+    dins = [torch.empty_like(t) for t in srcs]
+    houts = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in path.outs + [path.idx]]
+    h2d = sum(t.numel() * t.element_size() for t in hins)
+    d2h = sum(t.numel() * t.element_size() for t in houts)
+    nq = 3 if path.qs is not None else 2
+
+    def run():
+        qs_saved = path.qs
+        if path.qs is not None:
+            path.qs = dins[2]
+        try:
+            path.api_step(stream, dins[0], dins[1], dins[nq:])
+        finally:
+            path.qs = qs_saved
+
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+
+    def one(step_fn):
+        flush()
+        ev[0].record(stream)
+        for d, h in zip(dins, hins):
+            d.copy_(h, non_blocking=True)
+        ev[1].record(stream)
+        t0 = time.perf_counter()
+        step_fn()
+        host = time.perf_counter() - t0
+        ev[2].record(stream)
+        for h, d in zip(houts, path.outs + [path.idx]):
+            h.copy_(d, non_blocking=True)
+        ev[3].record(stream)
+        torch.cuda.synchronize()
+        return ev[0].elapsed_time(ev[3]), ev[0].elapsed_time(ev[1]), ev[1].elapsed_time(ev[2]), \
+            ev[2].elapsed_time(ev[3]), 1000 * host
+
+    for _ in range(3):
+        one(run)
+    rec = [one(run) for _ in range(K)]
+    # the same calls captured once in a CUDA graph by the application
+    g = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(stream)
+    with torch.cuda.graph(g, stream=cap, capture_error_mode="relaxed"):
+        s_saved = stream
+        stream = torch.cuda.current_stream(dev)
+        run()
+        stream = s_saved
+    torch.cuda.synchronize()
+    for _ in range(3):
+        one(g.replay)
+    recg = [one(g.replay) for _ in range(K)]
     del g
-    return {name: 1000 * sum(per[i]) / K for i, (name, _) in enumerate(stages)}, total_ms / K, clk.summary()
+    units = path.w.B * path.w.T * (int(os.environ.get("WORLD_SIZE", "1")))
+    tot = max_over_ranks(sum(r[0] for r in rec) / K, dev, pg)
+    totg = max_over_ranks(sum(r[0] for r in recg) / K, dev, pg)
+    mean = lambda rs, i: sum(r[i] for r in rs) / K
+    return {
+        "value": units / (tot / 1000.0), "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+        "ms_per_step": tot, "h2d_ms": mean(rec, 1), "compute_ms": mean(rec, 2), "d2h_ms": mean(rec, 3),
+        "host_issue_ms": mean(rec, 4),
+        "graph": {"value": units / (totg / 1000.0), "ms_per_step": totg, "h2d_ms": mean(recg, 1),
+                  "compute_ms": mean(recg, 2), "d2h_ms": mean(recg, 3), "host_issue_ms": mean(recg, 4)},
+        "note": "caches resident; per step the new queries go in and o, idx come out (pinned host memory); "
+                "value: the public calls issued per step; graph: the same calls captured once by the application",
+    }
 
 
-def device_bf16_normal(torch, shape, seed, dev):
-    """Seeded N(0,1) bf16 drawn on the device (timing inputs for long KV caches)."""
-    g = torch.Generator(device=dev)
-    g.manual_seed(int(seed))
-    return torch.randn(shape, generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+# ---------------------------------------------------------------------------
+# the oracle on the host cores (CPU baseline and the reference arm)
+# ---------------------------------------------------------------------------
 
 
-def run_workload(args, w, rank, world, dev, pg):
+def host_bf16(t):
     import numpy as np
     import torch
-    import torch.distributed as dist
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
 
-    from kv_indexing_b200 import inputs as I
-    from kv_indexing_b200 import lsa as L
 
-    seed = rank_seed(args.seed, rank)
-    if w.m:
-        # compressed entries: the indexer's keys are the entry keys [B, L/m, d]
-        x = I.make_compressed_inputs(w, seed)
-        x["k_idx"] = x.pop("entry_keys")
-        if "entry_keys_fp8" in x:
-            x["k_idx_fp8"] = x.pop("entry_keys_fp8")
-    else:
-        x = I.make_indexer_inputs(w, seed)
-    kv_rows = w.L // w.m if w.m else w.L
+class OraclePath:
+    """The whole path for a list of query rows on the C++ oracle: indexer scores,
+    streaming selection (flat, hierarchical or over entries), then the sparse
+    attention of every layer. Page keys are pooled once, outside the timed
+    part, as on the GPU."""
 
-    def up(arr, kind):
-        t = torch.from_numpy(np.ascontiguousarray(arr).view(np.int16) if kind == "bf16" else arr)
-        t = t.view(torch.bfloat16) if kind == "bf16" else t
-        return t.to(dev)
-
-    q, k, wt, sl = up(x["q_idx"], "bf16"), up(x["k_idx"], "bf16"), up(x["w"], "f32"), up(x["seq_len"], "i32")
-    B, T = w.B, w.T
-    budget = (w.k, w.sink, w.window)
-    layers = []
-    for li in range(w.n_layers):
-        qa = device_bf16_normal(torch, (B, T, w.Hq, w.d_qk), 7919 * seed + 2 * li, dev)
-        kv = device_bf16_normal(torch, (B, kv_rows, w.d_qk), 7919 * seed + 2 * li + 1, dev)
-        layers.append({"q": qa, "kv": kv, "scale": w.scale, "d_v": w.d_v})
-    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-
-    def flush():
-        flush_buf.random_(0, 255)
-
-    peaks, peak_src = measured_peaks()
-    idx = torch.empty((B, T, w.k), dtype=torch.int32, device=dev)
-    outs = [torch.empty((B, T, w.Hq, w.d_v), dtype=torch.bfloat16, device=dev) for _ in range(w.n_layers)]
-    extra = {}
-    ai = L.attn_in(layers[0]["q"], sl, w.scale, kv=layers[0]["kv"], d_v=w.d_v)
-    attn_ws = torch.empty(max(256, L.workspace_size(L.LSA_OP_SPARSE_ATTN, attn=ai, budget=(w.k, 0, 0))),
-                          dtype=torch.uint8, device=dev)
-
-    def attn_stage(li):
-        lay = layers[li]
-        return lambda s: L.lsa_sparse_attn(lay["q"], idx, sl, w.scale, kv=lay["kv"], d_v=w.d_v, out=outs[li],
-                                           workspace=attn_ws, stream=s)
-
-    if w.m:
-        kind = "compressed"
-        qk = dict(q=q, k=k)
-        if args.fp8:
-            qk = dict(q=up(x["q_idx_fp8"], "u8").view(torch.float8_e4m3fn),
-                      k=up(x["k_idx_fp8"], "u8").view(torch.float8_e4m3fn),
-                      q_scale=up(x["q_scale"], "f32"), k_scale=up(x["k_scale"], "f32"))
-        ii = L.indexer_in(qk["q"], wt, qk["k"], sl, qk.get("q_scale"), qk.get("k_scale"), m=w.m)
-        cws = torch.empty(max(256, L.workspace_size(L.LSA_OP_INDEX_COMPRESSED, indexer=ii, budget=budget, m=w.m)),
-                          dtype=torch.uint8, device=dev)
-        # one query per sequence (decode): its entry position is seq_len // m - 1
-        sl_e = torch.div(sl, w.m, rounding_mode="floor").to(torch.int32)
-        lay = layers[0]
-        ai_c = L.attn_in(lay["q"], sl_e, w.scale, kv=lay["kv"], d_v=w.d_v, stream_budget=budget)
-        cattn_ws = torch.empty(max(256, L.workspace_size(L.LSA_OP_SPARSE_ATTN, attn=ai_c, budget=(w.k, 0, 0))),
-                               dtype=torch.uint8, device=dev)
-        stages = [("index_compressed", lambda s: L.lsa_index_compressed(
-                      qk["q"], wt, qk["k"], sl, w.m, budget, q_scale=qk.get("q_scale"), k_scale=qk.get("k_scale"),
-                      idx=idx, workspace=cws, stream=s)),
-                  ("attention", lambda s: L.lsa_sparse_attn(lay["q"], idx, sl_e, w.scale, kv=lay["kv"], d_v=w.d_v,
-                                                            out=outs[0], workspace=cattn_ws, stream_budget=budget,
-                                                            stream=s))]
-    elif w.T > 1:
-        kind = "prefill"
-        qk = dict(q=q, k=k)
-        if args.fp8:
-            if "k_idx_fp8" not in x:
-                raise SystemExit(f"workload {w.name} has no e4m3 indexer inputs")
-            qk = dict(q=up(x["q_idx_fp8"], "u8").view(torch.float8_e4m3fn),
-                      k=up(x["k_idx_fp8"], "u8").view(torch.float8_e4m3fn),
-                      q_scale=up(x["q_scale"], "f32"), k_scale=up(x["k_scale"], "f32"))
-        ii = L.indexer_in(qk["q"], wt, qk["k"], sl, qk.get("q_scale"), qk.get("k_scale"))
-        scores = torch.empty((B, T, w.L), dtype=torch.float32, device=dev)
-        sel_ws = torch.empty(max(256, L.workspace_size(L.LSA_OP_SELECT, budget=budget, B=B, T=T, L_max=w.L)),
-                             dtype=torch.uint8, device=dev)
-        stages = [("indexer", lambda s: L.lsa_index_flat(qk["q"], wt, qk["k"], sl, budget,
-                                                         q_scale=qk.get("q_scale"), k_scale=qk.get("k_scale"),
-                                                         scores_out=scores, with_idx=False, stream=s)),
-                  ("select", lambda s: L.lsa_select_streaming(scores, sl, budget, idx=idx, workspace=sel_ws,
-                                                              stream=s)),
-                  ("attention", attn_stage(0))]
-    elif w.n_layers > 1:
-        kind = "group"
-        page_keys = L.lsa_pool_pages(k, sl, w.P) if w.P else None
-        ii = L.indexer_in(q, wt, k, sl)
-        ais = [L.attn_in(l["q"], sl, w.scale, kv=l["kv"], d_v=w.d_v) for l in layers]
-        ws = torch.empty(max(256, L.workspace_size(L.LSA_OP_LAYER_GROUP, indexer=ii, attn=ais, budget=budget,
-                                                   P=w.P, M=w.M, n_layers=w.n_layers)), dtype=torch.uint8, device=dev)
-        stages = [("group", lambda s: L.lsa_layer_group(q, wt, k, sl, budget, layers, P=w.P, M=w.M,
-                                                        page_keys=page_keys, outs=outs, idx=idx, workspace=ws,
-                                                        stream=s))]
-    else:
-        kind = "hier"
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        page_keys = torch.zeros((B, w.L // w.P, w.d), dtype=torch.bfloat16, device=dev)
-        e0.record()
-        L.lsa_pool_pages(k, sl, w.P, page_keys=page_keys)
-        e1.record()
-        torch.cuda.synchronize()
-        extra["page_pooling_once_us"] = 1000 * e0.elapsed_time(e1)
-        ii = L.indexer_in(q, wt, k, sl)
-        ws = torch.empty(max(256, L.workspace_size(L.LSA_OP_INDEX_HIER, indexer=ii, budget=budget, P=w.P, M=w.M)),
-                         dtype=torch.uint8, device=dev)
-        stages = [("hier_index", lambda s: L.lsa_index_hier(q, wt, k, sl, page_keys, w.P, w.M, budget, idx=idx,
-                                                            workspace=ws, stream=s)),
-                  ("attention", attn_stage(0))]
-
-    br, ms_per_step, clocks = time_stages(torch, stages, args.steps, args.warmup, flush, dev, pg)
-    L.lsa_device_status()
-    units = B * T * world
-    value = units / (ms_per_step / 1000.0)
-
-    # roofline of the dominant stage
-    if kind == "prefill":
-        pos = np.arange(w.L - w.T, w.L, dtype=np.float64)
-        flops = 2.0 * w.H * w.d * float(np.sum(pos + 1)) * B
-        us = br["indexer"]
-        peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * (2.0 if args.fp8 else 1.0)
-        roof = {"bound": "tensor", "kernel": "indexer (tcgen05 score GEMM over causal tiles, fused epilogue)",
-                "achieved": flops / (us * 1e-6) / 1e12, "peak": peak, "unit": "TFLOP/s",
-                "frac": flops / (us * 1e-6) / 1e12 / peak, "traffic": None, "algorithmic_flops_per_launch": flops,
-                "launch_us": us, "peak_source": peak_src + (" bf16 sustained x 2 (e4m3 nominal ratio)" if args.fp8
-                                                             else " bf16 sustained")}
-    elif kind == "compressed":
-        n_e = w.L // w.m
-        byts = (n_e * w.d * (1 if args.fp8 else 2) + (n_e * 4 if args.fp8 else 0) + w.H * w.d * 2 + w.H * 4) * B * T
-        us = br["index_compressed"]
-        roof = {"bound": "hbm", "kernel": "compressed-entry indexing call (entry scores, streaming top-k)",
-                "achieved": byts / (us * 1e-6) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": byts / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], "traffic": None,
-                "algorithmic_bytes_per_launch": byts, "launch_us": us, "peak_source": peak_src}
-    elif kind == "group":
+    def __init__(self, w, x, layers_host, fp8=False):
+        import oracle as O
+        self.O, self.w, self.x, self.layers, self.fp8 = O, w, x, layers_host, fp8
+        self.kind = kind_of(w)
         if w.P:
-            ib = (w.L // w.P) * w.d * 2 + w.M * w.P * w.d * 2
+            self.pk = O.pool_pages(x["k_idx"], x["seq_len"], w.P)
+
+    def run(self, rows):
+        import numpy as np
+        O, w, x = self.O, self.w, self.x
+        budget = (w.k, w.sink, w.window)
+        if self.fp8:
+            q, k = x["q_idx_fp8"], x["k_idx_fp8"]
+            kw = dict(fp8=True, q_scale=x["q_scale"], k_scale=x["k_scale"])
         else:
-            ib = indexer_bytes_per_query(w)
-        byts = (ib + w.n_layers * attention_bytes_per_query(w)) * B * T
-        us = br["group"]
-        roof = {"bound": "hbm", "kernel": "layer-group call (one indexing pass + %d attention layers)" % w.n_layers,
-                "achieved": byts / (us * 1e-6) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": byts / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], "traffic": None,
-                "algorithmic_bytes_per_launch": byts, "launch_us": us, "peak_source": peak_src}
-    else:
-        byts = ((w.L // w.P) * w.d * 2 + w.M * w.P * w.d * 2) * B * T
-        us = br["hier_index"]
-        roof = {"bound": "hbm", "kernel": "hierarchical indexing call (page scores, recall, fine scores, top-k)",
-                "achieved": byts / (us * 1e-6) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": byts / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], "traffic": None,
-                "algorithmic_bytes_per_launch": byts, "launch_us": us, "peak_source": peak_src}
-    if rank == 0:
-        line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "e4m3" if args.fp8 else "bf16",
-            "data": "synthetic (seeded N(0,1) bf16 indexer inputs with 1% needles from the host generator; "
-                    "latent KV and attention queries drawn on the device with a seeded generator)",
-            "config": workload_config(w, parallelism=f"replicas x{world} (independent batches)",
-                                      fp8_indexer=bool(args.fp8)),
-            "roofline": roof, "cpu_baseline": None, "e2e": None, "breakdown_us": br, **extra,
-            "tokens_scanned_per_s": value * w.L, "clocks": clocks,
-            "note": "extra workload line; the headline, e2e and CPU baseline are on flat_decode_128k",
-        }
-        print(json.dumps(line), flush=True)
-    if pg:
-        dist.destroy_process_group()
+            q, k, kw = x["q_idx"], x["k_idx"], {}
+        if self.kind == "compressed":
+            idx, _ = O.index_compressed(q, x["w"], k, x["seq_len"], m=w.m, budget=w.k, sink=w.sink,
+                                        window=w.window, **kw)
+        elif w.P:
+            idx, _ = O.index_hier(q, x["w"], k, self.pk, x["seq_len"], P=w.P, M=w.M, budget=w.k, sink=w.sink,
+                                  window=w.window, rows=rows)
+        else:
+            sc = O.indexer_scores_rows(q, x["w"], k, x["seq_len"], rows, **kw)
+            idx = np.full((w.B, w.T, w.k), -1, np.int32)
+            for i, (b, t) in enumerate(rows):
+                idx[b, t] = O.select_streaming_row(sc[i], int(x["seq_len"][b]) - w.T + t, *budget)
+        for lay in self.layers:
+            O.sparse_attention_rows(lay["qa"], idx, rows, scale=w.scale, d_v=w.d_v, kv=lay["kv"])
+
+    def all_rows(self):
+        return [(b, t) for b in range(self.w.B) for t in range(self.w.T)]
+
+
+def time_oracle(op: OraclePath, rows, budget_s: float):
+    """Repeat the rows until budget_s has passed (at least once): rows/s."""
+    n, t0 = 0, time.perf_counter()
+    while True:
+        op.run(rows)
+        n += len(rows)
+        dt = time.perf_counter() - t0
+        if dt >= budget_s:
+            return n / dt, n, dt
+
+
+def cpu_baseline(op: OraclePath, budget_s: float = 12.0):
+    import oracle as O
+    w = op.w
+    rows = op.all_rows()
+    if op.kind == "prefill":                      # a stride of query rows (the full chunk is ~2e12 MACs)
+        rows = [(0, t) for t in range(0, w.T, w.T // 32)]
+    if op.kind == "compressed":
+        rows = op.all_rows()
+    O.set_threads(0)
+    cores = O.threads()
+    op.run(rows[:1])                               # warm the caches and pages
+    v, n, dt = time_oracle(op, rows, budget_s)
+    O.set_threads(1)
+    try:
+        v1, n1, dt1 = time_oracle(op, rows[:1] if op.kind != "compressed" else rows, min(budget_s / 2, 6.0))
+    finally:
+        O.set_threads(0)
+    return {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{n} query rows ({len(rows)} per pass{', a stride of the chunk' if op.kind == 'prefill' else ''}"
+                      f") through the whole path in {dt:.1f} s on {cores} threads",
+            "one_thread": {"value": v1, "unit": UNIT, "sample": f"{n1} query rows in {dt1:.1f} s on 1 thread"}}
+
+
+def run_reference(args, rank: int, world: int):
+    """The C++ oracle as it stands on the host cores, same workload and metric."""
+    if rank != 0:
+        return 0
+    import oracle as O
+    from kv_indexing_b200 import inputs as I
+    w = I.WORKLOADS[args.workload if args.workload in I.WORKLOADS else "flat_decode_128k"]
+    x = host_inputs(w, args.seed)
+    kv_w = I.entry_workload(w) if w.m else w
+    layers = [I.make_attn_inputs(kv_w, args.seed, layer=li) for li in range(w.n_layers)]
+    op = OraclePath(w, x, layers, fp8=args.fp8)
+    rows = op.all_rows()
+    if op.kind == "prefill":
+        rows = [(0, t) for t in range(0, w.T, w.T // 32)]
+    O.set_threads(0)
+    t0 = time.perf_counter()
+    op.run(rows)
+    per_pass = time.perf_counter() - t0
+    # keep the whole --steps/--warmup run within a few minutes: each step runs
+    # the batch, or a bounded sample of its rows when the batch is slower
+    budget_step = 150.0 / max(1, args.steps + args.warmup)
+    if per_pass > budget_step and len(rows) > 1:
+        rows = rows[:max(1, int(len(rows) * budget_step / per_pass))]
+    for _ in range(args.warmup):
+        op.run(rows)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        op.run(rows)
+    dt = time.perf_counter() - t0
+    v = len(rows) * args.steps / dt
+    sample = f"{len(rows)} of the {w.B * w.T} query rows per step, whole path, {O.threads()} threads"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1000 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (the same seeded inputs as our arm's host generator)",
+        "config": workload_config(w, parallelism="host threads", l2="n/a (host run)"),
+        "cpu_baseline": {"value": v, "unit": UNIT, "cores": O.threads(), "kind": "oracle", "sample": sample},
+        "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
     return 0
 
 
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
+
+
+def roofline(path, br, peaks, peak_src, fp8, torch, dev):
+    w = path.w
+    us = br[path.dominant]
+    if path.kind == "prefill":
+        achieved = path.roof_flops / (us * 1e-6) / 1e12
+        peak, src = peaks["bf16_tflops"], peak_src + " bf16 burst (the indexer is timed in its own stage)"
+        if fp8:
+            fp8_peak = measure_fp8_peak(torch, dev)
+            if fp8_peak:
+                peak, src = fp8_peak, "e4m3 GEMM measured in this run (torch._scaled_mm 8192^3, best of 10)"
+            else:
+                peak, src = 2 * peaks["bf16_tflops"], peak_src + " bf16 burst x 2 (nominal e4m3 ratio)"
+        return {"bound": "tensor", "kernel": path.roof_kernel, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": None, "algorithmic_flops_per_launch": path.roof_flops,
+                "launch_us": us, "peak_source": src}
+    achieved = path.roof_bytes / (us * 1e-6) / 1e9
+    traffic = None
+    if path.kind == "flat" and not fp8 and w.name == "flat_decode_128k":
+        traffic = kernel_traffic("indexer_flat_decode_128k")
+    return {"bound": "hbm", "kernel": path.roof_kernel, "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "traffic": traffic, "algorithmic_bytes_per_launch": path.roof_bytes,
+            "launch_us": us, "peak_source": peak_src + " HBM copy"}
+
+
+def measure_fp8_peak(torch, dev):
+    try:
+        n = 8192
+        a = torch.randn((n, n), device=dev).to(torch.float8_e4m3fn)
+        b = torch.randn((n, n), device=dev).to(torch.float8_e4m3fn).t()
+        one = torch.tensor(1.0, device=dev)
+        for _ in range(3):
+            torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        best = None
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for _ in range(10):
+            e0.record()
+            torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+            e1.record()
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1)
+            best = ms if best is None else min(best, ms)
+        return 2.0 * n ** 3 / (best * 1e-3) / 1e12
+    except Exception:
+        return None
+
+
+def step_bytes(path) -> float:
+    w = path.w
+    if path.kind == "prefill":
+        return None
+    if path.kind == "hier":
+        ib = hier_index_bytes_per_query(w)
+    elif path.kind == "group":
+        return path.roof_bytes
+    else:
+        ib = indexer_bytes_per_query(w, path.fp8, w.L // w.m if w.m else w.L)
+    return (ib + attention_bytes_per_query(w) + w.k * 4) * w.B * w.T
+
+
+def run_workload(args, w, rank, world, dev, pg):
+    import torch
+    import torch.distributed as dist
+    from kv_indexing_b200 import lsa as L
+
+    seed = rank_seed(args.seed, rank)
+    x = host_inputs(w, seed)
+    path = Path(torch, L, w, x, dev, seed, args.fp8)
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def flush():
+        flush_buf.random_(0, 255)   # touch 256 MiB (> 126 MB L2)
+
+    t = time_device(torch, path.stages, args.steps, args.warmup, flush, dev, pg)
+    L.lsa_device_status()
+    extra = dict(path.extra)
+    if path.kind == "group":
+        ti = time_device(torch, path.index_alone, max(10, args.steps // 4), 3, flush, dev, pg)
+        extra["index_alone_us"] = ti["breakdown_us"]["index_alone"]
+        extra["index_per_layer_amortised_us"] = ti["breakdown_us"]["index_alone"] / w.n_layers
+    units = w.B * w.T * world
+    value = units / (t["ms_per_step"] / 1000.0)
+    peaks, peak_src = measured_peaks()
+    roof = roofline(path, t["breakdown_us"], peaks, peak_src, args.fp8, torch, dev)
+    sb = step_bytes(path)
+    if sb:
+        roof["step_frac_of_hbm_roofline"] = sb / (t["ms_per_step"] * 1e-3) / 1e9 / peaks["hbm_gbs"]
+        roof["step_algorithmic_bytes"] = sb
+    e2e = None if args.no_e2e else time_e2e(torch, path, max(20, min(args.steps, 100)), flush, dev, pg)
+    L.lsa_device_status()
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        layers_host = [{"qa": host_bf16(l["q"]), "kv": host_bf16(l["kv"])} for l in path.layers]
+        del flush_buf
+        torch.cuda.empty_cache()
+        cpu = cpu_baseline(OraclePath(w, x, layers_host, fp8=args.fp8))
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": t["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "e4m3" if args.fp8 else "bf16",
+            "data": "synthetic (seeded N(0,1) bf16 indexer inputs, U(0,1) head weights and 1% planted needles from "
+                    "the host generator; latent KV and attention queries drawn on the device with a seeded "
+                    "generator)",
+            "config": workload_config(w, parallelism=f"replicas x{world} (independent batches)",
+                                      fp8_indexer=bool(args.fp8)),
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": (t["launches_per_step"] or 0) * args.steps,
+            "launches_per_step": t["launches_per_step"],
+            "breakdown_us": t["breakdown_us"],
+            "plain_launches": {"ms_per_step": t["plain_ms_per_step"],
+                               "value": units / (t["plain_ms_per_step"] / 1000.0)},
+            "graph_note": "value: one CUDA graph per step with events only around it (consecutive kernels overlap "
+                          "their launch); breakdown_us: a second graph with events between the stages",
+            "tokens_scanned_per_s": value * w.L, "clocks": t["clocks"], **extra,
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_sweep(args, rank, world, dev, pg):
+    """Flat against hierarchical indexing on identical inputs (B=2, P=64, M=256,
+    k=2048), L = 64K .. 1M: the indexing call alone and the whole step."""
+    import torch
+    from kv_indexing_b200 import inputs as I
+    from kv_indexing_b200 import lsa as L
+
+    seed = rank_seed(args.seed, rank)
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def flush():
+        flush_buf.random_(0, 255)
+
+    peaks, peak_src = measured_peaks()
+    table = []
+    K = max(10, min(args.steps, 50))
+    for Lc in SWEEP_L:
+        wh = I.scaled(I.WORKLOADS["hier_decode_1m"], L=Lc, name=f"hier_decode_{Lc // 1024}k")
+        wf = I.scaled(I.WORKLOADS["flat_decode_1m"], L=Lc, name=f"flat_decode_{Lc // 1024}k")
+        x = host_inputs(wh, seed)                 # identical for both (same seed and shapes)
+        ph = Path(torch, L, wh, x, dev, seed, False)
+        pf = Path(torch, L, wf, x, dev, seed, False, layers=ph.layers)   # the same latent KV and queries
+        th = time_device(torch, ph.stages, K, 3, flush, dev, pg)
+        tf = time_device(torch, pf.stages, K, 3, flush, dev, pg)
+        flat_index = tf["breakdown_us"]["indexer"] + tf["breakdown_us"]["select"]
+        hier_index = th["breakdown_us"]["hier_index"]
+        table.append({
+            "L": Lc, "flat_index_us": flat_index, "hier_index_us": hier_index,
+            "index_speedup_hier_over_flat": flat_index / hier_index,
+            "flat_step_us": 1000 * tf["ms_per_step"], "hier_step_us": 1000 * th["ms_per_step"],
+            "step_speedup_hier_over_flat": tf["ms_per_step"] / th["ms_per_step"],
+            "flat_index_frac_of_hbm": indexer_bytes_per_query(wf) * wf.B / (flat_index * 1e-6) / 1e9
+            / peaks["hbm_gbs"],
+            "hier_index_frac_of_hbm": hier_index_bytes_per_query(wh) * wh.B / (hier_index * 1e-6) / 1e9
+            / peaks["hbm_gbs"],
+            "clocks_sm_mhz": th["clocks"]["sm_mhz"], "clock_reasons": sorted(set(th["clocks"]["reasons"]) |
+                                                                             set(tf["clocks"]["reasons"])),
+        })
+        del ph, pf
+        torch.cuda.empty_cache()
+    last = table[-1]
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC, "value": 2 * world / (last["hier_step_us"] * 1e-6), "unit": UNIT, "n_gpus": world,
+            "steps": K, "warmup": 3, "ms_per_step": last["hier_step_us"] / 1000, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "hier_sweep", "B": 2, "P": 64, "M": 256, "k": 2048, "L": list(SWEEP_L),
+                       "l2": "flushed between timed steps"},
+            "sweep": table, "peak_source": peak_src,
+            "note": "index = the indexing call(s) only (flat: scores + top-k; hierarchical: page scores, recall, "
+                    "fine scores, top-k; page pooling is once per filled page, outside); step = index + attention",
+        }), flush=True)
+    return 0
 
 
 def main():
@@ -509,7 +901,6 @@ def main():
     if args.impl == "reference":
         return run_reference(args, rank, world)
 
-    import numpy as np
     import torch
     import torch.distributed as dist
 
@@ -524,181 +915,13 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=180), device_id=dev)
         pg = True
     L.load()
-    w = I.WORKLOADS[args.workload]
-    if w.P or w.m or w.n_layers > 1 or w.T > 1 or args.fp8:
-        return run_workload(args, w, rank, world, dev, pg)
-    seed = rank_seed(args.seed, rank)                   # each rank its own batch
-    x = I.make_indexer_inputs(w, seed)
-    a = I.make_attn_inputs(w, seed)
-
-    def up(arr, kind):
-        t = torch.from_numpy(np.ascontiguousarray(arr).view(np.int16) if kind == "bf16" else arr)
-        t = t.view(torch.bfloat16) if kind == "bf16" else t
-        return t.to(dev)
-
-    q, k, wt = up(x["q_idx"], "bf16"), up(x["k_idx"], "bf16"), up(x["w"], "f32")
-    sl = up(x["seq_len"], "i32")
-    qa, kv = up(a["qa"], "bf16"), up(a["kv"], "bf16")
-    B, T = w.B, w.T
-    budget = (w.k, w.sink, w.window)
-    scores = torch.empty((B, T, w.L), dtype=torch.float32, device=dev)
-    idx = torch.empty((B, T, w.k), dtype=torch.int32, device=dev)
-    out = torch.empty((B, T, w.Hq, w.d_v), dtype=torch.bfloat16, device=dev)
-    ai = L.attn_in(qa, sl, w.scale, kv=kv, d_v=w.d_v, stream_budget=budget)
-    attn_ws_n = L.workspace_size(L.LSA_OP_SPARSE_ATTN, attn=ai, budget=(w.k, 0, 0))
-    attn_ws = torch.empty(max(attn_ws_n, 256), dtype=torch.uint8, device=dev)
-    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    flat_ws = torch.empty(L.workspace_size(L.LSA_OP_INDEX_FLAT, indexer=L.indexer_in(q, wt, k, sl), budget=budget),
-                          dtype=torch.uint8, device=dev)
-    sel_ws = torch.empty(max(256, L.workspace_size(L.LSA_OP_SELECT, budget=budget, B=B, T=T, L_max=w.L)),
-                         dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream(dev)
-
-    def k_index():
-        L.lsa_index_flat(q, wt, k, sl, budget, scores_out=scores, with_idx=False, stream=stream)
-
-    def k_select():
-        L.lsa_select_streaming(scores, sl, budget, idx=idx, workspace=sel_ws, stream=stream)
-
-    def k_attn():
-        L.lsa_sparse_attn(qa, idx, sl, w.scale, kv=kv, d_v=w.d_v, out=out, workspace=attn_ws, stream=stream,
-                          stream_budget=budget)
-
-    def flush():
-        flush_buf.random_(0, 255)   # touch 256 MiB (> 126 MB L2)
-
-    for _ in range(max(3, args.warmup)):
-        flush()
-        k_index(); k_select(); k_attn()
-    torch.cuda.synchronize()
-    L.lsa_device_status()
-
-    # One CUDA graph per step. The timed graph has events only around the whole
-    # step, so consecutive kernels may overlap their launch (programmatic
-    # dependent launch); a second graph with events between the stages gives
-    # the per-stage breakdown (stages then run back to back).
-    def capture(stage_events):
-        ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
-        g = torch.cuda.CUDAGraph()
-        cap = torch.cuda.Stream(dev)
-        cap.wait_stream(stream)
-        with torch.cuda.graph(g, stream=cap, capture_error_mode="relaxed"):
-            s = torch.cuda.current_stream(dev)
-            ev[0].record(s)
-            L.lsa_index_flat(q, wt, k, sl, budget, scores_out=scores, with_idx=False, stream=s)
-            if stage_events:
-                ev[1].record(s)
-            L.lsa_select_streaming(scores, sl, budget, idx=idx, workspace=sel_ws, stream=s)
-            if stage_events:
-                ev[2].record(s)
-            L.lsa_sparse_attn(qa, idx, sl, w.scale, kv=kv, d_v=w.d_v, out=out, workspace=attn_ws, stream=s,
-                              stream_budget=budget)
-            ev[3].record(s)
-        torch.cuda.synchronize()
-        for _ in range(3):
-            flush()
-            g.replay()
-        torch.cuda.synchronize()
-        return g, ev
-
-    g, ev = capture(False)
-    gb, evb = capture(True)
-
-    K = args.steps
-    t_step, t_idx, t_sel, t_att = [], [], [], []
-    if pg:
-        dist.barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(str(torch.cuda.get_device_properties(dev).uuid)) as clk:
-        for _ in range(K):
-            flush()
-            g.replay()
-            torch.cuda.synchronize()
-            t_step.append(ev[0].elapsed_time(ev[3]))
-    torch.cuda.synchronize()
-    if pg:
-        dist.barrier()
-    for _ in range(K):
-        flush()
-        gb.replay()
-        torch.cuda.synchronize()
-        t_idx.append(evb[0].elapsed_time(evb[1]))
-        t_sel.append(evb[1].elapsed_time(evb[2]))
-        t_att.append(evb[2].elapsed_time(evb[3]))
-    torch.cuda.synchronize()
-    L.lsa_device_status()
-    total_ms = max_over_ranks(float(sum(t_step)), dev, pg)
-    ms_per_step = total_ms / K
-    units = B * T * world
-    value = units / (ms_per_step / 1000.0)
-
-    # end to end through the public API with host buffers: per step copy the
-    # step's queries in (indexer q and w, attention q), read o and idx back
-    e2e = None
-    if not args.no_e2e:
-        hq = torch.from_numpy(x["q_idx"].view(np.int16)).view(torch.bfloat16).pin_memory()
-        hw = torch.from_numpy(x["w"]).pin_memory()
-        hqa = torch.from_numpy(a["qa"].view(np.int16)).view(torch.bfloat16).pin_memory()
-        ho = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
-        hi = torch.empty(idx.shape, dtype=torch.int32).pin_memory()
-        dq, dw, dqa = torch.empty_like(q), torch.empty_like(wt), torch.empty_like(qa)
-        h2d = sum(t.numel() * t.element_size() for t in (hq, hw, hqa))
-        d2h = ho.numel() * ho.element_size() + hi.numel() * hi.element_size()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e2e_ms = []
-        for i in range(3 + K):
-            flush()
-            e0.record(stream)
-            dq.copy_(hq, non_blocking=True); dw.copy_(hw, non_blocking=True); dqa.copy_(hqa, non_blocking=True)
-            ix = L.lsa_index_flat(dq, dw, k, sl, budget, idx=idx, workspace=flat_ws, stream=stream)
-            L.lsa_sparse_attn(dqa, ix, sl, w.scale, kv=kv, d_v=w.d_v, out=out, workspace=attn_ws, stream=stream,
-                              stream_budget=budget)
-            ho.copy_(out, non_blocking=True); hi.copy_(idx, non_blocking=True)
-            e1.record(stream)
-            torch.cuda.synchronize()
-            if i >= 3:
-                e2e_ms.append(e0.elapsed_time(e1))
-        em = max_over_ranks(sum(e2e_ms) / len(e2e_ms), dev, pg)
-        e2e = {"value": units / (em / 1000.0), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
-               "d2h_bytes_per_step": int(d2h), "ms_per_step": em,
-               "note": "KV and indexer-key caches resident; per step the new queries go in and o, idx come out"}
-
-    peaks, peak_src = measured_peaks()
-    idx_us = 1000 * sum(t_idx) / K
-    idx_bytes = indexer_bytes_per_query(w) * B * T
-    achieved = idx_bytes / (idx_us * 1e-6) / 1e9
-    roof = {"bound": "hbm", "kernel": "indexer (tcgen05 score GEMM + fused epilogue)", "achieved": achieved,
-            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-            "traffic": kernel_traffic("indexer_flat_decode_128k"),
-            "algorithmic_bytes_per_launch": idx_bytes, "launch_us": idx_us, "peak_source": peak_src,
-            "step_frac_of_hbm_roofline": (step_bytes_per_query(w) * B * T / (ms_per_step * 1e-3) / 1e9)
-            / peaks["hbm_gbs"]}
-
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, n, dt = time_oracle(w, x, a)
-        cpu = {"value": v, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-               "sample": f"{n} of {B * T} queries of the batch, whole path, {dt:.1f} s"}
-
-    if rank == 0:
-        line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
-            "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16, U(0,1) head weights, 1% planted needles)",
-            "config": workload_config(w, parallelism=f"replicas x{world} (independent batches)"),
-            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": 4 * K,
-            "breakdown_us": {"indexer": idx_us, "select": 1000 * sum(t_sel) / K, "attention": 1000 * sum(t_att) / K,
-                             "note": "stages timed back to back (events between them); the value's step lets "
-                                     "consecutive kernels overlap their launch"},
-            "tokens_scanned_per_s": value * w.L,
-            "clocks": clk.summary(),
-        }
-        print(json.dumps(line), flush=True)
-    del g, gb
-    if pg:
-        dist.destroy_process_group()
-    return 0
+    try:
+        if args.workload == "hier_sweep":
+            return run_sweep(args, rank, world, dev, pg)
+        return run_workload(args, I.WORKLOADS[args.workload], rank, world, dev, pg)
+    finally:
+        if pg:
+            dist.destroy_process_group()
 
 
 if __name__ == "__main__":

@@ -73,6 +73,17 @@ struct SelectArgs {
   // grid-cooperative path: per-row coordination blocks
   void* grid_ws;
   size_t grid_row_bytes;
+  // filter path: group maxima of 2^g0_shift slots (written by group_max_kernel
+  // or by the indexer's epilogue), the per-row pool of kept candidates, the
+  // per-warp segment table and the per-row counters (arrivals, pool fill)
+  uint32_t* gmax;         // [rows][gmax_stride] order-preserving keys, 0 = no candidate
+  int gmax_stride;
+  int g0_shift, fold;     // the lower bound uses groups of 2^g0_shift * fold slots
+  uint32_t* pool_keys;    // [rows][pool_cap]
+  int* pool_slots;        // [rows][pool_cap]
+  int pool_cap;
+  uint4* wtab;            // [rows][C * warps]: (pool base, kept, equal to the bound, 0)
+  unsigned* counters;     // [rows][2]
   int* status;
 };
 
@@ -83,13 +94,25 @@ struct SelectPlan {
   bool grid;              // grid-cooperative launch (rows * C CTAs co-resident)
   bool cluster;           // one thread-block cluster of C CTAs per row (no workspace)
   int cluster_rc;         // cluster path: keys per thread (32 or 64)
+  bool filter;            // filter path: group-maximum bound, C CTAs per row, last CTA finishes
+  int g0_shift, fold, gmax_stride, pool_cap;
 };
+
+// Workspace layout of the filter path (offsets from the selection workspace).
+struct FilterLayout {
+  size_t gmax, pool_keys, pool_slots, wtab, counters, total;
+};
+FilterLayout filter_layout(int rows, const SelectPlan& p);
 
 // d_bound: an upper bound on the dynamic budget of any row (k - sink - window for
 // token selection, M for page recall).
 SelectPlan select_plan(int rows, int n_slots, int d_bound, int num_sms);
 size_t select_ws_bytes(int rows, const SelectPlan& p);
-cudaError_t launch_select(const SelectArgs& a, const SelectPlan& p, void* ws, cudaStream_t stream);
+// gmax_ready: the group maxima are already in the workspace and the row
+// counters cleared (the indexer's epilogue did both); otherwise a pre-pass
+// computes them from the scores.
+cudaError_t launch_select(const SelectArgs& a, const SelectPlan& p, void* ws, cudaStream_t stream,
+                          bool gmax_ready = false);
 
 // ------------------------------------------------------------------ pooling --
 cudaError_t launch_pool(const uint16_t* k, const int* seq_len, int B, int L_max, int d, int P,

@@ -139,7 +139,7 @@ struct Thr {
 };
 
 struct Shared {
-  uint32_t hist[kDigits];
+  alignas(16) uint32_t hist[kDigits];   // 16-byte aligned: read four bins at a time
   uint32_t tmp[32];
   uint32_t red[3][kWarps];
   uint32_t cnt, mn, mx;
@@ -182,12 +182,14 @@ __device__ __noinline__ void block_cnt_min_max(uint32_t c, uint32_t mn, uint32_t
   __syncthreads();
 }
 
-// Exact threshold of the D-th best key of keys[0, n) (key 0 = not a candidate).
-__device__ Thr cta_threshold(const uint32_t* keys, int n, uint32_t D, Shared& sh) {
+// Exact threshold of the D-th best key of key(0) .. key(n - 1) (key 0 = not a
+// candidate); `key` reads element i (shared or global memory).
+template <class K>
+__device__ Thr cta_threshold_by(K&& key, int n, uint32_t D, Shared& sh) {
   const int tid = threadIdx.x;
   Thr r{0u, 0u, false};
   uint32_t c = 0u;
-  for (int i = tid; i < n; i += kThreads) c += keys[i] != 0u ? 1u : 0u;
+  for (int i = tid; i < n; i += kThreads) c += key(i) != 0u ? 1u : 0u;
   uint32_t total = 0u;
   block_incl_scan(c, sh.tmp, &total);
   if (total <= D) {
@@ -206,7 +208,7 @@ __device__ Thr cta_threshold(const uint32_t* keys, int n, uint32_t D, Shared& sh
     for (int i = tid; i < nb; i += kThreads) sh.hist[i] = 0u;
     __syncthreads();
     for (int i = tid; i < n; i += kThreads) {
-      const uint32_t k = keys[i];
+      const uint32_t k = key(i);
       if (k != 0u && (k & mask) == prefix) atomicAdd(&sh.hist[(k >> shift) & dmask], 1u);
     }
     __syncthreads();
@@ -237,6 +239,10 @@ __device__ Thr cta_threshold(const uint32_t* keys, int n, uint32_t D, Shared& sh
   r.thr = prefix;
   r.need_eq = need;
   return r;
+}
+
+__device__ Thr cta_threshold(const uint32_t* keys, int n, uint32_t D, Shared& sh) {
+  return cta_threshold_by([&](int i) { return keys[i]; }, n, D, sh);
 }
 
 // Emit the selected elements of keys[0, n) in index order: emit(out_pos, i).
@@ -1494,6 +1500,444 @@ __global__ void __launch_bounds__(kThreads, 1) select_cluster_kernel(const Selec
   cluster_sync_all();   // no CTA leaves while another may still read its lists or histograms
 }
 
+// ===========================================================================
+// Filter path (few rows, each split over C CTAs; no spin waits).
+//
+// A lower bound on the threshold comes from group maxima. Cut a row's slots
+// into groups of G and take each group's maximum key over its dynamic
+// candidates; let v be the D-th largest of these maxima. At least D groups have
+// a candidate >= v, so the D-th best candidate is >= v. And every candidate
+// strictly above v lies in one of the fewer than D groups whose maximum
+// exceeds v, so fewer than D * G candidates are above v (when at most D groups
+// hold candidates v = 0 and every candidate counts, again fewer than D * G + 1).
+// Each CTA finds v from the row's group maxima (the same v in every CTA),
+// streams its segment of the row and keeps the candidates above v in one run
+// per warp, in slot order, in a per-row pool; it also counts those equal to v.
+// The last CTA of the row to finish takes the exact top D of the kept
+// candidates -- or, when fewer than D are above v, all of them and the
+// lowest-slot candidates equal to v -- and writes the row.
+// ===========================================================================
+
+// Exact D-th best of the nonzero keys held in registers (R per thread, any
+// layout): radix rounds of 11-bit digits over key - kmin, each a 2048-bin
+// shared histogram whose target bin is found by a conflict-free warp-chunked
+// scan from the top. Same result as reg_threshold, fewer and cheaper steps.
+template <int R>
+__device__ Thr fast_threshold(const uint32_t (&k)[R], uint32_t D, Shared& sh) {
+  constexpr int kBits = 11, kBins = 1 << kBits;          // 2048 bins: 128 per warp, 4 per lane
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint32_t c = 0u, mn = 0xFFFFFFFFu, mx = 0u;
+#pragma unroll
+  for (int j = 0; j < R; ++j)
+    if (k[j] != 0u) {
+      ++c;
+      mn = min(mn, k[j]);
+      mx = max(mx, k[j]);
+    }
+  block_cnt_min_max(c, mn, mx, sh);
+  Thr r{0u, 0u, false};
+  const uint32_t total = sh.cnt, kmin = sh.mn, kmax = sh.mx;
+  if (total <= D) {
+    r.all = true;
+    return r;
+  }
+  if (D == 0u) {
+    r.thr = 0xFFFFFFFFu;
+    return r;
+  }
+  if (kmin == kmax) {
+    r.thr = kmax;
+    r.need_eq = D;
+    return r;
+  }
+  const int bits = 32 - __clz(kmax - kmin);               // every rel = key - kmin is < 2^bits
+  int prev = bits;                                         // keys in play satisfy rel >> prev == hi
+  int shift = bits > kBits ? bits - kBits : 0;
+  uint32_t hi = 0u, need = D;
+  uint4* h4 = reinterpret_cast<uint4*>(sh.hist);
+  while (true) {
+    const int width = prev - shift;                        // digit bits this round (<= 11)
+    const uint32_t dmask = (1u << width) - 1u;
+    if (tid < kBins / 4) h4[tid] = make_uint4(0u, 0u, 0u, 0u);
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < R; ++j) {
+      const uint32_t rel = k[j] - kmin;
+      const bool in = k[j] != 0u && (prev >= 32 || (rel >> prev) == hi);
+      if (in) atomicAdd(&sh.hist[(rel >> shift) & dmask], 1u);
+    }
+    __syncthreads();
+    // warp w owns bins [kBins - 128 (w + 1), kBins - 128 w) counted from the top;
+    // lane l holds four of them as one 16-byte load (conflict-free)
+    const int b0 = kBins - 128 * (warp + 1) + 4 * (31 - lane);   // lowest of the lane's four bins
+    const uint4 v = h4[b0 >> 2];
+    const uint32_t lsum = v.x + v.y + v.z + v.w;
+    uint32_t incl = lsum;                                  // inclusive scan from the top within the warp
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) sh.red[0][warp] = incl;
+    __syncthreads();
+    uint32_t before = 0u;                                  // bins above this warp's chunk
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) before += w < warp ? sh.red[0][w] : 0u;
+    const uint32_t excl = before + incl - lsum;
+    if (excl < need && need <= excl + lsum) {
+      const uint32_t cnt[4] = {v.w, v.z, v.y, v.x};       // top bin first
+      uint32_t above = excl;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (above + cnt[q] >= need) {
+          sh.bin = b0 + 3 - q;
+          sh.above = above;
+          break;
+        }
+        above += cnt[q];
+      }
+    }
+    __syncthreads();
+    hi = (width >= 32 ? 0u : (hi << width)) | static_cast<uint32_t>(sh.bin);
+    need -= sh.above;
+    __syncthreads();
+    if (shift == 0) break;
+    prev = shift;
+    shift = shift > kBits ? shift - kBits : 0;
+  }
+  r.thr = kmin + hi;
+  r.need_eq = need;
+  return r;
+}
+
+constexpr int kPhase1Per = 32;                    // group maxima per thread in phase 1
+constexpr int kStageCap = 8192;                   // kept candidates staged in shared memory by the finisher
+constexpr int kWarpSlots = 1024;                  // slots per warp in phase 2 (held in registers)
+constexpr int kPhase1Cap = kThreads * kPhase1Per; // 16384 per row
+
+// gmax[r][g] = max key over slots [g G0, g G0 + G0) of row r that are dynamic
+// candidates (0 if none); entries past the row's groups are 0.
+__global__ void __launch_bounds__(256) group_max_kernel(const SelectArgs a) {
+  pdl_wait();   // the scores come from the previous kernel
+  pdl_trigger();
+  const int r = blockIdx.y;
+  const Plan pl = make_plan(a, r);
+  const int G0 = 1 << a.g0_shift;
+  const float* row = a.scores + static_cast<long long>(r) * a.row_stride;
+  uint32_t* gm = a.gmax + static_cast<long long>(r) * a.gmax_stride;
+  const int lo = pl.valid ? pl.dyn_lo : 0, hi = pl.valid ? pl.dyn_hi : 0;
+  if (blockIdx.x == 0 && threadIdx.x < 2) a.counters[2 * r + threadIdx.x] = 0u;   // arrivals, pool fill
+  for (int g = blockIdx.x * blockDim.x + threadIdx.x; g < a.gmax_stride; g += gridDim.x * blockDim.x) {
+    const int s0 = g << a.g0_shift;
+    uint32_t m = 0u;
+    if (s0 < hi && s0 + G0 > lo) {
+      for (int i = 0; i < G0; ++i) {
+        const int s = s0 + i;
+        if (s >= lo && s < hi) m = max(m, score_key(__ldg(row + s)));
+      }
+    }
+    gm[g] = m;
+  }
+}
+
+// Slot range [lo, hi) of warp `w` of CTA `c` (C CTAs, kWarps warps each) within
+// the row's dynamic region.
+struct WarpRange {
+  int lo, hi;
+};
+__device__ __forceinline__ WarpRange warp_range(const Plan& pl, int C, int c, int w) {
+  const int len = pl.dyn_hi - pl.dyn_lo;
+  const int seg = (len + C - 1) / C;
+  const int c_lo = pl.dyn_lo + min(len, c * seg), c_hi = pl.dyn_lo + min(len, (c + 1) * seg);
+  const int sub = (seg + kWarps - 1) / kWarps;
+  const int lo = min(c_hi, c_lo + w * sub);
+  return WarpRange{lo, min(c_hi, lo + sub)};
+}
+
+__global__ void __launch_bounds__(kThreads, 1) select_filter_kernel(const SelectArgs a) {
+  pdl_wait();   // scores and group maxima come from the previous kernel(s)
+  pdl_trigger();
+  const int C = static_cast<int>(gridDim.x);
+  const int c = blockIdx.x, r = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t lt = (1u << lane) - 1u;
+  __shared__ Shared sh;
+  extern __shared__ __align__(16) uint32_t filt_dsm[];
+
+  const Plan pl = make_plan(a, r);
+  int* out = a.out + static_cast<long long>(r) * a.out_len;
+  if (!pl.valid) {
+    if (c == 0)
+      for (int i = tid; i < a.out_len; i += kThreads) out[i] = -1;
+    return;   // every CTA of the row returns; the row's counters are untouched
+  }
+  const uint32_t D = static_cast<uint32_t>(pl.D);
+  const int nreg = C * kWarps;
+  const float* row = a.scores + static_cast<long long>(r) * a.row_stride;
+  const long long pbase = static_cast<long long>(r) * a.pool_cap;
+  uint4* wt_row = a.wtab + static_cast<long long>(r) * nreg;
+
+  // ---- phase 1: the D-th largest group maximum v (0: keep every candidate)
+  uint32_t v = 0u;
+  if (D > 0u) {
+    const uint32_t* gm = a.gmax + static_cast<long long>(r) * a.gmax_stride;
+    const int F = a.fold;
+    const int n_fold = a.gmax_stride / F;
+    uint32_t k[kPhase1Per];
+    const int e0 = warp * 32 * kPhase1Per + lane;   // element of k[j]: e0 + 32 j
+    // predicated loads, all in flight at once (fold F in {1, 2, 4, 8})
+    if (F == 1) {
+#pragma unroll
+      for (int j = 0; j < kPhase1Per; ++j) {
+        const int e = e0 + 32 * j;
+        k[j] = e < n_fold ? __ldcg(gm + e) : 0u;
+      }
+    } else if (F == 2) {
+#pragma unroll
+      for (int j = 0; j < kPhase1Per; ++j) {
+        const int e = e0 + 32 * j;
+        const uint2 q = e < n_fold ? __ldcg(reinterpret_cast<const uint2*>(gm) + e) : make_uint2(0u, 0u);
+        k[j] = max(q.x, q.y);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < kPhase1Per; ++j) {
+        const int e = e0 + 32 * j;
+        const uint4 q = e < n_fold ? __ldcg(reinterpret_cast<const uint4*>(gm + e * F)) : make_uint4(0u, 0u, 0u, 0u);
+        k[j] = max(max(q.x, q.y), max(q.z, q.w));
+      }
+      if (F == 8) {
+#pragma unroll
+        for (int j = 0; j < kPhase1Per; ++j) {
+          const int e = e0 + 32 * j;
+          const uint4 q = e < n_fold ? __ldcg(reinterpret_cast<const uint4*>(gm + e * F + 4)) : make_uint4(0u, 0u, 0u, 0u);
+          k[j] = max(k[j], max(max(q.x, q.y), max(q.z, q.w)));
+        }
+      }
+    }
+    const Thr t = fast_threshold<kPhase1Per>(k, D, sh);
+    v = t.all ? 0u : t.thr;
+  }
+
+  // ---- phase 2: keep this warp's candidates above v (slot order), count those equal to v.
+  // The warp's slots (at most kWarpSlots: the plan gives every row enough CTAs)
+  // are loaded once, all in flight, and stay in registers for both passes.
+  if (D > 0u) {
+    const WarpRange wr = warp_range(pl, C, c, warp);
+    uint32_t kk[kWarpSlots / 32];
+#pragma unroll
+    for (int j = 0; j < kWarpSlots / 32; ++j) {
+      const int s = wr.lo + lane + 32 * j;
+      kk[j] = s < wr.hi ? score_key(__ldcg(row + s)) : 0u;
+    }
+    uint32_t kept = 0u, n_eq = 0u;
+#pragma unroll
+    for (int j = 0; j < kWarpSlots / 32; ++j) {
+      kept += __popc(__ballot_sync(0xffffffffu, kk[j] > v));
+      n_eq += __popc(__ballot_sync(0xffffffffu, v != 0u && kk[j] == v));
+    }
+    uint32_t base = 0u;
+    if (lane == 0 && kept) base = atomicAdd(a.counters + 2 * r + 1, kept);
+    base = __shfl_sync(0xffffffffu, base, 0);
+    if (base + kept > static_cast<uint32_t>(a.pool_cap)) {   // cannot happen (see above); never write past the pool
+      if (lane == 0) record_timeout(a.status);
+      kept = 0u;
+    }
+    if (kept) {
+      uint32_t run = base;
+#pragma unroll
+      for (int j = 0; j < kWarpSlots / 32; ++j) {
+        const uint32_t m = __ballot_sync(0xffffffffu, kk[j] > v);
+        if (kk[j] > v) {
+          const uint32_t p = run + __popc(m & lt);
+          a.pool_keys[pbase + p] = kk[j];
+          a.pool_slots[pbase + p] = wr.lo + lane + 32 * j;
+        }
+        run += __popc(m);
+      }
+    }
+    if (lane == 0) wt_row[c * kWarps + warp] = make_uint4(base, kept, n_eq, 0u);
+  }
+
+  // ---- phase 3: the last CTA of the row finishes it
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) sh.last = atomicAdd(a.counters + 2 * r, 1u) == static_cast<unsigned>(C - 1);
+  __syncthreads();
+  if (!sh.last) return;
+  __threadfence();
+
+  uint4* wt = reinterpret_cast<uint4*>(filt_dsm);                 // [nreg] this row's warp table
+  uint32_t* sel = reinterpret_cast<uint32_t*>(wt + nreg);         // [nreg] selected per warp run
+  uint32_t* take = sel + nreg;                                    // [nreg] ties taken per warp run
+  uint32_t* off = take + nreg;                                    // [nreg] output offset per warp run
+  const int M = a.M, P = a.P;
+  const long long prow = static_cast<long long>(r) * M;
+  auto token = [&](int slot) {
+    return a.mode == kSelectHierTokens ? __ldg(a.pages + prow + slot / P) * P + slot % P : slot;
+  };
+  int* dyn_out = out + pl.dyn_off;
+  // Exclusive prefix over the warp runs of x(i) into pre[i] (each thread a
+  // contiguous chunk of runs); returns the total.
+  auto run_prefix = [&](auto&& x, uint32_t* pre) -> uint32_t {
+    const int per = (nreg + kThreads - 1) / kThreads;
+    const int i0 = tid * per;
+    uint32_t loc = 0u;
+    for (int q = 0; q < per; ++q)
+      if (i0 + q < nreg) loc += x(i0 + q);
+    uint32_t total = 0u;
+    uint32_t run = block_incl_scan(loc, sh.tmp, &total) - loc;
+    for (int q = 0; q < per; ++q)
+      if (i0 + q < nreg) {
+        const uint32_t xv = x(i0 + q);
+        pre[i0 + q] = run;
+        run += xv;
+      }
+    __syncthreads();
+    return total;
+  };
+  // Ties to the lowest slots (the runs are in slot order): run i takes
+  // min(eq_i, need - ties before it); then output offsets of (above_i + take_i).
+  auto place = [&](auto&& above, uint32_t need) -> uint32_t {
+    run_prefix([&](int i) { return take[i]; }, off);   // off[i] = ties before run i
+    const int per = (nreg + kThreads - 1) / kThreads;
+    for (int q = 0; q < per; ++q) {
+      const int i = tid * per + q;
+      if (i < nreg) take[i] = need > off[i] ? min(take[i], need - off[i]) : 0u;
+    }
+    __syncthreads();
+    return run_prefix([&](int i) { return above(i) + take[i]; }, off);
+  };
+  uint32_t n_sel = 0u;
+  if (D > 0u) {
+    uint32_t g_loc = 0u;
+    for (int i = tid; i < nreg; i += kThreads) {
+      const uint4 e = __ldcg(wt_row + i);
+      wt[i] = e;
+      g_loc += e.y;
+    }
+    uint32_t G = 0u;
+    block_incl_scan(g_loc, sh.tmp, &G);   // also orders the table fill before its use
+    const uint32_t* pk = a.pool_keys + pbase;
+    const int* ps = a.pool_slots + pbase;
+    // the kept candidates in slot order: run i's land at sk[at[i] ..]; each
+    // thread copies whole runs, its loads independent of one another
+    uint32_t* at = sel;
+    run_prefix([&](int i) { return wt[i].y; }, at);
+    uint32_t* sk = off + nreg;                                   // [kStageCap] keys
+    int* ss = reinterpret_cast<int*>(sk + kStageCap);            // [kStageCap] slots
+    const bool staged = G <= static_cast<uint32_t>(kStageCap);
+    if (staged) {
+      for (int i = tid; i < nreg; i += kThreads) {
+        const uint4 e = wt[i];
+        const uint32_t d0 = at[i];
+        for (uint32_t j0 = 0; j0 < e.y; j0 += 8) {
+          uint32_t kv[8];
+          int sv[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const bool in = j0 + q < e.y;
+            kv[q] = in ? __ldcg(pk + e.x + j0 + q) : 0u;
+            sv[q] = in ? __ldcg(ps + e.x + j0 + q) : 0;
+          }
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            if (j0 + q < e.y) {
+              sk[d0 + j0 + q] = kv[q];
+              ss[d0 + j0 + q] = sv[q];
+            }
+        }
+      }
+      __syncthreads();
+    }
+    if (G >= D && staged) {
+      // the exact D-th best is among the kept candidates: registers, warp-striped
+      // (element w 32 R + 32 j + l in k[j] of lane l, warp w: slot order is (warp, j, lane))
+      constexpr int R = kStageCap / kThreads;
+      uint32_t k[R];
+      const int e0 = warp * 32 * R + lane;
+#pragma unroll
+      for (int j = 0; j < R; ++j) k[j] = e0 + 32 * j < static_cast<int>(G) ? sk[e0 + 32 * j] : 0u;
+      const Thr t = fast_threshold<R>(k, D, sh);
+      n_sel = reg_emit<R>(k, t, sh, [&](uint32_t p, int j) { dyn_out[p] = token(ss[e0 + 32 * j]); });
+    } else if (G >= D) {
+      // more kept candidates than shared memory holds (not expected for scores
+      // that are not adversarial): the same from the pool in global memory
+      const Thr t = cta_threshold_by([&](int i) { return __ldcg(pk + i); }, static_cast<int>(G), D, sh);
+      for (int i = warp; i < nreg; i += kWarps) {
+        const uint4 e = wt[i];
+        uint32_t gt = 0u, eq = 0u;
+        for (uint32_t j0 = 0; j0 < e.y; j0 += 32) {
+          const uint32_t kk = j0 + lane < e.y ? __ldcg(pk + e.x + j0 + lane) : 0u;
+          gt += __popc(__ballot_sync(0xffffffffu, kk != 0u && (t.all || kk > t.thr)));
+          eq += __popc(__ballot_sync(0xffffffffu, kk != 0u && !t.all && kk == t.thr));
+        }
+        if (lane == 0) {
+          sel[i] = gt;
+          take[i] = eq;
+        }
+      }
+      __syncthreads();
+      n_sel = place([&](int i) { return sel[i]; }, t.all ? 0u : t.need_eq);
+      for (int i = warp; i < nreg; i += kWarps) {
+        const uint4 e = wt[i];
+        uint32_t pos = off[i], eq_run = 0u;
+        const uint32_t tk = take[i];
+        for (uint32_t j0 = 0; j0 < e.y; j0 += 32) {
+          const bool in = j0 + lane < e.y;
+          const uint32_t kk = in ? __ldcg(pk + e.x + j0 + lane) : 0u;
+          const bool gt = kk != 0u && (t.all || kk > t.thr);
+          const bool eq = kk != 0u && !t.all && kk == t.thr;
+          const uint32_t em = __ballot_sync(0xffffffffu, eq);
+          const bool s = gt || (eq && eq_run + __popc(em & lt) < tk);
+          const uint32_t sm = __ballot_sync(0xffffffffu, s);
+          if (s) dyn_out[pos + __popc(sm & lt)] = token(__ldcg(ps + e.x + j0 + lane));
+          pos += __popc(sm);
+          eq_run += __popc(em);
+        }
+      }
+    } else {
+      // every kept candidate (G < D <= kStageCap, so they are staged), and the
+      // lowest-slot candidates equal to v
+      const bool ties = v != 0u;                                  // v = 0: the kept candidates are all there are
+      for (int i = tid; i < nreg; i += kThreads) take[i] = ties ? wt[i].z : 0u;
+      __syncthreads();
+      // at[] (staged offsets) is overwritten by place(); keep the runs' staged starts in wt[i].w
+      for (int i = tid; i < nreg; i += kThreads) wt[i].w = at[i];
+      __syncthreads();
+      n_sel = place([&](int i) { return wt[i].y; }, ties ? D - G : 0u);
+      for (int i = warp; i < nreg; i += kWarps) {
+        const uint4 e = wt[i];
+        uint32_t pos = off[i];
+        const uint32_t tk = take[i];
+        if (tk == 0u) {
+          for (uint32_t j0 = lane; j0 < e.y; j0 += 32) dyn_out[pos + j0] = token(ss[e.w + j0]);
+        } else {
+          // this run holds some of the ties: rescan its slots
+          const WarpRange wr = warp_range(pl, C, i / kWarps, i % kWarps);
+          uint32_t eq_run = 0u;
+          for (int s0 = wr.lo; s0 < wr.hi; s0 += 32) {
+            const int s = s0 + lane;
+            const uint32_t kk = s < wr.hi ? score_key(__ldcg(row + s)) : 0u;
+            const bool eq = kk == v;
+            const uint32_t em = __ballot_sync(0xffffffffu, eq);
+            const bool sl = kk > v || (eq && eq_run + __popc(em & lt) < tk);
+            const uint32_t sm = __ballot_sync(0xffffffffu, sl);
+            if (sl) dyn_out[pos + __popc(sm & lt)] = token(s);
+            pos += __popc(sm);
+            eq_run += __popc(em);
+          }
+        }
+      }
+    }
+  }
+  for (int i = tid; i < pl.lead_a_n; i += kThreads) out[i] = pl.lead_a_lo + i;
+  for (int i = tid; i < pl.lead_b_n; i += kThreads) out[pl.lead_a_n + i] = pl.lead_b_lo + i;
+  const int tr0 = pl.dyn_off + static_cast<int>(n_sel);
+  for (int i = tid; i < pl.trail_n; i += kThreads) out[tr0 + i] = pl.trail_lo + i;
+  for (int i = tr0 + pl.trail_n + tid; i < a.out_len; i += kThreads) out[i] = -1;
+}
+
 }  // namespace
 
 SelectPlan select_plan(int rows, int n_slots, int d_bound, int num_sms) {
@@ -1526,6 +1970,36 @@ SelectPlan select_plan(int rows, int n_slots, int d_bound, int num_sms) {
     p.cand_cap = 0;
     return p;
   }
+  // filter path: rows too long for one cluster and for the grid launch, few enough
+  // that each gets two or more CTAs
+  if (d_bound >= 1 && n_slots > kClusterMax * kThreads * 64 && n_slots <= (1 << 21) && 2 * rows <= num_sms) {
+    p.filter = true;
+    const int c_min = (n_slots + kWarps * kWarpSlots - 1) / (kWarps * kWarpSlots);   // warp slices fit registers
+    p.C = std::max(c_min, std::min((n_slots + 4095) / 4096, num_sms / rows));
+    p.seg = seg_of(p.C);
+    // groups of G slots: the bound is tight when there are many groups per
+    // dynamic slot (G <= n / (8 D)); phase 1 holds at most kPhase1Cap of them
+    int G = 1;
+    while (G < 64 && 16ll * G * d_bound <= n_slots) G *= 2;
+    while (true) {
+      const int g0 = std::min(G, 16);
+      int sh = 0;
+      while ((1 << sh) < g0) ++sh;
+      const int fold = G / g0;
+      const int ng0 = (n_slots + g0 - 1) / g0;
+      const int unit = std::max(fold, 4);
+      const int stride = (ng0 + unit - 1) / unit * unit;
+      if (stride / fold <= kPhase1Cap) {
+        p.g0_shift = sh;
+        p.fold = fold;
+        p.gmax_stride = stride;
+        break;
+      }
+      G *= 2;
+    }
+    p.pool_cap = d_bound * G + 32;
+    return p;
+  }
   // few rows: ~2K keys per CTA for latency; rows alone fill the GPU: register-sized segments
   int C = rows >= num_sms ? std::max(1, (n_slots + kLocalRegs - 1) / kLocalRegs)
                           : std::max(1, std::min(64, (n_slots + 2047) / 2048));
@@ -1539,16 +2013,61 @@ SelectPlan select_plan(int rows, int n_slots, int d_bound, int num_sms) {
   return p;
 }
 
+FilterLayout filter_layout(int rows, const SelectPlan& p) {
+  auto al = [](size_t x) { return (x + 255) / 256 * 256; };
+  FilterLayout L{};
+  size_t o = 0;
+  L.gmax = o;
+  o += al(static_cast<size_t>(rows) * p.gmax_stride * 4);
+  L.pool_keys = o;
+  o += al(static_cast<size_t>(rows) * p.pool_cap * 4);
+  L.pool_slots = o;
+  o += al(static_cast<size_t>(rows) * p.pool_cap * 4);
+  L.wtab = o;
+  o += al(static_cast<size_t>(rows) * p.C * kWarps * 16);
+  L.counters = o;
+  o += al(static_cast<size_t>(rows) * 8);
+  L.total = o;
+  return L;
+}
+
 size_t select_ws_bytes(int rows, const SelectPlan& p) {
+  if (p.filter) return filter_layout(rows, p).total;
   if (p.cluster) return 0;
   if (p.grid) return grid_blocks_bytes(rows) + grid_row_bytes(p.C) * rows;
   const size_t n = static_cast<size_t>(rows) * p.C * p.cand_cap;
   return ((n * 8 + rows * 4 + 255) / 256) * 256;
 }
 
-cudaError_t launch_select(const SelectArgs& a0, const SelectPlan& p, void* ws, cudaStream_t stream) {
+cudaError_t launch_select(const SelectArgs& a0, const SelectPlan& p, void* ws, cudaStream_t stream,
+                          bool gmax_ready) {
   SelectArgs a = a0;
   const int rows = a.B * a.T;
+  if (p.filter) {
+    const FilterLayout Ly = filter_layout(rows, p);
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    a.gmax = reinterpret_cast<uint32_t*>(w + Ly.gmax);
+    a.gmax_stride = p.gmax_stride;
+    a.g0_shift = p.g0_shift;
+    a.fold = p.fold;
+    a.pool_keys = reinterpret_cast<uint32_t*>(w + Ly.pool_keys);
+    a.pool_slots = reinterpret_cast<int*>(w + Ly.pool_slots);
+    a.pool_cap = p.pool_cap;
+    a.wtab = reinterpret_cast<uint4*>(w + Ly.wtab);
+    a.counters = reinterpret_cast<unsigned*>(w + Ly.counters);
+    void* args[] = {&a};
+    if (!gmax_ready) {
+      const int blocks = std::min((p.gmax_stride + 255) / 256, 64);
+      cudaError_t e = launch_pdl(reinterpret_cast<const void*>(&group_max_kernel), dim3(blocks, rows), dim3(256), 0,
+                                 stream, args);
+      if (e != cudaSuccess) return e;
+    }
+    const size_t smem = static_cast<size_t>(p.C) * kWarps * 28 + static_cast<size_t>(kStageCap) * 8;
+    const void* fn = reinterpret_cast<const void*>(&select_filter_kernel);
+    cudaError_t e = set_max_smem(fn, smem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(fn, dim3(p.C, rows), dim3(kThreads), smem, stream, args);
+  }
   if (p.cluster) {
     const size_t smem = cluster_smem_words(p.cluster_rc) * 4;
     const void* fn = p.cluster_rc == 64 ? reinterpret_cast<const void*>(&select_cluster_kernel<64>)

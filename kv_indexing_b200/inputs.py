@@ -83,6 +83,11 @@ WORKLOADS: Dict[str, Workload] = {
     "hier_decode_1m": Workload(
         name="hier_decode_1m", B=2, L=1048576, T=1, H=64, d=128, k=2048, sink=64,
         window=960, needle_frac=0.01, P=64, M=256),
+    # Flat decode at 1M tokens: the hierarchical workload's inputs with the
+    # hierarchy off (same seed => identical indexer inputs and needles).
+    "flat_decode_1m": Workload(
+        name="flat_decode_1m", B=2, L=1048576, T=1, H=64, d=128, k=2048, sink=64,
+        window=960, needle_frac=0.01),
     # Cross-layer group: two layers share one indexer pass.
     "cli_group_256k": Workload(
         name="cli_group_256k", B=4, L=262144, T=1, H=64, d=128, k=2048, sink=64,

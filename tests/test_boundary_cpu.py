@@ -86,7 +86,7 @@ def test_workspace_checks_and_sizes():
     n_ext = L.workspace_size(L.LSA_OP_INDEX_FLAT, indexer=ii, budget=(2048, 64, 960), scores_external=True)
     assert n - n_ext == 8 * 131072 * 4                     # the score buffer moves out of the workspace
     sel = L.workspace_size(L.LSA_OP_SELECT, budget=(2048, 64, 960), B=8, T=1, L_max=131072)
-    assert sel == n_ext == 0                               # rows of <= 128K keys select in cluster shared memory
+    assert sel == n_ext == 0                               # rows of <= 256K keys select in cluster shared memory
     st = lib.lsa_index_flat(ctypes.byref(ii), L.Budget(2048, 64, 960), 16, None, 256, n - 1, None)
     assert st == L.LSA_ERR_WORKSPACE
     big = L.workspace_size(L.LSA_OP_SELECT, budget=(2048, 64, 960), B=2, T=1, L_max=1 << 20)
@@ -95,8 +95,11 @@ def test_workspace_checks_and_sizes():
     assert st == L.LSA_ERR_WORKSPACE
     hi = L.workspace_size(L.LSA_OP_INDEX_HIER, indexer=_indexer(B=2, L_max=1 << 20), budget=(2048, 64, 960),
                           P=64, M=256)
-    # page scores + recalled pages + fine scores; 16K-candidate selections need no scratch
-    assert hi == 2 * (1 << 14) * 4 + 2 * 256 * 4 + 2 * 256 * 64 * 4
+    # page scores + recalled pages + fine scores, then the larger of the two selections' scratch
+    sel_pages = L.workspace_size(L.LSA_OP_SELECT, budget=(256, 0, 0), B=2, T=1, L_max=1 << 14)
+    sel_fine = L.workspace_size(L.LSA_OP_SELECT, budget=(2048, 64, 960), B=2, T=1, L_max=256 * 64)
+    fixed = 2 * (1 << 14) * 4 + 2 * 256 * 4 + 2 * 256 * 64 * 4
+    assert fixed <= hi <= fixed + max(sel_pages, sel_fine) + 256
 
 
 def test_hier_parameter_validation():
@@ -124,16 +127,24 @@ def test_compressed_entry_validation_and_sizes():
     assert lib.lsa_index_compressed(ctypes.byref(ii), 4, bu, None, None, None, 0, None) == L.LSA_ERR_INVALID_ARG
     big = _indexer(B=4, L_max=1 << 20)
     n = L.workspace_size(L.LSA_OP_INDEX_COMPRESSED, indexer=big, budget=(2048, 16, 240), m=4)
-    assert n == 4 * (1 << 18) * 4          # entry scores only: 262144-entry rows select in cluster shared memory
+    sel = L.workspace_size(L.LSA_OP_SELECT, budget=(2048, 16, 240), B=4, T=1, L_max=1 << 18)
+    assert n == 4 * (1 << 18) * 4 + sel    # entry scores + the selection's scratch over 262144-entry rows
     assert L.workspace_size(L.LSA_OP_INDEX_COMPRESSED, indexer=big, budget=(2048, 16, 240), m=4,
-                            scores_external=True) == 0
+                            scores_external=True) == sel
     st = lib.lsa_index_compressed(ctypes.byref(big), 4, bu, 16, None, 256, n - 1, None)
     assert st == L.LSA_ERR_WORKSPACE
 
 
-def test_cluster_selection_covers_rows_up_to_262144_slots():
+def test_selection_launch_shapes_by_workspace():
+    # rows of <= 262144 slots: one cluster per row, keys in shared memory, no scratch
+    assert L.workspace_size(L.LSA_OP_SELECT, budget=(2048, 64, 960), B=80, T=1, L_max=262144) == 0
     assert L.workspace_size(L.LSA_OP_SELECT, budget=(2048, 64, 960), B=4, T=1, L_max=262144) == 0
-    assert L.workspace_size(L.LSA_OP_SELECT, budget=(2048, 64, 960), B=4, T=1, L_max=262144 + 64 + 960 + 1) > 0
+    # many longer rows: per-segment candidate lists in the workspace
+    assert L.workspace_size(L.LSA_OP_SELECT, budget=(2048, 64, 960), B=80, T=1, L_max=262144 + 1025) > 0
+    # few longer rows: the filter launch -- group maxima, a candidate pool of at
+    # most D x G entries per row, per-warp tables, counters
+    few = L.workspace_size(L.LSA_OP_SELECT, budget=(2048, 64, 960), B=4, T=1, L_max=1 << 20)
+    assert 0 < few < 4 * (1 << 20) * 8
 
 
 def _mla_layer(q, kv, B=1, T=1, L_max=1024, Hq=128):

@@ -23,15 +23,15 @@ from tests.parity import dev, host
 
 
 def test_noalloc_rejects_oversized_shape_on_the_host():
-    # B*T=16 rows at L_max=1M need just over 16 MiB of selection scratch; the
+    # B*T=22 rows at L_max=1M need just over 16 MiB of selection scratch; the
     # call must refuse before touching the (fake, never dereferenced) pointers.
     lib = L.load()
     fake = ctypes.c_void_p(256)
-    st = lib.lsa_select_streaming_noalloc(fake, fake, 16, 1, 1 << 20, L.Budget(2048, 64, 960), fake, None)
+    st = lib.lsa_select_streaming_noalloc(fake, fake, 22, 1, 1 << 20, L.Budget(2048, 64, 960), fake, None)
     assert st == L.LSA_ERR_WORKSPACE
     msg = lib.lsa_last_error().decode()
     assert "static scratch" in msg and str(L.LSA_NOALLOC_SCRATCH_BYTES) in msg
-    need = L.workspace_size(L.LSA_OP_SELECT, budget=(2048, 64, 960), B=16, T=1, L_max=1 << 20)
+    need = L.workspace_size(L.LSA_OP_SELECT, budget=(2048, 64, 960), B=22, T=1, L_max=1 << 20)
     assert need > L.LSA_NOALLOC_SCRATCH_BYTES
 
 
@@ -58,26 +58,26 @@ def _scores(seed, B, T, L_max, seq_len, ties=False):
 
 # Consecutive calls on the two launch shapes that keep scratch in the static
 # buffer. Rows longer than 262144 slots go to the grid-cooperative launch while
-# rows x CTAs fit the GPU at once (4 rows of 300000 slots: about 1 MiB of
-# per-row coordination blocks, counters and flags); otherwise to per-segment
-# candidate lists merged by the last CTA of each row (15 rows of 1M slots: about
-# 15.7 MiB, just under the limit). Each shape runs twice with new scores and
-# interleaved with the other, so leftovers of one call sit in the scratch when
-# the next starts.
-GRID = (4, 1, 300000, (2048, 64, 960))
-TWO_LEVEL = (15, 1, 1 << 20, (2048, 64, 960))
+# rows x CTAs fit the GPU at once (4 rows of 300000 slots: per-row coordination
+# blocks, counters and flags, about 1 MiB); longer rows to the filter launch (15
+# rows of 1M slots: the rows' group maxima, candidate pools, per-warp tables and
+# counters, about 11.8 MiB, near the limit). Each shape runs twice with new
+# scores, interleaved with the other, so the leftovers of one call sit in the
+# scratch when the next starts.
+SHAPE_A = (4, 1, 300000, (2048, 64, 960))
+SHAPE_B = (15, 1, 1 << 20, (2048, 64, 960))
 CALLS = [
-    (21, GRID, [300000, 300000, 123457, 299999], True),
-    (22, TWO_LEVEL, [1 << 20] * 12 + [700001, 5000, 1 << 20], False),
-    (23, GRID, [299000, 300000, 300000, 65536], False),
-    (24, TWO_LEVEL, [1 << 20, 999999] + [1 << 20] * 13, True),
+    (21, SHAPE_A, [300000, 300000, 123457, 299999], True),
+    (22, SHAPE_B, [1 << 20] * 12 + [700001, 5000, 1 << 20], False),
+    (23, SHAPE_A, [299000, 300000, 300000, 65536], False),
+    (24, SHAPE_B, [1 << 20, 999999] + [1 << 20] * 13, True),
 ]
 
 
 def test_noalloc_shapes_use_the_static_scratch():
     # guard: if a plan change stopped these shapes from using scratch, the GPU
     # test below would no longer reach the static buffer
-    for B, T, L_max, budget in (GRID, TWO_LEVEL):
+    for B, T, L_max, budget in (SHAPE_A, SHAPE_B):
         need = L.workspace_size(L.LSA_OP_SELECT, budget=budget, B=B, T=T, L_max=L_max)
         assert 0 < need <= L.LSA_NOALLOC_SCRATCH_BYTES, (B, L_max, need)
 
