@@ -266,6 +266,7 @@ class Path:
         self.idx = torch.empty((B, T, w.k), dtype=torch.int32, device=dev)
         self.outs = [torch.empty((B, T, w.Hq, w.d_v), dtype=torch.bfloat16, device=dev) for _ in range(w.n_layers)]
         self.extra = {}
+        self.breakdown_stages = None
         self._build()
 
     def _ws(self, n):
@@ -304,10 +305,21 @@ class Path:
                 self.api_ws = self._ws(L.workspace_size(L.LSA_OP_INDEX_FLAT, indexer=ii, budget=budget))
                 index_scores = lambda s: L.lsa_index_flat(q, wt, k, sl, budget, q_scale=qs, k_scale=ks,
                                                           scores_out=self.scores, with_idx=False, stream=s)
-            self.stages = [("indexer", index_scores),
-                           ("select", lambda s: L.lsa_select_streaming(self.scores, sl_sel, budget, idx=self.idx,
-                                                                       workspace=self.sel_ws, stream=s)),
-                           ("attention", attn(0))]
+            if w.m:
+                index_call = lambda s: L.lsa_index_compressed(q, wt, k, sl, w.m, budget, q_scale=qs, k_scale=ks,
+                                                              idx=self.idx, workspace=self.api_ws, stream=s)
+            else:
+                index_call = lambda s: L.lsa_index_flat(q, wt, k, sl, budget, q_scale=qs, k_scale=ks, idx=self.idx,
+                                                        workspace=self.api_ws, stream=s)
+            # the step: the indexing call (scores and selection, fused where the
+            # selection uses the indexer's summaries) then attention; the
+            # breakdown splits the indexing call into scores alone and selection
+            self.stages = [("index", index_call), ("attention", attn(0))]
+            self.breakdown_stages = [("indexer", index_scores),
+                                     ("select", lambda s: L.lsa_select_streaming(self.scores, sl_sel, budget,
+                                                                                 idx=self.idx, workspace=self.sel_ws,
+                                                                                 stream=s)),
+                                     ("attention", attn(0))]
             self.dominant = "indexer"
             if kind == "prefill":
                 self.roof_kernel = "indexer (tcgen05 score GEMM over causal tiles, fused epilogue)"
@@ -450,19 +462,25 @@ def graph_kernel_count(g):
         return None
 
 
-def time_device(torch, stages, K, warmup, flush, dev, pg):
+def time_device(torch, stages, K, warmup, flush, dev, pg, breakdown_stages=None):
     """Whole step as one graph (events only around it), per-stage breakdown from
-    a second graph, and the same step as plain launches. Returns a dict."""
+    a second graph (of breakdown_stages when given: the same work split into
+    finer calls), and the same step as plain launches. Returns a dict."""
     import torch.distributed as dist
     stream = torch.cuda.current_stream(dev)
+    bstages = breakdown_stages or stages
     for _ in range(max(3, warmup)):
         flush()
         for _, fn in stages:
             fn(stream)
+        flush()
+        for _, fn in bstages:
+            fn(stream)
     torch.cuda.synchronize()
     g, ev, launches = capture(torch, stages, dev, stream, inner_events=False, keep_graph=True)
-    gb, evb, _ = capture(torch, stages, dev, stream, inner_events=True)
+    gb, evb, _ = capture(torch, bstages, dev, stream, inner_events=True)
     n = len(stages)
+    nb = len(bstages)
     for _ in range(3):
         flush()
         g.replay()
@@ -482,12 +500,12 @@ def time_device(torch, stages, K, warmup, flush, dev, pg):
     torch.cuda.synchronize()
     if pg:
         dist.barrier()
-    per = [[] for _ in range(n)]
+    per = [[] for _ in range(nb)]
     for _ in range(K):
         flush()
         gb.replay()
         torch.cuda.synchronize()
-        for i in range(n):
+        for i in range(nb):
             per[i].append(evb[i].elapsed_time(evb[i + 1]))
     # plain launches: the same calls issued on the stream, no graph
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -504,7 +522,7 @@ def time_device(torch, stages, K, warmup, flush, dev, pg):
     return {
         "ms_per_step": max_over_ranks(float(sum(step)) / K, dev, pg),
         "step_ms_median": statistics.median(step),
-        "breakdown_us": {name: 1000 * sum(per[i]) / K for i, (name, _) in enumerate(stages)},
+        "breakdown_us": {name: 1000 * sum(per[i]) / K for i, (name, _) in enumerate(bstages)},
         "plain_ms_per_step": max_over_ranks(float(sum(plain)) / K, dev, pg),
         "clocks": clk.summary(),
         "launches_per_step": launches,
@@ -791,7 +809,7 @@ def run_workload(args, w, rank, world, dev, pg):
     def flush():
         flush_buf.random_(0, 255)   # touch 256 MiB (> 126 MB L2)
 
-    t = time_device(torch, path.stages, args.steps, args.warmup, flush, dev, pg)
+    t = time_device(torch, path.stages, args.steps, args.warmup, flush, dev, pg, path.breakdown_stages)
     L.lsa_device_status()
     extra = dict(path.extra)
     if path.kind == "group":
@@ -831,7 +849,8 @@ def run_workload(args, w, rank, world, dev, pg):
             "plain_launches": {"ms_per_step": t["plain_ms_per_step"],
                                "value": units / (t["plain_ms_per_step"] / 1000.0)},
             "graph_note": "value: one CUDA graph per step with events only around it (consecutive kernels overlap "
-                          "their launch); breakdown_us: a second graph with events between the stages",
+                          "their launch); breakdown_us: a second graph with events between the stages (the "
+                          "indexing call split into scores alone and the selection)",
             "tokens_scanned_per_s": value * w.L, "clocks": t["clocks"], **extra,
         }
         print(json.dumps(line), flush=True)
@@ -862,7 +881,7 @@ def run_sweep(args, rank, world, dev, pg):
         pf = Path(torch, L, wf, x, dev, seed, False, layers=ph.layers)   # the same latent KV and queries
         th = time_device(torch, ph.stages, K, 3, flush, dev, pg)
         tf = time_device(torch, pf.stages, K, 3, flush, dev, pg)
-        flat_index = tf["breakdown_us"]["indexer"] + tf["breakdown_us"]["select"]
+        flat_index = tf["breakdown_us"]["index"]
         hier_index = th["breakdown_us"]["hier_index"]
         table.append({
             "L": Lc, "flat_index_us": flat_index, "hier_index_us": hier_index,

@@ -277,8 +277,17 @@ size_t flat_ws_bytes(const lsa_indexer_in_t* in, lsa_budget_t bu, bool scores_ex
 }
 
 // ------------------------------------------------------------ launchers --
+// Where the indexer writes the selection's group maxima (FLAT scores feeding a
+// filter-launch selection), or nothing.
+struct FusedSummary {
+  uint32_t* gmax = nullptr;
+  int gmax_stride = 0, g0_shift = 0;
+  unsigned* counters = nullptr;
+  int sink = 0, window = 0;
+};
+
 lsa_status_t run_flat_scores(const lsa_indexer_in_t* in, const void* keys, int L_rows, int vis_shift,
-                             float* scores, cudaStream_t st) {
+                             float* scores, cudaStream_t st, const FusedSummary& fs = FusedSummary{}) {
   const bool fp8 = in->dtype == LSA_E4M3;
   const FlatPlan fp = flat_plan(in->T, in->H, L_rows);
   CUtensorMap tm_k, tm_q;
@@ -298,6 +307,8 @@ lsa_status_t run_flat_scores(const lsa_indexer_in_t* in, const void* keys, int L
   a.seq_len = in->seq_len; a.w = in->w; a.q_scale = in->q_scale; a.k_scale = in->k_scale;
   a.out = scores; a.out_row_stride = L_rows;
   a.inv_sqrt_d = 1.0f / std::sqrt(static_cast<float>(in->d));
+  a.gmax = fs.gmax; a.gmax_stride = fs.gmax_stride; a.g0_shift = fs.g0_shift; a.sel_counters = fs.counters;
+  if (fs.gmax) { a.sink = fs.sink; a.window = fs.window; }
   a.status = device_status_ptr();
   const int grid = static_cast<int>(std::min<long long>(a.n_items, device_sm_count()));
   if (grid < 1) return LSA_OK;
@@ -307,7 +318,8 @@ lsa_status_t run_flat_scores(const lsa_indexer_in_t* in, const void* keys, int L
 
 lsa_status_t run_select(int mode, int B, int T, int L_max, const int* seq_len, const float* scores,
                         long long row_stride, int n_slots, lsa_budget_t bu, int P, int M, const int* pages,
-                        int* out, int out_len, void* sws, cudaStream_t st, int entry_shift = 0) {
+                        int* out, int out_len, void* sws, cudaStream_t st, int entry_shift = 0,
+                        bool summary_ready = false) {
   SelectArgs a{};
   a.mode = mode; a.B = B; a.T = T; a.L_max = L_max; a.seq_len = seq_len;
   a.entry_shift = entry_shift;
@@ -317,8 +329,26 @@ lsa_status_t run_select(int mode, int B, int T, int L_max, const int* seq_len, c
   a.status = device_status_ptr();
   const SelectPlan p = mode == kSelectPages ? page_select_plan(B * T, n_slots, M)
                                             : token_select_plan(B * T, n_slots, bu);
-  LSA_CHECK_CUDA(launch_select(a, p, sws, st), "select launch");
+  LSA_CHECK_CUDA(launch_select(a, p, sws, st, summary_ready && p.filter), "select launch");
   return LSA_OK;
+}
+
+// The indexer-side half of the fused decode selection: when token selection
+// over n_slots will take the filter launch, the FLAT indexer writes its group
+// maxima (and clears its counters) into the selection workspace `sws`.
+FusedSummary fused_summary(int rows, int n_slots, lsa_budget_t bu, void* sws) {
+  FusedSummary fs;
+  const SelectPlan p = token_select_plan(rows, n_slots, bu);
+  if (!p.filter) return fs;
+  const FilterLayout Ly = filter_layout(rows, p);
+  uint8_t* w = static_cast<uint8_t*>(sws);
+  fs.gmax = reinterpret_cast<uint32_t*>(w + Ly.gmax);
+  fs.gmax_stride = p.gmax_stride;
+  fs.g0_shift = p.g0_shift;
+  fs.counters = reinterpret_cast<unsigned*>(w + Ly.counters);
+  fs.sink = bu.sink;
+  fs.window = bu.window;
+  return fs;
 }
 
 lsa_status_t run_hier(const lsa_indexer_in_t* in, const void* page_keys, int P, int M, lsa_budget_t bu,
@@ -660,10 +690,11 @@ lsa_status_t lsa_index_flat(const lsa_indexer_in_t* in, lsa_budget_t budget, int
     scores = reinterpret_cast<float*>(w);
     w += align_up(static_cast<size_t>(in->B) * in->T * in->L_max * 4, 256);
   }
-  if ((s = run_flat_scores(in, in->k, in->L_max, 0, scores, st)) != LSA_OK) return s;
+  const FusedSummary fs = idx ? fused_summary(in->B * in->T, in->L_max, budget, w) : FusedSummary{};
+  if ((s = run_flat_scores(in, in->k, in->L_max, 0, scores, st, fs)) != LSA_OK) return s;
   if (idx)
     return run_select(kSelectTokens, in->B, in->T, in->L_max, in->seq_len, scores, in->L_max, in->L_max, budget, 0,
-                      0, nullptr, idx, budget.k, w, st);
+                      0, nullptr, idx, budget.k, w, st, 0, fs.gmax != nullptr);
   return LSA_OK;
 }
 
@@ -687,10 +718,11 @@ lsa_status_t lsa_index_compressed(const lsa_indexer_in_t* in, int32_t m, lsa_bud
     scores = reinterpret_cast<float*>(w);
     w += align_up(static_cast<size_t>(in->B) * in->T * n_e * 4, 256);
   }
-  if ((s = run_flat_scores(in, in->k, n_e, shift, scores, st)) != LSA_OK) return s;
+  const FusedSummary fs = idx ? fused_summary(in->B * in->T, n_e, budget, w) : FusedSummary{};
+  if ((s = run_flat_scores(in, in->k, n_e, shift, scores, st, fs)) != LSA_OK) return s;
   if (idx)
     return run_select(kSelectTokens, in->B, in->T, in->L_max, in->seq_len, scores, n_e, n_e, budget, 0, 0, nullptr,
-                      idx, budget.k, w, st, shift);
+                      idx, budget.k, w, st, shift, fs.gmax != nullptr);
   return LSA_OK;
 }
 
@@ -805,9 +837,10 @@ lsa_status_t lsa_layer_group(const lsa_indexer_in_t* in, const void* page_keys, 
   } else {
     float* scores = reinterpret_cast<float*>(w);
     uint8_t* sws = w + align_up(static_cast<size_t>(in->B) * in->T * in->L_max * 4, 256);
-    if ((s = run_flat_scores(in, in->k, in->L_max, 0, scores, st)) != LSA_OK) return s;
+    const FusedSummary fs = fused_summary(in->B * in->T, in->L_max, budget, sws);
+    if ((s = run_flat_scores(in, in->k, in->L_max, 0, scores, st, fs)) != LSA_OK) return s;
     if ((s = run_select(kSelectTokens, in->B, in->T, in->L_max, in->seq_len, scores, in->L_max, in->L_max, budget,
-                        0, 0, nullptr, idx_buf, budget.k, sws, st)) != LSA_OK)
+                        0, 0, nullptr, idx_buf, budget.k, sws, st, 0, fs.gmax != nullptr)) != LSA_OK)
       return s;
   }
   for (int i = 0; i < n_layers;) {

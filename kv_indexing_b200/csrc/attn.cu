@@ -375,10 +375,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 // accumulates its half of the output columns (O += P V over 256 of the 512
 // latent columns, with P in tensor memory as the MMA A operand).
 //
-// Roles (320 threads):
-//   warp 0      TMA producer: index entries (prefetched one ring ahead) ->
-//               validity mask, tiled boxes for contiguous runs, tile::gather4
-//               row gathers otherwise, into a kStages-deep ring of 64-row blocks
+// Roles (352 threads):
+//   warps 0, 10 TMA producers, each for half of every block (rows 0-31 and
+//               32-63): index entries (prefetched one ring ahead) -> validity
+//               mask, tiled boxes for contiguous runs, tile::gather4 row
+//               gathers otherwise, into a kStages-deep ring of 64-row blocks.
+//               Two warps issue the 80 gather operations of a block: measured
+//               on B200, one issuing warp is what limits a random-row gather
+//               (3.2 us per 64-row block against 2.2 us with two)
 //   warp 1      TMEM owner; lane 0 issues QK(b) then PV(b - 1)
 //   warps 2..9  softmax: two threads per head, each on 32 of a block's 64
 //               columns. Software-pipelined: the partial scores of block b + 1
@@ -387,8 +391,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 //               threads of a head agree on the block max through a tagged
 //               shared-memory slot (bounded wait, no block-wide barrier).
 namespace mla {
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;
 constexpr int kSoftThreads = 256;
+constexpr int kProducer2 = 10;                      // the second producer warp
 constexpr int BN = 64;                              // KV rows per block
 constexpr int kStages = 3;
 constexpr int kChunks = 5;                          // 64-column chunks per CTA and block
@@ -524,7 +529,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_full[i], 2);    // one expect_tx arrive per producer warp
       mbar_init(&kv_empty[i], 1);
     }
     mbar_init(s_full, 1);
@@ -559,9 +564,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t tO = tmem + kColO, tQ = tmem + kColQ, tS = tmem + kColS, tP = tmem + kColP;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer --
-    if (lane == 0) {
+  if (warp == 0 || warp == kProducer2) {
+    // ----------------------------------------------------------- producers --
+    const int part = warp == 0 ? 0 : 1;   // rows [32 part, 32 part + 32) of every block
+    if (part == 0 && lane == 0) {
       // q rows [r Hq, r Hq + 128) x this CTA's chunks, 128-byte swizzled, into the exchange buffers
       mbar_arrive_expect_tx(q_full, nq * 16384);
       for (int j = 0; j < nq; ++j) tma_load_2d(sX + j * 16384, tm_q, q_full, (q_chunk0 + j) * 64, r * a.Hq);
@@ -609,32 +615,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int id0 = __shfl_sync(0xffffffffu, id_lo, 0);
         const bool contiguous =
             __all_sync(0xffffffffu, id0 >= 0 && id_lo == id0 + lane && id_hi == id0 + 32 + lane);
-        const int y_lo = row0 + (id_lo >= 0 ? id_lo : 0), y_hi = row0 + (id_hi >= 0 ? id_hi : 0);
+        const int y_mine = row0 + (part == 0 ? (id_lo >= 0 ? id_lo : 0) : (id_hi >= 0 ? id_hi : 0));
         int yg[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int src = (4 * lane + q) & 31;
-          const int a_lo = __shfl_sync(0xffffffffu, y_lo, src), a_hi = __shfl_sync(0xffffffffu, y_hi, src);
-          yg[q] = lane < 8 ? a_lo : a_hi;   // lane g gathers block rows 4g .. 4g + 3
-        }
+        for (int q = 0; q < 4; ++q)   // lane g < 8 gathers block rows 32 part + 4g .. + 3
+          yg[q] = __shfl_sync(0xffffffffu, y_mine, (4 * lane + q) & 31);
         if (lane == 0) {
-          mask_s[2 * j] = valid_lo;
-          mask_s[2 * j + 1] = valid_hi;
-          mbar_arrive_expect_tx(&kv_full[j], kStageBytes);
+          if (part == 0) {
+            mask_s[2 * j] = valid_lo;
+            mask_s[2 * j + 1] = valid_hi;
+          }
+          mbar_arrive_expect_tx(&kv_full[j], kStageBytes / 2);
         }
         __syncwarp();
         uint8_t* st = sStage + j * kStageBytes;
         if (contiguous) {
-          if (lane < 2 * kChunks) {
-            const int c = lane >> 1, hrow = lane & 1;   // two 32-row boxes per chunk
-            tma_load_2d(st + c * kChunkBytes + hrow * (kChunkBytes / 2), tm_kt, &kv_full[j], (chunk0 + c) * 64,
-                        row0 + id0 + 32 * hrow);
-          }
-        } else if (lane < BN / 4) {
+          if (lane < kChunks)   // one 32-row box per chunk
+            tma_load_2d(st + lane * kChunkBytes + part * (kChunkBytes / 2), tm_kt, &kv_full[j],
+                        (chunk0 + lane) * 64, row0 + id0 + 32 * part);
+        } else if (lane < BN / 8) {
 #pragma unroll
           for (int c = 0; c < kChunks; ++c)
-            tma_gather4(st + c * kChunkBytes + lane * 512, tm_kg, &kv_full[j], (chunk0 + c) * 64, yg[0], yg[1],
-                        yg[2], yg[3]);
+            tma_gather4(st + c * kChunkBytes + (8 * part + lane) * 512, tm_kg, &kv_full[j], (chunk0 + c) * 64,
+                        yg[0], yg[1], yg[2], yg[3]);
         }
       }
     }

@@ -122,6 +122,21 @@ __device__ __forceinline__ void relu_dot_acc(const float* wcol, const uint32_t (
   }
 }
 
+// Selection summary written beside a FLAT score (the selection's filter launch
+// reads it): the maximum score key of each group of 2^g0_shift consecutive
+// slots over the query's dynamic candidates -- visible, neither sink nor
+// window -- from the 32 consecutive slots of this warp (one per lane).
+// Warp-uniform: every lane calls it.
+__device__ __forceinline__ void flat_group_max(const IndexerArgs& a, long long qrow, int s, int nvis, float v,
+                                               int lane) {
+  const int pe = nvis - 1;                           // the query's last visible slot
+  const int sink_end = min(a.sink, max(pe + 1, 0));
+  const int w_lo = max(sink_end, pe - a.window + 1);
+  uint32_t key = (s >= sink_end && s < w_lo) ? score_key(v) : 0u;
+  for (int o = 1; o < (1 << a.g0_shift); o <<= 1) key = max(key, __shfl_xor_sync(0xffffffffu, key, o));
+  if ((lane & ((1 << a.g0_shift) - 1)) == 0) a.gmax[qrow * a.gmax_stride + (s >> a.g0_shift)] = key;
+}
+
 __device__ __forceinline__ float sum8(const float (&a)[8]) {
   return ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
 }
@@ -180,6 +195,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   pdl_wait();   // inputs may come from the previous kernel in the stream
   pdl_trigger();
+  if (a.sel_counters && blockIdx.x == 0)   // the selection that follows starts from zero counters
+    for (int i = threadIdx.x; i < 2 * a.B * a.T; i += blockDim.x) a.sel_counters[i] = 0u;
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
@@ -320,6 +337,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!a.gather) {
           if (s < a.L_rows)
             for (int qi = 0; qi < g.nq; ++qi) a.out[orow + qi * a.out_row_stride + s] = -INFINITY;
+          if (a.gmax && (lane & ((1 << a.g0_shift) - 1)) == 0)
+            for (int qi = 0; qi < g.nq; ++qi)
+              a.gmax[(static_cast<long long>(g.b) * a.T + g.q0 + qi) * a.gmax_stride + (s >> a.g0_shift)] = 0u;
         } else if (s < a.M * a.P) {
           a.out[orow + s] = -INFINITY;
         }
@@ -365,7 +385,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!a.gather) {
               const int pos = g.pos0 + qi;   // key s visible iff s < (pos + 1) >> vis_shift
               const int nvis = pos < 0 ? 0 : (pos + 1) >> a.vis_shift;
-              if (s < a.L_rows) a.out[orow + qi * a.out_row_stride + s] = s < nvis ? sc * kscale : -INFINITY;
+              const float v = s < nvis ? sc * kscale : -INFINITY;
+              if (s < a.L_rows) a.out[orow + qi * a.out_row_stride + s] = v;
+              if (a.gmax) flat_group_max(a, static_cast<long long>(g.b) * a.T + g.q0 + qi, s, nvis, v, lane);
             } else if (s < a.M * a.P) {
               const int page = __ldg(a.pages + (static_cast<long long>(g.b) * a.T + g.q0) * a.M + s / a.P);
               const int tok = page * a.P + (s & (a.P - 1));
@@ -389,7 +411,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!a.gather) {
               const int pos = g.pos0 + qi;
               const int nvis = pos < 0 ? 0 : (pos + 1) >> a.vis_shift;
-              if (s < a.L_rows) a.out[orow + qi * a.out_row_stride + s] = s < nvis ? sc * kscale : -INFINITY;
+              const float v = s < nvis ? sc * kscale : -INFINITY;
+              if (s < a.L_rows) a.out[orow + qi * a.out_row_stride + s] = v;
+              if (a.gmax) flat_group_max(a, static_cast<long long>(g.b) * a.T + g.q0 + qi, s, nvis, v, lane);
             } else if (s < a.M * a.P) {
               const int page = __ldg(a.pages + (static_cast<long long>(g.b) * a.T + g.q0) * a.M + s / a.P);
               const int tok = page * a.P + (s & (a.P - 1));

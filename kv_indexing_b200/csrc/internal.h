@@ -37,6 +37,13 @@ struct IndexerArgs {
   // GATHER
   const int* pages;
   int M, P, sink, window;
+  // FLAT, feeding the selection's filter launch (gmax != null): per query row
+  // the maximum score key over each group of 2^g0_shift slots that are dynamic
+  // candidates (sink and window excluded, visible only), and the selection's
+  // per-row counters cleared
+  uint32_t* gmax;
+  int gmax_stride, g0_shift;
+  unsigned* sel_counters;
   int* status;           // per-device status word
 };
 
@@ -47,6 +54,17 @@ cudaError_t launch_indexer(const CUtensorMap& tm_k, const CUtensorMap& tm_q, con
                            bool fp8, int grid, cudaStream_t stream);
 
 // --------------------------------------------------------- streaming select --
+// Order-preserving key of a score: larger score, larger key; -inf -> 0 (not a
+// candidate), -0 ranks as +0. NaN is not supported.
+#ifdef __CUDACC__
+__device__ __forceinline__ uint32_t score_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  if (u == 0x80000000u) u = 0u;                         // -0 ranks as +0
+  const uint32_t k = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return k <= 0x007FFFFFu ? 0u : k;                     // -inf: not a candidate
+}
+#endif
+
 enum SelectMode { kSelectTokens = 0, kSelectHierTokens = 1, kSelectPages = 2 };
 
 struct SelectArgs {

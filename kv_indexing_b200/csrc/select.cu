@@ -35,12 +35,6 @@ constexpr int kPer = 8;          // consecutive elements per thread per compacti
 constexpr int kRL = 16;          // keys per thread, local phase
 constexpr int kRF = 32;          // keys per thread, merge phase
 
-__device__ __forceinline__ uint32_t score_key(float f) {
-  uint32_t u = __float_as_uint(f);
-  if (u == 0x80000000u) u = 0u;                         // -0 ranks as +0
-  const uint32_t k = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-  return k <= 0x007FFFFFu ? 0u : k;                     // -inf: not a candidate
-}
 
 struct Plan {
   bool valid;

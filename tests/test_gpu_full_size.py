@@ -59,6 +59,29 @@ def test_flat_decode_128k_full_size():
     assert_attention_close(O.bf16_to_f64(host(out)), o_ref)
 
 
+def test_flat_decode_1m_full_size_fused_selection():
+    # 2 x 1M: the indexer writes the selection's group maxima beside the scores
+    # (fused scoring + selection); its index rows must equal the oracle's, and
+    # bit for bit the selection over the same scores without the fused summaries
+    w = I.WORKLOADS["flat_decode_1m"]
+    x = I.make_indexer_inputs(w, 1)
+    budget = budget_of(w)
+    q, k, ww, sl = dev(x["q_idx"], "bf16"), dev(x["k_idx"], "bf16"), dev(x["w"], "f32"), dev(x["seq_len"], "i32")
+    scores = torch.empty((w.B, 1, w.L), dtype=torch.float32, device="cuda")
+    gi = host(L.lsa_index_flat(q, ww, k, sl, budget, scores_out=scores))   # scores out: the selection reads them
+    idx_ws = L.lsa_index_flat(q, ww, k, sl, budget)                          # scores in the workspace
+    sel = L.lsa_select_streaming(scores, sl, budget)
+    torch.cuda.synchronize()
+    L.lsa_device_status()
+    assert np.array_equal(gi, host(idx_ws))
+    assert np.array_equal(gi, host(sel))
+    rows = [(b, 0) for b in range(w.B)]
+    os_ = O.indexer_scores_rows(x["q_idx"], x["w"], x["k_idx"], x["seq_len"], rows)
+    for b in range(w.B):
+        check_index_row(gi[b, 0], O.select_streaming_row(os_[b], w.L - 1, *budget), os_[b], w.L - 1, w.sink,
+                        w.window)
+
+
 @pytest.mark.parametrize("fp8", [False, True])
 def test_prefill_64k_full_size_strided_rows(fp8):
     w = I.WORKLOADS["prefill_64k"]

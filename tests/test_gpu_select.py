@@ -80,3 +80,43 @@ def test_select_long_rows_all_launch_paths(B, L_max, ties):
     got = run_select(sc, sl, 1, (2048, 64, 960))
     ref = O.select_streaming(sc, sl, 1, 2048, 64, 960)
     assert np.array_equal(got, ref)
+
+
+def _filter_rows(B, L_max, seq_len, kind, seed):
+    rng = np.random.default_rng(seed)
+    if kind == "all_equal":                    # every candidate ties: the lowest slots win
+        sc = np.full((B, 1, L_max), 2.5, np.float32)
+    elif kind == "tie_block":                  # a block of exact ties straddles the threshold
+        sc = (np.abs(rng.standard_normal((B, 1, L_max))) + 3.0).astype(np.float32)
+        sc[:, :, rng.integers(0, L_max, size=3000)] = np.float32(5.25)
+    elif kind == "holes":                      # -inf holes (not candidates) and -0
+        sc = rng.standard_normal((B, 1, L_max)).astype(np.float32)
+        sc[rng.random(sc.shape) < 0.3] = -np.inf
+        sc[rng.random(sc.shape) < 0.01] = -0.0
+    else:                                      # plain normal scores
+        sc = rng.standard_normal((B, 1, L_max)).astype(np.float32)
+    for b in range(B):
+        sc[b, 0, seq_len[b]:] = -np.inf
+    return sc
+
+
+@pytest.mark.parametrize("kind", ["normal", "all_equal", "tie_block", "holes"])
+def test_select_filter_launch_bit_exact(kind):
+    # rows longer than a cluster holds and than the grid launch takes: the filter
+    # launch (group-maximum bound, per-warp kept runs, last-CTA finish)
+    B, L_max = 2, 1 << 20
+    sl = np.array([L_max, 700001], np.int32)
+    assert L.workspace_size(L.LSA_OP_SELECT, budget=(2048, 64, 960), B=B, T=1, L_max=L_max) > 0
+    sc = _filter_rows(B, L_max, sl, kind, 7)
+    for budget in [(2048, 64, 960), (300, 0, 0), (4096, 16, 16)]:
+        got = run_select(sc, sl, 1, budget)
+        assert np.array_equal(got, O.select_streaming(sc, sl, 1, *budget)), (kind, budget)
+
+
+def test_select_filter_launch_short_and_empty_rows():
+    B, L_max = 4, 600000
+    sl = np.array([600000, 3000, 0, 599999], np.int32)   # a row shorter than the budget and an empty one
+    sc = _filter_rows(B, L_max, sl, "normal", 8)
+    got = run_select(sc, sl, 1, (2048, 64, 960))
+    assert np.array_equal(got, O.select_streaming(sc, sl, 1, 2048, 64, 960))
+    assert (got[2] == -1).all()
