@@ -111,7 +111,7 @@ struct SelectPlan {
   bool final_in_smem;
   bool grid;              // grid-cooperative launch (rows * C CTAs co-resident)
   bool cluster;           // one thread-block cluster of C CTAs per row (no workspace)
-  int cluster_rc;         // cluster path: keys per thread (32 or 64)
+  int cluster_rc;         // cluster path: keys per thread (4, 8, 16, 32 or 64)
   bool filter;            // filter path: group-maximum bound, C CTAs per row, last CTA finishes
   int g0_shift, fold, gmax_stride, pool_cap;
 };

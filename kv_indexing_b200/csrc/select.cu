@@ -1219,10 +1219,10 @@ constexpr size_t cluster_smem_words(int RC) {
 }
 static_assert(kClusterMax * kListCapC <= kSubHist * kWHStride, "list copies fit the sub-histogram space");
 
-// RC keys per thread: 32 (16384 slots per CTA) or 64 (32768).
+// RC keys per thread: 4, 8, 16, 32 or 64 (2048 .. 32768 slots per CTA).
 template <int RC>
 __global__ void __launch_bounds__(kThreads, 1) select_cluster_kernel(const SelectArgs a) {
-  static_assert(RC == 32 || RC == 64, "keys per thread");
+  static_assert(RC == 4 || RC == 8 || RC == 16 || RC == 32 || RC == 64, "keys per thread");
   pdl_wait();
   pdl_trigger();
   const int C = static_cast<int>(gridDim.x);
@@ -1259,14 +1259,15 @@ __global__ void __launch_bounds__(kThreads, 1) select_cluster_kernel(const Selec
 
   // ---- (1) keys (coalesced fill), local max and count; broadcast
   uint32_t nz = 0u, mx = 0u;
+  constexpr int kBatch = RC < 32 ? RC : 32;   // loads in flight per thread at a time
 #pragma unroll 1
-  for (int h = 0; h < RC / 32; ++h) {   // 32 loads in flight per thread at a time
-    const int e0 = warp * 32 * RC + lane + 1024 * h;
-    float f[32];
+  for (int h = 0; h < RC / kBatch; ++h) {
+    const int e0 = warp * 32 * RC + lane + 32 * kBatch * h;
+    float f[kBatch];
 #pragma unroll
-    for (int j = 0; j < 32; ++j) f[j] = e0 + 32 * j < my_n ? __ldg(row + e0 + 32 * j) : -INFINITY;
+    for (int j = 0; j < kBatch; ++j) f[j] = e0 + 32 * j < my_n ? __ldg(row + e0 + 32 * j) : -INFINITY;
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
+    for (int j = 0; j < kBatch; ++j) {
       const uint32_t k = score_key(f[j]);
       const int e = e0 + 32 * j;
       keys[e + 4 * (e / RC)] = k;
@@ -1940,11 +1941,15 @@ SelectPlan select_plan(int rows, int n_slots, int d_bound, int num_sms) {
   constexpr int kSegMax = 32768;            // fallback: keys per CTA in shared memory
   SelectPlan p{};
   auto seg_of = [&](int C) { return (n_slots + C - 1) / C; };
-  // cluster path: one cluster of up to 8 CTAs per row, any number of rows;
-  // 32 keys per thread up to 131072 slots, 64 up to 262144
-  for (const int rc : {32, 64}) {
+  // cluster path: one cluster of up to 8 CTAs per row, any number of rows. The
+  // cost of a CTA's passes grows with its keys per thread (each pass is
+  // instruction-bound on one SM), so few rows spread over more CTAs with fewer
+  // keys each (down to 4 per thread); many rows keep 32 (up to 131072 slots)
+  // or 64 (up to 262144) to bound the CTA count
+  for (const int rc : {4, 8, 16, 32, 64}) {
     const int cta_keys = kThreads * rc;
-    if (n_slots <= kClusterMax * cta_keys) {
+    const int C = (n_slots + cta_keys - 1) / cta_keys;
+    if (n_slots <= kClusterMax * cta_keys && (rows * C <= num_sms || rc >= 32)) {
       p.cluster = true;
       p.cluster_rc = rc;
       p.C = std::max(1, (n_slots + cta_keys - 1) / cta_keys);
@@ -2064,8 +2069,11 @@ cudaError_t launch_select(const SelectArgs& a0, const SelectPlan& p, void* ws, c
   }
   if (p.cluster) {
     const size_t smem = cluster_smem_words(p.cluster_rc) * 4;
-    const void* fn = p.cluster_rc == 64 ? reinterpret_cast<const void*>(&select_cluster_kernel<64>)
-                                        : reinterpret_cast<const void*>(&select_cluster_kernel<32>);
+    const void* fn = p.cluster_rc == 64   ? reinterpret_cast<const void*>(&select_cluster_kernel<64>)
+                     : p.cluster_rc == 32 ? reinterpret_cast<const void*>(&select_cluster_kernel<32>)
+                     : p.cluster_rc == 16 ? reinterpret_cast<const void*>(&select_cluster_kernel<16>)
+                     : p.cluster_rc == 8  ? reinterpret_cast<const void*>(&select_cluster_kernel<8>)
+                                          : reinterpret_cast<const void*>(&select_cluster_kernel<4>);
     cudaError_t e = set_max_smem(fn, smem);
     if (e != cudaSuccess) return e;
     cudaLaunchAttribute attr[1];

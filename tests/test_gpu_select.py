@@ -120,3 +120,18 @@ def test_select_filter_launch_short_and_empty_rows():
     got = run_select(sc, sl, 1, (2048, 64, 960))
     assert np.array_equal(got, O.select_streaming(sc, sl, 1, 2048, 64, 960))
     assert (got[2] == -1).all()
+
+
+@pytest.mark.parametrize("L_max", [16384, 30000, 65536, 100000])
+def test_select_cluster_keys_per_thread_variants_bit_exact(L_max):
+    # two rows: the cluster of up to 8 CTAs per row holds 4, 8, 16 or 32 keys per
+    # thread depending on the row length (the hierarchical selections' shapes)
+    rng = np.random.default_rng(L_max)
+    B = 2
+    sl = np.array([L_max, L_max * 3 // 4], np.int32)
+    sc = (rng.integers(0, 50, size=(B, 1, L_max)) * 0.125).astype(np.float32)   # many ties
+    for b in range(B):
+        sc[b, 0, sl[b]:] = -np.inf
+    for budget in [(2048, 64, 960), (256, 0, 0), (1024, 8, 100)]:
+        got = run_select(sc, sl, 1, budget)
+        assert np.array_equal(got, O.select_streaming(sc, sl, 1, *budget)), budget
