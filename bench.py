@@ -78,8 +78,11 @@ def indexer_bytes_per_query(w, fp8=False, n_keys=None) -> int:
     return n * w.d * 2 + w.H * w.d * 2 + w.H * 4
 
 
-def hier_index_bytes_per_query(w) -> int:
-    """Page keys of the whole sequence + the recalled pages' token keys + q, w."""
+def hier_index_bytes_per_query(w, fp8=False) -> int:
+    """Page keys of the whole sequence + the recalled pages' token keys + q, w
+    (e4m3: one byte per element plus a 4-byte scale per page, token and query head)."""
+    if fp8:
+        return ((w.L // w.P) * (w.d + 4) + w.M * w.P * (w.d + 4) + w.H * (w.d + 4) + w.H * 4)
     return (w.L // w.P) * w.d * 2 + w.M * w.P * w.d * 2 + w.H * w.d * 2 + w.H * 4
 
 
@@ -214,10 +217,13 @@ def kind_of(w) -> str:
     return "prefill" if w.T > 1 else "flat"
 
 
-def host_inputs(w, seed):
+def host_inputs(w, seed, fp8=False):
     """Indexer inputs from the seeded host generator (needles included); for
-    compressed entries the entry keys take the place of the token keys."""
+    compressed entries the entry keys take the place of the token keys. With
+    fp8, e4m3 codes and row scales are drawn too."""
     from kv_indexing_b200 import inputs as I
+    if fp8 and not w.fp8:
+        w = I.scaled(w, fp8=True)
     if w.m:
         x = I.make_compressed_inputs(w, seed)
         x["k_idx"] = x.pop("entry_keys")
@@ -330,14 +336,19 @@ class Path:
                 self.roof_bytes = indexer_bytes_per_query(w, self.fp8, n_keys) * B * T
         elif kind == "hier":
             self._pool_once()
-            ii = L.indexer_in(q, wt, k, sl)
+            ii = L.indexer_in(q, wt, k, sl, qs, ks)
             self.api_ws = self._ws(L.workspace_size(L.LSA_OP_INDEX_HIER, indexer=ii, budget=budget, P=w.P, M=w.M))
-            self.stages = [("hier_index", lambda s: L.lsa_index_hier(q, wt, k, sl, self.page_keys, w.P, w.M, budget,
-                                                                     idx=self.idx, workspace=self.api_ws, stream=s)),
-                           ("attention", attn(0))]
+            if self.fp8:
+                hier_call = lambda s: L.lsa_index_hier_e4m3(q, qs, wt, k, ks, sl, self.page_keys, self.page_scales,
+                                                            w.P, w.M, budget, idx=self.idx, workspace=self.api_ws,
+                                                            stream=s)
+            else:
+                hier_call = lambda s: L.lsa_index_hier(q, wt, k, sl, self.page_keys, w.P, w.M, budget, idx=self.idx,
+                                                       workspace=self.api_ws, stream=s)
+            self.stages = [("hier_index", hier_call), ("attention", attn(0))]
             self.dominant = "hier_index"
             self.roof_kernel = "hierarchical indexing call (page scores, page recall, fine scores, token top-k)"
-            self.roof_bytes = hier_index_bytes_per_query(w) * B * T
+            self.roof_bytes = hier_index_bytes_per_query(w, self.fp8) * B * T
         else:   # group
             if w.P:
                 self._pool_once()
@@ -369,10 +380,19 @@ class Path:
         torch, L, w = self.torch, self.L, self.w
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        self.page_keys = torch.zeros((w.B, w.L // w.P, w.d), dtype=torch.bfloat16, device=self.dev)
-        e0.record()
-        L.lsa_pool_pages(self.k, self.sl, w.P, page_keys=self.page_keys)
-        e1.record()
+        if self.fp8:
+            self.page_keys = torch.zeros((w.B, w.L // w.P, w.d), dtype=torch.uint8,
+                                         device=self.dev).view(torch.float8_e4m3fn)
+            self.page_scales = torch.ones((w.B, w.L // w.P), dtype=torch.float32, device=self.dev)
+            e0.record()
+            L.lsa_pool_pages_e4m3(self.k, self.ks, self.sl, w.P, page_codes=self.page_keys,
+                                  page_scales=self.page_scales)
+            e1.record()
+        else:
+            self.page_keys = torch.zeros((w.B, w.L // w.P, w.d), dtype=torch.bfloat16, device=self.dev)
+            e0.record()
+            L.lsa_pool_pages(self.k, self.sl, w.P, page_keys=self.page_keys)
+            e1.record()
         torch.cuda.synchronize()
         self.extra["page_pooling_once_us"] = 1000 * e0.elapsed_time(e1)
 
@@ -388,7 +408,10 @@ class Path:
                               page_keys=self.page_keys if w.P else None, outs=self.outs, idx=self.idx,
                               workspace=self.api_ws, stream=s)
             return
-        if self.kind == "hier":
+        if self.kind == "hier" and self.fp8:
+            L.lsa_index_hier_e4m3(q, qs, wt, k, ks, sl, self.page_keys, self.page_scales, w.P, w.M, budget,
+                                  idx=self.idx, workspace=self.api_ws, stream=s)
+        elif self.kind == "hier":
             L.lsa_index_hier(q, wt, k, sl, self.page_keys, w.P, w.M, budget, idx=self.idx, workspace=self.api_ws,
                              stream=s)
         elif self.kind == "compressed":
@@ -625,7 +648,9 @@ class OraclePath:
         import oracle as O
         self.O, self.w, self.x, self.layers, self.fp8 = O, w, x, layers_host, fp8
         self.kind = kind_of(w)
-        if w.P:
+        if w.P and fp8:
+            self.pk, self.ps = O.pool_pages_e4m3(x["k_idx_fp8"], x["k_scale"], x["seq_len"], w.P)
+        elif w.P:
             self.pk = O.pool_pages(x["k_idx"], x["seq_len"], w.P)
 
     def run(self, rows):
@@ -640,6 +665,9 @@ class OraclePath:
         if self.kind == "compressed":
             idx, _ = O.index_compressed(q, x["w"], k, x["seq_len"], m=w.m, budget=w.k, sink=w.sink,
                                         window=w.window, **kw)
+        elif w.P and self.fp8:
+            idx, _ = O.index_hier_e4m3(q, x["q_scale"], x["w"], k, x["k_scale"], self.pk, self.ps, x["seq_len"], P=w.P,
+                                       M=w.M, budget=w.k, sink=w.sink, window=w.window, rows=rows)
         elif w.P:
             idx, _ = O.index_hier(q, x["w"], k, self.pk, x["seq_len"], P=w.P, M=w.M, budget=w.k, sink=w.sink,
                                   window=w.window, rows=rows)
@@ -696,7 +724,7 @@ def run_reference(args, rank: int, world: int):
     import oracle as O
     from kv_indexing_b200 import inputs as I
     w = I.WORKLOADS[args.workload if args.workload in I.WORKLOADS else "flat_decode_128k"]
-    x = host_inputs(w, args.seed)
+    x = host_inputs(w, args.seed, args.fp8)
     kv_w = I.entry_workload(w) if w.m else w
     layers = [I.make_attn_inputs(kv_w, args.seed, layer=li) for li in range(w.n_layers)]
     op = OraclePath(w, x, layers, fp8=args.fp8)
@@ -788,7 +816,7 @@ def step_bytes(path) -> float:
     if path.kind == "prefill":
         return None
     if path.kind == "hier":
-        ib = hier_index_bytes_per_query(w)
+        ib = hier_index_bytes_per_query(w, path.fp8)
     elif path.kind == "group":
         return path.roof_bytes
     else:
@@ -802,7 +830,7 @@ def run_workload(args, w, rank, world, dev, pg):
     from kv_indexing_b200 import lsa as L
 
     seed = rank_seed(args.seed, rank)
-    x = host_inputs(w, seed)
+    x = host_inputs(w, seed, args.fp8)
     path = Path(torch, L, w, x, dev, seed, args.fp8)
     flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 

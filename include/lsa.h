@@ -240,12 +240,38 @@ lsa_status_t lsa_pool_pages(const void* k, const int32_t* seq_len, int32_t B, in
  * tokens are forced in; the rest are the top full, fully visible pages of the
  * dynamic region by page score, ties to the lower page), then fine token
  * scores inside the recalled pages and the streaming selection restricted to
- * them. bf16 only. Requires M >= ceil(sink/P) + ceil(window/P) + 1.
+ * them. bf16 inputs (e4m3: lsa_index_hier_e4m3). Requires
+ * M >= ceil(sink/P) + ceil(window/P) + 1.
  *   idx       [B,T,k] int32 out (layout as lsa_index_flat)
  *   pages_out [B,T,M] int32 out, optional: recalled pages ascending, -1 padded. */
 lsa_status_t lsa_index_hier(const lsa_indexer_in_t* in, const void* page_keys, int32_t P,
                             int32_t M, lsa_budget_t budget, int32_t* idx, int32_t* pages_out,
                             void* workspace, size_t workspace_bytes, lsa_stream_t stream);
+
+/* FP8 page pooling for Hierarchical Indexing [LSA abstract (3); DSA "Quantized
+ * computation"]: page keys of e4m3 token keys, themselves in e4m3 with one fp32
+ * scale per page. For every full page (pP + P <= seq_len[b]):
+ *   mean[i]  = (sum_{j<P} fp32(code(k8[b,pP+j,i]) * k_scale[b,pP+j])) / P
+ *              (fp32 products and sum, ascending j, one division)
+ *   scale    = max_i |mean[i]| / 448 (fp32), or 1 for an all-zero page
+ *   code[i]  = e4m3(mean[i] / scale), round to nearest even, saturating to 448
+ * page_codes [B,L_max/P,d] e4m3 codes; page_scales [B,L_max/P] fp32; rows of
+ * pages that are not full are left untouched. d = 128; P in {16,32,64,128};
+ * L_max % P == 0. Called when pages fill, not per query. */
+lsa_status_t lsa_pool_pages_e4m3(const void* k8, const float* k_scale, const int32_t* seq_len, int32_t B,
+                                 int32_t L_max, int32_t d, int32_t P, void* page_codes, float* page_scales,
+                                 lsa_stream_t stream);
+
+/* FP8 hierarchical indexing [LSA abstract (3); DSA "Quantized computation"]:
+ * lsa_index_hier on e4m3 inputs (in->dtype == LSA_E4M3: q codes with q_scale,
+ * token key codes with k_scale) and e4m3 page keys with their page scales as
+ * lsa_pool_pages_e4m3 writes them. Page scores and fine scores are the
+ * indexer's formula on the dequantized values (code times scale); recall and
+ * selection as lsa_index_hier. Workspace: lsa_workspace_size with
+ * LSA_OP_INDEX_HIER and the same descriptor. Requires d = 128. */
+lsa_status_t lsa_index_hier_e4m3(const lsa_indexer_in_t* in, const void* page_codes, const float* page_scales,
+                                 int32_t P, int32_t M, lsa_budget_t budget, int32_t* idx, int32_t* pages_out,
+                                 void* workspace, size_t workspace_bytes, lsa_stream_t stream);
 
 /* Sparse MQA/MLA attention over an index set [DSA "Sparse Attention
  * Calculator"]: idx [B,T,k] int32 (entries < 0 are skipped; entries must be

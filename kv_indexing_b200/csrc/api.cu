@@ -351,8 +351,11 @@ FusedSummary fused_summary(int rows, int n_slots, lsa_budget_t bu, void* sws) {
   return fs;
 }
 
+// Hierarchical indexing; e4m3 inputs (in->dtype) come with page_scales, the
+// per-page fp32 scales of the e4m3 page codes.
 lsa_status_t run_hier(const lsa_indexer_in_t* in, const void* page_keys, int P, int M, lsa_budget_t bu,
-                      int* idx, int* pages_out, void* ws, cudaStream_t st) {
+                      int* idx, int* pages_out, void* ws, cudaStream_t st, const float* page_scales = nullptr) {
+  const bool fp8 = in->dtype == LSA_E4M3;
   const size_t rows = static_cast<size_t>(in->B) * in->T;
   const int n_pages = in->L_max / P;
   uint8_t* w = static_cast<uint8_t*>(ws);
@@ -370,7 +373,9 @@ lsa_status_t run_hier(const lsa_indexer_in_t* in, const void* page_keys, int P, 
   // 1) coarse scores over full, fully visible pages
   int p_shift = 0;
   while ((1 << p_shift) < P) ++p_shift;
-  lsa_status_t s = run_flat_scores(in, page_keys, n_pages, p_shift, page_scores, st);
+  lsa_indexer_in_t pin = *in;   // the page keys (and, for e4m3, their scales) take the keys' place
+  pin.k_scale = page_scales;
+  lsa_status_t s = run_flat_scores(&pin, page_keys, n_pages, p_shift, page_scores, st);
   if (s != LSA_OK) return s;
   // 2) recall: forced sink/window pages + top pages of the dynamic region (ascending)
   s = run_select(kSelectPages, in->B, in->T, in->L_max, in->seq_len, page_scores, n_pages, n_pages, bu, P, M,
@@ -379,10 +384,11 @@ lsa_status_t run_hier(const lsa_indexer_in_t* in, const void* page_keys, int P, 
   // 3) fine scores over the recalled pages' tokens
   {
     CUtensorMap tm_k, tm_q;
-    s = make_tmap(&tm_k, in->k, false, in->d, static_cast<uint64_t>(in->B) * in->L_max, 64, P);
+    const uint32_t box_inner = fp8 ? 128 : 64;   // one 128-byte swizzle span per box row
+    s = make_tmap(&tm_k, in->k, fp8, in->d, static_cast<uint64_t>(in->B) * in->L_max, box_inner, P);
     if (s != LSA_OK) return s;
     const int N = in->H < 16 ? 16 : in->H;
-    s = make_tmap(&tm_q, in->q, false, in->d, static_cast<uint64_t>(in->B) * in->T * in->H, 64, N);
+    s = make_tmap(&tm_q, in->q, fp8, in->d, static_cast<uint64_t>(in->B) * in->T * in->H, box_inner, N);
     if (s != LSA_OK) return s;
     IndexerArgs a{};
     a.B = in->B; a.T = in->T; a.H = in->H; a.d = in->d;
@@ -390,16 +396,16 @@ lsa_status_t run_hier(const lsa_indexer_in_t* in, const void* page_keys, int P, 
     a.NQ = 1; a.N = N; a.G = in->T;
     a.n_tiles = (M * P + 127) / 128;
     a.vis_shift = 0; a.gather = 1;
-    indexer_pick_pipeline(in->d, false, N, &a.stages, &a.nbuf_b);
+    indexer_pick_pipeline(in->d, fp8, N, &a.stages, &a.nbuf_b);
     a.n_acc = indexer_n_acc(N);
     a.n_items = static_cast<long long>(rows) * a.n_tiles;
-    a.seq_len = in->seq_len; a.w = in->w;
+    a.seq_len = in->seq_len; a.w = in->w; a.q_scale = in->q_scale; a.k_scale = in->k_scale;
     a.out = cand; a.out_row_stride = static_cast<long long>(M) * P;
     a.inv_sqrt_d = 1.0f / std::sqrt(static_cast<float>(in->d));
     a.pages = pages; a.M = M; a.P = P; a.sink = bu.sink; a.window = bu.window;
     a.status = device_status_ptr();
     const int grid = static_cast<int>(std::min<long long>(a.n_items, device_sm_count()));
-    LSA_CHECK_CUDA(launch_indexer(tm_k, tm_q, a, false, grid, st), "fine indexer launch");
+    LSA_CHECK_CUDA(launch_indexer(tm_k, tm_q, a, fp8, grid, st), "fine indexer launch");
   }
   // 4) token selection restricted to the recalled pages
   return run_select(kSelectHierTokens, in->B, in->T, in->L_max, in->seq_len, cand, static_cast<long long>(M) * P,
@@ -472,7 +478,6 @@ lsa_status_t check_entry_size(const lsa_indexer_in_t* in, int m) {
 }
 
 lsa_status_t check_hier_params(const lsa_indexer_in_t* in, int P, int M, lsa_budget_t bu) {
-  if (in->dtype != LSA_BF16) return fail(LSA_ERR_UNSUPPORTED, "hierarchical indexing takes bf16 inputs");
   if (!is_pow2_in(P, 16, 128)) return fail(LSA_ERR_UNSUPPORTED, "page size P=%d not in {16,32,64,128}", P);
   if (in->L_max % P) return fail(LSA_ERR_INVALID_ARG, "L_max must be a multiple of P");
   const int forced_max = (bu.sink + P - 1) / P + (bu.window + P - 1) / P + 1;
@@ -625,7 +630,7 @@ lsa_status_t lsa_workspace_size(lsa_op_t op, const lsa_op_args_t* args, size_t* 
       *bytes = compressed_ws_bytes(args->indexer, args->m, args->budget, args->scores_external != 0);
       return LSA_OK;
     case LSA_OP_INDEX_HIER:
-      if ((s = check_indexer(args->indexer, false)) != LSA_OK) return s;
+      if ((s = check_indexer(args->indexer, true)) != LSA_OK) return s;
       if ((s = check_hier_params(args->indexer, args->P, args->M, args->budget)) != LSA_OK) return s;
       if ((s = check_budget(args->budget)) != LSA_OK) return s;
       *bytes = hier_ws_bytes(args->indexer, args->P, args->M, args->budget, false);
@@ -758,6 +763,8 @@ lsa_status_t lsa_index_hier(const lsa_indexer_in_t* in, const void* page_keys, i
                             lsa_budget_t budget, int32_t* idx, int32_t* pages_out, void* workspace,
                             size_t workspace_bytes, lsa_stream_t stream) {
   lsa_status_t s;
+  if (in && in->dtype == LSA_E4M3)
+    return fail(LSA_ERR_UNSUPPORTED, "e4m3 inputs: use lsa_index_hier_e4m3 (page keys come with page scales)");
   if ((s = check_indexer(in, false)) != LSA_OK) return s;
   if ((s = check_budget(budget)) != LSA_OK) return s;
   if ((s = check_hier_params(in, P, M, budget)) != LSA_OK) return s;
@@ -768,6 +775,41 @@ lsa_status_t lsa_index_hier(const lsa_indexer_in_t* in, const void* page_keys, i
   const size_t need = hier_ws_bytes(in, P, M, budget, pages_out != nullptr);
   if ((s = check_ws(workspace, workspace_bytes, need)) != LSA_OK) return s;
   return run_hier(in, page_keys, P, M, budget, idx, pages_out, workspace, reinterpret_cast<cudaStream_t>(stream));
+}
+
+lsa_status_t lsa_pool_pages_e4m3(const void* k8, const float* k_scale, const int32_t* seq_len, int32_t B,
+                                 int32_t L_max, int32_t d, int32_t P, void* page_codes, float* page_scales,
+                                 lsa_stream_t stream) {
+  if (!k8 || !k_scale || !seq_len || !page_codes || !page_scales) return fail(LSA_ERR_INVALID_ARG, "null tensor");
+  if (!aligned16(k8) || !aligned16(page_codes) || !aligned16(k_scale) || !aligned16(page_scales))
+    return fail(LSA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  if (B < 1 || L_max < 1) return fail(LSA_ERR_INVALID_ARG, "B and L_max must be >= 1");
+  if (d != 128) return fail(LSA_ERR_UNSUPPORTED, "e4m3 page pooling requires d = 128");
+  if (!is_pow2_in(P, 16, 128)) return fail(LSA_ERR_UNSUPPORTED, "page size P=%d not in {16,32,64,128}", P);
+  if (L_max % P) return fail(LSA_ERR_INVALID_ARG, "L_max must be a multiple of P");
+  LSA_CHECK_CUDA(launch_pool_e4m3(static_cast<const uint8_t*>(k8), k_scale, seq_len, B, L_max, d, P,
+                                  static_cast<uint8_t*>(page_codes), page_scales,
+                                  reinterpret_cast<cudaStream_t>(stream)),
+                 "e4m3 pool launch");
+  return LSA_OK;
+}
+
+lsa_status_t lsa_index_hier_e4m3(const lsa_indexer_in_t* in, const void* page_codes, const float* page_scales,
+                                 int32_t P, int32_t M, lsa_budget_t budget, int32_t* idx, int32_t* pages_out,
+                                 void* workspace, size_t workspace_bytes, lsa_stream_t stream) {
+  lsa_status_t s;
+  if ((s = check_indexer(in, true)) != LSA_OK) return s;
+  if (in->dtype != LSA_E4M3) return fail(LSA_ERR_INVALID_ARG, "lsa_index_hier_e4m3 takes e4m3 inputs");
+  if ((s = check_budget(budget)) != LSA_OK) return s;
+  if ((s = check_hier_params(in, P, M, budget)) != LSA_OK) return s;
+  if (!page_codes || !page_scales || !idx) return fail(LSA_ERR_INVALID_ARG, "null page codes, page scales or idx");
+  if (!aligned16(page_codes) || !aligned16(page_scales) || !aligned16(idx) || (pages_out && !aligned16(pages_out)))
+    return fail(LSA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  if (static_cast<long long>(in->B) * in->T > 65535) return fail(LSA_ERR_UNSUPPORTED, "at most 65535 query rows per call");
+  const size_t need = hier_ws_bytes(in, P, M, budget, pages_out != nullptr);
+  if ((s = check_ws(workspace, workspace_bytes, need)) != LSA_OK) return s;
+  return run_hier(in, page_codes, P, M, budget, idx, pages_out, workspace, reinterpret_cast<cudaStream_t>(stream),
+                  page_scales);
 }
 
 lsa_status_t lsa_sparse_attn(const lsa_attn_in_t* in, const int32_t* idx, int32_t k, void* out, float* lse,

@@ -352,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(qw * 32) << 16) + static_cast<uint32_t>(acc * N);
       float kscale = 1.f;
-      if (FP8 && s < a.L_rows) kscale = __ldg(a.k_scale + static_cast<long long>(g.b) * a.L_rows + s);
+      if (FP8 && !a.gather && s < a.L_rows) kscale = __ldg(a.k_scale + static_cast<long long>(g.b) * a.L_rows + s);
       if (a.H >= 16) {
         for (int qi = 0; qi < a.NQ; ++qi) {
           float acc8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -391,7 +391,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else if (s < a.M * a.P) {
               const int page = __ldg(a.pages + (static_cast<long long>(g.b) * a.T + g.q0) * a.M + s / a.P);
               const int tok = page * a.P + (s & (a.P - 1));
-              a.out[orow + s] = (page >= 0 && tok >= sink_end && tok < w_lo) ? sc : -INFINITY;
+              // e4m3: the recalled token's own key scale
+              const float ks = (FP8 && page >= 0) ? __ldg(a.k_scale + static_cast<long long>(g.b) * a.L_max + tok) : 1.f;
+              a.out[orow + s] = (page >= 0 && tok >= sink_end && tok < w_lo) ? sc * ks : -INFINITY;
             }
           }
         }
@@ -417,7 +419,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else if (s < a.M * a.P) {
               const int page = __ldg(a.pages + (static_cast<long long>(g.b) * a.T + g.q0) * a.M + s / a.P);
               const int tok = page * a.P + (s & (a.P - 1));
-              a.out[orow + s] = (page >= 0 && tok >= sink_end && tok < w_lo) ? sc : -INFINITY;
+              // e4m3: the recalled token's own key scale
+              const float ks = (FP8 && page >= 0) ? __ldg(a.k_scale + static_cast<long long>(g.b) * a.L_max + tok) : 1.f;
+              a.out[orow + s] = (page >= 0 && tok >= sink_end && tok < w_lo) ? sc * ks : -INFINITY;
             }
           }
         }

@@ -135,6 +135,9 @@ cudaError_t launch_select(const SelectArgs& a, const SelectPlan& p, void* ws, cu
 // ------------------------------------------------------------------ pooling --
 cudaError_t launch_pool(const uint16_t* k, const int* seq_len, int B, int L_max, int d, int P,
                         uint16_t* page_keys, cudaStream_t stream);
+// d must be 128 (one warp of four columns per page).
+cudaError_t launch_pool_e4m3(const uint8_t* k8, const float* k_scale, const int* seq_len, int B, int L_max, int d,
+                             int P, uint8_t* page_codes, float* page_scales, cudaStream_t stream);
 
 // ---------------------------------------------------------- sparse attention --
 struct AttnArgs {

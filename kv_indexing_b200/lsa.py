@@ -24,7 +24,7 @@ LSA_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024   # static scratch of lsa_select_st
 EXPORTS = [
     "lsa_status_string", "lsa_last_error", "lsa_workspace_size", "lsa_index_flat", "lsa_select_streaming",
     "lsa_pool_pages", "lsa_index_hier", "lsa_sparse_attn", "lsa_layer_group", "lsa_device_status",
-    "lsa_select_streaming_noalloc", "lsa_index_compressed",
+    "lsa_select_streaming_noalloc", "lsa_index_compressed", "lsa_pool_pages_e4m3", "lsa_index_hier_e4m3",
 ]
 
 
@@ -88,6 +88,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.lsa_select_streaming_noalloc.argtypes = [vp, vp, i32, i32, i32, Budget, vp, vp]
     lib.lsa_pool_pages.restype = i32
     lib.lsa_pool_pages.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp]
+    lib.lsa_pool_pages_e4m3.restype = i32
+    lib.lsa_pool_pages_e4m3.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp, vp]
+    lib.lsa_index_hier_e4m3.restype = i32
+    lib.lsa_index_hier_e4m3.argtypes = [ctypes.POINTER(IndexerIn), vp, vp, i32, i32, Budget, vp, vp, vp, sz, vp]
     lib.lsa_index_hier.restype = i32
     lib.lsa_index_hier.argtypes = [ctypes.POINTER(IndexerIn), vp, i32, i32, Budget, vp, vp, vp, sz, vp]
     lib.lsa_sparse_attn.restype = i32
@@ -321,6 +325,42 @@ def lsa_index_hier(q, w, k, seq_len, page_keys, P, M, budget, *, idx=None, pages
     ws = _workspace(need, q.device, workspace)
     _check(lib.lsa_index_hier(ctypes.byref(ii), _ptr(page_keys), P, M, Budget(*budget), _ptr(idx), _ptr(pages_out),
                               _ptr(ws), _nbytes(ws), _stream(stream)))
+    return idx, pages_out
+
+
+def lsa_pool_pages_e4m3(k8, k_scale, seq_len, P, *, page_codes=None, page_scales=None, stream=None):
+    """FP8 page keys from e4m3 token keys k8 [B, L_max, 128] with k_scale [B, L_max]:
+    (page codes [B, L_max/P, 128] e4m3, page scales [B, L_max/P] fp32)."""
+    torch = _torch()
+    lib = load()
+    _need(k8, "k8", (torch.float8_e4m3fn, torch.uint8), 3)
+    _need(k_scale, "k_scale", torch.float32, 2)
+    _need(seq_len, "seq_len", torch.int32, 1)
+    B, L_max, d = k8.shape
+    if page_codes is None:
+        page_codes = torch.zeros((B, L_max // P, d), dtype=torch.uint8, device=k8.device).view(k8.dtype)
+    if page_scales is None:
+        page_scales = torch.ones((B, L_max // P), dtype=torch.float32, device=k8.device)
+    _check(lib.lsa_pool_pages_e4m3(_ptr(k8), _ptr(k_scale), _ptr(seq_len), B, L_max, d, P, _ptr(page_codes),
+                                   _ptr(page_scales), _stream(stream)))
+    return page_codes, page_scales
+
+
+def lsa_index_hier_e4m3(q8, q_scale, w, k8, k_scale, seq_len, page_codes, page_scales, P, M, budget, *, idx=None,
+                        pages_out=None, workspace=None, stream=None):
+    """FP8 hierarchical indexing. Returns (idx [B,T,k], pages [B,T,M] or None)."""
+    torch = _torch()
+    lib = load()
+    ii = indexer_in(q8, w, k8, seq_len, q_scale, k_scale)
+    _need(page_codes, "page_codes", (torch.float8_e4m3fn, torch.uint8), 3)
+    _need(page_scales, "page_scales", torch.float32, 2)
+    B, T = q8.shape[0], q8.shape[1]
+    if idx is None:
+        idx = torch.empty((B, T, budget[0]), dtype=torch.int32, device=q8.device)
+    need = workspace_size(LSA_OP_INDEX_HIER, indexer=ii, budget=budget, P=P, M=M)
+    ws = _workspace(need, q8.device, workspace)
+    _check(lib.lsa_index_hier_e4m3(ctypes.byref(ii), _ptr(page_codes), _ptr(page_scales), P, M, Budget(*budget),
+                                   _ptr(idx), _ptr(pages_out), _ptr(ws), _nbytes(ws), _stream(stream)))
     return idx, pages_out
 
 

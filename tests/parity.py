@@ -163,7 +163,7 @@ def check_row_valid_over(g, cands, scores, pos, sink, window, tol=TIE_RTOL):
         assert float(np.max(scores[rest])) <= tau + tol * abs(tau), "a better candidate was left out"
 
 
-def check_hier_rows(x, seq_len, P, M, budget, gi, gp, rows):
+def check_hier_rows(x, seq_len, P, M, budget, gi, gp, rows, fp8=False):
     """Recalled pages and index rows of the listed (b, t) against the oracle.
 
     Pages: the forced pages exactly; the others eligible and equal to the
@@ -175,11 +175,20 @@ def check_hier_rows(x, seq_len, P, M, budget, gi, gp, rows):
     sink, window = budget[1], budget[2]
     T = x["q_idx"].shape[1]
     L_max = x["k_idx"].shape[1]
-    pk_o = O.pool_pages(x["k_idx"], seq_len, P)
-    oi, op = O.index_hier(x["q_idx"], x["w"], x["k_idx"], pk_o, seq_len, P=P, M=M, budget=budget[0], sink=sink,
-                          window=window, rows=rows)
-    psc = O.indexer_scores_rows(x["q_idx"], x["w"], pk_o, seq_len, rows, vis_shift=P.bit_length() - 1, L_max=L_max)
-    tsc_all = O.indexer_scores_rows(x["q_idx"], x["w"], x["k_idx"], seq_len, rows)
+    kw = dict(P=P, M=M, budget=budget[0], sink=sink, window=window, rows=rows)
+    if fp8:   # e4m3 queries, token keys and pooled page keys, each with its scales
+        q, k, qs, ks = x["q_idx_fp8"], x["k_idx_fp8"], x["q_scale"], x["k_scale"]
+        pk_o, ps_o = O.pool_pages_e4m3(k, ks, seq_len, P)
+        oi, op = O.index_hier_e4m3(q, qs, x["w"], k, ks, pk_o, ps_o, seq_len, **kw)
+        psc = O.indexer_scores_rows(q, x["w"], pk_o, seq_len, rows, vis_shift=P.bit_length() - 1, L_max=L_max,
+                                    fp8=True, q_scale=qs, k_scale=ps_o)
+        tsc_all = O.indexer_scores_rows(q, x["w"], k, seq_len, rows, fp8=True, q_scale=qs, k_scale=ks)
+    else:
+        pk_o = O.pool_pages(x["k_idx"], seq_len, P)
+        oi, op = O.index_hier(x["q_idx"], x["w"], x["k_idx"], pk_o, seq_len, **kw)
+        psc = O.indexer_scores_rows(x["q_idx"], x["w"], pk_o, seq_len, rows, vis_shift=P.bit_length() - 1,
+                                    L_max=L_max)
+        tsc_all = O.indexer_scores_rows(x["q_idx"], x["w"], x["k_idx"], seq_len, rows)
     for i, (b, t) in enumerate(rows):
         pos = int(seq_len[b]) - T + t
         if pos < 0:

@@ -15,7 +15,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 def header_functions():
     src = open(os.path.join(ROOT, "include", "lsa.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(lsa_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(lsa_[a-z0-9_]+)\s*\(", src)))
 
 
 def test_header_declares_the_boundary():
@@ -100,6 +100,25 @@ def test_workspace_checks_and_sizes():
     sel_fine = L.workspace_size(L.LSA_OP_SELECT, budget=(2048, 64, 960), B=2, T=1, L_max=256 * 64)
     fixed = 2 * (1 << 14) * 4 + 2 * 256 * 4 + 2 * 256 * 64 * 4
     assert fixed <= hi <= fixed + max(sel_pages, sel_fine) + 256
+
+
+def test_hier_e4m3_validation():
+    lib = L.load()
+    ii = _indexer(L_max=4096)
+    ii.dtype = L.LSA_E4M3
+    ii.q_scale, ii.k_scale = 1 << 20, 2 << 20
+    bu = L.Budget(2048, 64, 960)
+    # the bf16 entry point points e4m3 callers at the e4m3 one
+    assert lib.lsa_index_hier(ctypes.byref(ii), 16, 64, 256, bu, 16, None, None, 0, None) == L.LSA_ERR_UNSUPPORTED
+    assert b"lsa_index_hier_e4m3" in lib.lsa_last_error()
+    assert lib.lsa_index_hier_e4m3(ctypes.byref(ii), 16, None, 64, 256, bu, 16, None, None, 0, None) \
+        == L.LSA_ERR_INVALID_ARG                                  # page scales missing
+    assert lib.lsa_pool_pages_e4m3(16, 16, 16, 1, 4096, 64, 64, 16, 16, None) == L.LSA_ERR_UNSUPPORTED   # d != 128
+    assert lib.lsa_pool_pages_e4m3(16, 16, 16, 1, 4096, 128, 24, 16, 16, None) == L.LSA_ERR_UNSUPPORTED  # P
+    # the workspace of the e4m3 call is the bf16 call's
+    ii_bf = _indexer(L_max=4096)
+    assert L.workspace_size(L.LSA_OP_INDEX_HIER, indexer=ii, budget=(2048, 64, 960), P=64, M=256) == \
+        L.workspace_size(L.LSA_OP_INDEX_HIER, indexer=ii_bf, budget=(2048, 64, 960), P=64, M=256)
 
 
 def test_hier_parameter_validation():
