@@ -34,8 +34,9 @@
  *     pos(t) = seq_len[b] - T + t. Values are clamped to [0, L_max]; a query with
  *     pos < 0 yields an all -1 index row.
  *   - Kernels that wait on on-chip barriers give up after a bounded number of
- *     polls, record LSA_ERR_TIMEOUT in a per-device status word and return;
- *     lsa_device_status() reads (and clears) it.
+ *     polls, record a timeout in a per-device status word and return;
+ *     lsa_device_status() reads (and clears) it. The attention records there
+ *     too any index entry it skipped for being >= L_max.
  *   - No exceptions cross the ABI.
  */
 #ifndef LSA_H_
@@ -274,8 +275,9 @@ lsa_status_t lsa_index_hier_e4m3(const lsa_indexer_in_t* in, const void* page_co
                                  void* workspace, size_t workspace_bytes, lsa_stream_t stream);
 
 /* Sparse MQA/MLA attention over an index set [DSA "Sparse Attention
- * Calculator"]: idx [B,T,k] int32 (entries < 0 are skipped; entries must be
- * < L_max -- not checked on the device). out [B,T,Hq,d_v] bf16;
+ * Calculator"]: idx [B,T,k] int32 (entries < 0 are skipped; entries >= L_max
+ * are skipped too and make the next lsa_device_status() return
+ * LSA_ERR_INVALID_ARG: the device checks every entry). out [B,T,Hq,d_v] bf16;
  * lse [B,T,Hq] fp32 optional (-inf and out = 0 when a row has no valid index). */
 lsa_status_t lsa_sparse_attn(const lsa_attn_in_t* in, const int32_t* idx, int32_t k, void* out,
                              float* lse, void* workspace, size_t workspace_bytes,
@@ -302,8 +304,9 @@ lsa_status_t lsa_layer_group(const lsa_indexer_in_t* in, const void* page_keys, 
                              size_t workspace_bytes, lsa_stream_t stream);
 
 /* Synchronises `stream`, then returns and clears the device status word of the
- * current device: LSA_OK, or LSA_ERR_TIMEOUT if a kernel gave up waiting since
- * the last call. */
+ * current device, for everything since the last call: LSA_OK; LSA_ERR_TIMEOUT
+ * if a kernel gave up waiting; LSA_ERR_INVALID_ARG if an attention index row
+ * held an entry >= L_max; LSA_ERR_CUDA if an internal bound did not hold. */
 lsa_status_t lsa_device_status(lsa_stream_t stream);
 
 #ifdef __cplusplus

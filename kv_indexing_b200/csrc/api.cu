@@ -908,7 +908,10 @@ lsa_status_t lsa_device_status(lsa_stream_t stream) {
   LSA_CHECK_CUDA(cudaMemcpyFromSymbol(&v, lsa::g_device_status, sizeof(int)), "status read");
   const int zero = 0;
   LSA_CHECK_CUDA(cudaMemcpyToSymbol(lsa::g_device_status, &zero, sizeof(int)), "status reset");
-  if (v) return fail(LSA_ERR_TIMEOUT, "a kernel gave up waiting on a barrier");
+  if (v & kStatusTimeout) return fail(LSA_ERR_TIMEOUT, "a kernel gave up waiting on a barrier");
+  if (v & kStatusInternal) return fail(LSA_ERR_CUDA, "a selection candidate pool bound did not hold");
+  if (v & kStatusBadIndex)
+    return fail(LSA_ERR_INVALID_ARG, "an attention index row held an entry >= L_max (it was skipped)");
   return LSA_OK;
 }
 

@@ -139,7 +139,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto idx_at = [&](int blk) -> int {
     const int ip = (blk0 + blk) * BN + tid;
     int id = (blk < nblk && ip < a.k) ? __ldg(idx_row + ip) : -1;
-    return id >= a.L_max ? -1 : id;
+    if (id >= a.L_max) {   // out of range: skipped, and flagged in the status word
+      record_bad_index(a.status);
+      id = -1;
+    }
+    return id;
   };
   int idx_reg = tid < BN ? idx_at(0) : -1;
   constexpr uint32_t kBlockBytes = BN * (DQK + (SEP_V ? DV : 0)) * 2;
@@ -583,7 +587,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (bb >= nblk || ip >= a.k) return -1;
       if (fixed) return ip < f_sink_end ? ip : f_wlo + (ip - f_sink_end);
       const int v = __ldg(idx_row + ip);
-      return v >= a.L_max ? -1 : v;
+      if (v >= a.L_max) {   // out of range: skipped, and flagged in the status word
+        record_bad_index(a.status);
+        return -1;
+      }
+      return v;
     };
     int ids_lo[kStages], ids_hi[kStages];   // entries lane and lane + 32 of the next kStages blocks
 #pragma unroll

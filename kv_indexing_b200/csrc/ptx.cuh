@@ -1,8 +1,8 @@
 // Inline-PTX helpers for sm_100a: mbarriers, TMA tile loads, tcgen05 (TMEM
 // allocation, UMMA issue/commit, TMEM loads/stores) and shared-memory matrix
 // descriptors. Every barrier wait here is bounded: after kWaitLimitNs of
-// polling it records LSA_ERR_TIMEOUT in the caller's status word and returns
-// false, so no kernel can spin forever.
+// polling it records a timeout in the caller's status word and returns false,
+// so no kernel can spin forever.
 #pragma once
 
 #include <cuda.h>
@@ -12,7 +12,10 @@
 namespace lsa {
 
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s
-constexpr int kStatusTimeout = 5;                            // == LSA_ERR_TIMEOUT
+// Bits of the per-device status word (lsa_device_status maps them to codes).
+constexpr int kStatusTimeout = 1;    // a kernel gave up waiting on a barrier
+constexpr int kStatusBadIndex = 2;   // an index row held an entry >= L_max (skipped)
+constexpr int kStatusInternal = 4;   // an internal capacity bound did not hold
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -27,6 +30,12 @@ __device__ __forceinline__ unsigned long long globaltimer_ns() {
 // `status` points at the per-device status word (0 = ok) owned by the C-ABI layer.
 __device__ __forceinline__ void record_timeout(int* status) {
   if (status) atomicOr(status, kStatusTimeout);
+}
+__device__ __forceinline__ void record_bad_index(int* status) {
+  if (status) atomicOr(status, kStatusBadIndex);
+}
+__device__ __forceinline__ void record_internal(int* status) {
+  if (status) atomicOr(status, kStatusInternal);
 }
 
 // ------------------------------------------------- programmatic launch --

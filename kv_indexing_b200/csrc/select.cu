@@ -1735,7 +1735,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_filter_kernel(const Select
     if (lane == 0 && kept) base = atomicAdd(a.counters + 2 * r + 1, kept);
     base = __shfl_sync(0xffffffffu, base, 0);
     if (base + kept > static_cast<uint32_t>(a.pool_cap)) {   // cannot happen (see above); never write past the pool
-      if (lane == 0) record_timeout(a.status);
+      if (lane == 0) record_internal(a.status);
       kept = 0u;
     }
     if (kept) {

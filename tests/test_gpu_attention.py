@@ -129,3 +129,36 @@ def test_attention_streaming_prefix_promise_matches_reading_idx():
     assert_attention_close(O.bf16_to_f64(host(o2)), o)
     assert np.allclose(host(lse2), ol, atol=1e-3, rtol=1e-3)
     assert np.allclose(host(lse1), host(lse2), atol=1e-3, rtol=1e-3)
+
+
+@pytest.mark.parametrize("mla", [True, False])
+def test_attention_out_of_range_index_is_skipped_and_flagged(mla):
+    # entries >= L_max are skipped by the kernel and flagged in the device status
+    # word: lsa_device_status reports LSA_ERR_INVALID_ARG once, then clears
+    if mla:
+        w = I.scaled(I.WORKLOADS["flat_decode_128k"], B=1, L=4096, T=2)
+    else:
+        w = I.scaled(I.WORKLOADS["tiny_l2k"], T=2)
+    x = I.make_attn_inputs(w, 21)
+    sl = np.array([w.L], np.int32)
+    rng = np.random.default_rng(21)
+    idx = rand_idx(rng, w.B, w.T, w.k, w.L, sl, n_valid=min(w.k, 300))
+    bad = idx.copy()
+    bad[0, 0, 5] = w.L            # first slot past the cache
+    bad[0, 1, 17] = w.L + 999
+    sl_d = dev(sl, "i32")
+    q = dev(x["qa"], "bf16")
+    L.lsa_device_status()         # start clean
+    if mla:
+        out, _ = L.lsa_sparse_attn(q, dev(bad, "i32"), sl_d, w.scale, kv=dev(x["kv"], "bf16"), d_v=w.d_v)
+    else:
+        out, _ = L.lsa_sparse_attn(q, dev(bad, "i32"), sl_d, w.scale, k=dev(x["k"], "bf16"), v=dev(x["v"], "bf16"))
+    torch.cuda.synchronize()
+    with pytest.raises(L.LsaError) as e:
+        L.lsa_device_status()
+    assert e.value.status == L.LSA_ERR_INVALID_ARG
+    assert L.lsa_device_status() == L.LSA_OK        # cleared by the read
+    skipped = bad.copy()
+    skipped[skipped >= w.L] = -1                    # what the kernel computes: the row without those entries
+    o_ref, _ = oracle_attn(w, x, skipped, sl)
+    assert_attention_close(O.bf16_to_f64(host(out)), o_ref)
