@@ -1075,7 +1075,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_grid_kernel(const SelectAr
 // CTAs take three exact radix rounds over the full key instead (the decision
 // is made from the same cluster-wide data in every CTA, so the barriers stay
 // uniform). No global workspace and no spin waits: only barriers.
-constexpr int kClusterMax = 8;
+constexpr int kClusterMax = 8;    // CTAs per row cluster (the portable maximum)
 constexpr int kListCapC = 512;                  // boundary-bin keys per CTA
 enum { kXMax = 0, kXCnt = 1, kXIn = 2, kXDef = 3, kXLen = 4, kXGt = 5, kXEq = 6, kXSlots = 7 };
 
@@ -1649,6 +1649,47 @@ __device__ __forceinline__ WarpRange warp_range(const Plan& pl, int C, int c, in
   return WarpRange{lo, min(c_hi, lo + sub)};
 }
 
+// The D-th largest of the row's n_fold group maxima (each the maximum of F
+// consecutive stored maxima), R per thread; 0 when at most D are nonzero.
+// Loads are predicated and all in flight at once.
+template <int R>
+__device__ uint32_t phase1_bound(const uint32_t* gm, int F, int n_fold, uint32_t D, Shared& sh) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t k[R];
+  const int e0 = warp * 32 * R + lane;   // element of k[j]: e0 + 32 j
+  if (F == 1) {
+#pragma unroll
+    for (int j = 0; j < R; ++j) {
+      const int e = e0 + 32 * j;
+      k[j] = e < n_fold ? __ldcg(gm + e) : 0u;
+    }
+  } else if (F == 2) {
+#pragma unroll
+    for (int j = 0; j < R; ++j) {
+      const int e = e0 + 32 * j;
+      const uint2 q = e < n_fold ? __ldcg(reinterpret_cast<const uint2*>(gm) + e) : make_uint2(0u, 0u);
+      k[j] = max(q.x, q.y);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < R; ++j) {
+      const int e = e0 + 32 * j;
+      const uint4 q = e < n_fold ? __ldcg(reinterpret_cast<const uint4*>(gm + e * F)) : make_uint4(0u, 0u, 0u, 0u);
+      k[j] = max(max(q.x, q.y), max(q.z, q.w));
+    }
+    if (F == 8) {
+#pragma unroll
+      for (int j = 0; j < R; ++j) {
+        const int e = e0 + 32 * j;
+        const uint4 q = e < n_fold ? __ldcg(reinterpret_cast<const uint4*>(gm + e * F + 4)) : make_uint4(0u, 0u, 0u, 0u);
+        k[j] = max(k[j], max(max(q.x, q.y), max(q.z, q.w)));
+      }
+    }
+  }
+  const Thr t = fast_threshold<R>(k, D, sh);
+  return t.all ? 0u : t.thr;
+}
+
 __global__ void __launch_bounds__(kThreads, 1) select_filter_kernel(const SelectArgs a) {
   pdl_wait();   // scores and group maxima come from the previous kernel(s)
   pdl_trigger();
@@ -1676,42 +1717,9 @@ __global__ void __launch_bounds__(kThreads, 1) select_filter_kernel(const Select
   uint32_t v = 0u;
   if (D > 0u) {
     const uint32_t* gm = a.gmax + static_cast<long long>(r) * a.gmax_stride;
-    const int F = a.fold;
-    const int n_fold = a.gmax_stride / F;
-    uint32_t k[kPhase1Per];
-    const int e0 = warp * 32 * kPhase1Per + lane;   // element of k[j]: e0 + 32 j
-    // predicated loads, all in flight at once (fold F in {1, 2, 4, 8})
-    if (F == 1) {
-#pragma unroll
-      for (int j = 0; j < kPhase1Per; ++j) {
-        const int e = e0 + 32 * j;
-        k[j] = e < n_fold ? __ldcg(gm + e) : 0u;
-      }
-    } else if (F == 2) {
-#pragma unroll
-      for (int j = 0; j < kPhase1Per; ++j) {
-        const int e = e0 + 32 * j;
-        const uint2 q = e < n_fold ? __ldcg(reinterpret_cast<const uint2*>(gm) + e) : make_uint2(0u, 0u);
-        k[j] = max(q.x, q.y);
-      }
-    } else {
-#pragma unroll
-      for (int j = 0; j < kPhase1Per; ++j) {
-        const int e = e0 + 32 * j;
-        const uint4 q = e < n_fold ? __ldcg(reinterpret_cast<const uint4*>(gm + e * F)) : make_uint4(0u, 0u, 0u, 0u);
-        k[j] = max(max(q.x, q.y), max(q.z, q.w));
-      }
-      if (F == 8) {
-#pragma unroll
-        for (int j = 0; j < kPhase1Per; ++j) {
-          const int e = e0 + 32 * j;
-          const uint4 q = e < n_fold ? __ldcg(reinterpret_cast<const uint4*>(gm + e * F + 4)) : make_uint4(0u, 0u, 0u, 0u);
-          k[j] = max(k[j], max(max(q.x, q.y), max(q.z, q.w)));
-        }
-      }
-    }
-    const Thr t = fast_threshold<kPhase1Per>(k, D, sh);
-    v = t.all ? 0u : t.thr;
+    const int n_fold = a.gmax_stride / a.fold;
+    v = n_fold <= kThreads * 16 ? phase1_bound<16>(gm, a.fold, n_fold, D, sh)
+                                : phase1_bound<kPhase1Per>(gm, a.fold, n_fold, D, sh);
   }
 
   // ---- phase 2: keep this warp's candidates above v (slot order), count those equal to v.
@@ -1949,7 +1957,7 @@ SelectPlan select_plan(int rows, int n_slots, int d_bound, int num_sms) {
   for (const int rc : {4, 8, 16, 32, 64}) {
     const int cta_keys = kThreads * rc;
     const int C = (n_slots + cta_keys - 1) / cta_keys;
-    if (n_slots <= kClusterMax * cta_keys && (rows * C <= num_sms || rc >= 32)) {
+    if (C <= kClusterMax && (rows * C <= num_sms || rc >= 32)) {
       p.cluster = true;
       p.cluster_rc = rc;
       p.C = std::max(1, (n_slots + cta_keys - 1) / cta_keys);
@@ -1979,7 +1987,7 @@ SelectPlan select_plan(int rows, int n_slots, int d_bound, int num_sms) {
     // groups of G slots: the bound is tight when there are many groups per
     // dynamic slot (G <= n / (8 D)); phase 1 holds at most kPhase1Cap of them
     int G = 1;
-    while (G < 64 && 16ll * G * d_bound <= n_slots) G *= 2;
+    while (G < 64 && 16ll * G * d_bound <= 2ll * n_slots) G *= 2;   // largest G <= n / (8 D)
     while (true) {
       const int g0 = std::min(G, 16);
       int sh = 0;
