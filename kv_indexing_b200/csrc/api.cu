@@ -301,6 +301,7 @@ lsa_status_t run_flat_scores(const lsa_indexer_in_t* in, const void* keys, int L
   a.L_rows = L_rows; a.L_max = in->L_max;
   a.NQ = fp.NQ; a.N = fp.N; a.G = fp.G; a.n_tiles = fp.n_tiles;
   a.vis_shift = vis_shift; a.gather = 0;
+  a.multi_group = fp.G > 1;
   indexer_pick_pipeline(in->d, fp8, fp.N, &a.stages, &a.nbuf_b);
   a.n_acc = indexer_n_acc(fp.N);
   a.n_items = static_cast<long long>(in->B) * fp.G * fp.n_tiles;

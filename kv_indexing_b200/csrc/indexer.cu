@@ -137,6 +137,16 @@ __device__ __forceinline__ void flat_group_max(const IndexerArgs& a, long long q
   if ((lane & ((1 << a.g0_shift) - 1)) == 0) a.gmax[qrow * a.gmax_stride + (s >> a.g0_shift)] = key;
 }
 
+// A FLAT score. Rows of a multi-group (prefill) launch are far larger than L2
+// and read only by a later selection, so they bypass it (streaming store);
+// decode rows stay in L2 for the selection that follows at once.
+__device__ __forceinline__ void store_score(const IndexerArgs& a, long long i, float v) {
+  if (a.multi_group)
+    __stcs(a.out + i, v);
+  else
+    a.out[i] = v;
+}
+
 __device__ __forceinline__ float sum8(const float (&a)[8]) {
   return ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
 }
@@ -203,7 +213,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_q);
-      const uint64_t pol = policy_evict_first();   // keys are streamed once
+      const uint64_t pol = policy_evict_first();   // keys read by one query group are streamed once
       long long na = 0, ng = 0, cur = -1;
       TileIter it;
       for (it.begin(a, it_begin, it_end); it.valid(); it.next(a)) {
@@ -229,9 +239,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* dst = sA + static_cast<size_t>(s) * C::kATileBytes;
         if (!a.gather) {
           const int y = it.g.b * a.L_rows + kTileM * it.j;
+          if (a.multi_group) {   // the sequence's other query groups read this tile again: normal L2 policy
 #pragma unroll
-          for (int bx = 0; bx < C::kBoxes; ++bx)
-            tma_load_2d_hint(dst + bx * kTileM * 128, &tm_k, &a_full[s], bx * C::kBoxElems, y, pol);
+            for (int bx = 0; bx < C::kBoxes; ++bx)
+              tma_load_2d(dst + bx * kTileM * 128, &tm_k, &a_full[s], bx * C::kBoxElems, y);
+          } else {
+#pragma unroll
+            for (int bx = 0; bx < C::kBoxes; ++bx)
+              tma_load_2d_hint(dst + bx * kTileM * 128, &tm_k, &a_full[s], bx * C::kBoxElems, y, pol);
+          }
         } else {
           const int per_tile = kTileM / a.P;
           const long long r = it.grp;
@@ -336,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!live) {
         if (!a.gather) {
           if (s < a.L_rows)
-            for (int qi = 0; qi < g.nq; ++qi) a.out[orow + qi * a.out_row_stride + s] = -INFINITY;
+            for (int qi = 0; qi < g.nq; ++qi) store_score(a, orow + qi * a.out_row_stride + s, -INFINITY);
           if (a.gmax && (lane & ((1 << a.g0_shift) - 1)) == 0)
             for (int qi = 0; qi < g.nq; ++qi)
               a.gmax[(static_cast<long long>(g.b) * a.T + g.q0 + qi) * a.gmax_stride + (s >> a.g0_shift)] = 0u;
@@ -386,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int pos = g.pos0 + qi;   // key s visible iff s < (pos + 1) >> vis_shift
               const int nvis = pos < 0 ? 0 : (pos + 1) >> a.vis_shift;
               const float v = s < nvis ? sc * kscale : -INFINITY;
-              if (s < a.L_rows) a.out[orow + qi * a.out_row_stride + s] = v;
+              if (s < a.L_rows) store_score(a, orow + qi * a.out_row_stride + s, v);
               if (a.gmax) flat_group_max(a, static_cast<long long>(g.b) * a.T + g.q0 + qi, s, nvis, v, lane);
             } else if (s < a.M * a.P) {
               const int page = __ldg(a.pages + (static_cast<long long>(g.b) * a.T + g.q0) * a.M + s / a.P);
@@ -414,7 +430,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int pos = g.pos0 + qi;
               const int nvis = pos < 0 ? 0 : (pos + 1) >> a.vis_shift;
               const float v = s < nvis ? sc * kscale : -INFINITY;
-              if (s < a.L_rows) a.out[orow + qi * a.out_row_stride + s] = v;
+              if (s < a.L_rows) store_score(a, orow + qi * a.out_row_stride + s, v);
               if (a.gmax) flat_group_max(a, static_cast<long long>(g.b) * a.T + g.q0 + qi, s, nvis, v, lane);
             } else if (s < a.M * a.P) {
               const int page = __ldg(a.pages + (static_cast<long long>(g.b) * a.T + g.q0) * a.M + s / a.P);

@@ -1513,25 +1513,57 @@ __global__ void __launch_bounds__(kThreads, 1) select_cluster_kernel(const Selec
 // lowest-slot candidates equal to v -- and writes the row.
 // ===========================================================================
 
-// Exact D-th best of the nonzero keys held in registers (R per thread, any
-// layout): radix rounds of 11-bit digits over key - kmin, each a 2048-bin
-// shared histogram whose target bin is found by a conflict-free warp-chunked
-// scan from the top. Same result as reg_threshold, fewer and cheaper steps.
-template <int R>
-__device__ Thr fast_threshold(const uint32_t (&k)[R], uint32_t D, Shared& sh) {
-  constexpr int kBits = 11, kBins = 1 << kBits;          // 2048 bins: 128 per warp, 4 per lane
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  uint32_t c = 0u, mn = 0xFFFFFFFFu, mx = 0u;
+// Range-radix thresholds: the exact D-th best nonzero key by rounds of 11-bit
+// digits over key - kmin, each a 2048-bin shared histogram whose target bin is
+// found by a conflict-free warp-chunked scan from the top.
+constexpr int kFastBits = 11, kFastBins = 1 << kFastBits;   // 2048 bins: 128 per warp, 4 per lane
+
+// After a round's histogram (kFastBins bins in sh.hist, counted from the top):
+// the bin holding the need-th key (sh.bin) and the keys above it (sh.above).
+// Warp w owns bins [kFastBins - 128 (w + 1), kFastBins - 128 w); lane l reads
+// four of them as one 16-byte load (conflict-free). Not inlined: every caller
+// shares one copy of the code.
+__device__ __noinline__ void pick_bin_from_top(uint32_t need, Shared& sh) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint4* h4 = reinterpret_cast<const uint4*>(sh.hist);
+  const int b0 = kFastBins - 128 * (warp + 1) + 4 * (31 - lane);   // lowest of the lane's four bins
+  const uint4 v = h4[b0 >> 2];
+  const uint32_t lsum = v.x + v.y + v.z + v.w;
+  uint32_t incl = lsum;                                  // inclusive scan from the top within the warp
 #pragma unroll
-  for (int j = 0; j < R; ++j)
-    if (k[j] != 0u) {
-      ++c;
-      mn = min(mn, k[j]);
-      mx = max(mx, k[j]);
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) sh.red[0][warp] = incl;
+  __syncthreads();
+  uint32_t before = 0u;                                  // bins above this warp's chunk
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) before += w < warp ? sh.red[0][w] : 0u;
+  const uint32_t excl = before + incl - lsum;
+  if (excl < need && need <= excl + lsum) {
+    const uint32_t cnt[4] = {v.w, v.z, v.y, v.x};       // top bin first
+    uint32_t above = excl;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (above + cnt[q] >= need) {
+        sh.bin = b0 + 3 - q;
+        sh.above = above;
+        break;
+      }
+      above += cnt[q];
     }
-  block_cnt_min_max(c, mn, mx, sh);
+  }
+  __syncthreads();
+}
+
+// The rounds of a range-radix threshold: digits of
+// rel = key - kmin from the top, kFastBits at a time. `count(prev, hi, shift,
+// dmask)` adds this round's in-play keys (rel >> prev == hi) to sh.hist.
+template <class Count>
+__device__ Thr range_rounds(uint32_t total, uint32_t kmin, uint32_t kmax, uint32_t D, Shared& sh, Count&& count) {
+  const int tid = threadIdx.x;
   Thr r{0u, 0u, false};
-  const uint32_t total = sh.cnt, kmin = sh.mn, kmax = sh.mx;
   if (total <= D) {
     r.all = true;
     return r;
@@ -1547,67 +1579,82 @@ __device__ Thr fast_threshold(const uint32_t (&k)[R], uint32_t D, Shared& sh) {
   }
   const int bits = 32 - __clz(kmax - kmin);               // every rel = key - kmin is < 2^bits
   int prev = bits;                                         // keys in play satisfy rel >> prev == hi
-  int shift = bits > kBits ? bits - kBits : 0;
+  int shift = bits > kFastBits ? bits - kFastBits : 0;
   uint32_t hi = 0u, need = D;
   uint4* h4 = reinterpret_cast<uint4*>(sh.hist);
   while (true) {
     const int width = prev - shift;                        // digit bits this round (<= 11)
     const uint32_t dmask = (1u << width) - 1u;
-    if (tid < kBins / 4) h4[tid] = make_uint4(0u, 0u, 0u, 0u);
+    if (tid < kFastBins / 4) h4[tid] = make_uint4(0u, 0u, 0u, 0u);
     __syncthreads();
-#pragma unroll
-    for (int j = 0; j < R; ++j) {
-      const uint32_t rel = k[j] - kmin;
-      const bool in = k[j] != 0u && (prev >= 32 || (rel >> prev) == hi);
-      if (in) atomicAdd(&sh.hist[(rel >> shift) & dmask], 1u);
-    }
+    count(prev, hi, shift, dmask);
     __syncthreads();
-    // warp w owns bins [kBins - 128 (w + 1), kBins - 128 w) counted from the top;
-    // lane l holds four of them as one 16-byte load (conflict-free)
-    const int b0 = kBins - 128 * (warp + 1) + 4 * (31 - lane);   // lowest of the lane's four bins
-    const uint4 v = h4[b0 >> 2];
-    const uint32_t lsum = v.x + v.y + v.z + v.w;
-    uint32_t incl = lsum;                                  // inclusive scan from the top within the warp
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    if (lane == 31) sh.red[0][warp] = incl;
-    __syncthreads();
-    uint32_t before = 0u;                                  // bins above this warp's chunk
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) before += w < warp ? sh.red[0][w] : 0u;
-    const uint32_t excl = before + incl - lsum;
-    if (excl < need && need <= excl + lsum) {
-      const uint32_t cnt[4] = {v.w, v.z, v.y, v.x};       // top bin first
-      uint32_t above = excl;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        if (above + cnt[q] >= need) {
-          sh.bin = b0 + 3 - q;
-          sh.above = above;
-          break;
-        }
-        above += cnt[q];
-      }
-    }
-    __syncthreads();
+    pick_bin_from_top(need, sh);
     hi = (width >= 32 ? 0u : (hi << width)) | static_cast<uint32_t>(sh.bin);
     need -= sh.above;
     __syncthreads();
     if (shift == 0) break;
     prev = shift;
-    shift = shift > kBits ? shift - kBits : 0;
+    shift = shift > kFastBits ? shift - kFastBits : 0;
   }
   r.thr = kmin + hi;
   r.need_eq = need;
   return r;
 }
 
-constexpr int kPhase1Per = 32;                    // group maxima per thread in phase 1
+// Exact threshold of the D-th best of key(0) .. key(n - 1) (key 0 = not a
+// candidate), read through an accessor (shared memory), by range-radix
+// rounds. Rolled loops: code that runs once per CTA pays more for instruction
+// fetch than for loop overhead.
+template <class K>
+__device__ Thr range_threshold_by(K&& key, int n, uint32_t D, Shared& sh) {
+  uint32_t c = 0u, mn = 0xFFFFFFFFu, mx = 0u;
+#pragma unroll 4
+  for (int i = threadIdx.x; i < n; i += kThreads) {
+    const uint32_t k = key(i);
+    if (k != 0u) {
+      ++c;
+      mn = min(mn, k);
+      mx = max(mx, k);
+    }
+  }
+  block_cnt_min_max(c, mn, mx, sh);
+  const uint32_t kmin = sh.mn;
+  return range_rounds(sh.cnt, kmin, sh.mx, D, sh, [&](int prev, uint32_t hi, int shift, uint32_t dmask) {
+#pragma unroll 4
+    for (int i = threadIdx.x; i < n; i += kThreads) {
+      const uint32_t k = key(i);
+      const uint32_t rel = k - kmin;
+      if (k != 0u && (prev >= 32 || (rel >> prev) == hi)) atomicAdd(&sh.hist[(rel >> shift) & dmask], 1u);
+    }
+  });
+}
+
+// The same over keys held in registers, R per thread (any layout).
+template <int R>
+__device__ Thr fast_threshold(const uint32_t (&k)[R], uint32_t D, Shared& sh) {
+  uint32_t c = 0u, mn = 0xFFFFFFFFu, mx = 0u;
+#pragma unroll
+  for (int j = 0; j < R; ++j)
+    if (k[j] != 0u) {
+      ++c;
+      mn = min(mn, k[j]);
+      mx = max(mx, k[j]);
+    }
+  block_cnt_min_max(c, mn, mx, sh);
+  const uint32_t kmin = sh.mn;
+  return range_rounds(sh.cnt, kmin, sh.mx, D, sh, [&](int prev, uint32_t hi, int shift, uint32_t dmask) {
+#pragma unroll
+    for (int j = 0; j < R; ++j) {
+      const uint32_t rel = k[j] - kmin;
+      if (k[j] != 0u && (prev >= 32 || (rel >> prev) == hi)) atomicAdd(&sh.hist[(rel >> shift) & dmask], 1u);
+    }
+  });
+}
+
 constexpr int kStageCap = 8192;                   // kept candidates staged in shared memory by the finisher
 constexpr int kWarpSlots = 1024;                  // slots per warp in phase 2 (held in registers)
+constexpr int kPhase1Per = 32;                    // folded group maxima per thread in phase 1
 constexpr int kPhase1Cap = kThreads * kPhase1Per; // 16384 per row
 
 // gmax[r][g] = max key over slots [g G0, g G0 + G0) of row r that are dynamic
@@ -1651,7 +1698,8 @@ __device__ __forceinline__ WarpRange warp_range(const Plan& pl, int C, int c, in
 
 // The D-th largest of the row's n_fold group maxima (each the maximum of F
 // consecutive stored maxima), R per thread; 0 when at most D are nonzero.
-// Loads are predicated and all in flight at once.
+// Loads are predicated and all in flight at once. Rows of maxima start on
+// 16-byte boundaries and hold a multiple of max(F, 4).
 template <int R>
 __device__ uint32_t phase1_bound(const uint32_t* gm, int F, int n_fold, uint32_t D, Shared& sh) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -1854,15 +1902,9 @@ __global__ void __launch_bounds__(kThreads, 1) select_filter_kernel(const Select
       __syncthreads();
     }
     if (G >= D && staged) {
-      // the exact D-th best is among the kept candidates: registers, warp-striped
-      // (element w 32 R + 32 j + l in k[j] of lane l, warp w: slot order is (warp, j, lane))
-      constexpr int R = kStageCap / kThreads;
-      uint32_t k[R];
-      const int e0 = warp * 32 * R + lane;
-#pragma unroll
-      for (int j = 0; j < R; ++j) k[j] = e0 + 32 * j < static_cast<int>(G) ? sk[e0 + 32 * j] : 0u;
-      const Thr t = fast_threshold<R>(k, D, sh);
-      n_sel = reg_emit<R>(k, t, sh, [&](uint32_t p, int j) { dyn_out[p] = token(ss[e0 + 32 * j]); });
+      // the exact D-th best is among the kept candidates, staged in slot order
+      const Thr t = range_threshold_by([&](int i) { return sk[i]; }, static_cast<int>(G), D, sh);
+      n_sel = cta_emit(sk, static_cast<int>(G), t, sh, [&](uint32_t p, int i) { dyn_out[p] = token(ss[i]); });
     } else if (G >= D) {
       // more kept candidates than shared memory holds (not expected for scores
       // that are not adversarial): the same from the pool in global memory
