@@ -151,6 +151,36 @@ __device__ __forceinline__ float sum8(const float (&a)[8]) {
   return ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
 }
 
+// The eight chains of relu_dot_acc held as four packed pairs (chain 2j in the
+// low half of acc2[j], 2j + 1 in the high half), advanced with the paired fp32
+// FMA: each lane is an ordinary round-to-nearest fmaf, so the chains and their
+// sum equal relu_dot_acc's bit for bit.
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+
+__device__ __forceinline__ void relu_dot_acc2(const float* wcol, const uint32_t (&v)[32], uint64_t (&acc2)[4]) {
+#pragma unroll
+  for (int i = 0; i < 32; i += 4) {
+    const float4 wv = *reinterpret_cast<const float4*>(wcol + i);
+    const uint64_t r01 = pack2(fmaxf(__uint_as_float(v[i + 0]), 0.f), fmaxf(__uint_as_float(v[i + 1]), 0.f));
+    const uint64_t r23 = pack2(fmaxf(__uint_as_float(v[i + 2]), 0.f), fmaxf(__uint_as_float(v[i + 3]), 0.f));
+    uint64_t& a01 = acc2[(i & 7) >> 1];
+    uint64_t& a23 = acc2[((i + 2) & 7) >> 1];
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(a01) : "l"(pack2(wv.x, wv.y)), "l"(r01));
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(a23) : "l"(pack2(wv.z, wv.w)), "l"(r23));
+  }
+}
+
+__device__ __forceinline__ float sum8x2(const uint64_t (&acc2)[4]) {
+  float a[8];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) asm("mov.b64 {%0, %1}, %2;" : "=f"(a[2 * j]), "=f"(a[2 * j + 1]) : "l"(acc2[j]));
+  return sum8(a);
+}
+
 template <int DK, bool FP8>
 __global__ void __launch_bounds__(kThreads, 1)
     indexer_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
@@ -213,7 +243,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_q);
-      const uint64_t pol = policy_evict_first();   // keys read by one query group are streamed once
+      const uint64_t pol = policy_evict_first();   // recalled pages' keys are read once
       long long na = 0, ng = 0, cur = -1;
       TileIter it;
       for (it.begin(a, it_begin, it_end); it.valid(); it.next(a)) {
@@ -238,16 +268,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(&a_full[s], C::kATileBytes);
         uint8_t* dst = sA + static_cast<size_t>(s) * C::kATileBytes;
         if (!a.gather) {
+          // default L2 policy: measured faster than evict-first for keys read
+          // once, and a prefill chunk's other query groups re-read them from L2
           const int y = it.g.b * a.L_rows + kTileM * it.j;
-          if (a.multi_group) {   // the sequence's other query groups read this tile again: normal L2 policy
 #pragma unroll
-            for (int bx = 0; bx < C::kBoxes; ++bx)
-              tma_load_2d(dst + bx * kTileM * 128, &tm_k, &a_full[s], bx * C::kBoxElems, y);
-          } else {
-#pragma unroll
-            for (int bx = 0; bx < C::kBoxes; ++bx)
-              tma_load_2d_hint(dst + bx * kTileM * 128, &tm_k, &a_full[s], bx * C::kBoxElems, y, pol);
-          }
+          for (int bx = 0; bx < C::kBoxes; ++bx)
+            tma_load_2d(dst + bx * kTileM * 128, &tm_k, &a_full[s], bx * C::kBoxElems, y);
         } else {
           const int per_tile = kTileM / a.P;
           const long long r = it.grp;
@@ -369,20 +395,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(qw * 32) << 16) + static_cast<uint32_t>(acc * N);
       float kscale = 1.f;
       if (FP8 && !a.gather && s < a.L_rows) kscale = __ldg(a.k_scale + static_cast<long long>(g.b) * a.L_rows + s);
-      if (a.H >= 16) {
+      // the score of query qi of the group from its head sum sc
+      auto finish = [&](int qi, float sc) {
+        if (qi >= g.nq) return;
+        if (!a.gather) {
+          const int pos = g.pos0 + qi;   // key s visible iff s < (pos + 1) >> vis_shift
+          const int nvis = pos < 0 ? 0 : (pos + 1) >> a.vis_shift;
+          const float v = s < nvis ? sc * kscale : -INFINITY;
+          if (s < a.L_rows) store_score(a, orow + qi * a.out_row_stride + s, v);
+          if (a.gmax) flat_group_max(a, static_cast<long long>(g.b) * a.T + g.q0 + qi, s, nvis, v, lane);
+        } else if (s < a.M * a.P) {
+          const int page = __ldg(a.pages + (static_cast<long long>(g.b) * a.T + g.q0) * a.M + s / a.P);
+          const int tok = page * a.P + (s & (a.P - 1));
+          // e4m3: the recalled token's own key scale
+          const float ks = (FP8 && page >= 0) ? __ldg(a.k_scale + static_cast<long long>(g.b) * a.L_max + tok) : 1.f;
+          a.out[orow + s] = (page >= 0 && tok >= sink_end && tok < w_lo) ? sc * ks : -INFINITY;
+        }
+      };
+      if ((a.H & 63) == 0) {
+        // 64 columns per load round, summed with paired FMAs
+        for (int qi = 0; qi < a.NQ; ++qi) {
+          uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
+          for (int c0 = qi * a.H; c0 < (qi + 1) * a.H; c0 += 64) {
+            uint32_t v0[32], v1[32];
+            tmem_ld32(tbase + c0, v0);
+            tmem_ld32(tbase + c0 + 32, v1);
+            tmem_ld_wait();
+            relu_dot_acc2(wcol + c0, v0, acc2);
+            relu_dot_acc2(wcol + c0 + 32, v1, acc2);
+          }
+          finish(qi, sum8x2(acc2));
+        }
+      } else if (a.H >= 16) {
         for (int qi = 0; qi < a.NQ; ++qi) {
           float acc8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
           const int c_end = (qi + 1) * a.H;
           for (int c0 = qi * a.H; c0 < c_end;) {
-            if (c_end - c0 >= 64) {
-              uint32_t v0[32], v1[32];
-              tmem_ld32(tbase + c0, v0);
-              tmem_ld32(tbase + c0 + 32, v1);
-              tmem_ld_wait();
-              relu_dot_acc<32>(wcol + c0, v0, acc8);
-              relu_dot_acc<32>(wcol + c0 + 32, v1, acc8);
-              c0 += 64;
-            } else if (c_end - c0 >= 32) {
+            if (c_end - c0 >= 32) {
               uint32_t v0[32];
               tmem_ld32(tbase + c0, v0);
               tmem_ld_wait();
@@ -396,22 +445,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               c0 += 16;
             }
           }
-          if (qi < g.nq) {
-            const float sc = sum8(acc8);
-            if (!a.gather) {
-              const int pos = g.pos0 + qi;   // key s visible iff s < (pos + 1) >> vis_shift
-              const int nvis = pos < 0 ? 0 : (pos + 1) >> a.vis_shift;
-              const float v = s < nvis ? sc * kscale : -INFINITY;
-              if (s < a.L_rows) store_score(a, orow + qi * a.out_row_stride + s, v);
-              if (a.gmax) flat_group_max(a, static_cast<long long>(g.b) * a.T + g.q0 + qi, s, nvis, v, lane);
-            } else if (s < a.M * a.P) {
-              const int page = __ldg(a.pages + (static_cast<long long>(g.b) * a.T + g.q0) * a.M + s / a.P);
-              const int tok = page * a.P + (s & (a.P - 1));
-              // e4m3: the recalled token's own key scale
-              const float ks = (FP8 && page >= 0) ? __ldg(a.k_scale + static_cast<long long>(g.b) * a.L_max + tok) : 1.f;
-              a.out[orow + s] = (page >= 0 && tok >= sink_end && tok < w_lo) ? sc * ks : -INFINITY;
-            }
-          }
+          finish(qi, sum8(acc8));
         }
       } else {
         // H in {4, 8}: one 16-column load covers 16 / H queries
@@ -424,21 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             float sc = 0.f;
             for (int i = 0; i < a.H; ++i)
               sc = fmaf(wcol[c0 + qq * a.H + i], fmaxf(__uint_as_float(v[qq * a.H + i]), 0.f), sc);
-            const int qi = c0 / a.H + qq;
-            if (qi >= g.nq) continue;
-            if (!a.gather) {
-              const int pos = g.pos0 + qi;
-              const int nvis = pos < 0 ? 0 : (pos + 1) >> a.vis_shift;
-              const float v = s < nvis ? sc * kscale : -INFINITY;
-              if (s < a.L_rows) store_score(a, orow + qi * a.out_row_stride + s, v);
-              if (a.gmax) flat_group_max(a, static_cast<long long>(g.b) * a.T + g.q0 + qi, s, nvis, v, lane);
-            } else if (s < a.M * a.P) {
-              const int page = __ldg(a.pages + (static_cast<long long>(g.b) * a.T + g.q0) * a.M + s / a.P);
-              const int tok = page * a.P + (s & (a.P - 1));
-              // e4m3: the recalled token's own key scale
-              const float ks = (FP8 && page >= 0) ? __ldg(a.k_scale + static_cast<long long>(g.b) * a.L_max + tok) : 1.f;
-              a.out[orow + s] = (page >= 0 && tok >= sink_end && tok < w_lo) ? sc * ks : -INFINITY;
-            }
+            finish(c0 / a.H + qq, sc);
           }
         }
       }
