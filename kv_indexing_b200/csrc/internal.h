@@ -24,8 +24,8 @@ struct IndexerArgs {
   int n_tiles;           // tiles per group (FLAT) or per query row (GATHER)
   int vis_shift;         // FLAT: key s visible to pos iff s < (pos + 1) >> vis_shift (rows of 2^shift tokens)
   int gather;            // 0 = FLAT, 1 = GATHER
-  int multi_group;       // FLAT with several query groups per sequence: every group
-                         // re-reads the keys (kept in L2); score rows are streamed out
+  int multi_group;       // FLAT with several query groups per sequence (prefill):
+                         // the score rows are streamed out past L2
   int stages, nbuf_b;    // A-tile ring depth, B-tile buffers (1 or 2)
   int n_acc;             // TMEM accumulators (2 or 4)
   long long n_items;
