@@ -846,13 +846,14 @@ def roofline(path, br, peaks, peak_src, fp8, torch, dev):
                 peak, src = fp8_peak, "e4m3 GEMM measured in this run (torch._scaled_mm 8192^3, best of 10)"
             else:
                 peak, src = 2 * peaks["bf16_tflops"], peak_src + " bf16 burst x 2 (nominal e4m3 ratio)"
+        traffic = kernel_traffic("indexer_" + w.name) if not fp8 else None
         return {"bound": "tensor", "kernel": path.roof_kernel, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": None, "algorithmic_flops_per_launch": path.roof_flops,
+                "frac": achieved / peak, "traffic": traffic, "algorithmic_flops_per_launch": path.roof_flops,
                 "launch_us": us, "peak_source": src}
     achieved = path.roof_bytes / (us * 1e-6) / 1e9
     traffic = None
-    if path.kind == "flat" and not fp8 and w.name == "flat_decode_128k":
-        traffic = kernel_traffic("indexer_flat_decode_128k")
+    if path.kind == "flat" and not fp8:
+        traffic = kernel_traffic("indexer_" + w.name)
     return {"bound": "hbm", "kernel": path.roof_kernel, "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": achieved / peaks["hbm_gbs"], "traffic": traffic, "algorithmic_bytes_per_launch": path.roof_bytes,
             "launch_us": us, "peak_source": peak_src + " HBM copy"}
