@@ -115,6 +115,8 @@ struct SelectPlan {
   bool cluster;           // one thread-block cluster of C CTAs per row (no workspace)
   int cluster_rc;         // cluster path: keys per thread (4, 8, 16, 32 or 64)
   bool filter;            // filter path: group-maximum bound, C CTAs per row, last CTA finishes
+  bool row;               // row path: one CTA per row, the row's keys in registers
+  int row_rc;             // row path: keys per thread (8 or 16)
   int g0_shift, fold, gmax_stride, pool_cap;
 };
 

@@ -12,15 +12,22 @@
 //
 // Scores map to order-preserving uint32 keys (-inf -> 0 = not a candidate,
 // -0 -> +0); ties go to the lower slot, so every path equals the definition
-// exactly. Three launch shapes, chosen by select_plan:
-//   cluster  rows of <= 8 x 16384 dynamic slots: one thread-block cluster per
-//            row, keys in shared memory, agreement through DSMEM and cluster
-//            barriers (select_cluster_kernel; no workspace)
+// exactly. Launch shapes, chosen by select_plan in this order:
+//   row      rows of <= 8192 dynamic slots: one CTA per row, keys in registers,
+//            range-radix threshold, ordered emission (select_row_kernel)
+//   cluster  rows of <= 8 x 512 x 64 slots: one thread-block cluster of up to
+//            8 CTAs per row, 4..64 keys per thread in shared memory, agreement
+//            through DSMEM and cluster barriers (select_cluster_kernel)
 //   grid     longer rows when rows x CTAs fit the GPU at once: one cooperative
 //            launch, agreement through per-row blocks in global memory
 //            (select_grid_kernel)
+//   filter   rows too long for a cluster, few enough for two CTAs each: a
+//            bound from per-group maxima (written by the indexer when fused),
+//            per-warp candidate runs, the last CTA of the row finishes
+//            (select_filter_kernel)
 //   two-level otherwise: each CTA keeps its segment's local top-D candidates,
 //            the last CTA of the row merges them (select_kernel)
+// None but grid, filter and two-level use a workspace.
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -1333,16 +1340,22 @@ __global__ void __launch_bounds__(kThreads, 1) select_cluster_kernel(const Selec
       if (tid == 0) s_cnt = 0u;
       __syncthreads();
       uint32_t nd = 0u;
-      for_keys<RC, 2>(kvb, [&](uint32_t k, int) {
+      const uint32_t lt = (1u << lane) - 1u;
+      for_keys<RC, 2>(kvb, [&](uint32_t k, int) {   // warp-uniform: every thread holds RC keys
         const uint32_t rel = kmax - k;
         const uint32_t d = rel >> kRangeShift;
-        if (k != 0u && d <= b1) {
-          if (d < b1) {
-            ++nd;
-          } else {
-            const unsigned p = atomicAdd(&s_cnt, 1u);
-            if (p < kListCapC) list[p] = rel;
-          }
+        nd += (k != 0u && d < b1) ? 1u : 0u;
+        // boundary-bin keys: one shared-counter reservation per warp (the list is
+        // unordered), so a crowded bin does not serialise on the counter
+        const bool inb = k != 0u && d == b1;
+        const uint32_t m = __ballot_sync(0xffffffffu, inb);
+        if (m != 0u) {
+          const int leader = __ffs(m) - 1;
+          unsigned base = 0u;
+          if (lane == leader) base = atomicAdd(&s_cnt, static_cast<unsigned>(__popc(m)));
+          base = __shfl_sync(0xffffffffu, base, leader);
+          const unsigned p = base + static_cast<unsigned>(__popc(m & lt));
+          if (inb && p < kListCapC) list[p] = rel;
         }
       });
       uint32_t my_def = 0u;
@@ -1983,6 +1996,48 @@ __global__ void __launch_bounds__(kThreads, 1) select_filter_kernel(const Select
   for (int i = tr0 + pl.trail_n + tid; i < a.out_len; i += kThreads) out[i] = -1;
 }
 
+// One CTA per row for rows of at most kThreads * RC dynamic slots: the keys
+// stay in registers (warp-striped: lane l of warp w holds element
+// w 32 RC + 32 j + l in k[j]), the exact D-th key comes from range-radix
+// rounds over one shared histogram, and the selection is emitted in index
+// order. No cluster barriers, no distributed shared memory, no workspace.
+template <int RC>
+__global__ void __launch_bounds__(kThreads, 1) select_row_kernel(const SelectArgs a) {
+  pdl_wait();   // the scores come from the previous kernel
+  pdl_trigger();
+  __shared__ Shared sh;
+  const int r = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const Plan pl = make_plan(a, r);
+  int* out = a.out + static_cast<long long>(r) * a.out_len;
+  if (!pl.valid) {
+    for (int i = tid; i < a.out_len; i += kThreads) out[i] = -1;
+    return;
+  }
+  const int len = pl.dyn_hi - pl.dyn_lo;
+  const float* row = a.scores + static_cast<long long>(r) * a.row_stride + pl.dyn_lo;
+  const int e0 = warp * 32 * RC + lane;
+  uint32_t k[RC];
+#pragma unroll
+  for (int j = 0; j < RC; ++j) {
+    const int e = e0 + 32 * j;
+    k[j] = e < len ? score_key(__ldg(row + e)) : 0u;
+  }
+  const Thr t = fast_threshold<RC>(k, static_cast<uint32_t>(pl.D), sh);
+  int* dyn_out = out + pl.dyn_off;
+  const long long prow = static_cast<long long>(r) * a.M;
+  const bool hier = a.mode == kSelectHierTokens;
+  const uint32_t n_sel = reg_emit<RC>(k, t, sh, [&](uint32_t p, int j) {
+    const int slot = pl.dyn_lo + e0 + 32 * j;
+    dyn_out[p] = hier ? __ldg(a.pages + prow + slot / a.P) * a.P + slot % a.P : slot;
+  });
+  for (int i = tid; i < pl.lead_a_n; i += kThreads) out[i] = pl.lead_a_lo + i;
+  for (int i = tid; i < pl.lead_b_n; i += kThreads) out[pl.lead_a_n + i] = pl.lead_b_lo + i;
+  const int tr0 = pl.dyn_off + static_cast<int>(n_sel);
+  for (int i = tid; i < pl.trail_n; i += kThreads) out[tr0 + i] = pl.trail_lo + i;
+  for (int i = tr0 + pl.trail_n + tid; i < a.out_len; i += kThreads) out[i] = -1;
+}
+
 }  // namespace
 
 SelectPlan select_plan(int rows, int n_slots, int d_bound, int num_sms) {
@@ -1991,6 +2046,18 @@ SelectPlan select_plan(int rows, int n_slots, int d_bound, int num_sms) {
   constexpr int kSegMax = 32768;            // fallback: keys per CTA in shared memory
   SelectPlan p{};
   auto seg_of = [&](int C) { return (n_slots + C - 1) / C; };
+  // row path: rows of at most 8192 slots, one CTA each, keys in registers.
+  // Measured: faster than a cluster up to 8192 slots; at 16384 (32 keys per
+  // thread on one SM) the 8-CTA cluster with 4 keys per thread is faster
+  for (const int rc : {8, 16}) {
+    if (n_slots <= kThreads * rc) {
+      p.row = true;
+      p.row_rc = rc;
+      p.C = 1;
+      p.seg = n_slots;
+      return p;
+    }
+  }
   // cluster path: one cluster of up to 8 CTAs per row, any number of rows. The
   // cost of a CTA's passes grows with its keys per thread (each pass is
   // instruction-bound on one SM), so few rows spread over more CTAs with fewer
@@ -2082,7 +2149,7 @@ FilterLayout filter_layout(int rows, const SelectPlan& p) {
 
 size_t select_ws_bytes(int rows, const SelectPlan& p) {
   if (p.filter) return filter_layout(rows, p).total;
-  if (p.cluster) return 0;
+  if (p.cluster || p.row) return 0;
   if (p.grid) return grid_blocks_bytes(rows) + grid_row_bytes(p.C) * rows;
   const size_t n = static_cast<size_t>(rows) * p.C * p.cand_cap;
   return ((n * 8 + rows * 4 + 255) / 256) * 256;
@@ -2116,6 +2183,12 @@ cudaError_t launch_select(const SelectArgs& a0, const SelectPlan& p, void* ws, c
     cudaError_t e = set_max_smem(fn, smem);
     if (e != cudaSuccess) return e;
     return launch_pdl(fn, dim3(p.C, rows), dim3(kThreads), smem, stream, args);
+  }
+  if (p.row) {
+    const void* fn = p.row_rc == 16 ? reinterpret_cast<const void*>(&select_row_kernel<16>)
+                                    : reinterpret_cast<const void*>(&select_row_kernel<8>);
+    void* args[] = {&a};
+    return launch_pdl(fn, dim3(rows, 1, 1), dim3(kThreads, 1, 1), 0, stream, args);
   }
   if (p.cluster) {
     const size_t smem = cluster_smem_words(p.cluster_rc) * 4;
