@@ -214,7 +214,7 @@ lsa_status_t lsa_select_streaming(const float* scores, const int32_t* seq_len, i
  *     LSA_NOALLOC_SCRATCH_BYTES are rejected with LSA_ERR_WORKSPACE before
  *     anything is launched. Rows of up to 262144 score slots need no
  *     scratch at all (any number of rows); longer rows do: with k=2048 and
- *     sink+window=1024 on a 148-SM B200, L_max=1M admits up to 21 rows.
+ *     sink+window=1024 on a 148-SM B200, L_max=1M admits up to 20 rows.
  *   - The first call on a device (and the first after its context changes,
  *     e.g. after cudaDeviceReset) looks up the buffer's device address, which
  *     may load the library's device code onto that device; make that first

@@ -23,16 +23,19 @@ from tests.parity import dev, host
 
 
 def test_noalloc_rejects_oversized_shape_on_the_host():
-    # B*T=22 rows at L_max=1M need just over 16 MiB of selection scratch; the
-    # call must refuse before touching the (fake, never dereferenced) pointers.
+    # B*T=21 rows at L_max=1M need just over 16 MiB of selection scratch (20
+    # fit); the call must refuse before touching the (fake, never
+    # dereferenced) pointers.
     lib = L.load()
     fake = ctypes.c_void_p(256)
-    st = lib.lsa_select_streaming_noalloc(fake, fake, 22, 1, 1 << 20, L.Budget(2048, 64, 960), fake, None)
+    st = lib.lsa_select_streaming_noalloc(fake, fake, 21, 1, 1 << 20, L.Budget(2048, 64, 960), fake, None)
     assert st == L.LSA_ERR_WORKSPACE
     msg = lib.lsa_last_error().decode()
     assert "static scratch" in msg and str(L.LSA_NOALLOC_SCRATCH_BYTES) in msg
-    need = L.workspace_size(L.LSA_OP_SELECT, budget=(2048, 64, 960), B=22, T=1, L_max=1 << 20)
+    need = L.workspace_size(L.LSA_OP_SELECT, budget=(2048, 64, 960), B=21, T=1, L_max=1 << 20)
     assert need > L.LSA_NOALLOC_SCRATCH_BYTES
+    fits = L.workspace_size(L.LSA_OP_SELECT, budget=(2048, 64, 960), B=20, T=1, L_max=1 << 20)
+    assert 0 < fits <= L.LSA_NOALLOC_SCRATCH_BYTES
 
 
 def test_noalloc_rejects_bad_arguments_on_the_host():
