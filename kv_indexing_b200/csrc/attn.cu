@@ -956,6 +956,7 @@ cudaError_t launch(const AttnMaps* m, const AttnArgs* a, int n, cudaStream_t str
 
 // Merge KV-split partials (o_s = O_s / l_s in bf16, with m_s and l_s):
 //   f_s = l_s 2^(m_s - m*),  m* = max m_s;  o = sum f_s o_s / sum f_s.
+template <int kInFlight>
 __global__ void __launch_bounds__(128) combine_kernel(const __grid_constant__ LayerOuts lo, const AttnArgs a) {
   pdl_wait();
   pdl_trigger();
@@ -1001,14 +1002,36 @@ __global__ void __launch_bounds__(128) combine_kernel(const __grid_constant__ La
   const int c = threadIdx.x * 4;
   if (c >= a.d_v) return;
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  if constexpr (kInFlight <= 4) {
 #pragma unroll 4
-  for (int sidx = 0; sidx < ns; ++sidx) {
-    const float f = s_f[sidx];
-    const uint2 o = *reinterpret_cast<const uint2*>(Lo.part_o + (base + static_cast<long long>(sidx) * a.Hq) * a.d_v + c);
-    acc[0] = fmaf(__uint_as_float(o.x << 16), f, acc[0]);
-    acc[1] = fmaf(__uint_as_float(o.x & 0xFFFF0000u), f, acc[1]);
-    acc[2] = fmaf(__uint_as_float(o.y << 16), f, acc[2]);
-    acc[3] = fmaf(__uint_as_float(o.y & 0xFFFF0000u), f, acc[3]);
+    for (int sidx = 0; sidx < ns; ++sidx) {
+      const float f = s_f[sidx];
+      const uint2 o = *reinterpret_cast<const uint2*>(Lo.part_o + (base + static_cast<long long>(sidx) * a.Hq) * a.d_v + c);
+      acc[0] = fmaf(__uint_as_float(o.x << 16), f, acc[0]);
+      acc[1] = fmaf(__uint_as_float(o.x & 0xFFFF0000u), f, acc[1]);
+      acc[2] = fmaf(__uint_as_float(o.y << 16), f, acc[2]);
+      acc[3] = fmaf(__uint_as_float(o.y & 0xFFFF0000u), f, acc[3]);
+    }
+  } else {
+    // many splits: their partials are independent loads, kInFlight in flight
+    // per thread, then accumulated in split order (the same arithmetic)
+    const uint16_t* po = Lo.part_o + base * a.d_v + c;
+    const long long sstride = static_cast<long long>(a.Hq) * a.d_v;
+    for (int s0 = 0; s0 < ns; s0 += kInFlight) {
+      uint2 o[kInFlight];
+#pragma unroll
+      for (int j = 0; j < kInFlight; ++j)
+        o[j] = s0 + j < ns ? *reinterpret_cast<const uint2*>(po + (s0 + j) * sstride) : make_uint2(0u, 0u);
+#pragma unroll
+      for (int j = 0; j < kInFlight; ++j) {
+        if (s0 + j >= ns) break;
+        const float f = s_f[s0 + j];
+        acc[0] = fmaf(__uint_as_float(o[j].x << 16), f, acc[0]);
+        acc[1] = fmaf(__uint_as_float(o[j].x & 0xFFFF0000u), f, acc[1]);
+        acc[2] = fmaf(__uint_as_float(o[j].y << 16), f, acc[2]);
+        acc[3] = fmaf(__uint_as_float(o[j].y & 0xFFFF0000u), f, acc[3]);
+      }
+    }
   }
   const float inv = s_den > 0.f ? 1.f / s_den : 0.f;
   const __nv_bfloat162 v01 = __floats2bfloat162_rn(acc[0] * inv, acc[1] * inv);
@@ -1059,7 +1082,11 @@ cudaError_t launch_attn_combine(const AttnArgs* args, int n, cudaStream_t stream
   AttnArgs shared = a;
   const dim3 grid(a.B * a.T, a.Hq, n);
   void* kargs[] = {&lo, &shared};
-  return launch_pdl(reinterpret_cast<const void*>(&combine_kernel), grid, dim3(a.d_v / 4 < 32 ? 32 : a.d_v / 4),
+  // rows with many splits (few rows on the GPU) take 16 partial loads in flight
+  // per thread; many rows keep 4 (registers: the grid is rows x heads CTAs)
+  const void* fn = a.n_split >= 24 ? reinterpret_cast<const void*>(&combine_kernel<16>)
+                                   : reinterpret_cast<const void*>(&combine_kernel<4>);
+  return launch_pdl(fn, grid, dim3(a.d_v / 4 < 32 ? 32 : a.d_v / 4),
                     0, stream, kargs);
 }
 
