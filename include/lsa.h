@@ -105,7 +105,12 @@ typedef struct lsa_indexer_in {
  * v + (b*L_max + s)*v_row_stride (d_v elements). For MLA (one latent row per
  * token) pass v = k: V is then the first d_v columns of the latent row.
  *   q [B,T,Hq,d_qk] bf16; K, V bf16. Strides in elements, multiples of 8.
- * Supported: (d_qk, d_v) in {(64, 64), (576, 512)}; 1 <= Hq <= 128. */
+ * Supported: (d_qk, d_v) in {(64, 64), (576, 512)}; 1 <= Hq <= 128.
+ * FP8 KV (kv_dtype = LSA_E4M3, MLA only; the quantised storage of the DSA
+ * article's "Quantized computation" applied to the latent cache): k = v holds
+ * e4m3 codes (row stride in elements = bytes, a multiple of 16) and k_scale
+ * [B*L_max] the fp32 scale of each token's row, so K = V = code * scale.
+ * Scores and outputs are those of the formula above on those values. */
 typedef struct lsa_attn_in {
   int32_t B, T, Hq, d_qk, d_v, L_max;
   float scale;
@@ -125,6 +130,8 @@ typedef struct lsa_attn_in {
    * workspace or outputs (q, k, v and seq_len are read before it ends). A row
    * that breaks the promise gives undefined results. */
   int32_t stream_sink, stream_window;
+  int32_t kv_dtype;        /* LSA_BF16 (0, the default) or LSA_E4M3 */
+  const float* k_scale;    /* LSA_E4M3: per-token scale [B*L_max]; else NULL */
 } lsa_attn_in_t;
 
 typedef enum lsa_op {

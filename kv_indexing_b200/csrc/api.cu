@@ -140,6 +140,16 @@ lsa_status_t check_attn(const lsa_attn_in_t* at, int k) {
     return fail(LSA_ERR_INVALID_ARG, "row strides must cover the row and be multiples of 8 elements");
   const bool alias = at->v == at->k && at->v_row_stride == at->k_row_stride;
   if (mla && !alias) return fail(LSA_ERR_UNSUPPORTED, "d_qk=576/d_v=512 requires v == k (MLA latent rows)");
+  if (at->kv_dtype != LSA_BF16 && at->kv_dtype != LSA_E4M3)
+    return fail(LSA_ERR_INVALID_ARG, "kv_dtype %d is neither LSA_BF16 nor LSA_E4M3", at->kv_dtype);
+  if (at->kv_dtype == LSA_E4M3) {
+    if (!mla) return fail(LSA_ERR_UNSUPPORTED, "e4m3 KV needs the MLA shape (d_qk=576, d_v=512)");
+    if (!at->k_scale || (reinterpret_cast<uintptr_t>(at->k_scale) & 3u))
+      return fail(LSA_ERR_INVALID_ARG, "e4m3 KV needs k_scale (fp32, 4-byte aligned)");
+    if (at->k_row_stride % 16) return fail(LSA_ERR_INVALID_ARG, "e4m3 KV row stride must be a multiple of 16 bytes");
+  } else if (at->k_scale) {
+    return fail(LSA_ERR_INVALID_ARG, "k_scale is for e4m3 KV only");
+  }
   if (!(at->scale > 0.f) || !std::isfinite(at->scale)) return fail(LSA_ERR_INVALID_ARG, "scale must be finite and > 0");
   if (k < 1 || k > 8192) return fail(LSA_ERR_UNSUPPORTED, "index row length %d outside [1, 8192]", k);
   if (at->stream_sink < -1 || at->stream_window < -1)
@@ -220,13 +230,13 @@ size_t attn_ws_bytes(const lsa_attn_in_t* at, int k, int layers = 1) {
 }
 
 // Layers [i, i + n) of a group that go into one attention launch: consecutive
-// MLA layers with the same head count, at most kMaxLaunchLayers.
+// MLA layers with the same head count and KV type, at most kMaxLaunchLayers.
 int group_launch_layers(const lsa_attn_in_t* layers, int i, int n_layers) {
   const lsa_attn_in_t& f = layers[i];
   if (!(f.d_qk == 576 && f.d_v == 512)) return 1;
   int n = 1;
   while (n < kMaxLaunchLayers && i + n < n_layers && layers[i + n].d_qk == 576 && layers[i + n].d_v == 512 &&
-         layers[i + n].Hq == f.Hq)
+         layers[i + n].Hq == f.Hq && layers[i + n].kv_dtype == f.kv_dtype)
     ++n;
   return n;
 }
@@ -427,10 +437,15 @@ lsa_status_t run_attn(const lsa_attn_in_t* ats, int n, const int* idx, int k, vo
     lsa_status_t s = make_tmap(&m.q, at->q, false, at->d_qk, static_cast<uint64_t>(at->B) * at->T * at->Hq, 64, 128);
     if (s != LSA_OK) return s;
     const uint64_t kv_rows = static_cast<uint64_t>(at->B) * at->L_max;
-    if ((s = make_tmap_strided(&m.k_tile, at->k, at->d_qk, kv_rows, at->k_row_stride, 64, kAttnBN)) != LSA_OK) return s;
-    if ((s = make_tmap_strided(&m.k_rows, at->k, at->d_qk, kv_rows, at->k_row_stride, 64, 1)) != LSA_OK) return s;
-    if ((s = make_tmap_strided(&m.v_tile, at->v, at->d_v, kv_rows, at->v_row_stride, 64, kAttnBN)) != LSA_OK) return s;
-    if ((s = make_tmap_strided(&m.v_rows, at->v, at->d_v, kv_rows, at->v_row_stride, 64, 1)) != LSA_OK) return s;
+    m.k_tile = m.k_rows = m.v_tile = m.v_rows = CUtensorMap{};   // e4m3 KV: rows staged by the producer threads
+    if (at->kv_dtype != LSA_E4M3) {
+      if ((s = make_tmap_strided(&m.k_tile, at->k, at->d_qk, kv_rows, at->k_row_stride, 64, kAttnBN)) != LSA_OK)
+        return s;
+      if ((s = make_tmap_strided(&m.k_rows, at->k, at->d_qk, kv_rows, at->k_row_stride, 64, 1)) != LSA_OK) return s;
+      if ((s = make_tmap_strided(&m.v_tile, at->v, at->d_v, kv_rows, at->v_row_stride, 64, kAttnBN)) != LSA_OK)
+        return s;
+      if ((s = make_tmap_strided(&m.v_rows, at->v, at->d_v, kv_rows, at->v_row_stride, 64, 1)) != LSA_OK) return s;
+    }
     AttnArgs& a = args[i];
     a = AttnArgs{};
     a.B = at->B; a.T = at->T; a.Hq = at->Hq; a.L_max = at->L_max;
@@ -442,6 +457,8 @@ lsa_status_t run_attn(const lsa_attn_in_t* ats, int n, const int* idx, int k, vo
     a.vp = static_cast<const uint16_t*>(at->v);
     a.k_stride = at->k_row_stride; a.v_stride = at->v_row_stride;
     a.sep_v = !(at->v == at->k && at->v_row_stride == at->k_row_stride);
+    a.kv8 = at->kv_dtype == LSA_E4M3;
+    a.k_scale = at->k_scale;
     a.n_split = p.n_split; a.blocks_per_split = p.bps;
     a.fixed_blocks = p.fixed_blocks; a.fixed_splits = p.fixed_splits; a.bps_fixed = p.bps_fixed;
     a.stream_sink = at->stream_sink > 0 ? at->stream_sink : 0;

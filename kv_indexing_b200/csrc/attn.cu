@@ -18,6 +18,7 @@
 // writes bf16 P to shared memory for the PV MMA. With several KV splits each
 // CTA writes an unnormalised partial (O, m, l) and a combine kernel merges them.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -33,6 +34,9 @@ struct LayerOut {
   float* part_m;          // [rows, n_split, Hq]
   float* part_l;          // [rows, n_split, Hq]
   float scale_log2;       // the layer's softmax scale * log2(e)
+  const uint8_t* kv8;     // e4m3 KV: the layer's latent rows of codes (else null)
+  long long kv8_stride;   // bytes between consecutive latent rows
+  const float* k_scale;   // e4m3 KV: per-token scale [B * L_max]
 };
 struct LayerOuts {
   LayerOut l[kMaxLaunchLayers];
@@ -43,7 +47,15 @@ LayerOuts layer_outs(const AttnArgs* args, int n) {
   LayerOuts lo{};
   lo.n = n;
   for (int i = 0; i < n; ++i)
-    lo.l[i] = LayerOut{args[i].out, args[i].lse, args[i].part_o, args[i].part_m, args[i].part_l, args[i].scale_log2};
+    lo.l[i] = LayerOut{args[i].out,
+                       args[i].lse,
+                       args[i].part_o,
+                       args[i].part_m,
+                       args[i].part_l,
+                       args[i].scale_log2,
+                       args[i].kv8 ? reinterpret_cast<const uint8_t*>(args[i].kp) : nullptr,
+                       args[i].k_stride,
+                       args[i].k_scale};
   return lo;
 }
 
@@ -411,7 +423,8 @@ constexpr int kOffX = kStages * kStageBytes;        // [2] receive buffers
 constexpr int kOffSend = kOffX + 2 * kXBytes;       // outgoing partial scores (same layout)
 constexpr int kOffTag = kOffSend + kXBytes;         // [2][2][128] u64 tagged max slots + [2][128] u64 sums
 constexpr int kOffMask = kOffTag + (4 * 128 + 2 * 128) * 8;
-constexpr int kOffBars = kOffMask + kStages * 8;
+constexpr int kOffKScale = kOffMask + kStages * 8;   // e4m3 KV: [kStages][BN] token scales of the staged rows
+constexpr int kOffBars = kOffKScale + kStages * BN * 4;
 constexpr int kNumBars = 2 * kStages + 11;
 constexpr int kOffMisc = kOffBars + kNumBars * 8;
 constexpr size_t kSmem = 1024 + kOffMisc + 16;
@@ -465,6 +478,21 @@ struct MapSet {
   CUtensorMap kt[kMaxLaunchLayers], kg[kMaxLaunchLayers], q[kMaxLaunchLayers];
 };
 
+// e4m3 pair -> bf16 pair, exact (every e4m3 value is a bf16 value): through
+// the paired e4m3 -> f16 conversion and fp32.
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t two_codes) {
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<uint16_t>(two_codes)));
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+  const __nv_bfloat162 b = __floats2bfloat162_rn(f.x, f.y);
+  return *reinterpret_cast<const uint32_t*>(&b);
+}
+
+// KV8: the latent rows are e4m3 codes with a per-token scale. The producer
+// threads stage each block's codes as bf16 (exact) in the same swizzled tiles
+// and the token scales beside them; the softmax multiplies each score column
+// by its token's scale, and P by it before the PV product (V = code * scale).
+template <bool KV8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mla_pair_kernel(const __grid_constant__ MapSet maps, const __grid_constant__ LayerOuts lo, const AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -475,6 +503,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   volatile unsigned long long* tag_max = reinterpret_cast<volatile unsigned long long*>(base + kOffTag);  // [2][2][128]
   volatile unsigned long long* tag_sum = tag_max + 4 * 128;                                              // [2][128]
   uint32_t* mask_s = reinterpret_cast<uint32_t*>(base + kOffMask);                                       // [kStages][2]
+  float* kscale_s = reinterpret_cast<float*>(base + kOffKScale);                                         // [kStages][BN]
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + kOffBars);
   uint64_t* kv_full = bars;
   uint64_t* kv_empty = bars + kStages;
@@ -533,7 +562,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&kv_full[i], 2);    // one expect_tx arrive per producer warp
+      mbar_init(&kv_full[i], KV8 ? 64 : 2);   // KV8: every producer thread; else one expect_tx arrive per warp
       mbar_init(&kv_empty[i], 1);
     }
     mbar_init(s_full, 1);
@@ -578,8 +607,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
     cluster_arrive_release();
-    prefetch_tmap(tm_kt);
-    prefetch_tmap(tm_kg);
+    if (!KV8) {   // e4m3 KV: no K tensor maps (the rows are staged by these threads)
+      prefetch_tmap(tm_kt);
+      prefetch_tmap(tm_kg);
+    }
     const int row0 = b * a.L_max;
     // index entry e of block `bb`, -1 outside the split / row
     auto load_id = [&](int bb, int e) -> int {
@@ -623,6 +654,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int id0 = __shfl_sync(0xffffffffu, id_lo, 0);
         const bool contiguous =
             __all_sync(0xffffffffu, id0 >= 0 && id_lo == id0 + lane && id_hi == id0 + 32 + lane);
+        if constexpr (KV8) {
+          // this lane's row of the block, 320 codes of it (this CTA's columns),
+          // staged as bf16 in the swizzled tile; invalid entries stage row 0 of
+          // the sequence (finite, masked out) with scale 0
+          const int id = part == 0 ? id_lo : id_hi;
+          const int row = 32 * part + lane;
+          const int y = id >= 0 ? id : 0;
+          if (lane == 0 && part == 0) {
+            mask_s[2 * j] = valid_lo;
+            mask_s[2 * j + 1] = valid_hi;
+          }
+          kscale_s[j * BN + row] = id >= 0 ? __ldg(Lo.k_scale + row0 + y) : 0.f;
+          const uint4* src = reinterpret_cast<const uint4*>(Lo.kv8 + static_cast<long long>(row0 + y) * Lo.kv8_stride +
+                                                            chunk0 * 64);
+          uint8_t* trow = sStage + j * kStageBytes + row * 128;
+          const int swz = row & 7;
+#pragma unroll
+          for (int c = 0; c < kChunks; ++c) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {   // codes 16q .. 16q + 15 of chunk c -> bf16 units 2q, 2q + 1
+              const uint4 v = __ldg(src + 4 * c + q);
+              const uint4 u0 = make_uint4(e4m3x2_to_bf16x2(v.x), e4m3x2_to_bf16x2(v.x >> 16), e4m3x2_to_bf16x2(v.y),
+                                          e4m3x2_to_bf16x2(v.y >> 16));
+              const uint4 u1 = make_uint4(e4m3x2_to_bf16x2(v.z), e4m3x2_to_bf16x2(v.z >> 16), e4m3x2_to_bf16x2(v.w),
+                                          e4m3x2_to_bf16x2(v.w >> 16));
+              *reinterpret_cast<uint4*>(trow + c * kChunkBytes + (((2 * q) ^ swz) << 4)) = u0;
+              *reinterpret_cast<uint4*>(trow + c * kChunkBytes + (((2 * q + 1) ^ swz) << 4)) = u1;
+            }
+          }
+          fence_proxy_async_smem();   // generic-proxy stores, read by the tensor cores
+          mbar_arrive(&kv_full[j]);
+          continue;
+        }
         const int y_mine = row0 + (part == 0 ? (id_lo >= 0 ? id_lo : 0) : (id_hi >= 0 ? id_hi : 0));
         int yg[4];
 #pragma unroll
@@ -796,9 +860,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, wait_ph<false>(&kv_full[s], (blk / kStages) & 1, a.status, abort_flag));
       if (!ok) break;
       const uint32_t valid = mask_s[2 * s + half];
+      const float4* ks4 = reinterpret_cast<const float4*>(kscale_s + s * BN + 32 * half);   // KV8: token scales
       float mloc[8];
+      if constexpr (KV8) {
 #pragma unroll
-      for (int j = 0; j < 32; ++j) x[j] = ((valid >> j) & 1u) ? x[j] * Lo.scale_log2 : -INFINITY;
+        for (int t = 0; t < 8; ++t) {
+          const float4 k4 = ks4[t];
+          const float kk[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int j = 4 * t + e;
+            x[j] = ((valid >> j) & 1u) ? x[j] * kk[e] * Lo.scale_log2 : -INFINITY;
+          }
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) x[j] = ((valid >> j) & 1u) ? x[j] * Lo.scale_log2 : -INFINITY;
+      }
 #pragma unroll
       for (int t = 0; t < 8; ++t) mloc[t] = fmaxf(fmaxf(x[4 * t], x[4 * t + 1]), fmaxf(x[4 * t + 2], x[4 * t + 3]));
       const float mb_mine = fmaxf(fmaxf(fmaxf(mloc[0], mloc[1]), fmaxf(mloc[2], mloc[3])),
@@ -841,7 +919,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const float p0 = m_run == -INFINITY ? 0.f : exp2f(x[j] - m_run);
         const float p1 = m_run == -INFINITY ? 0.f : exp2f(x[j + 1] - m_run);
         ps[(j >> 1) & 3] += p0 + p1;
-        const __nv_bfloat162 v2 = __floats2bfloat162_rn(p0, p1);
+        float w0 = p0, w1 = p1;
+        if constexpr (KV8) {   // V row = code * scale: the scale rides on P
+          const float2 k2 = reinterpret_cast<const float2*>(ks4)[j >> 1];
+          w0 *= k2.x;
+          w1 *= k2.y;
+        }
+        const __nv_bfloat162 v2 = __floats2bfloat162_rn(w0, w1);
         pk[j >> 1] = *reinterpret_cast<const uint32_t*>(&v2);
       }
       l_part += (ps[0] + ps[1]) + (ps[2] + ps[3]);
@@ -938,7 +1022,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 }
 
 cudaError_t launch(const AttnMaps* m, const AttnArgs* a, int n, cudaStream_t stream) {
-  const void* fn = reinterpret_cast<const void*>(&mla_pair_kernel);
+  for (int i = 1; i < n; ++i)
+    if (a[i].kv8 != a[0].kv8) return cudaErrorInvalidValue;   // one KV type per launch
+  const void* fn = a[0].kv8 ? reinterpret_cast<const void*>(&mla_pair_kernel<true>)
+                            : reinterpret_cast<const void*>(&mla_pair_kernel<false>);
   cudaError_t e = set_max_smem(fn, kSmem);
   if (e != cudaSuccess) return e;
   MapSet maps{};

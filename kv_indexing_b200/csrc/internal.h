@@ -155,6 +155,8 @@ struct AttnArgs {
   const uint16_t* vp;     // V rows (may alias kp)
   long long k_stride, v_stride;
   int sep_v;              // V rows loaded separately (not a prefix of the K row)
+  int kv8;                // MLA: K = V rows are e4m3 codes (row stride in bytes), times k_scale
+  const float* k_scale;   // kv8: per-token scale [B * L_max]
   int n_split, blocks_per_split;
   int fixed_blocks, fixed_splits, bps_fixed;   // splits [0, fixed_splits) cover blocks [0, fixed_blocks) in
                                                // bps_fixed-block pieces; the others blocks_per_split each

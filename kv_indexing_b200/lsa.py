@@ -50,7 +50,8 @@ class AttnIn(ctypes.Structure):
                 ("d_v", ctypes.c_int32), ("L_max", ctypes.c_int32), ("scale", ctypes.c_float),
                 ("seq_len", ctypes.c_void_p), ("q", ctypes.c_void_p), ("k", ctypes.c_void_p),
                 ("v", ctypes.c_void_p), ("k_row_stride", ctypes.c_int64), ("v_row_stride", ctypes.c_int64),
-                ("stream_sink", ctypes.c_int32), ("stream_window", ctypes.c_int32)]
+                ("stream_sink", ctypes.c_int32), ("stream_window", ctypes.c_int32),
+                ("kv_dtype", ctypes.c_int32), ("k_scale", ctypes.c_void_p)]
 
 
 class OpArgs(ctypes.Structure):
@@ -165,15 +166,28 @@ def indexer_in(q, w, k, seq_len, q_scale=None, k_scale=None, m=1) -> IndexerIn:
                      _ptr(q_scale) if fp8 else None, _ptr(w), _ptr(k), _ptr(k_scale) if fp8 else None)
 
 
-def attn_in(q, seq_len, scale, *, kv=None, k=None, v=None, d_v=None, stream_budget=None) -> AttnIn:
+def attn_in(q, seq_len, scale, *, kv=None, k=None, v=None, d_v=None, stream_budget=None, kv_scale=None) -> AttnIn:
     """Describe attention tensors: q [B,T,Hq,d_qk]; MLA kv [B,L_max,d_qk] (V = first d_v
-    columns) or separate k [B,L_max,d_qk], v [B,L_max,d_v]; all bf16. stream_budget
+    columns) or separate k [B,L_max,d_qk], v [B,L_max,d_v]; all bf16, or an MLA kv of
+    e4m3 codes (torch.float8_e4m3fn) with kv_scale [B,L_max] fp32 per token. stream_budget
     (k, sink, window) promises the index rows start with that streaming prefix."""
     torch = _torch()
     _need(q, "q", torch.bfloat16, 4)
     _need(seq_len, "seq_len", torch.int32, 1)
     B, T, Hq, d_qk = q.shape
     ss, sw = (-1, -1) if stream_budget is None else (int(stream_budget[1]), int(stream_budget[2]))
+    if kv is not None and kv.dtype == torch.float8_e4m3fn:
+        _need(kv, "kv", torch.float8_e4m3fn, 3)
+        if kv_scale is None:
+            raise ValueError("an e4m3 kv needs kv_scale [B, L_max] float32")
+        _need(kv_scale, "kv_scale", torch.float32, 2)
+        if tuple(kv_scale.shape) != (kv.shape[0], kv.shape[1]):
+            raise ValueError("kv_scale must be [B, L_max]")
+        dv = d_v if d_v is not None else 512
+        return AttnIn(B, T, Hq, d_qk, dv, kv.shape[1], float(scale), _ptr(seq_len), _ptr(q), _ptr(kv), _ptr(kv),
+                      kv.shape[2], kv.shape[2], ss, sw, LSA_E4M3, _ptr(kv_scale))
+    if kv_scale is not None:
+        raise ValueError("kv_scale is for an e4m3 kv only")
     if kv is not None:
         _need(kv, "kv", torch.bfloat16, 3)
         dv = d_v if d_v is not None else (512 if d_qk == 576 else d_qk)
@@ -365,13 +379,14 @@ def lsa_index_hier_e4m3(q8, q_scale, w, k8, k_scale, seq_len, page_codes, page_s
 
 
 def lsa_sparse_attn(q, idx, seq_len, scale, *, kv=None, k=None, v=None, d_v=None, out=None, lse=None,
-                    workspace=None, stream=None, stream_budget=None):
+                    workspace=None, stream=None, stream_budget=None, kv_scale=None):
     """Sparse attention over idx [B,T,k]. Returns (out [B,T,Hq,d_v] bf16, lse or None).
     stream_budget (k, sink, window): idx rows come from the streaming selection with
-    that budget, so their sink/window prefix may be computed instead of read."""
+    that budget, so their sink/window prefix may be computed instead of read.
+    An e4m3 MLA kv (torch.float8_e4m3fn) takes kv_scale [B, L_max] fp32."""
     torch = _torch()
     lib = load()
-    ai = attn_in(q, seq_len, scale, kv=kv, k=k, v=v, d_v=d_v, stream_budget=stream_budget)
+    ai = attn_in(q, seq_len, scale, kv=kv, k=k, v=v, d_v=d_v, stream_budget=stream_budget, kv_scale=kv_scale)
     _need(idx, "idx", torch.int32, 3)
     if out is None:
         out = torch.empty((ai.B, ai.T, ai.Hq, ai.d_v), dtype=torch.bfloat16, device=q.device)
@@ -390,7 +405,8 @@ def lsa_layer_group(q, w, k, seq_len, budget, layers: Sequence[dict], *, P=0, M=
     torch = _torch()
     lib = load()
     ii = indexer_in(q, w, k, seq_len)
-    ais = [attn_in(l["q"], seq_len, l["scale"], kv=l.get("kv"), k=l.get("k"), v=l.get("v"), d_v=l.get("d_v"))
+    ais = [attn_in(l["q"], seq_len, l["scale"], kv=l.get("kv"), k=l.get("k"), v=l.get("v"), d_v=l.get("d_v"),
+                   kv_scale=l.get("kv_scale"))
            for l in layers]
     n = len(ais)
     if outs is None:

@@ -63,6 +63,8 @@ def _load():
             "orc_sparse_attention_row": (i32, [P, P, P, i64, i32, i32, i32, P, i64, f64, P, P]),
             "orc_sparse_attention": (i32, [i32, i32, i32, i32, i32, i32, P, P, i32, P, i64, P, i64, f64, P, i32, P,
                                            P, i32]),
+            "orc_sparse_attention_e4m3": (i32, [i32, i32, i32, i32, i32, i32, P, P, i32, P, i64, P, f64, P, i32, P,
+                                                P, i32]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -382,6 +384,27 @@ def sparse_attention_rows(qa, idx, rows, *, scale: float, d_v: int, kv=None, k=N
     _ok(_load().orc_sparse_attention(B, T, Hq, d_qk, d_v, L_max, _p(q), _p(ix), ix.shape[2], _p(kk), kk.shape[2],
                                      _p(vv), vv.shape[2], float(scale), _p(r), n, _p(o), _p(lse), _threads),
         "sparse_attention")
+    return o, lse
+
+
+def sparse_attention_e4m3_rows(qa, idx, rows, *, scale: float, d_v: int, kv8, k_scale):
+    """Attention over an e4m3 latent cache (K = code * scale, V = its first d_v
+    columns), for the listed (b, t) rows (None = all), compact: (o [n, Hq, d_v],
+    lse [n, Hq]) in float64. kv8 [B,L_max,d_qk] e4m3 codes; k_scale [B,L_max] fp32."""
+    q = _c(qa, np.uint16)
+    B, T, Hq, d_qk = q.shape
+    ix = _c(idx, np.int32)
+    kc = _c(kv8, np.uint8)
+    ks = _c(k_scale, np.float32)
+    L_max = kc.shape[1]
+    if ks.shape != (kc.shape[0], L_max):
+        raise ValueError("k_scale must be [B, L_max]")
+    r, n = _rows_arg(rows, B, T)
+    o = np.empty((n, Hq, d_v), np.float64)
+    lse = np.empty((n, Hq), np.float64)
+    _ok(_load().orc_sparse_attention_e4m3(B, T, Hq, d_qk, d_v, L_max, _p(q), _p(ix), ix.shape[2], _p(kc), kc.shape[2],
+                                          _p(ks), float(scale), _p(r), n, _p(o), _p(lse), _threads),
+        "sparse_attention_e4m3")
     return o, lse
 
 

@@ -753,4 +753,46 @@ int orc_sparse_attention(int B, int T, int Hq, int d_qk, int d_v, int L_max, con
   return bad ? -1 : 0;
 }
 
+// Attention over an FP8 latent cache (DSA article, "Quantized computation",
+// applied to the KV): row s of sequence b holds d_qk e4m3 codes at
+// kv8 + (b*L_max + s)*kv_stride (bytes) and its fp32 scale k_scale[b*L_max + s];
+// K = code * scale (all d_qk columns), V = the first d_v columns of K. The
+// dequantised rows then enter the same attention as orc_sparse_attention.
+int orc_sparse_attention_e4m3(int B, int T, int Hq, int d_qk, int d_v, int L_max, const uint16_t* qa,
+                              const int32_t* idx, int kk, const uint8_t* kv8, int64_t kv_stride,
+                              const float* k_scale, double scale, const int32_t* rows, int n_rows, double* o,
+                              double* lse, int n_threads) {
+  if (B < 1 || T < 1 || Hq < 1 || d_qk < 1 || d_v < 1 || d_v > d_qk || kk < 0) return -1;
+  const auto list = row_list(B, T, rows, n_rows);
+  std::atomic<int> bad(0);
+  parallel_for(static_cast<int64_t>(list.size()), n_threads, [&](int64_t i) {
+    const int b = list[i].first, t = list[i].second;
+    if (b < 0 || b >= B || t < 0 || t >= T) {
+      bad = 1;
+      return;
+    }
+    const int64_t r = static_cast<int64_t>(b) * T + t;
+    std::vector<int64_t> sel(kk);
+    for (int j = 0; j < kk; ++j) {
+      sel[j] = idx[r * kk + j];
+      if (sel[j] >= L_max) {
+        bad = 1;
+        return;
+      }
+    }
+    std::vector<double> qd(static_cast<size_t>(Hq) * d_qk);
+    for (int64_t e = 0; e < static_cast<int64_t>(Hq) * d_qk; ++e) qd[e] = bf16_value(qa[r * Hq * d_qk + e]);
+    auto row_of = [&](int64_t s, int width, double* out) {
+      const int64_t tok = static_cast<int64_t>(b) * L_max + s;
+      const uint8_t* src = kv8 + tok * kv_stride;
+      const double sc = static_cast<double>(k_scale[tok]);
+      for (int c = 0; c < width; ++c) out[c] = e4m3_value(src[c]) * sc;
+    };
+    attention_row(
+        qd.data(), Hq, d_qk, d_v, sel.data(), kk, [&](int64_t s, double* out) { row_of(s, d_qk, out); },
+        [&](int64_t s, double* out) { row_of(s, d_v, out); }, scale, o + i * Hq * d_v, lse + i * Hq);
+  });
+  return bad ? -1 : 0;
+}
+
 }  // extern "C"

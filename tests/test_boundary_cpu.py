@@ -186,3 +186,23 @@ def test_layer_group_rejects_overlapping_outputs_on_host():
     idx_over = base + out_bytes + 512                  # idx inside the second layer's output
     st = lib.lsa_layer_group(ctypes.byref(ii), None, 0, 0, bu, 2, layers, outs, None, idx_over, None, 0, None)
     assert st == L.LSA_ERR_INVALID_ARG and b"idx" in lib.lsa_last_error()
+
+
+def test_attention_e4m3_kv_validation():
+    lib = L.load()
+    idx = 5 << 20
+    out = 6 << 20
+
+    def call(**kw):
+        ai = _mla_layer(1 << 20, 2 << 20)
+        for f, v in kw.items():
+            setattr(ai, f, v)
+        return lib.lsa_sparse_attn(ctypes.byref(ai), idx, 256, out, None, None, 0, None)
+
+    assert call(kv_dtype=L.LSA_E4M3) == L.LSA_ERR_INVALID_ARG                       # scales missing
+    assert call(kv_dtype=L.LSA_E4M3, k_scale=(3 << 20) + 2) == L.LSA_ERR_INVALID_ARG  # misaligned scales
+    assert call(kv_dtype=L.LSA_E4M3, k_scale=3 << 20, k_row_stride=584, v_row_stride=584) == L.LSA_ERR_INVALID_ARG
+    assert call(kv_dtype=7) == L.LSA_ERR_INVALID_ARG
+    assert call(k_scale=3 << 20) == L.LSA_ERR_INVALID_ARG                            # scales on a bf16 cache
+    small = L.AttnIn(1, 1, 8, 64, 64, 1024, 0.1, 16, 1 << 20, 2 << 20, 2 << 20, 64, 64, -1, -1, L.LSA_E4M3, 3 << 20)
+    assert lib.lsa_sparse_attn(ctypes.byref(small), idx, 256, out, None, None, 0, None) == L.LSA_ERR_UNSUPPORTED

@@ -162,3 +162,87 @@ def test_attention_out_of_range_index_is_skipped_and_flagged(mla):
     skipped[skipped >= w.L] = -1                    # what the kernel computes: the row without those entries
     o_ref, _ = oracle_attn(w, x, skipped, sl)
     assert_attention_close(O.bf16_to_f64(host(out)), o_ref)
+
+
+# ---- FP8 latent cache (e4m3 codes with a per-token scale): K = V = code * scale
+
+def kv_e4m3(x):
+    """The workload's latent rows quantised per token (scale = amax / 448)."""
+    return I.quantize_e4m3_rows(I.bf16_bits_to_f32(x["kv"]))
+
+
+def run_e4m3(w, x, kv8, ks, idx, seq_len, stream_budget=None):
+    sl = dev(seq_len, "i32")
+    lse = torch.empty(idx.shape[:2] + (w.Hq,), dtype=torch.float32, device="cuda")
+    out, _ = L.lsa_sparse_attn(dev(x["qa"], "bf16"), dev(idx, "i32"), sl, w.scale, kv=dev(kv8, "e4m3"),
+                               kv_scale=dev(ks, "f32"), d_v=w.d_v, lse=lse, stream_budget=stream_budget)
+    torch.cuda.synchronize()
+    L.lsa_device_status()
+    return O.bf16_to_f64(host(out)), host(lse)
+
+
+@pytest.mark.parametrize("B,L_,T,n_valid", [(2, 8192, 1, None), (1, 4096, 40, 700), (2, 2048, 3, 5)])
+def test_attention_mla_e4m3_kv_matches_oracle(B, L_, T, n_valid):
+    # splits, ragged lengths, -1 padding and an empty row, against the oracle's
+    # attention over the dequantised cache
+    w = I.scaled(I.WORKLOADS["flat_decode_128k"], B=B, L=L_, T=T)
+    rng = np.random.default_rng(31 + B + T)
+    x = I.make_attn_inputs(w, 31)
+    kv8, ks = kv_e4m3(x)
+    sl = np.array([L_, L_ - 1234][:B], np.int32)
+    idx = rand_idx(rng, w.B, w.T, w.k, w.L, sl, n_valid=n_valid)
+    if T > 2:
+        idx[0, 1] = -1
+    g, gl = run_e4m3(w, x, kv8, ks, idx, sl)
+    o, ol = O.sparse_attention_e4m3_rows(x["qa"], idx, None, scale=w.scale, d_v=w.d_v, kv8=kv8, k_scale=ks)
+    o, ol = o.reshape(g.shape), ol.reshape(gl.shape)
+    assert_attention_close(g, o)
+    fin = np.isfinite(ol)
+    assert np.allclose(gl[fin], ol[fin], atol=1e-3, rtol=1e-3)
+    if T > 2:
+        assert (g[0, 1] == 0).all() and np.isneginf(gl[0, 1]).all()
+
+
+def test_attention_mla_e4m3_kv_streaming_prefix_and_bad_index():
+    w = I.scaled(I.WORKLOADS["flat_decode_128k"], B=2, L=8192)
+    x = I.make_attn_inputs(w, 33)
+    kv8, ks = kv_e4m3(x)
+    sl = np.array([8192, 3000], np.int32)
+    rng = np.random.default_rng(33)
+    sc = rng.standard_normal((2, 1, 8192)).astype(np.float32)
+    for b in range(2):
+        sc[b, 0, sl[b]:] = -np.inf
+    budget = (w.k, w.sink, w.window)
+    oi = O.select_streaming(sc, sl, 1, *budget)
+    g, _ = run_e4m3(w, x, kv8, ks, oi, sl, stream_budget=budget)      # prefix computed, not read
+    o, _ = O.sparse_attention_e4m3_rows(x["qa"], oi, None, scale=w.scale, d_v=w.d_v, kv8=kv8, k_scale=ks)
+    assert_attention_close(g, o.reshape(g.shape))
+    bad = oi.copy()
+    bad[1, 0, 1500] = w.L + 7
+    L.lsa_device_status()
+    L.lsa_sparse_attn(dev(x["qa"], "bf16"), dev(bad, "i32"), dev(sl, "i32"), w.scale, kv=dev(kv8, "e4m3"),
+                      kv_scale=dev(ks, "f32"), d_v=w.d_v)
+    torch.cuda.synchronize()
+    with pytest.raises(L.LsaError) as e:
+        L.lsa_device_status()
+    assert e.value.status == L.LSA_ERR_INVALID_ARG
+
+
+def test_layer_group_e4m3_kv_layers():
+    # two layers with their own e4m3 caches share one attention launch
+    w = I.scaled(I.WORKLOADS["cli_group_256k"], B=2, L=8192)
+    xi = I.make_indexer_inputs(w, 35)
+    lnps = [I.make_attn_inputs(w, 35, layer=i) for i in range(2)]
+    quant = [kv_e4m3(l) for l in lnps]
+    budget = (w.k, w.sink, w.window)
+    q, k, ww, sl = dev(xi["q_idx"], "bf16"), dev(xi["k_idx"], "bf16"), dev(xi["w"], "f32"), dev(xi["seq_len"], "i32")
+    layers = [{"q": dev(l["qa"], "bf16"), "kv": dev(kv8, "e4m3"), "kv_scale": dev(ks, "f32"), "scale": w.scale,
+               "d_v": w.d_v} for l, (kv8, ks) in zip(lnps, quant)]
+    idx, outs = L.lsa_layer_group(q, ww, k, sl, budget, layers)
+    torch.cuda.synchronize()
+    L.lsa_device_status()
+    gi = host(idx)
+    for l, (kv8, ks), out in zip(lnps, quant, outs):
+        o, _ = O.sparse_attention_e4m3_rows(l["qa"], gi, None, scale=w.scale, d_v=w.d_v, kv8=kv8, k_scale=ks)
+        g = O.bf16_to_f64(host(out))
+        assert_attention_close(g, o.reshape(g.shape))

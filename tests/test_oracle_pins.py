@@ -457,6 +457,44 @@ def test_attention_mla_alias_v_is_prefix_of_latent_row():
     assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
 
 
+def test_attention_e4m3_kv_equals_dense_sdpa_on_dequantised_rows():
+    # e4m3 latent cache: K = code * scale (torch's e4m3 decode, float64), V its
+    # first d_v columns; selecting every visible row must equal dense SDPA
+    rng = np.random.default_rng(24)
+    B, T, Hq, dqk, dv, L = 1, 5, 3, 32, 16, 36
+    qa = I.normal_bf16((B, T, Hq, dqk), rng)
+    kv8, ks = I.quantize_e4m3_rows(rng.standard_normal((B, L, dqk)).astype(np.float32) * 3)
+    idx = np.full((B, T, L), -1, np.int32)
+    for t in range(T):
+        pos = L - T + t
+        idx[0, t, :pos + 1] = rng.permutation(pos + 1)
+    o, lse = O.sparse_attention_e4m3_rows(qa, idx, None, scale=0.21, d_v=dv, kv8=kv8, k_scale=ks)
+    kdq = torch.from_numpy(kv8[0].copy()).view(torch.float8_e4m3fn).to(torch.float64) * \
+        torch.from_numpy(ks[0].astype(np.float64))[:, None]
+    qt = torch.from_numpy(O.bf16_to_f64(qa[0])).permute(1, 0, 2)
+    mask = torch.zeros(T, L, dtype=torch.bool)
+    for t in range(T):
+        mask[t, :L - T + t + 1] = True
+    ref = torch.nn.functional.scaled_dot_product_attention(qt, kdq[None].expand(Hq, L, dqk),
+                                                           kdq[None, :, :dv].expand(Hq, L, dv), attn_mask=mask,
+                                                           scale=0.21)
+    assert np.allclose(o.reshape(T, Hq, dv), ref.permute(1, 0, 2).numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_attention_e4m3_kv_single_index_returns_the_scaled_row():
+    rng = np.random.default_rng(25)
+    Hq, dqk, dv, L = 2, 16, 8, 10
+    qa = I.normal_bf16((1, 1, Hq, dqk), rng)
+    kv8 = rng.integers(0, 256, (1, L, dqk)).astype(np.uint8)
+    kv8[(kv8 & 0x7F) == 0x7F] = 0x01                                # no NaN codes
+    ks = np.full((1, L), 0.375, np.float32)
+    o, lse = O.sparse_attention_e4m3_rows(qa, np.array([[[4, -1, -1]]], np.int32), None, scale=0.5, d_v=dv,
+                                          kv8=kv8, k_scale=ks)
+    row = O.e4m3_to_f64(kv8[0, 4]) * 0.375
+    assert np.array_equal(o[0], np.broadcast_to(row[:dv], (Hq, dv)))
+    assert np.allclose(lse[0], 0.5 * O.bf16_to_f64(qa[0, 0]) @ row, rtol=1e-13)
+
+
 # ---------------------------------------------------------------------------
 # cross-layer group
 # ---------------------------------------------------------------------------
