@@ -9,7 +9,7 @@ d_qk 576 / d_v 512). Inputs are seeded synthetic data resident in HBM; L2 is
 flushed (256 MiB write) between timed steps, outside the timed events.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME] [--fp8]
+                    [--workload NAME] [--fp8] [--fp8-kv]
 
 Workloads (kv_indexing_b200.inputs.WORKLOADS): flat_decode_128k (default),
 flat_decode_1m and hier_decode_1m (the same 2 x 1M inputs, hierarchy off / on;
@@ -17,7 +17,8 @@ page pooling timed once, outside the step), cli_group_256k(_flat) (one indexing
 pass feeding two layers), prefill_64k (4096 causal queries; --fp8 for e4m3
 indexer inputs), compressed_decode_1m (262144 entries of 4 tokens; --fp8 for
 e4m3 entry keys), and hier_sweep: flat against hierarchical indexing on the
-same inputs at L = 64K, 256K, 512K and 1M (B=2).
+same inputs at L = 64K, 256K, 512K and 1M (B=2). --fp8-kv stores every
+workload's latent attention cache as e4m3 codes with a per-token fp32 scale.
 
 Each line carries: the device-timed step (one CUDA graph per step, no events
 inside) and its per-stage breakdown (a second graph with events between the
@@ -62,6 +63,8 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--fp8", action="store_true", help="e4m3 indexer keys and queries (prefill, compressed)")
+    p.add_argument("--fp8-kv", action="store_true",
+                   help="e4m3 latent KV cache (per-token scale) for the sparse MLA attention")
     return p.parse_args()
 
 
@@ -86,9 +89,10 @@ def hier_index_bytes_per_query(w, fp8=False) -> int:
     return (w.L // w.P) * w.d * 2 + w.M * w.P * w.d * 2 + w.H * w.d * 2 + w.H * 4
 
 
-def attention_bytes_per_query(w) -> int:
-    """Gathered latent KV rows + q + o."""
-    return w.k * w.d_qk * 2 + w.Hq * w.d_qk * 2 + w.Hq * w.d_v * 2
+def attention_bytes_per_query(w, kv8=False) -> int:
+    """Gathered latent KV rows (e4m3: codes + a 4-byte scale per row) + q + o."""
+    row = w.d_qk + 4 if kv8 else w.d_qk * 2
+    return w.k * row + w.Hq * w.d_qk * 2 + w.Hq * w.d_v * 2
 
 
 def prefill_indexer_flops(w) -> float:
@@ -240,9 +244,9 @@ def host_inputs(w, seed, fp8=False):
 
 
 class Path:
-    def __init__(self, torch, L, w, x, dev, seed, fp8, layers=None):
+    def __init__(self, torch, L, w, x, dev, seed, fp8, layers=None, kv8=False):
         import numpy as np
-        self.torch, self.L, self.w, self.x, self.dev, self.fp8 = torch, L, w, x, dev, fp8
+        self.torch, self.L, self.w, self.x, self.dev, self.fp8, self.kv8 = torch, L, w, x, dev, fp8, kv8
         self.kind = kind_of(w)
         B, T = w.B, w.T
         self.budget = (w.k, w.sink, w.window)
@@ -268,7 +272,15 @@ class Path:
         for li in range(0 if layers is not None else w.n_layers):
             qa = device_bf16_normal(torch, (B, T, w.Hq, w.d_qk), 7919 * seed + 2 * li, dev)
             kv = device_bf16_normal(torch, (B, kv_rows, w.d_qk), 7919 * seed + 2 * li + 1, dev)
-            self.layers.append({"q": qa, "kv": kv, "scale": w.scale, "d_v": w.d_v})
+            lay = {"q": qa, "kv": kv, "scale": w.scale, "d_v": w.d_v}
+            if kv8:   # per-token e4m3: scale = amax / 448, codes = kv / scale (round to nearest even)
+                kf = kv.float()
+                amax = kf.abs().amax(dim=-1)
+                sc = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax)).contiguous()
+                lay["kv"] = (kf / sc[..., None]).to(torch.float8_e4m3fn).contiguous()
+                lay["kv_scale"] = sc
+                del kf
+            self.layers.append(lay)
         self.idx = torch.empty((B, T, w.k), dtype=torch.int32, device=dev)
         self.outs = [torch.empty((B, T, w.Hq, w.d_v), dtype=torch.bfloat16, device=dev) for _ in range(w.n_layers)]
         self.extra = {}
@@ -286,14 +298,15 @@ class Path:
         # attention rows: entries for compressed indexing (decode: the query's entry
         # position is seq_len // m - 1), tokens otherwise
         self.sl_attn = torch.div(sl, w.m, rounding_mode="floor").to(torch.int32) if w.m else sl
-        ai = L.attn_in(lay0["q"], self.sl_attn, w.scale, kv=lay0["kv"], d_v=w.d_v, stream_budget=budget)
+        ai = L.attn_in(lay0["q"], self.sl_attn, w.scale, kv=lay0["kv"], d_v=w.d_v, stream_budget=budget,
+                       kv_scale=lay0.get("kv_scale"))
         self.attn_ws = self._ws(L.workspace_size(L.LSA_OP_SPARSE_ATTN, attn=ai, budget=(w.k, 0, 0)))
 
         def attn(li, idx=None):
             lay = self.layers[li]
             return lambda s: L.lsa_sparse_attn(lay["q"], self.idx if idx is None else idx, self.sl_attn, w.scale,
                                                kv=lay["kv"], d_v=w.d_v, out=self.outs[li], workspace=self.attn_ws,
-                                               stream_budget=budget, stream=s)
+                                               stream_budget=budget, stream=s, kv_scale=lay.get("kv_scale"))
 
         kind = self.kind
         if kind in ("flat", "prefill", "compressed"):
@@ -353,7 +366,7 @@ class Path:
             if w.P:
                 self._pool_once()
             ii = L.indexer_in(q, wt, k, sl)
-            ais = [L.attn_in(l["q"], sl, w.scale, kv=l["kv"], d_v=w.d_v) for l in self.layers]
+            ais = [L.attn_in(l["q"], sl, w.scale, kv=l["kv"], d_v=w.d_v, kv_scale=l.get("kv_scale")) for l in self.layers]
             self.api_ws = self._ws(L.workspace_size(L.LSA_OP_LAYER_GROUP, indexer=ii, attn=ais, budget=budget,
                                                     P=w.P, M=w.M, n_layers=w.n_layers))
             pk = self.page_keys if w.P else None
@@ -374,7 +387,7 @@ class Path:
             self.dominant = "group"
             self.roof_kernel = f"layer-group call (one indexing pass + {w.n_layers} attention layers)"
             ib = hier_index_bytes_per_query(w) if w.P else indexer_bytes_per_query(w)
-            self.roof_bytes = (ib + w.n_layers * attention_bytes_per_query(w)) * B * T
+            self.roof_bytes = (ib + w.n_layers * attention_bytes_per_query(w, self.kv8)) * B * T
 
     def _pool_once(self):
         torch, L, w = self.torch, self.L, self.w
@@ -418,7 +431,8 @@ class Path:
         """The attention call of the step over self.idx (not for the layer group)."""
         lay = self.layers[0]
         self.L.lsa_sparse_attn(qas[0], self.idx, self.sl_attn, self.w.scale, kv=lay["kv"], d_v=self.w.d_v,
-                               out=self.outs[0], workspace=self.attn_ws, stream_budget=self.budget, stream=s)
+                               out=self.outs[0], workspace=self.attn_ws, stream_budget=self.budget, stream=s,
+                               kv_scale=lay.get("kv_scale"))
 
     def api_step(self, s, q, wt, qas):
         """The path through the library's public calls (what an application
@@ -707,6 +721,16 @@ def host_bf16(t):
     return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
 
 
+def host_layer(lay):
+    """A device layer's query and cache as the oracle takes them (e4m3 codes and scales, or bf16)."""
+    import numpy as np
+    import torch
+    if "kv_scale" in lay:
+        return {"qa": host_bf16(lay["q"]), "kv8": lay["kv"].view(torch.uint8).cpu().numpy(),
+                "ks": lay["kv_scale"].cpu().numpy().astype(np.float32)}
+    return {"qa": host_bf16(lay["q"]), "kv": host_bf16(lay["kv"])}
+
+
 class OraclePath:
     """The whole path for a list of query rows on the C++ oracle: indexer scores,
     streaming selection (flat, hierarchical or over entries), then the sparse
@@ -746,7 +770,11 @@ class OraclePath:
             for i, (b, t) in enumerate(rows):
                 idx[b, t] = O.select_streaming_row(sc[i], int(x["seq_len"][b]) - w.T + t, *budget)
         for lay in self.layers:
-            O.sparse_attention_rows(lay["qa"], idx, rows, scale=w.scale, d_v=w.d_v, kv=lay["kv"])
+            if "kv8" in lay:
+                O.sparse_attention_e4m3_rows(lay["qa"], idx, rows, scale=w.scale, d_v=w.d_v, kv8=lay["kv8"],
+                                             k_scale=lay["ks"])
+            else:
+                O.sparse_attention_rows(lay["qa"], idx, rows, scale=w.scale, d_v=w.d_v, kv=lay["kv"])
 
     def all_rows(self):
         return [(b, t) for b in range(self.w.B) for t in range(self.w.T)]
@@ -796,6 +824,9 @@ def run_reference(args, rank: int, world: int):
     x = host_inputs(w, args.seed, args.fp8)
     kv_w = I.entry_workload(w) if w.m else w
     layers = [I.make_attn_inputs(kv_w, args.seed, layer=li) for li in range(w.n_layers)]
+    if args.fp8_kv:   # the same per-token e4m3 quantisation the device path applies
+        for lay in layers:
+            lay["kv8"], lay["ks"] = I.quantize_e4m3_rows(I.bf16_bits_to_f32(lay.pop("kv")))
     op = OraclePath(w, x, layers, fp8=args.fp8)
     rows = op.all_rows()
     if op.kind == "prefill":
@@ -821,7 +852,8 @@ def run_reference(args, rank: int, world: int):
         "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1000 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (the same seeded inputs as our arm's host generator)",
-        "config": workload_config(w, parallelism="host threads", l2="n/a (host run)"),
+        "config": workload_config(w, parallelism="host threads", l2="n/a (host run)", fp8_indexer=bool(args.fp8),
+                                  kv_cache="e4m3 (per-token fp32 scale)" if args.fp8_kv else "bf16"),
         "cpu_baseline": {"value": v, "unit": UNIT, "cores": O.threads(), "kind": "oracle", "sample": sample},
         "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -891,7 +923,7 @@ def step_bytes(path) -> float:
         return path.roof_bytes
     else:
         ib = indexer_bytes_per_query(w, path.fp8, w.L // w.m if w.m else w.L)
-    return (ib + attention_bytes_per_query(w) + w.k * 4) * w.B * w.T
+    return (ib + attention_bytes_per_query(w, path.kv8) + w.k * 4) * w.B * w.T
 
 
 def run_workload(args, w, rank, world, dev, pg):
@@ -901,7 +933,7 @@ def run_workload(args, w, rank, world, dev, pg):
 
     seed = rank_seed(args.seed, rank)
     x = host_inputs(w, seed, args.fp8)
-    path = Path(torch, L, w, x, dev, seed, args.fp8)
+    path = Path(torch, L, w, x, dev, seed, args.fp8, kv8=args.fp8_kv)
     flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
     def flush():
@@ -926,7 +958,7 @@ def run_workload(args, w, rank, world, dev, pg):
     L.lsa_device_status()
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        layers_host = [{"qa": host_bf16(l["q"]), "kv": host_bf16(l["kv"])} for l in path.layers]
+        layers_host = [host_layer(l) for l in path.layers]
         del flush_buf
         torch.cuda.empty_cache()
         cpu = cpu_baseline(OraclePath(w, x, layers_host, fp8=args.fp8))
@@ -939,7 +971,8 @@ def run_workload(args, w, rank, world, dev, pg):
                     "the host generator; latent KV and attention queries drawn on the device with a seeded "
                     "generator)",
             "config": workload_config(w, parallelism=f"replicas x{world} (independent batches)",
-                                      fp8_indexer=bool(args.fp8)),
+                                      fp8_indexer=bool(args.fp8),
+                                      kv_cache="e4m3 (per-token fp32 scale)" if args.fp8_kv else "bf16"),
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": (t["launches_per_step"] or 0) * args.steps,
             "launches_per_step": t["launches_per_step"],
