@@ -425,7 +425,7 @@ constexpr int kOffTag = kOffSend + kXBytes;         // [2][2][128] u64 tagged ma
 constexpr int kOffMask = kOffTag + (4 * 128 + 2 * 128) * 8;
 constexpr int kOffKScale = kOffMask + kStages * 8;   // e4m3 KV: [kStages][BN] token scales of the staged rows
 constexpr int kOffBars = kOffKScale + kStages * BN * 4;
-constexpr int kNumBars = 2 * kStages + 11;
+constexpr int kNumBars = 2 * kStages + 13;
 constexpr int kOffMisc = kOffBars + kNumBars * 8;
 constexpr size_t kSmem = 1024 + kOffMisc + 16;
 static_assert(kOffBars % 8 == 0, "mbarriers need 8-byte alignment");
@@ -517,6 +517,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   uint64_t* send_full = q_ready + 1;  // the outgoing buffer is written
   uint64_t* send_free = send_full + 1;  // the bulk copy has read it
   uint64_t* q_full = send_free + 1;     // q chunks staged in shared memory
+  uint64_t* x_free = q_full + 1;        // [2] the partner has read what this CTA sent into its buffer i
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -575,6 +576,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mbar_init(send_full, kSoftThreads);
     mbar_init(send_free, 1);
     mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) mbar_init(&x_free[i], 1);   // the partner's MMA issuer, remotely
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -726,6 +728,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (lane == 0 && nblk > 0) {
       const uint32_t idesc_qk = make_idesc(1, 1, 128, BN, 0, 0);
       const uint32_t idesc_pv = make_idesc(1, 1, 128, 256, 0, 1);
+      const uint32_t peer_xfree = mapa_shared(smem_u32(x_free), peer);
       auto issue_pv = [&](int pb) -> bool {
         if (!wait_ph<false>(p_full, pb & 1, a.status, abort_flag)) return false;
         tc_fence_after();
@@ -737,6 +740,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         umma_commit(pv_done);
         umma_commit(&kv_empty[pb % kStages]);
+        // P(pb) is stored, so every softmax thread has read block pb's partial
+        // scores from exchange buffer pb & 1: the partner may copy block pb + 2
+        // into it (a cumulative release of what p_full acquired)
+        mbar_arrive_remote(peer_xfree + (pb & 1) * 8);
         return true;
       };
       bool ok = wait_ph<false>(q_ready, 0, a.status, abort_flag);
@@ -828,6 +835,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (leader) {
         mbar_arrive_expect_tx(&x_full[i], kXTotalBytes);
         lok = wait_ph<false>(send_full, bb & 1, a.status, abort_flag);
+        // the partner's buffer i still holds block bb - 2 until its readers have
+        // signalled (remote arrivals on this CTA's x_free[i])
+        if (lok && bb >= 2) lok = wait_ph<true>(&x_free[i], ((bb - 2) >> 1) & 1, a.status, abort_flag);
         if (lok) {
           bulk_copy_to_peer(peer_x + i * kXBytes, sSend, kXBytes, peer_xfull + i * 8);
           bulk_commit();

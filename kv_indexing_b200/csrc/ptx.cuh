@@ -292,6 +292,12 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
 
 // Bulk copy of `bytes` (multiple of 16) from this CTA's shared memory into
 // another CTA's (cluster address), counted on that CTA's mbarrier.
+// Arrive (release, cluster scope) on an mbarrier in another CTA of the
+// cluster; remote_bar is its shared::cluster address (mapa).
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t remote_bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
+}
+
 __device__ __forceinline__ void bulk_copy_to_peer(uint32_t remote_dst, const void* src, uint32_t bytes,
                                                   uint32_t remote_bar) {
   asm volatile(
