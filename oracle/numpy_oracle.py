@@ -60,12 +60,12 @@ R11 Compressed entries (the DSA article's "Technical Evolution": the indexer
     name no compressor). Scores are R1 on the entry keys; the selection is
     R3-R5 over entries, at entry position (pos + 1) // m - 1, with budget, sink
     and window counted in entries. m = 1 is flat indexing.
-R12 FP8 hierarchical indexing (the survey's next item; the pages only name
-    "quantized computation"): token keys and queries as R10. A page key is the
-    float32 mean of its tokens' dequantized keys (R6's order and division),
-    stored as e4m3 with a float32 page scale amax / 448 (round to nearest even,
-    saturating), like the token keys. Page and fine scores are R1 on the
-    dequantized values; recall and selection as R7.
+R12 FP8 hierarchical indexing (the pages only name "quantized computation"):
+    token keys and queries as R10. A page key is the float32 mean of its
+    tokens' dequantized keys (R6's order and division), stored as e4m3 with a
+    float32 page scale amax / 448 (round to nearest even, saturating), like
+    the token keys. Page and fine scores are R1 on the dequantized values;
+    recall and selection as R7.
 """
 from __future__ import annotations
 
