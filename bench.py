@@ -824,6 +824,10 @@ def run_reference(args, rank: int, world: int):
     x = host_inputs(w, args.seed, args.fp8)
     kv_w = I.entry_workload(w) if w.m else w
     layers = [I.make_attn_inputs(kv_w, args.seed, layer=li) for li in range(w.n_layers)]
+    if not w.mla:   # our arm's cache has one row per token, V its first d_v columns: the same here
+        for lay in layers:
+            lay["kv"] = lay.pop("k")
+            del lay["v"]
     if args.fp8_kv:   # the same per-token e4m3 quantisation the device path applies
         for lay in layers:
             lay["kv8"], lay["ks"] = I.quantize_e4m3_rows(I.bf16_bits_to_f32(lay.pop("kv")))
