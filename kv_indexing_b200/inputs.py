@@ -163,16 +163,24 @@ def f32_to_e4m3_bits(x: np.ndarray) -> np.ndarray:
     return out.astype(np.uint8)
 
 
-def quantize_e4m3_rows(x: np.ndarray) -> tuple:
+def quantize_e4m3_rows(x: np.ndarray, chunk_rows: int = 1 << 14) -> tuple:
     """Quantise along the last axis: scale = amax / 448, codes = e4m3(x / scale).
 
     Rows that are entirely zero get scale 1. Returns (codes uint8, scale float32).
+    Rows are encoded chunk_rows at a time, so a 1M-token latent cache needs no
+    more than a few hundred MB of temporaries; every row is independent.
     """
     x = np.asarray(x, dtype=np.float32)
-    amax = np.max(np.abs(x), axis=-1)
-    scale = np.where(amax > 0, amax / np.float32(_E4M3_MAX), np.float32(1.0)).astype(np.float32)
-    codes = f32_to_e4m3_bits(x / scale[..., None])
-    return codes, scale
+    flat = x.reshape(-1, x.shape[-1])
+    codes = np.empty(flat.shape, dtype=np.uint8)
+    scale = np.empty(flat.shape[0], dtype=np.float32)
+    for r0 in range(0, flat.shape[0], chunk_rows):
+        blk = flat[r0:r0 + chunk_rows]
+        amax = np.max(np.abs(blk), axis=-1)
+        sc = np.where(amax > 0, amax / np.float32(_E4M3_MAX), np.float32(1.0)).astype(np.float32)
+        codes[r0:r0 + chunk_rows] = f32_to_e4m3_bits(blk / sc[:, None])
+        scale[r0:r0 + chunk_rows] = sc
+    return codes.reshape(x.shape), scale.reshape(x.shape[:-1])
 
 
 # ---------------------------------------------------------------------------

@@ -85,6 +85,23 @@ def test_input_e4m3_encoder_matches_torch():
     assert np.array_equal(I.f32_to_e4m3_bits(x), ref)
 
 
+@pytest.mark.parametrize("shape", [(5,), (3, 7, 64), (2, 4001, 16)])
+def test_input_e4m3_row_quantiser_is_per_row_amax_over_448(shape):
+    # scale = amax / 448 per row (1 for an all-zero row), codes = torch's e4m3 of
+    # x / scale; rows are encoded in chunks, which must not change a byte
+    rng = np.random.default_rng(5)
+    x = (rng.standard_normal(shape) * 5).astype(np.float32)
+    x.reshape(-1, shape[-1])[0] = 0
+    t = torch.from_numpy(x)
+    amax = t.abs().amax(dim=-1)
+    sc = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+    ref = (t / sc[..., None]).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    for chunk in (1 << 14, 997):
+        codes, scale = I.quantize_e4m3_rows(x, chunk_rows=chunk)
+        assert codes.shape == x.shape and scale.shape == x.shape[:-1]
+        assert np.array_equal(scale, sc.numpy()) and np.array_equal(codes, ref)
+
+
 # ---------------------------------------------------------------------------
 # indexer score
 # ---------------------------------------------------------------------------
