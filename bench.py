@@ -58,7 +58,8 @@ def parse():
     p.add_argument("--steps", type=int, default=200)
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    p.add_argument("--workload", default="flat_decode_128k")
+    from kv_indexing_b200.inputs import WORKLOADS
+    p.add_argument("--workload", default="flat_decode_128k", choices=sorted(WORKLOADS) + ["hier_sweep"])
     p.add_argument("--seed", type=int, default=1)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
@@ -818,9 +819,14 @@ def run_reference(args, rank: int, world: int):
     """The C++ oracle as it stands on the host cores, same workload and metric."""
     if rank != 0:
         return 0
+    if args.workload == "hier_sweep":
+        print(json.dumps({"impl": "reference", "unavailable": "hier_sweep is a table of device timings (flat against "
+                          "hierarchical indexing at four lengths); the oracle arm times single workloads, e.g. "
+                          "--workload hier_decode_1m"}), flush=True)
+        return 0
     import oracle as O
     from kv_indexing_b200 import inputs as I
-    w = I.WORKLOADS[args.workload if args.workload in I.WORKLOADS else "flat_decode_128k"]
+    w = I.WORKLOADS[args.workload]
     x = host_inputs(w, args.seed, args.fp8)
     kv_w = I.entry_workload(w) if w.m else w
     layers = [I.make_attn_inputs(kv_w, args.seed, layer=li) for li in range(w.n_layers)]

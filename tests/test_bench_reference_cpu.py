@@ -39,3 +39,14 @@ def test_reference_arm_line():
 def test_reference_arm_fp8_indexer_line():
     j = _reference_line("--fp8")
     assert j["config"]["fp8_indexer"] is True and j["value"] > 0
+
+
+def test_reference_arm_declines_the_sweep_and_unknown_workloads():
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", "hier_sweep"],
+                       cwd=ROOT, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0
+    j = json.loads(r.stdout.strip().splitlines()[-1])
+    assert j["impl"] == "reference" and "hier_sweep" in j["unavailable"]
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", "no_such_workload"],
+                       cwd=ROOT, capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0 and "invalid choice" in r.stderr
