@@ -138,6 +138,9 @@ def _need(t, name, dtype=None, dim=None):
         raise ValueError(f"{name} is required")
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
+    cur = torch.cuda.current_device()
+    if t.device.index != cur:   # the kernels launch on the current device and would read another GPU's memory
+        raise ValueError(f"{name} is on {t.device}, but the calls launch on the current device cuda:{cur}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if dtype is not None:
@@ -146,6 +149,17 @@ def _need(t, name, dtype=None, dim=None):
             raise ValueError(f"{name} has dtype {t.dtype}, expected {dts}")
     if dim is not None and t.dim() != dim:
         raise ValueError(f"{name} must have {dim} dims")
+    return t
+
+
+def _out(t, name, dtype, shape):
+    """A caller-supplied output (or None): a contiguous CUDA tensor on the current
+    device with exactly the documented shape, since the kernels write all of it."""
+    if t is None:
+        return None
+    _need(t, name, dtype, len(shape))
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
     return t
 
 
@@ -227,6 +241,7 @@ def _workspace(nbytes: int, device, workspace=None):
     if nbytes == 0:
         return None
     if workspace is not None:
+        _need(workspace, "workspace")
         if workspace.numel() * workspace.element_size() < nbytes:
             raise ValueError(f"workspace smaller than the {nbytes} bytes required")
         return workspace
@@ -251,6 +266,9 @@ def lsa_index_flat(q, w, k, seq_len, budget, *, q_scale=None, k_scale=None, idx=
     B, T = q.shape[0], q.shape[1]
     if with_idx and idx is None:
         idx = torch.empty((B, T, budget[0]), dtype=torch.int32, device=q.device)
+    if with_idx:
+        _out(idx, "idx", torch.int32, (B, T, budget[0]))
+    _out(scores_out, "scores_out", torch.float32, (B, T, k.shape[1]))
     need = workspace_size(LSA_OP_INDEX_FLAT, indexer=ii, budget=budget, scores_external=scores_out is not None)
     ws = _workspace(need, q.device, workspace)
     _check(lib.lsa_index_flat(ctypes.byref(ii), Budget(*budget), _ptr(idx) if with_idx else None, _ptr(scores_out),
@@ -269,6 +287,9 @@ def lsa_index_compressed(q, w, entry_keys, seq_len, m, budget, *, q_scale=None, 
     B, T = q.shape[0], q.shape[1]
     if with_idx and idx is None:
         idx = torch.empty((B, T, budget[0]), dtype=torch.int32, device=q.device)
+    if with_idx:
+        _out(idx, "idx", torch.int32, (B, T, budget[0]))
+    _out(scores_out, "scores_out", torch.float32, (B, T, entry_keys.shape[1]))
     need = workspace_size(LSA_OP_INDEX_COMPRESSED, indexer=ii, budget=budget, m=m,
                           scores_external=scores_out is not None)
     ws = _workspace(need, q.device, workspace)
@@ -286,6 +307,7 @@ def lsa_select_streaming(scores, seq_len, budget, *, idx=None, workspace=None, s
     B, T, L_max = scores.shape
     if idx is None:
         idx = torch.empty((B, T, budget[0]), dtype=torch.int32, device=scores.device)
+    _out(idx, "idx", torch.int32, (B, T, budget[0]))
     need = workspace_size(LSA_OP_SELECT, budget=budget, B=B, T=T, L_max=L_max)
     ws = _workspace(need, scores.device, workspace)
     _check(lib.lsa_select_streaming(_ptr(scores), _ptr(seq_len), B, T, L_max, Budget(*budget), _ptr(idx), _ptr(ws),
@@ -306,7 +328,7 @@ def lsa_select_streaming_noalloc(scores, seq_len, budget, *, idx=None, stream=No
     B, T, L_max = scores.shape
     if idx is None:
         idx = torch.empty((B, T, budget[0]), dtype=torch.int32, device=scores.device)
-    _need(idx, "idx", torch.int32, 3)
+    _out(idx, "idx", torch.int32, (B, T, budget[0]))
     _check(lib.lsa_select_streaming_noalloc(_ptr(scores), _ptr(seq_len), B, T, L_max, Budget(*budget), _ptr(idx),
                                             _stream(stream)))
     return idx
@@ -321,6 +343,7 @@ def lsa_pool_pages(k, seq_len, P, *, page_keys=None, stream=None):
     B, L_max, d = k.shape
     if page_keys is None:
         page_keys = torch.zeros((B, L_max // P, d), dtype=torch.bfloat16, device=k.device)
+    _out(page_keys, "page_keys", torch.bfloat16, (B, L_max // P, d))
     _check(lib.lsa_pool_pages(_ptr(k), _ptr(seq_len), B, L_max, d, P, _ptr(page_keys), _stream(stream)))
     return page_keys
 
@@ -335,6 +358,8 @@ def lsa_index_hier(q, w, k, seq_len, page_keys, P, M, budget, *, idx=None, pages
     B, T = q.shape[0], q.shape[1]
     if idx is None:
         idx = torch.empty((B, T, budget[0]), dtype=torch.int32, device=q.device)
+    _out(idx, "idx", torch.int32, (B, T, budget[0]))
+    _out(pages_out, "pages_out", torch.int32, (B, T, M))
     need = workspace_size(LSA_OP_INDEX_HIER, indexer=ii, budget=budget, P=P, M=M)
     ws = _workspace(need, q.device, workspace)
     _check(lib.lsa_index_hier(ctypes.byref(ii), _ptr(page_keys), P, M, Budget(*budget), _ptr(idx), _ptr(pages_out),
@@ -355,6 +380,8 @@ def lsa_pool_pages_e4m3(k8, k_scale, seq_len, P, *, page_codes=None, page_scales
         page_codes = torch.zeros((B, L_max // P, d), dtype=torch.uint8, device=k8.device).view(k8.dtype)
     if page_scales is None:
         page_scales = torch.ones((B, L_max // P), dtype=torch.float32, device=k8.device)
+    _out(page_codes, "page_codes", (torch.float8_e4m3fn, torch.uint8), (B, L_max // P, d))
+    _out(page_scales, "page_scales", torch.float32, (B, L_max // P))
     _check(lib.lsa_pool_pages_e4m3(_ptr(k8), _ptr(k_scale), _ptr(seq_len), B, L_max, d, P, _ptr(page_codes),
                                    _ptr(page_scales), _stream(stream)))
     return page_codes, page_scales
@@ -371,6 +398,8 @@ def lsa_index_hier_e4m3(q8, q_scale, w, k8, k_scale, seq_len, page_codes, page_s
     B, T = q8.shape[0], q8.shape[1]
     if idx is None:
         idx = torch.empty((B, T, budget[0]), dtype=torch.int32, device=q8.device)
+    _out(idx, "idx", torch.int32, (B, T, budget[0]))
+    _out(pages_out, "pages_out", torch.int32, (B, T, M))
     need = workspace_size(LSA_OP_INDEX_HIER, indexer=ii, budget=budget, P=P, M=M)
     ws = _workspace(need, q8.device, workspace)
     _check(lib.lsa_index_hier_e4m3(ctypes.byref(ii), _ptr(page_codes), _ptr(page_scales), P, M, Budget(*budget),
@@ -388,8 +417,12 @@ def lsa_sparse_attn(q, idx, seq_len, scale, *, kv=None, k=None, v=None, d_v=None
     lib = load()
     ai = attn_in(q, seq_len, scale, kv=kv, k=k, v=v, d_v=d_v, stream_budget=stream_budget, kv_scale=kv_scale)
     _need(idx, "idx", torch.int32, 3)
+    if tuple(idx.shape[:2]) != (ai.B, ai.T):
+        raise ValueError(f"idx has shape {tuple(idx.shape)}, expected [{ai.B}, {ai.T}, k]")
     if out is None:
         out = torch.empty((ai.B, ai.T, ai.Hq, ai.d_v), dtype=torch.bfloat16, device=q.device)
+    _out(out, "out", torch.bfloat16, (ai.B, ai.T, ai.Hq, ai.d_v))
+    _out(lse, "lse", torch.float32, (ai.B, ai.T, ai.Hq))
     need = workspace_size(LSA_OP_SPARSE_ATTN, attn=ai, budget=(idx.shape[2], 0, 0))
     ws = _workspace(need, q.device, workspace)
     _check(lib.lsa_sparse_attn(ctypes.byref(ai), _ptr(idx), idx.shape[2], _ptr(out), _ptr(lse), _ptr(ws), _nbytes(ws),
@@ -413,6 +446,15 @@ def lsa_layer_group(q, w, k, seq_len, budget, layers: Sequence[dict], *, P=0, M=
         outs = [torch.empty((a.B, a.T, a.Hq, a.d_v), dtype=torch.bfloat16, device=q.device) for a in ais]
     if idx is None:
         idx = torch.empty((q.shape[0], q.shape[1], budget[0]), dtype=torch.int32, device=q.device)
+    _out(idx, "idx", torch.int32, (q.shape[0], q.shape[1], budget[0]))
+    if len(outs) != n or (lses is not None and len(lses) != n):
+        raise ValueError(f"outs and lses need one entry per layer ({n})")
+    for i, a in enumerate(ais):
+        _out(outs[i], f"outs[{i}]", torch.bfloat16, (a.B, a.T, a.Hq, a.d_v))
+        if lses is not None:
+            _out(lses[i], f"lses[{i}]", torch.float32, (a.B, a.T, a.Hq))
+    if page_keys is not None:
+        _out(page_keys, "page_keys", torch.bfloat16, (q.shape[0], k.shape[1] // P if P else 0, k.shape[2]))
     need = workspace_size(LSA_OP_LAYER_GROUP, indexer=ii, attn=ais, budget=budget, P=P, M=M, n_layers=n)
     ws = _workspace(need, q.device, workspace)
     arr = (AttnIn * n)(*ais)

@@ -206,3 +206,49 @@ def test_attention_e4m3_kv_validation():
     assert call(k_scale=3 << 20) == L.LSA_ERR_INVALID_ARG                            # scales on a bf16 cache
     small = L.AttnIn(1, 1, 8, 64, 64, 1024, 0.1, 16, 1 << 20, 2 << 20, 2 << 20, 64, 64, -1, -1, L.LSA_E4M3, 3 << 20)
     assert lib.lsa_sparse_attn(ctypes.byref(small), idx, 256, out, None, None, 0, None) == L.LSA_ERR_UNSUPPORTED
+
+
+class _DeviceTensor:
+    """Stands in for a CUDA tensor in the binding's argument checks (no GPU here)."""
+
+    def __init__(self, shape, dtype, device=0, contiguous=True):
+        import torch
+        self.shape, self.dtype, self.is_cuda = torch.Size(shape), dtype, True
+        self.device = torch.device("cuda", device)
+        self._contiguous = contiguous
+
+    def is_contiguous(self):
+        return self._contiguous
+
+    def dim(self):
+        return len(self.shape)
+
+    def numel(self):
+        return self.shape.numel()
+
+    def element_size(self):
+        import torch
+        return torch.empty((), dtype=self.dtype).element_size()
+
+
+def test_binding_checks_device_layout_dtype_and_shape(monkeypatch):
+    import torch
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    i32 = torch.int32
+    assert L._out(_DeviceTensor((2, 1, 2048), i32), "idx", i32, (2, 1, 2048)) is not None
+    assert L._out(None, "idx", i32, (2, 1, 2048)) is None
+    cases = [
+        (torch.empty((2, 1, 2048), dtype=i32), "must be a CUDA tensor"),
+        (_DeviceTensor((2, 1, 2048), i32, device=1), "current device"),
+        (_DeviceTensor((2, 1, 2048), i32, contiguous=False), "contiguous"),
+        (_DeviceTensor((2, 1, 2048), torch.int64), "dtype"),
+        (_DeviceTensor((2, 2048), i32), "dims"),
+        (_DeviceTensor((2, 1, 1024), i32), "shape"),   # a short idx would be written past its end
+    ]
+    for t, msg in cases:
+        with pytest.raises(ValueError, match=msg):
+            L._out(t, "idx", i32, (2, 1, 2048))
+    with pytest.raises(ValueError, match="current device"):
+        L._workspace(4096, None, _DeviceTensor((4096,), torch.uint8, device=1))
+    with pytest.raises(ValueError, match="smaller"):
+        L._workspace(4096, None, _DeviceTensor((4095,), torch.uint8))
