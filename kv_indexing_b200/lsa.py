@@ -152,14 +152,20 @@ def _need(t, name, dtype=None, dim=None):
     return t
 
 
+def _dims(t, name, shape):
+    """t's shape must equal `shape` (None = any size in that place)."""
+    if len(t.shape) != len(shape) or any(want is not None and got != want for got, want in zip(t.shape, shape)):
+        want = tuple("*" if n is None else n for n in shape)
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {want}")
+
+
 def _out(t, name, dtype, shape):
     """A caller-supplied output (or None): a contiguous CUDA tensor on the current
     device with exactly the documented shape, since the kernels write all of it."""
     if t is None:
         return None
     _need(t, name, dtype, len(shape))
-    if tuple(t.shape) != tuple(shape):
-        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    _dims(t, name, shape)
     return t
 
 
@@ -173,9 +179,14 @@ def indexer_in(q, w, k, seq_len, q_scale=None, k_scale=None, m=1) -> IndexerIn:
     _need(w, "w", torch.float32, 3)
     _need(seq_len, "seq_len", torch.int32, 1)
     B, T, H, d = q.shape
+    _dims(k, "k", (B, None, d))
+    _dims(w, "w", (B, T, H))
+    _dims(seq_len, "seq_len", (B,))
     if fp8:
         _need(q_scale, "q_scale", torch.float32, 3)
         _need(k_scale, "k_scale", torch.float32, 2)
+        _dims(q_scale, "q_scale", (B, T, H))
+        _dims(k_scale, "k_scale", (B, k.shape[1]))
     return IndexerIn(B, T, H, d, k.shape[1] * m, LSA_E4M3 if fp8 else LSA_BF16, _ptr(seq_len), _ptr(q),
                      _ptr(q_scale) if fp8 else None, _ptr(w), _ptr(k), _ptr(k_scale) if fp8 else None)
 
@@ -189,9 +200,11 @@ def attn_in(q, seq_len, scale, *, kv=None, k=None, v=None, d_v=None, stream_budg
     _need(q, "q", torch.bfloat16, 4)
     _need(seq_len, "seq_len", torch.int32, 1)
     B, T, Hq, d_qk = q.shape
+    _dims(seq_len, "seq_len", (B,))
     ss, sw = (-1, -1) if stream_budget is None else (int(stream_budget[1]), int(stream_budget[2]))
     if kv is not None and kv.dtype == torch.float8_e4m3fn:
         _need(kv, "kv", torch.float8_e4m3fn, 3)
+        _dims(kv, "kv", (B, None, None))
         if kv_scale is None:
             raise ValueError("an e4m3 kv needs kv_scale [B, L_max] float32")
         _need(kv_scale, "kv_scale", torch.float32, 2)
@@ -204,11 +217,14 @@ def attn_in(q, seq_len, scale, *, kv=None, k=None, v=None, d_v=None, stream_budg
         raise ValueError("kv_scale is for an e4m3 kv only")
     if kv is not None:
         _need(kv, "kv", torch.bfloat16, 3)
+        _dims(kv, "kv", (B, None, None))
         dv = d_v if d_v is not None else (512 if d_qk == 576 else d_qk)
         return AttnIn(B, T, Hq, d_qk, dv, kv.shape[1], float(scale), _ptr(seq_len), _ptr(q), _ptr(kv), _ptr(kv),
                       kv.shape[2], kv.shape[2], ss, sw)
     _need(k, "k", torch.bfloat16, 3)
     _need(v, "v", torch.bfloat16, 3)
+    _dims(k, "k", (B, None, None))
+    _dims(v, "v", (B, k.shape[1], None))
     return AttnIn(B, T, Hq, d_qk, v.shape[2], k.shape[1], float(scale), _ptr(seq_len), _ptr(q), _ptr(k), _ptr(v),
                   k.shape[2], v.shape[2], ss, sw)
 
@@ -305,6 +321,7 @@ def lsa_select_streaming(scores, seq_len, budget, *, idx=None, workspace=None, s
     _need(scores, "scores", torch.float32, 3)
     _need(seq_len, "seq_len", torch.int32, 1)
     B, T, L_max = scores.shape
+    _dims(seq_len, "seq_len", (B,))
     if idx is None:
         idx = torch.empty((B, T, budget[0]), dtype=torch.int32, device=scores.device)
     _out(idx, "idx", torch.int32, (B, T, budget[0]))
@@ -326,6 +343,7 @@ def lsa_select_streaming_noalloc(scores, seq_len, budget, *, idx=None, stream=No
     _need(scores, "scores", torch.float32, 3)
     _need(seq_len, "seq_len", torch.int32, 1)
     B, T, L_max = scores.shape
+    _dims(seq_len, "seq_len", (B,))
     if idx is None:
         idx = torch.empty((B, T, budget[0]), dtype=torch.int32, device=scores.device)
     _out(idx, "idx", torch.int32, (B, T, budget[0]))
@@ -341,6 +359,7 @@ def lsa_pool_pages(k, seq_len, P, *, page_keys=None, stream=None):
     _need(k, "k", torch.bfloat16, 3)
     _need(seq_len, "seq_len", torch.int32, 1)
     B, L_max, d = k.shape
+    _dims(seq_len, "seq_len", (B,))
     if page_keys is None:
         page_keys = torch.zeros((B, L_max // P, d), dtype=torch.bfloat16, device=k.device)
     _out(page_keys, "page_keys", torch.bfloat16, (B, L_max // P, d))
@@ -355,6 +374,8 @@ def lsa_index_hier(q, w, k, seq_len, page_keys, P, M, budget, *, idx=None, pages
     lib = load()
     ii = indexer_in(q, w, k, seq_len)
     _need(page_keys, "page_keys", torch.bfloat16, 3)
+    if P > 0:
+        _dims(page_keys, "page_keys", (q.shape[0], k.shape[1] // P, q.shape[3]))
     B, T = q.shape[0], q.shape[1]
     if idx is None:
         idx = torch.empty((B, T, budget[0]), dtype=torch.int32, device=q.device)
@@ -376,6 +397,8 @@ def lsa_pool_pages_e4m3(k8, k_scale, seq_len, P, *, page_codes=None, page_scales
     _need(k_scale, "k_scale", torch.float32, 2)
     _need(seq_len, "seq_len", torch.int32, 1)
     B, L_max, d = k8.shape
+    _dims(k_scale, "k_scale", (B, L_max))
+    _dims(seq_len, "seq_len", (B,))
     if page_codes is None:
         page_codes = torch.zeros((B, L_max // P, d), dtype=torch.uint8, device=k8.device).view(k8.dtype)
     if page_scales is None:
@@ -395,6 +418,9 @@ def lsa_index_hier_e4m3(q8, q_scale, w, k8, k_scale, seq_len, page_codes, page_s
     ii = indexer_in(q8, w, k8, seq_len, q_scale, k_scale)
     _need(page_codes, "page_codes", (torch.float8_e4m3fn, torch.uint8), 3)
     _need(page_scales, "page_scales", torch.float32, 2)
+    if P > 0:
+        _dims(page_codes, "page_codes", (q8.shape[0], k8.shape[1] // P, q8.shape[3]))
+        _dims(page_scales, "page_scales", (q8.shape[0], k8.shape[1] // P))
     B, T = q8.shape[0], q8.shape[1]
     if idx is None:
         idx = torch.empty((B, T, budget[0]), dtype=torch.int32, device=q8.device)

@@ -252,3 +252,22 @@ def test_binding_checks_device_layout_dtype_and_shape(monkeypatch):
         L._workspace(4096, None, _DeviceTensor((4096,), torch.uint8, device=1))
     with pytest.raises(ValueError, match="smaller"):
         L._workspace(4096, None, _DeviceTensor((4095,), torch.uint8))
+
+
+def test_binding_checks_input_shapes_against_each_other(monkeypatch):
+    import torch
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    bf, f32, i32 = torch.bfloat16, torch.float32, torch.int32
+    q, k = _DeviceTensor((2, 1, 64, 128), bf), _DeviceTensor((2, 4096, 128), bf)
+    w, sl = _DeviceTensor((2, 1, 64), f32), _DeviceTensor((2,), i32)
+    for args, msg in [((q, w, _DeviceTensor((3, 4096, 128), bf), sl), "k has shape"),
+                      ((q, w, _DeviceTensor((2, 4096, 64), bf), sl), "k has shape"),
+                      ((q, _DeviceTensor((2, 1, 32), f32), k, sl), "w has shape"),
+                      ((q, w, k, _DeviceTensor((1,), i32)), "seq_len has shape")]:
+        with pytest.raises(ValueError, match=msg):
+            L.indexer_in(*args)
+    qa = _DeviceTensor((2, 1, 16, 64), bf)
+    with pytest.raises(ValueError, match="v has shape"):
+        L.attn_in(qa, sl, 0.125, k=_DeviceTensor((2, 4096, 64), bf), v=_DeviceTensor((2, 2048, 64), bf))
+    with pytest.raises(ValueError, match="kv has shape"):
+        L.attn_in(_DeviceTensor((2, 1, 128, 576), bf), sl, 0.04, kv=_DeviceTensor((1, 4096, 576), bf))
